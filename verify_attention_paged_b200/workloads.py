@@ -1,0 +1,291 @@
+"""Seeded synthetic inputs for paged decode / verification attention.
+
+This module only draws random numbers and lays them out; it holds none of the
+attention arithmetic.  Both the CUDA path's tests and the oracle's tests take
+their inputs from here, and it imports neither of them.
+
+Layout it produces (the fragment-addressed cache of the LSE releases page,
+v0.4.20 "K/V memory management and automatic split attention"):
+
+* the arena is ``n_chunks`` chunks of ``chunk_bytes`` each, cut into
+  fragments of ``fragment_bytes``; fragment id ``f`` lives in chunk
+  ``f // (chunk_bytes // fragment_bytes)``;
+* a fragment holds ``T`` consecutive tokens of K (or of V) for every kv head,
+  token-major: ``[token][kv_head][dim]``;
+* sequence ``s`` reaches key ``j`` through ``k_pages[s, j // T]`` (and
+  ``v_pages`` for V); K and V use separate fragments;
+* fragments are handed out in a shuffled order; unused page-table entries
+  hold -1; every byte of the arena not holding a live key is 0xFF, which is
+  NaN in all five storage formats, so any read of a dead slot shows up.
+
+The five named workloads follow the benchmark configurations of the
+specification: tiny FP32 decode, batched BF16 decode, BF16 chain verify,
+long-context FP8 (E4M3) and a mixed FP16 tree-verify batch.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+TORCH_DTYPES = {
+    "f32": torch.float32,
+    "f16": torch.float16,
+    "bf16": torch.bfloat16,
+    "e4m3": torch.float8_e4m3fn,
+    "e5m2": torch.float8_e5m2,
+}
+ELEM_SIZE = {"f32": 4, "f16": 2, "bf16": 2, "e4m3": 1, "e5m2": 1}
+DEAD_BYTE = 0xFF
+
+
+@dataclass
+class Workload:
+    name: str
+    dtype: str
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    fragment_bytes: int
+    chunk_bytes: int
+    chunks: list                 # list of np.uint8 arrays (host arena)
+    k_pages: np.ndarray          # int32 [S, max_pages]
+    v_pages: np.ndarray          # int32 [S, max_pages]
+    seq_lens: np.ndarray         # int32 [S]
+    row_offsets: np.ndarray      # int32 [S + 1]
+    row_masks: np.ndarray | None  # uint64 [total_rows]; None means chain
+    q: np.ndarray                # float32 [total_rows, Hq, D]
+    scale: float
+    seed: int
+    logical_k: list = field(default_factory=list)  # per seq torch [L, Hkv, D] storage dtype
+    logical_v: list = field(default_factory=list)
+    parents: list = field(default_factory=list)    # per seq list of draft parents (-1 = root)
+
+    @property
+    def n_seqs(self) -> int:
+        return int(len(self.seq_lens))
+
+    @property
+    def max_pages(self) -> int:
+        return int(self.k_pages.shape[1])
+
+    @property
+    def tokens_per_fragment(self) -> int:
+        return self.fragment_bytes // (self.n_kv_heads * self.head_dim * ELEM_SIZE[self.dtype])
+
+    @property
+    def total_rows(self) -> int:
+        return int(self.row_offsets[-1])
+
+    @property
+    def max_rows(self) -> int:
+        return int(np.max(np.diff(self.row_offsets))) if self.n_seqs else 0
+
+    def kv_bytes(self) -> int:
+        """Bytes of live K and V (every key of every sequence, all kv heads)."""
+        return int(np.sum(self.seq_lens.astype(np.int64))) * 2 * self.n_kv_heads * \
+            self.head_dim * ELEM_SIZE[self.dtype]
+
+    def call_bytes(self) -> int:
+        """K + V + Q + out bytes of one call (Q and out in FP32)."""
+        qo = 2 * self.total_rows * self.n_q_heads * self.head_dim * 4
+        return self.kv_bytes() + qo
+
+
+def _chain_masks(R: int) -> list[int]:
+    return [(1 << (r + 1)) - 1 for r in range(R)]
+
+
+def _tree_masks(parents: list[int]) -> list[int]:
+    """Self + ancestors bit masks for a topologically ordered parent list."""
+    masks = []
+    for i, p in enumerate(parents):
+        m = 1 << i
+        if p >= 0:
+            m |= masks[p]
+        masks.append(m)
+    return masks
+
+
+def build(
+    name: str,
+    dtype: str,
+    seq_lens: list[int],
+    rows: list[int],
+    n_q_heads: int,
+    n_kv_heads: int,
+    head_dim: int,
+    fragment_bytes: int,
+    chunk_bytes: int,
+    max_pages: int,
+    seed: int,
+    parents: list[list[int]] | None = None,
+    kv_std: float = 1.0,
+    q_std: float = 1.0,
+    keep_logical: bool = False,
+    n_chunks: int | None = None,
+    gen: torch.Generator | None = None,
+) -> Workload:
+    """Lay out one seeded problem.
+
+    ``rows[s]`` query rows are the last positions of sequence ``s``;
+    ``parents[s]`` (optional) gives each draft row's parent row, -1 for a row
+    hanging off the cached context; without it the rows form a chain.
+    """
+    g = gen if gen is not None else torch.Generator().manual_seed(seed)
+    es = ELEM_SIZE[dtype]
+    row_bytes = n_kv_heads * head_dim * es
+    assert fragment_bytes % row_bytes == 0 and chunk_bytes % fragment_bytes == 0
+    T = fragment_bytes // row_bytes
+    fpc = chunk_bytes // fragment_bytes
+    S = len(seq_lens)
+    pages_needed = [math.ceil(L / T) for L in seq_lens]
+    assert all(p <= max_pages for p in pages_needed)
+    need = 2 * sum(pages_needed)
+    if n_chunks is None:
+        n_chunks = max(1, math.ceil(need / fpc))
+    assert need <= n_chunks * fpc, "arena too small"
+
+    # shuffled fragment assignment
+    perm = torch.randperm(n_chunks * fpc, generator=g)[:need].to(torch.int64).numpy()
+    k_pages = np.full((S, max_pages), -1, np.int32)
+    v_pages = np.full((S, max_pages), -1, np.int32)
+    cursor = 0
+    for s in range(S):
+        n = pages_needed[s]
+        k_pages[s, :n] = perm[cursor:cursor + n]
+        v_pages[s, :n] = perm[cursor + n:cursor + 2 * n]
+        cursor += 2 * n
+
+    row_offsets = np.zeros(S + 1, np.int32)
+    row_offsets[1:] = np.cumsum(rows)
+    masks: list[int] = []
+    for s in range(S):
+        if parents is not None:
+            assert len(parents[s]) == rows[s]
+            masks += _tree_masks(parents[s])
+        else:
+            masks += _chain_masks(rows[s])
+    row_masks = np.array(masks, dtype=np.uint64) if parents is not None else None
+
+    total_rows = int(row_offsets[-1])
+    q = (torch.randn((total_rows, n_q_heads, head_dim), generator=g, dtype=torch.float32)
+         * q_std).numpy()
+
+    chunks = [np.full(chunk_bytes, DEAD_BYTE, np.uint8) for _ in range(n_chunks)]
+    tdt = TORCH_DTYPES[dtype]
+    logical_k, logical_v = [], []
+    for s in range(S):
+        L = seq_lens[s]
+        for which, table in (("k", k_pages), ("v", v_pages)):
+            x = torch.randn((L, n_kv_heads, head_dim), generator=g, dtype=torch.float32)
+            x = (x * kv_std).to(tdt)
+            if keep_logical:
+                (logical_k if which == "k" else logical_v).append(x)
+            raw = x.contiguous().view(torch.uint8).reshape(L, row_bytes).numpy()
+            for p in range(pages_needed[s]):
+                f = int(table[s, p])
+                c, off = divmod(f, fpc)
+                t0, t1 = p * T, min((p + 1) * T, L)
+                base = off * fragment_bytes
+                chunks[c][base:base + (t1 - t0) * row_bytes] = raw[t0:t1].reshape(-1)
+
+    return Workload(
+        name=name, dtype=dtype, n_q_heads=n_q_heads, n_kv_heads=n_kv_heads, head_dim=head_dim,
+        fragment_bytes=fragment_bytes, chunk_bytes=chunk_bytes, chunks=chunks,
+        k_pages=k_pages, v_pages=v_pages, seq_lens=np.array(seq_lens, np.int32),
+        row_offsets=row_offsets, row_masks=row_masks, q=q, scale=1.0 / math.sqrt(head_dim),
+        seed=seed, logical_k=logical_k, logical_v=logical_v,
+        parents=parents if parents is not None else [])
+
+
+# ---------------------------------------------------------------------------
+# The five benchmark workloads.  Seed = 1234 + index (index 0..4).
+# ---------------------------------------------------------------------------
+
+MIB = 1 << 20
+KIB = 1 << 10
+NAMES = ["tiny_decode", "batched_decode", "chain_verify", "long_fp8", "tree_verify"]
+
+
+def tiny_decode(keep_logical=False) -> Workload:
+    """1 sequence, 1 query row, 4 query heads / 1 kv head, head_dim 64, 512
+    keys, FP32 K/V in 16-token pages in random order."""
+    return build("tiny_decode", "f32", [512], [1], 4, 1, 64, fragment_bytes=16 * 64 * 4,
+                 chunk_bytes=1 * MIB, max_pages=32, seed=1234, keep_logical=keep_logical)
+
+
+def batched_decode(keep_logical=False) -> Workload:
+    """8 sequences, lengths uniform in [1024, 16384], 1 row each, 24/4 heads,
+    head_dim 128, BF16 K/V in 256 KiB fragments of one 256 MiB arena."""
+    g = torch.Generator().manual_seed(1235)
+    lens = torch.randint(1024, 16385, (8,), generator=g).tolist()
+    return build("batched_decode", "bf16", lens, [1] * 8, 24, 4, 128,
+                 fragment_bytes=256 * KIB, chunk_bytes=256 * MIB, max_pages=64, seed=1235,
+                 n_chunks=1, gen=g, keep_logical=keep_logical)
+
+
+def chain_verify(keep_logical=False) -> Workload:
+    """1 sequence, 32768 cached keys + 8 chained draft rows, 24/4 heads,
+    head_dim 128, BF16 in 256 KiB fragments."""
+    return build("chain_verify", "bf16", [32768 + 8], [8], 24, 4, 128,
+                 fragment_bytes=256 * KIB, chunk_bytes=256 * MIB, max_pages=129, seed=1236,
+                 n_chunks=1, keep_logical=keep_logical)
+
+
+def long_fp8(keep_logical=False) -> Workload:
+    """1 sequence, 68173 keys (4 chained query rows included), 24/4 heads,
+    head_dim 128, FP8 E4M3 cast from N(0, 0.5^2), 512-token fragments;
+    capacity 256 pages (131072 keys)."""
+    return build("long_fp8", "e4m3", [68173], [4], 24, 4, 128, fragment_bytes=512 * 4 * 128,
+                 chunk_bytes=256 * MIB, max_pages=256, seed=1237, kv_std=0.5, n_chunks=1,
+                 keep_logical=keep_logical)
+
+
+def tree_verify(keep_logical=False) -> Workload:
+    """16 sequences, context log-uniform in [256, 131072], each with a random
+    draft tree of 1..16 nodes, 24/4 heads, head_dim 128, FP16 in 256 KiB
+    fragments across several 256 MiB chunks; capacity 513 pages."""
+    g = torch.Generator().manual_seed(1238)
+    lo, hi = math.log(256), math.log(131072)
+    ctx = [int(math.exp(lo + (hi - lo) * float(u)))
+           for u in torch.rand(16, generator=g, dtype=torch.float64)]
+    nodes = torch.randint(1, 17, (16,), generator=g).tolist()
+    parents = []
+    for n in nodes:
+        parents.append([int(torch.randint(-1, i, (1,), generator=g)) for i in range(n)])
+    lens = [c + n for c, n in zip(ctx, nodes)]
+    return build("tree_verify", "f16", lens, nodes, 24, 4, 128, fragment_bytes=256 * KIB,
+                 chunk_bytes=256 * MIB, max_pages=513, seed=1238, parents=parents, gen=g,
+                 keep_logical=keep_logical)
+
+
+BUILDERS = {
+    "tiny_decode": tiny_decode,
+    "batched_decode": batched_decode,
+    "chain_verify": chain_verify,
+    "long_fp8": long_fp8,
+    "tree_verify": tree_verify,
+}
+
+
+def small_case(dtype: str, seq_lens, rows, n_q_heads=8, n_kv_heads=2, head_dim=64,
+               tokens_per_fragment=16, max_pages=None, seed=7, tree=False, kv_std=1.0,
+               keep_logical=True, n_chunks=None) -> Workload:
+    """A small seeded problem of any shape, for parity and pin tests."""
+    g = torch.Generator().manual_seed(seed)
+    es = ELEM_SIZE[dtype]
+    fb = tokens_per_fragment * n_kv_heads * head_dim * es
+    need = 2 * sum(math.ceil(L / tokens_per_fragment) for L in seq_lens)
+    if max_pages is None:
+        max_pages = max(1, max(math.ceil(L / tokens_per_fragment) for L in seq_lens))
+    fpc = max(4, need)
+    parents = None
+    if tree:
+        parents = [[int(torch.randint(-1, i, (1,), generator=g)) for i in range(R)] for R in rows]
+    return build(f"small_{dtype}", dtype, list(seq_lens), list(rows), n_q_heads, n_kv_heads,
+                 head_dim, fragment_bytes=fb, chunk_bytes=fb * fpc, max_pages=max_pages,
+                 seed=seed, parents=parents, kv_std=kv_std, keep_logical=keep_logical,
+                 n_chunks=n_chunks, gen=g)
