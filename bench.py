@@ -1,0 +1,368 @@
+#!/usr/bin/env python
+"""Benchmark: split-KV paged attention (decode / speculative verification).
+
+One step = one pass of the whole hot path over one batch: the partial pass
+(lse_attn_run) and the merge pass (lse_attn_merge) through the C ABI, on
+resident inputs.  The default workload is the batched BF16 decode
+(8 sequences, lengths uniform in [1024, 16384], 24 query / 4 kv heads,
+head_dim 128, 256 KiB fragments).  L2 is flushed (a 256 MiB write) before
+every timed step, outside the step's CUDA-event interval.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--impl ours|reference]
+
+Prints one JSON line.  ``value`` is effective GB/s: (K + V + Q + out bytes of
+every call on every rank) / (max over ranks of the summed step times).
+``--impl reference`` times the float64 CPU oracle on a bounded sample of
+the same workload (rank 0 only under torchrun).
+Multi-GPU runs are independent replicas (the path needs no exchange).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged attention us/call and effective KV GB/s (% of B200 HBM peak)"
+FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--workload", default="batched_decode")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="budget of the oracle CPU-baseline sample")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "verify_attention_paged_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload):
+    """DRAM bytes per launch of the partial kernel from the committed ncu
+    summary, when it was taken on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """SM clock and throttle reasons sampled through NVML while running."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            pass
+        self._stop = threading.Event()
+
+    def _loop(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._loop, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def cpu_baseline(w, budget_s):
+    """The oracle as it stands, single-threaded, on a bounded sample of the
+    workload's outputs; extrapolated to one whole call."""
+    from oracle import oracle as orc
+    from verify_attention_paged_b200.workloads import ELEM_SIZE
+    pb = orc.Problem(chunks=w.chunks, chunk_bytes=w.chunk_bytes, fragment_bytes=w.fragment_bytes,
+                     dtype=w.dtype, n_kv_heads=w.n_kv_heads, head_dim=w.head_dim,
+                     n_q_heads=w.n_q_heads, k_pages=w.k_pages, v_pages=w.v_pages,
+                     seq_lens=w.seq_lens, row_offsets=w.row_offsets, row_masks=w.row_masks,
+                     q=w.q, scale=w.scale)
+    m = orc.marshal(pb)
+    outputs = [(s, r, h) for s in range(w.n_seqs)
+               for r in range(int(w.row_offsets[s + 1] - w.row_offsets[s]))
+               for h in range(w.n_q_heads)]
+    rng = np.random.default_rng(0)
+    order = rng.permutation(len(outputs))
+    done_keys, n_done = 0, 0
+    t0 = time.perf_counter()
+    for i in order:
+        s, r, h = outputs[i]
+        orc.attention_one(pb, s, r, h, marshalled=m)
+        done_keys += int(w.seq_lens[s])
+        n_done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    all_keys = sum(int(w.seq_lens[s]) for (s, r, h) in outputs)
+    call_s = dt * all_keys / max(done_keys, 1)   # extrapolate by keys visited
+    gbs = w.call_bytes() / call_s / 1e9
+    return {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "us_per_call": call_s * 1e6,
+            "sample": f"{n_done} of {len(outputs)} (row, head) outputs in {dt:.1f} s, "
+                      f"extrapolated by keys visited to one call"}
+
+
+def run_reference(args, w, world, rank):
+    if rank != 0:
+        return
+    # each step is a bounded sample; the whole run stays within minutes
+    per_step = max(0.05, min(5.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline(w, per_step / 4)
+    vals = []
+    t_all = 0.0
+    for _ in range(args.steps):
+        r = cpu_baseline(w, per_step)
+        vals.append(r["value"])
+        t_all += r["us_per_call"]
+    v = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_all / args.steps / 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w),
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"each step: oracle on ~{per_step:.2f} s of "
+                                       f"(row, head) outputs, extrapolated to one call"},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w):
+    return {"workload": w.name, "seqs": w.n_seqs, "keys_total": int(np.sum(w.seq_lens)),
+            "query_rows": w.total_rows, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
+            "head_dim": w.head_dim, "kv_dtype": w.dtype,
+            "fragment_bytes": w.fragment_bytes, "chunk_bytes": w.chunk_bytes,
+            "bytes_per_call": w.call_bytes(), "l2": "flushed before every step (256 MiB write)"}
+
+
+def run_ours(args, w, world, rank, local):
+    import torch
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    from verify_attention_paged_b200 import binding as b
+
+    call = b.DeviceCall(w)
+    stream = call.stream
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    bytes_call = w.call_bytes()
+    bytes_partial = w.kv_bytes() + w.total_rows * w.n_q_heads * w.head_dim * 4
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        call.run()
+    torch.cuda.synchronize()
+    assert call.device_error() == 0, "device error during warm-up"
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xff)                  # L2 flush, outside the interval
+            ev[i][0].record(stream)
+            call.run_partial()
+            ev[i][1].record(stream)
+            call.run_merge()
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    part = [e[0].elapsed_time(e[1]) for e in ev]
+    merge = [e[1].elapsed_time(e[2]) for e in ev]
+    total_ms = sum(p + m for p, m in zip(part, merge))
+    t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+    if dist:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+
+    # end to end: pinned host inputs -> device -> run -> result back to host
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(call, w, args, stream, flush, dist)
+
+    if rank != 0:
+        if dist:
+            dist.destroy_process_group()
+        return
+    peak, peak_kind = measured_peaks()
+    part_ms = statistics.mean(part)
+    achieved = bytes_partial / (part_ms * 1e-3) / 1e9
+    value = world * bytes_call * args.steps / (total_ms * 1e-3) / 1e9
+    info = call.info
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "us_per_call": total_ms / args.steps * 1e3,
+        "us_per_call_median": statistics.median([p + m for p, m in zip(part, merge)]) * 1e3,
+        "partial_us_mean": part_ms * 1e3, "merge_us_mean": statistics.mean(merge) * 1e3,
+        "pct_of_8tbs": value / world / 8000.0 * 100.0,
+        "pct_of_measured_hbm": value / world / peak * 100.0,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16-mma/f32" if info["kernel"] == 1 else "f32",
+        "data": "synthetic", "config": {**workload_config(w), "parallelism": f"replicas{world}",
+                                        "kernel": info["kernel_name"],
+                                        "n_splits": info["n_splits"],
+                                        "keys_per_split": info["keys_per_split"]},
+        "roofline": {"bound": "hbm", "kernel": "partial", "achieved": achieved, "peak": peak,
+                     "peak_kind": f"{peak_kind} (copy, burst)", "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": ncu_traffic(w.name),
+                     "algorithmic_bytes_per_launch": bytes_partial},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if e2e:
+        line["e2e"] = e2e
+    if world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
+
+
+def measure_e2e(call, w, args, stream, flush, dist):
+    """Same metric through the public API with this step's inputs (Q, page
+    tables, lengths, row offsets, masks) copied from pinned host memory and
+    the result (out and lse) read back, inside the timed interval."""
+    import torch
+    host_in = [torch.from_numpy(np.ascontiguousarray(w.q)).pin_memory(),
+               torch.from_numpy(np.ascontiguousarray(w.k_pages)).pin_memory(),
+               torch.from_numpy(np.ascontiguousarray(w.v_pages)).pin_memory(),
+               torch.from_numpy(np.ascontiguousarray(w.seq_lens)).pin_memory(),
+               torch.from_numpy(np.ascontiguousarray(w.row_offsets)).pin_memory()]
+    dev_in = [call.q, call.k_pages, call.v_pages, call.seq_lens, call.row_offsets]
+    if w.row_masks is not None:
+        host_in.append(torch.from_numpy(np.ascontiguousarray(w.row_masks).view(np.int64))
+                       .pin_memory())
+        dev_in.append(call.row_masks)
+    rows = w.total_rows
+    host_out = torch.empty((rows, w.n_q_heads, w.head_dim), dtype=torch.float32).pin_memory()
+    host_lse = torch.empty((rows, w.n_q_heads), dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = host_out.numel() * 4 + host_lse.numel() * 4
+    steps = max(10, args.steps // 5)
+
+    def step():
+        with torch.cuda.stream(stream):
+            for h, d in zip(host_in, dev_in):
+                d.copy_(h, non_blocking=True)
+            call.run()
+            host_out.copy_(call.out[:rows], non_blocking=True)
+            host_lse.copy_(call.lse[:rows], non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    if dist:
+        dist.barrier()
+    for i in range(steps):
+        flush.fill_(i & 0xff)
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in evs)
+    t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+    if dist:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    world = dist.get_world_size() if dist else 1
+    ms = float(t.item())
+    return {"value": world * w.call_bytes() * steps / (ms * 1e-3) / 1e9, "unit": "GB/s",
+            "us_per_call": ms / steps * 1e3, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h}
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    from verify_attention_paged_b200 import workloads as wl
+    w = wl.BUILDERS[args.workload]()
+    if args.impl == "reference":
+        run_reference(args, w, world, rank)
+    else:
+        run_ours(args, w, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,272 @@
+/*
+ * lse_attn.h — split-KV paged attention for single-token decode and
+ * speculative verification over a fragment-addressed K/V cache, on NVIDIA
+ * B200 (sm_100a).
+ *
+ * What is computed (sources: the LSE README (Geramy/LSE), "KV cache
+ * formats"; LSE releases, v0.4.19 "Long-context split attention", v0.4.20
+ * "K/V memory management and automatic split attention", v0.4.21 "joint
+ * decode attention", v0.4.14 "Improvements"):
+ *
+ *   For sequence s with L_s keys, the last R_s of which are the query rows
+ *   (context C_s = L_s - R_s), query row r (position C_s + r), query head h,
+ *   kv head g = h / (Hq / Hkv):
+ *     visible(j)  <=>  j < C_s  or  bit (j - C_s) of mask_r is set
+ *     x_j  = softmax_scale * <q[r][h], K[j][g]>
+ *     out  = sum_vis exp(x_j - m) V[j][g] / sum_vis exp(x_j - m),  m = max_vis x_j
+ *     lse  = m + ln sum_vis exp(x_j - m)
+ *   mask_r defaults to the chain (rows 0..r); for a draft tree it is the row
+ *   itself plus its ancestors (nodes in topological order, R_s <= 64).
+ *
+ *   K/V elements are stored as FP32, FP16, BF16, FP8-E4M3 ("fp8") or
+ *   FP8-E5M2 ("bf8"); accumulation, softmax state and output are FP32.
+ *   The work is split along the keys into partitions whose count comes from
+ *   page-table capacity and on-chip memory limits (lse_attn_plan); each
+ *   partition writes a normalised partial output and its log-sum-exp
+ *   (lse_attn_run); a merge pass combines them (lse_attn_merge).  A
+ *   partition with no live key loads nothing and writes nothing.
+ *
+ * Memory layout
+ *   Arena: n_chunks device allocations ("arenas" on the pages) of chunk_bytes
+ *   each, cut into fragments of fragment_bytes.  Fragment id f lives in chunk
+ *   f / (chunk_bytes / fragment_bytes) at byte offset
+ *   (f % (chunk_bytes / fragment_bytes)) * fragment_bytes.  A fragment holds
+ *   T = fragment_bytes / (Hkv * D * esize) consecutive tokens of K (or of V)
+ *   for every kv head, token-major: [token][kv_head][dim].  K and V use
+ *   separate fragments and separate page tables.
+ *   Page tables: int32 [n_seqs][max_pages_per_seq]; key j of sequence s is
+ *   token j % T of fragment table[s][j / T].  Entries past the live pages are
+ *   ignored.
+ *   q:   FP32 [total_rows][Hq][D]; the rows of sequence s are
+ *        row_offsets[s] .. row_offsets[s+1]-1.
+ *   out: FP32 [total_rows][Hq][D];  lse_out (optional): FP32 [total_rows][Hq].
+ *
+ * Ownership and threading
+ *   The library never allocates, frees or owns device memory: the caller
+ *   allocates the arena chunks, page tables, q, out and the workspace (size
+ *   from lse_attn_plan).  Handles (arena, plan) are host objects owned by the
+ *   library and released by their destroy calls.  Device pointers are passed
+ *   as plain pointers; every launch goes to the caller's cudaStream_t (passed
+ *   as void*; NULL = legacy default stream).  No call synchronises except
+ *   lse_attn_read_error.  A plan may be used from one thread at a time.
+ *
+ * Errors
+ *   Every call returns LSE_OK (0) or an lse_status code.  When err is not
+ *   NULL and a call fails, *err receives a message the caller releases with
+ *   lse_free (the convention of libLSE's C API in the LSE README).  Host
+ *   checks cover every size and shape.  Device-resident inputs (page tables,
+ *   lengths, masks) are not read on the host by lse_attn_run; the kernels
+ *   bound-check them instead: a bad fragment id or length sets a bit in the
+ *   workspace's error word (read with lse_attn_read_error), the offending
+ *   keys are treated as absent, and no out-of-bounds access is made.
+ *   lse_attn_validate checks host copies of those arrays up front.
+ */
+#ifndef LSE_ATTN_H
+#define LSE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LSE_API __attribute__((visibility("default")))
+#else
+#define LSE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LSE_OK = 0,
+  LSE_ERR_INVALID_ARG = 1,      /* a size, shape, pointer or dtype is out of range */
+  LSE_ERR_UNSUPPORTED = 2,      /* valid, but no kernel here handles it             */
+  LSE_ERR_OUT_OF_FRAGMENTS = 3, /* the arena has fewer free fragments than asked   */
+  LSE_ERR_CUDA = 4,             /* a CUDA runtime call or launch failed             */
+  LSE_ERR_NO_MEMORY = 5,        /* a host allocation failed                         */
+  LSE_ERR_BAD_INPUT = 6         /* validated input violates the layout/mask rules   */
+} lse_status;
+
+typedef enum {
+  LSE_KV_F32 = 0,
+  LSE_KV_F16 = 1,
+  LSE_KV_BF16 = 2,
+  LSE_KV_FP8_E4M3 = 3, /* OCP E4M3: finite only, max 448, NaN = S.1111.111 */
+  LSE_KV_FP8_E5M2 = 4  /* OCP E5M2: IEEE-style inf and NaN                  */
+} lse_kv_dtype;
+
+/* Bits of the device error word (lse_attn_read_error). */
+#define LSE_DEVERR_BAD_FRAGMENT 0x1u /* a page-table entry named no fragment   */
+#define LSE_DEVERR_BAD_LENGTH 0x2u   /* L_s > capacity, R_s > L_s, R_s > max rows or rows past max_total_rows */
+
+#define LSE_MAX_CHUNKS 64     /* arena chunks a kernel can address          */
+#define LSE_MAX_ROWS_PER_SEQ 64
+
+typedef struct lse_kv_arena lse_kv_arena;
+typedef struct lse_attn_plan_s lse_attn_plan_t;
+
+/* ---------------------------------------------------------------------------
+ * K/V arena (LSE releases, v0.4.20: 256 MiB arenas of 256 KiB fragments,
+ * shared across layers and sessions; free slots are reused before another
+ * arena is added; growth never moves existing fragments).
+ * ------------------------------------------------------------------------- */
+
+/* Describe an arena over caller-owned device chunks.
+ *   chunk_bases: n_chunks device pointers (host array), each 256-byte aligned
+ *                and chunk_bytes long; 1 <= n_chunks <= LSE_MAX_CHUNKS.
+ *   fragment_bytes must divide chunk_bytes, be a multiple of
+ *   Hkv * D * esize and of 16.  head_dim in {64, 128, 256}.
+ *   All fragments start free.  *out receives the handle. */
+LSE_API int lse_kv_arena_create(void *const *chunk_bases, int n_chunks, size_t chunk_bytes,
+                        size_t fragment_bytes, int kv_dtype, int n_kv_heads, int head_dim,
+                        lse_kv_arena **out, char **err);
+
+/* Append one more caller-owned chunk (growth without copying).  Its
+ * fragments get the next ids; *first_id (optional) receives the first. */
+LSE_API int lse_kv_arena_add_chunk(lse_kv_arena *arena, void *chunk_base, int32_t *first_id,
+                           char **err);
+
+/* Take n free fragment ids, lowest id first (so earlier chunks fill before
+ * later ones); on LSE_ERR_OUT_OF_FRAGMENTS nothing is taken. */
+LSE_API int lse_kv_arena_alloc(lse_kv_arena *arena, int n, int32_t *frag_ids_out, char **err);
+
+/* Return fragment ids; a double free or an unknown id is LSE_ERR_INVALID_ARG
+ * and frees nothing. */
+LSE_API int lse_kv_arena_free(lse_kv_arena *arena, int n, const int32_t *frag_ids, char **err);
+
+typedef struct {
+  int32_t tokens_per_fragment; /* T */
+  int32_t n_fragments;         /* all chunks */
+  int32_t n_free;
+  int32_t n_chunks;
+  int32_t n_empty_chunks;      /* chunks whose fragments are all free (releasable) */
+} lse_kv_arena_info;
+
+LSE_API int lse_kv_arena_query(const lse_kv_arena *arena, lse_kv_arena_info *info);
+
+LSE_API void lse_kv_arena_destroy(lse_kv_arena *arena);
+
+/* ---------------------------------------------------------------------------
+ * Plan (LSE releases, v0.4.20: the partition count is derived from the
+ * actual K/V table capacity and checked against on-chip memory limits;
+ * partitions past a sequence's live keys are skipped).
+ *   n_seqs, max_rows_per_seq (<= 64), max_total_rows (>= rows of one call),
+ *   n_q_heads (multiple of Hkv), max_pages_per_seq (page-table row length:
+ *   the capacity).  Uses the current CUDA device's SM count and shared
+ *   memory limit.  *workspace_bytes receives the device workspace size the
+ *   caller allocates (256-byte aligned; zero it once with
+ *   lse_attn_workspace_init).  The plan does not depend on live lengths, so
+ *   one plan serves every step up to the capacity.
+ * ------------------------------------------------------------------------- */
+LSE_API int lse_attn_plan(const lse_kv_arena *arena, int n_seqs, int max_rows_per_seq,
+                  int max_total_rows, int n_q_heads, int max_pages_per_seq,
+                  lse_attn_plan_t **out, size_t *workspace_bytes, char **err);
+
+/* Device figures the planner uses.  lse_attn_plan reads them from the
+ * current CUDA device; lse_attn_plan_ex takes them from the caller and then
+ * makes no CUDA call (planning for another device, or on a host without
+ * one).  ctas_per_sm = 0 asks the CUDA occupancy calculator. */
+typedef struct {
+  int32_t n_sms;          /* streaming multiprocessors                     */
+  int32_t smem_optin;     /* shared memory per block, opt-in maximum       */
+  int32_t ctas_per_sm;    /* resident partial-pass CTAs per SM (0 = query)  */
+  int32_t allow_tcgen05;  /* 1: the tensor-core kernel may be chosen        */
+} lse_device_limits;
+
+LSE_API int lse_attn_plan_ex(const lse_kv_arena *arena, int n_seqs, int max_rows_per_seq,
+                             int max_total_rows, int n_q_heads, int max_pages_per_seq,
+                             const lse_device_limits *limits, lse_attn_plan_t **out,
+                             size_t *workspace_bytes, char **err);
+
+/* Kernel families a plan can select. */
+#define LSE_KERNEL_CUDA_CORE 0 /* FP32 math on CUDA cores (any dtype, any P) */
+#define LSE_KERNEL_TCGEN05 1   /* tensor-core (tcgen05) partial pass           */
+
+typedef struct {
+  int32_t n_splits;        /* partitions per (sequence, kv head)            */
+  int32_t keys_per_split;  /* K_p                                           */
+  int32_t kernel;          /* LSE_KERNEL_*                                  */
+  int32_t key_tile;        /* keys per pipeline stage                      */
+  int32_t pairs;           /* (row, head) pairs per kv head: G * max rows   */
+  int32_t smem_bytes;      /* dynamic shared memory of the partial kernel  */
+  int64_t workspace_bytes;
+} lse_attn_plan_info;
+
+LSE_API int lse_attn_plan_query(const lse_attn_plan_t *plan, lse_attn_plan_info *info);
+
+/* Same partition rule as lse_attn_plan, for explicit device figures (no
+ * CUDA call): capacity_keys = max_pages * T; units = n_seqs * Hkv;
+ * slots = n_sms * ctas_per_sm; key_tile = the kernel's keys per stage.
+ * K_p = clamp(roundup(ceil(capacity_keys * units / slots), key_tile),
+ *             key_tile, roundup(capacity_keys, key_tile));
+ * n_splits = ceil(capacity_keys / K_p).  Returns n_splits; *keys_per_split
+ * receives K_p. */
+LSE_API int lse_attn_split_rule(int64_t capacity_keys, int units, int n_sms, int ctas_per_sm,
+                        int key_tile, int32_t *keys_per_split);
+
+/* Zero the workspace's error word (once after allocation; any time to clear). */
+LSE_API int lse_attn_workspace_init(const lse_attn_plan_t *plan, void *workspace, void *stream,
+                            char **err);
+
+LSE_API void lse_attn_plan_destroy(lse_attn_plan_t *plan);
+
+/* ---------------------------------------------------------------------------
+ * Partial pass (LSE releases, v0.4.19: one partial family, verifier rows
+ * share K/V loads; v0.4.21: K/V reads shared across query heads and rows).
+ *   q:           device FP32 [total_rows][Hq][D]
+ *   k_pages,
+ *   v_pages:     device int32 [n_seqs][max_pages_per_seq]
+ *   seq_lens:    device int32 [n_seqs]      (L_s, query rows included)
+ *   row_offsets: device int32 [n_seqs + 1]  (R_s = difference, <= max rows)
+ *   row_masks:   device uint64 [total_rows] ancestor masks, or NULL = chain
+ *   softmax_scale: multiplies <q, k> (1/sqrt(D) in the usual case)
+ *   workspace:   device, workspace_bytes, 256-byte aligned
+ *   stream:      cudaStream_t
+ * Each live partition of each (sequence, kv head) reads its K/V tiles once
+ * for every query head of the group and every query row.
+ * ------------------------------------------------------------------------- */
+LSE_API int lse_attn_run(const lse_attn_plan_t *plan, const float *q, const int32_t *k_pages,
+                 const int32_t *v_pages, const int32_t *seq_lens, const int32_t *row_offsets,
+                 const uint64_t *row_masks, float softmax_scale, void *workspace, void *stream,
+                 char **err);
+
+/* ---------------------------------------------------------------------------
+ * Merge pass (LSE releases, v0.4.19: one merge family).  For each row and
+ * head, with partials (o_p, lse_p) over the live partitions:
+ *   M = max_p lse_p, w_p = exp(lse_p - M),
+ *   out = sum_p w_p o_p / sum_p w_p,  lse = M + ln sum_p w_p.
+ *   out: device FP32 [total_rows][Hq][D]; lse_out: device FP32
+ *   [total_rows][Hq] or NULL.  seq_lens / row_offsets as given to run.
+ * ------------------------------------------------------------------------- */
+LSE_API int lse_attn_merge(const lse_attn_plan_t *plan, const int32_t *seq_lens,
+                   const int32_t *row_offsets, const void *workspace, float *out,
+                   float *lse_out, void *stream, char **err);
+
+/* ---------------------------------------------------------------------------
+ * Host-side validation of HOST copies of the device inputs: every live page
+ * names a fragment of the arena (sequences may share read-only fragments),
+ * L_s <= capacity,
+ * 1 <= R_s <= min(L_s, 64) (R_s = 0 allowed: the sequence is idle), total
+ * rows <= max_total_rows, each mask has bit r set and no bit above r.
+ * Returns LSE_OK or LSE_ERR_BAD_INPUT with a message naming the first fault.
+ * ------------------------------------------------------------------------- */
+LSE_API int lse_attn_validate(const lse_attn_plan_t *plan, const int32_t *k_pages,
+                      const int32_t *v_pages, const int32_t *seq_lens,
+                      const int32_t *row_offsets, const uint64_t *row_masks, char **err);
+
+/* Read (and clear) the workspace's device error word.  Synchronises the
+ * stream.  *device_error receives LSE_DEVERR_* bits, 0 when clean. */
+LSE_API int lse_attn_read_error(const lse_attn_plan_t *plan, void *workspace, void *stream,
+                        uint32_t *device_error, char **err);
+
+/* Release a string returned through an err argument. */
+LSE_API void lse_free(void *p);
+
+/* Static description of a status code. */
+LSE_API const char *lse_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSE_ATTN_H */

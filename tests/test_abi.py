@@ -1,0 +1,144 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads and
+exports every declared entry point; arena bookkeeping; the split rule; plan
+shapes and argument checks; validation of host copies of the inputs."""
+import ctypes
+
+import numpy as np
+import pytest
+
+from verify_attention_paged_b200 import binding as b
+from verify_attention_paged_b200 import workloads as wl
+
+B200 = dict(n_sms=148, smem_optin=232448, ctas_per_sm=2)
+FAKE = 1 << 32  # 256-byte-aligned stand-in device address (never dereferenced here)
+
+
+def test_library_exports_every_declared_symbol():
+    declared = b.declared_symbols()
+    assert len(declared) >= 17
+    for name in declared:
+        assert hasattr(b._lib, name), name
+        assert hasattr(b, name), f"binding lacks {name}"
+
+
+def test_status_strings():
+    assert b.lse_status_string(0) == "ok"
+    assert "fragments" in b.lse_status_string(3)
+
+
+def test_arena_alloc_free_lowest_first_and_growth():
+    a = b.lse_kv_arena_create([FAKE], 1 << 20, 256 << 10, "bf16", 4, 128)
+    info = b.lse_kv_arena_query(a)
+    assert info["tokens_per_fragment"] == 256 and info["n_fragments"] == 4
+    ids = b.lse_kv_arena_alloc(a, 3)
+    assert list(ids) == [0, 1, 2]
+    b.lse_kv_arena_free(a, [1])
+    assert list(b.lse_kv_arena_alloc(a, 1)) == [1]          # free slot reused first
+    with pytest.raises(b.LseError, match="out of fragments"):
+        b.lse_kv_arena_alloc(a, 2)                           # only 1 free
+    assert b.lse_kv_arena_query(a)["n_free"] == 1            # nothing taken
+    first = b.lse_kv_arena_add_chunk(a, FAKE * 2)            # grow without moving
+    assert first == 4
+    assert list(b.lse_kv_arena_alloc(a, 2)) == [3, 4]
+    info = b.lse_kv_arena_query(a)
+    assert info["n_chunks"] == 2 and info["n_free"] == 3 and info["n_empty_chunks"] == 0
+    b.lse_kv_arena_free(a, [4])
+    assert b.lse_kv_arena_query(a)["n_empty_chunks"] == 1    # second chunk releasable
+    with pytest.raises(b.LseError, match="not in use"):
+        b.lse_kv_arena_free(a, [4])                          # double free
+    with pytest.raises(b.LseError, match="twice"):
+        b.lse_kv_arena_free(a, [0, 0])
+    assert b.lse_kv_arena_query(a)["n_free"] == 4            # failed frees took nothing
+    b.lse_kv_arena_destroy(a)
+
+
+@pytest.mark.parametrize("args,msg", [
+    (([FAKE], 1 << 20, 256 << 10, "bf16", 4, 96), "head_dim"),
+    (([FAKE], 1 << 20, 1000, "bf16", 4, 128), "fragment_bytes"),
+    (([FAKE], (1 << 20) + 5, 256 << 10, "bf16", 4, 128), "chunk_bytes"),
+    (([FAKE + 16], 1 << 20, 256 << 10, "bf16", 4, 128), "aligned"),
+    (([FAKE], 1 << 20, 256 << 10, 9, 4, 128), "dtype"),
+])
+def test_arena_rejects_bad_arguments(args, msg):
+    with pytest.raises(b.LseError, match=msg):
+        b.lse_kv_arena_create(*args)
+
+
+def test_split_rule():
+    # one full sequence of 33024 keys, 4 kv heads, 148 SMs x 2 CTAs, tile 128
+    n, kp = b.lse_attn_split_rule(33024, 4, 148, 2, 128)
+    assert kp % 128 == 0 and n == -(-33024 // kp)
+    assert n * 4 <= 2 * 148 + 4 * 2   # about one wave of resident CTAs at full capacity
+    # never smaller than a tile, never larger than the (rounded) capacity
+    assert b.lse_attn_split_rule(100, 1, 148, 8, 128) == (1, 128)
+    assert b.lse_attn_split_rule(10 ** 6 + 1, 1000, 1, 1, 64) == (1, 10 ** 6 // 64 * 64 + 64)
+    assert b.lse_attn_split_rule(0, 1, 1, 1, 1)[0] == 0
+
+
+def _plan_for(w, **lim):
+    a = b.lse_kv_arena_create([FAKE * (i + 1) for i in range(len(w.chunks))], w.chunk_bytes,
+                              w.fragment_bytes, w.dtype, w.n_kv_heads, w.head_dim)
+    p, ws = b.lse_attn_plan_ex(a, w.n_seqs, w.max_rows, w.total_rows, w.n_q_heads,
+                               w.max_pages, **(lim or B200))
+    return a, p, ws
+
+
+def test_plan_depends_on_capacity_not_live_lengths():
+    w1 = wl.small_case("bf16", [40, 9], [1, 1], max_pages=64, tokens_per_fragment=16)
+    w2 = wl.small_case("bf16", [1000, 3], [1, 1], max_pages=64, tokens_per_fragment=16)
+    i1 = b.lse_attn_plan_query(_plan_for(w1)[1])
+    i2 = b.lse_attn_plan_query(_plan_for(w2)[1])
+    assert (i1["n_splits"], i1["keys_per_split"]) == (i2["n_splits"], i2["keys_per_split"])
+    cap = 64 * 16
+    assert i1["n_splits"] == -(-cap // i1["keys_per_split"])
+
+
+def test_plan_workspace_size():
+    w = wl.small_case("f16", [100, 50, 7], [4, 2, 1], n_q_heads=8, n_kv_heads=2,
+                      head_dim=128, max_pages=20)
+    _, p, ws = _plan_for(w)
+    info = b.lse_attn_plan_query(p)
+    n = w.total_rows * 8 * info["n_splits"]
+    assert ws >= 256 + n * 128 * 4 + n * 4 and ws % 256 == 0
+    assert info["workspace_bytes"] == ws and info["pairs"] == 4 * 4
+
+
+def test_plan_rejects_bad_shapes():
+    a = b.lse_kv_arena_create([FAKE], 1 << 20, 256 << 10, "bf16", 4, 128)
+    for args in [(1, 65, 65, 24, 10), (1, 0, 1, 24, 10), (1, 1, 1, 22, 10), (0, 1, 1, 24, 10),
+                 (2, 4, 9, 24, 10)]:
+        with pytest.raises(b.LseError):
+            b.lse_attn_plan_ex(a, *args, **B200)
+
+
+def test_validate_accepts_generated_workloads_and_flags_faults():
+    w = wl.small_case("e4m3", [70, 33, 8], [2, 4, 1], n_q_heads=6, n_kv_heads=3, head_dim=64,
+                      tokens_per_fragment=8, tree=True, seed=4)
+    _, p, _ = _plan_for(w)
+    b.lse_attn_validate(p, w.k_pages, w.v_pages, w.seq_lens, w.row_offsets, w.row_masks)
+    bad = w.k_pages.copy(); bad[1, 2] = 10 ** 6
+    with pytest.raises(b.LseError, match="unknown"):
+        b.lse_attn_validate(p, bad, w.v_pages, w.seq_lens, w.row_offsets, w.row_masks)
+    m = w.row_masks.copy(); m[0] = 2
+    with pytest.raises(b.LseError, match="misses itself"):
+        b.lse_attn_validate(p, w.k_pages, w.v_pages, w.seq_lens, w.row_offsets, m)
+    m = w.row_masks.copy(); m[2] = 0b11
+    with pytest.raises(b.LseError, match="later row"):
+        b.lse_attn_validate(p, w.k_pages, w.v_pages, w.seq_lens, w.row_offsets, m)
+    lens = w.seq_lens.copy(); lens[0] = 10 ** 5
+    with pytest.raises(b.LseError, match="capacity"):
+        b.lse_attn_validate(p, w.k_pages, w.v_pages, lens, w.row_offsets, w.row_masks)
+    lens = w.seq_lens.copy(); lens[2] = 0
+    with pytest.raises(b.LseError, match="rows"):
+        b.lse_attn_validate(p, w.k_pages, w.v_pages, lens, w.row_offsets, w.row_masks)
+
+
+def test_run_rejects_null_pointers_without_launching():
+    w = wl.small_case("bf16", [10], [1])
+    _, p, _ = _plan_for(w)
+    with pytest.raises(b.LseError, match="NULL"):
+        b.lse_attn_run(p, 0, 0, 0, 0, 0, None, 0.1, 0)
+    with pytest.raises(b.LseError, match="aligned"):
+        b.lse_attn_run(p, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0.1, FAKE + 8)
+    with pytest.raises(b.LseError, match="finite"):
+        b.lse_attn_run(p, FAKE, FAKE, FAKE, FAKE, FAKE, None, float("nan"), FAKE)

@@ -1,0 +1,159 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle
+on the same seeded inputs.  Small cases compare every element; the five
+full-size workloads compare sampled outputs the oracle computes one by one,
+in the launch configuration the benchmark times, plus properties that hold
+at any size."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as orc
+from verify_attention_paged_b200 import workloads as wl
+from conftest import to_problem
+from parity_util import assert_close, lse_tol
+
+pytestmark = pytest.mark.gpu
+
+DTYPES = ["f32", "f16", "bf16", "e4m3", "e5m2"]
+
+
+@pytest.fixture(scope="module")
+def binding():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from verify_attention_paged_b200 import binding as b
+    return b
+
+
+def gpu_run(b, w, **kw):
+    call = b.DeviceCall(w, **kw)
+    out, lse = call.run()
+    torch.cuda.synchronize()
+    err = call.device_error()
+    res = out[:w.total_rows].cpu().numpy(), lse[:w.total_rows].cpu().numpy(), call.info
+    call.close()
+    return res, err
+
+
+def check_full(b, w, **kw):
+    (out, lse, info), err = gpu_run(b, w, **kw)
+    assert err == 0, f"device error word {err:#x}"
+    ref_out, ref_lse = orc.attention(to_problem(w))
+    assert_close(out, ref_out, w.dtype)
+    np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=lse_tol(w.dtype) * 4)
+    return info
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("tree", [False, True])
+def test_small_ragged_all_formats(binding, dtype, tree):
+    # lengths span many 32/128-key tiles with ragged tails; rows 1..16
+    w = wl.small_case(dtype, [1, 7, 33, 300, 517, 129], [1, 1, 3, 8, 16, 5], n_q_heads=12,
+                      n_kv_heads=2, head_dim=128, tokens_per_fragment=16, tree=tree, seed=101)
+    check_full(binding, w)
+
+
+@pytest.mark.parametrize("head_dim", [64, 128, 256])
+@pytest.mark.parametrize("groups", [(4, 4), (8, 1), (24, 4)])
+def test_head_dims_and_group_sizes(binding, head_dim, groups):
+    hq, hkv = groups
+    for dtype in ("bf16", "f32"):
+        w = wl.small_case(dtype, [200, 45], [4, 2], n_q_heads=hq, n_kv_heads=hkv,
+                          head_dim=head_dim, tokens_per_fragment=8, seed=102)
+        check_full(binding, w)
+
+
+def test_rows_at_the_limit_and_tiny_fragments(binding):
+    # R = 64 draft rows (the mask limit), 1-token fragments, GQA 3
+    w = wl.small_case("f16", [64, 100], [64, 33], n_q_heads=6, n_kv_heads=2, head_dim=64,
+                      tokens_per_fragment=1, tree=True, seed=103)
+    check_full(binding, w)
+
+
+def test_idle_sequence_and_drafts_only(binding):
+    # an idle sequence (R = 0), one of only draft rows (L = R), one single key
+    w = wl.small_case("bf16", [50, 6, 1], [0, 6, 1], n_q_heads=4, n_kv_heads=2, head_dim=64,
+                      tokens_per_fragment=4, tree=True, seed=104)
+    check_full(binding, w)
+
+
+def test_capacity_far_above_live_lengths(binding):
+    # most planned partitions are empty and must be skipped
+    w = wl.small_case("e4m3", [40, 3, 250], [2, 1, 4], n_q_heads=8, n_kv_heads=2,
+                      head_dim=128, tokens_per_fragment=16, max_pages=400, seed=105)
+    info = check_full(binding, w)
+    assert info["n_splits"] * info["keys_per_split"] >= 400 * 16
+
+
+def test_arena_spanning_several_chunks(binding):
+    w = wl.build("multi_chunk", "f16", [700, 90, 333], [3, 1, 2], 8, 2, 64,
+                 fragment_bytes=16 * 2 * 64 * 2, chunk_bytes=16 * 2 * 64 * 2 * 24, max_pages=50,
+                 seed=106, n_chunks=7)
+    assert len(w.chunks) == 7
+    check_full(binding, w)
+
+
+def test_fragment_placement_does_not_change_output(binding):
+    from test_oracle_pins import _replace_fragments
+    w = wl.small_case("bf16", [300, 77], [3, 2], n_q_heads=8, n_kv_heads=2, head_dim=128,
+                      tokens_per_fragment=16, seed=107)
+    (out1, lse1, _), e1 = gpu_run(binding, w)
+    chunks, kp, vp = _replace_fragments(w, seed=5)
+    w2 = wl.Workload(**{**w.__dict__, "chunks": chunks, "k_pages": kp, "v_pages": vp})
+    (out2, lse2, _), e2 = gpu_run(binding, w2)
+    assert e1 == 0 and e2 == 0
+    # same arithmetic in the same order: identical bits
+    assert np.array_equal(out1, out2) and np.array_equal(lse1, lse2)
+
+
+def test_bad_page_entry_sets_error_word_without_faulting(binding):
+    w = wl.small_case("bf16", [100], [2], n_q_heads=4, n_kv_heads=2, head_dim=64,
+                      tokens_per_fragment=16, seed=108)
+    kp = w.k_pages.copy()
+    kp[0, 2] = 10 ** 6          # names no fragment: the kernel must skip it and flag
+    w2 = wl.Workload(**{**w.__dict__, "k_pages": kp})
+    (_, _, _), err = gpu_run(binding, w2)
+    assert err & binding.DEVERR_BAD_FRAGMENT
+
+
+def test_bad_length_sets_error_word(binding):
+    w = wl.small_case("bf16", [100], [2], n_q_heads=4, n_kv_heads=2, head_dim=64,
+                      tokens_per_fragment=16, seed=109)
+    lens = w.seq_lens.copy()
+    lens[0] = 10 ** 6           # beyond the page-table capacity
+    w2 = wl.Workload(**{**w.__dict__, "seq_lens": lens})
+    (_, _, _), err = gpu_run(binding, w2)
+    assert err & binding.DEVERR_BAD_LENGTH
+
+
+# ---- the five full-size workloads, in the benchmark's launch configuration ----
+
+SAMPLES = {"tiny_decode": None, "batched_decode": 24, "chain_verify": 24, "long_fp8": 16,
+           "tree_verify": 24}
+
+
+@pytest.mark.parametrize("name", wl.NAMES)
+def test_full_size_workload(binding, name):
+    w = wl.BUILDERS[name]()
+    (out, lse, info), err = gpu_run(binding, w)
+    assert err == 0
+    assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
+    pb = to_problem(w)
+    n = SAMPLES[name]
+    if n is None:
+        ref_out, ref_lse = orc.attention(pb)
+        assert_close(out, ref_out, w.dtype)
+        np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=lse_tol(w.dtype) * 4)
+        return
+    rng = np.random.default_rng(2024)
+    m = orc.marshal(pb)
+    seqs = rng.integers(0, w.n_seqs, n)
+    for s in seqs:
+        r0, r1 = int(w.row_offsets[s]), int(w.row_offsets[s + 1])
+        if r1 == r0:
+            continue
+        r = int(rng.integers(0, r1 - r0))
+        h = int(rng.integers(0, w.n_q_heads))
+        ref, ref_lse = orc.attention_one(pb, int(s), r, h, marshalled=m)
+        assert_close(out[r0 + r, h], ref, w.dtype, what=f"{name} seq {s} row {r} head {h}")
+        assert abs(lse[r0 + r, h] - ref_lse) <= lse_tol(w.dtype) * 4

@@ -1,0 +1,92 @@
+// Internal declarations shared by the host side (lse_host.cpp) and the
+// kernels (lse_kernels.cu) of liblse_attn.so.  Not part of the C ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "lse_attn.h"
+
+struct lse_kv_arena {
+  std::vector<uint64_t> chunk_base;  // device addresses
+  size_t chunk_bytes = 0;
+  size_t fragment_bytes = 0;
+  int dtype = 0;
+  int n_kv_heads = 0;
+  int head_dim = 0;
+  int esize = 0;
+  int tokens_per_fragment = 0;
+  int frags_per_chunk = 0;
+  std::vector<uint8_t> used;        // per fragment id
+  std::vector<int32_t> chunk_live;  // live fragments per chunk
+  int32_t n_free = 0;
+  int32_t scan_from = 0;            // lowest id that may be free
+};
+
+struct lse_attn_plan_s {
+  const lse_kv_arena *arena = nullptr;
+  int n_seqs = 0;
+  int max_rows = 0;
+  int max_total_rows = 0;
+  int n_q_heads = 0;
+  int n_kv_heads = 0;
+  int group = 0;        // G = Hq / Hkv
+  int head_dim = 0;
+  int dtype = 0;
+  int max_pages = 0;
+  int tokens_per_fragment = 0;
+  int n_splits = 0;
+  int keys_per_split = 0;
+  int kernel = 0;
+  int key_tile = 0;
+  int pairs = 0;        // G * max_rows
+  int smem_bytes = 0;
+  int n_sms = 0;
+  size_t ws_bytes = 0;
+  size_t ws_o_off = 0;   // partial outputs  FP32 [rows][Hq][n_splits][D]
+  size_t ws_lse_off = 0; // partial lse (log2 units) FP32 [rows][Hq][n_splits]
+};
+
+// Bytes reserved at the head of the workspace (error word + padding).
+constexpr size_t kWsHeader = 256;
+
+// Parameters passed by value to the partial and merge kernels.
+struct LseKernelParams {
+  unsigned long long chunk_base[LSE_MAX_CHUNKS];
+  long long fragment_bytes;
+  int frags_per_chunk;
+  int n_fragments;
+  int n_q_heads;
+  int n_kv_heads;
+  int group;
+  int head_dim;
+  int tokens_per_fragment;
+  int max_pages;
+  int n_splits;
+  int keys_per_split;
+  int max_rows;
+  int max_total_rows;
+  int n_seqs;
+  float scale_log2;  // softmax_scale * log2(e)
+  const float *q;
+  const int32_t *k_pages;
+  const int32_t *v_pages;
+  const int32_t *seq_lens;
+  const int32_t *row_offsets;
+  const unsigned long long *row_masks;
+  float *o_part;
+  float *lse_part;
+  unsigned int *err;
+  float *out;
+  float *lse_out;
+};
+
+// Kernel entry points (lse_kernels.cu).  Return a cudaError_t value.
+int lse_launch_partial_cuda_core(const LseKernelParams &p, int dtype, int head_dim, int grid_x,
+                                 int grid_y, int grid_z, int smem, void *stream);
+int lse_launch_merge(const LseKernelParams &p, int head_dim, void *stream);
+int lse_partial_cuda_core_smem(int head_dim);
+int lse_partial_cuda_core_occupancy(int dtype, int head_dim, int smem, int *ctas_per_sm);
+const char *lse_cuda_error_string(int code);

@@ -1,0 +1,473 @@
+// CUDA-core partial pass and the log-sum-exp merge pass of split-KV paged
+// attention (sm_100a).
+//
+// Partial pass (LSE releases, v0.4.19 "Long-context split attention": one
+// partial family; v0.4.21: K/V reads shared across query heads and rows).
+// One CTA per (partition, kv head, sequence).  The CTA streams the
+// partition's keys in tiles of 32, reading each K/V row of its kv head once
+// through the page table and converting it to FP32 in shared memory; every
+// (query row, query head) pair of the group then uses that tile.  Scores,
+// online softmax (running max / sum in log2 units) and the P.V accumulation
+// run in FP32 on CUDA cores.  A partition past the sequence's live keys
+// returns before loading anything (v0.4.20: empty-partition skipping).
+//
+// Merge pass (v0.4.19: one merge family): for each (row, head) the live
+// partials are combined with weights exp(lse_p - max lse).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+
+#include <cfloat>
+#include <cstdint>
+
+#include "lse_internal.h"
+
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int kTileKeys = 32;   // keys per tile
+constexpr int kPairChunk = 16;  // (row, head) pairs per pass over the keys
+
+// ---- loads and conversions ---------------------------------------------
+
+template <int DT>
+struct KvFormat;
+template <>
+struct KvFormat<LSE_KV_F32> {
+  static constexpr int kElemBytes = 4;
+  static __device__ __forceinline__ void to_float(const uint4 &v, float *o) {
+    o[0] = __uint_as_float(v.x);
+    o[1] = __uint_as_float(v.y);
+    o[2] = __uint_as_float(v.z);
+    o[3] = __uint_as_float(v.w);
+  }
+};
+template <>
+struct KvFormat<LSE_KV_F16> {
+  static constexpr int kElemBytes = 2;
+  static __device__ __forceinline__ void to_float(const uint4 &v, float *o) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __half2 h = *reinterpret_cast<const __half2 *>(&w[i]);
+      float2 f = __half22float2(h);
+      o[2 * i] = f.x;
+      o[2 * i + 1] = f.y;
+    }
+  }
+};
+template <>
+struct KvFormat<LSE_KV_BF16> {
+  static constexpr int kElemBytes = 2;
+  static __device__ __forceinline__ void to_float(const uint4 &v, float *o) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162 *>(&w[i]);
+      float2 f = __bfloat1622float2(h);
+      o[2 * i] = f.x;
+      o[2 * i + 1] = f.y;
+    }
+  }
+};
+template <__nv_fp8_interpretation_t I>
+struct Fp8Format {
+  static constexpr int kElemBytes = 1;
+  static __device__ __forceinline__ void to_float(const uint4 &v, float *o) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)((w[i] >> (16 * k)) & 0xffffu);
+        __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, I);
+        float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hr));
+        o[4 * i + 2 * k] = f.x;
+        o[4 * i + 2 * k + 1] = f.y;
+      }
+    }
+  }
+};
+template <>
+struct KvFormat<LSE_KV_FP8_E4M3> : Fp8Format<__NV_E4M3> {};
+template <>
+struct KvFormat<LSE_KV_FP8_E5M2> : Fp8Format<__NV_E5M2> {};
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// Checks shared by both passes; returns false (and flags) on bad lengths.
+__device__ __forceinline__ bool seq_shape(const LseKernelParams &p, int s, int &L, int &row0,
+                                          int &R) {
+  L = p.seq_lens[s];
+  row0 = p.row_offsets[s];
+  R = p.row_offsets[s + 1] - row0;
+  const long long cap = (long long)p.max_pages * p.tokens_per_fragment;
+  if (row0 < 0 || R < 0 || R > p.max_rows || row0 + R > p.max_total_rows || R > L ||
+      (long long)L > cap) {
+    if (threadIdx.x == 0) atomicOr(p.err, LSE_DEVERR_BAD_LENGTH);
+    return false;
+  }
+  return true;
+}
+
+// Device address of key `key` of kv head g through a page table, or null
+// when the entry names no fragment (flagged).
+__device__ __forceinline__ const uint8_t *kv_addr(const LseKernelParams &p, const int32_t *table,
+                                                  int s, int key, int g, int row_bytes_head) {
+  const int T = p.tokens_per_fragment;
+  const int page = key / T;
+  const int off = key - page * T;
+  const int frag = table[(long long)s * p.max_pages + page];
+  if (frag < 0 || frag >= p.n_fragments) {
+    atomicOr(p.err, LSE_DEVERR_BAD_FRAGMENT);
+    return nullptr;
+  }
+  const int chunk = frag / p.frags_per_chunk;
+  const long long byte = (long long)(frag - chunk * p.frags_per_chunk) * p.fragment_bytes +
+                         ((long long)off * p.n_kv_heads + g) * row_bytes_head;
+  return reinterpret_cast<const uint8_t *>(p.chunk_base[chunk]) + byte;
+}
+
+// ---- partial pass on CUDA cores ------------------------------------------
+
+template <int D>
+struct CcShape {
+  static constexpr int kRow = D + 4;  // padded FP32 row in shared memory
+  static constexpr int kDimsPerThread = D >= kThreads ? D / kThreads : 1;
+  static constexpr int kDimCover = D / kDimsPerThread;     // threads covering D
+  static constexpr int kPairSets = kThreads / kDimCover;   // 1 or 2
+  static constexpr int kPairsPerThread = kPairChunk / kPairSets;
+  static constexpr int kSmemFloats =
+      kPairChunk * D + 2 * kTileKeys * kRow + kPairChunk * kTileKeys + 4 * kPairChunk;
+  static constexpr int kSmemBytes = kSmemFloats * 4 + kPairChunk * 8;
+};
+
+template <int DT, int D>
+__global__ void __launch_bounds__(kThreads)
+    partial_cuda_core_kernel(const __grid_constant__ LseKernelParams p) {
+  using Fmt = KvFormat<DT>;
+  using Sh = CcShape<D>;
+  constexpr int kEsz = Fmt::kElemBytes;
+  constexpr int kVecPerRow = D * kEsz / 16;  // 16-byte vectors per key row
+  constexpr int kElemPerVec = 16 / kEsz;
+
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float *Qs = reinterpret_cast<float *>(smem_raw);  // [PC][D], pre-scaled
+  float *Ks = Qs + kPairChunk * D;                   // [TK][kRow]
+  float *Vs = Ks + kTileKeys * Sh::kRow;             // [TK][kRow]
+  float *Ps = Vs + kTileKeys * Sh::kRow;             // [PC][TK]
+  float *alpha_s = Ps + kPairChunk * kTileKeys;      // [PC]
+  float *m_s = alpha_s + kPairChunk;                 // [PC]
+  float *l_s = m_s + kPairChunk;                     // [PC]
+  unsigned long long *mask_s =
+      reinterpret_cast<unsigned long long *>(l_s + 2 * kPairChunk);  // [PC]
+
+  const int split = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int L, row0, R;
+  if (!seq_shape(p, s, L, row0, R)) return;
+  const int kb = split * p.keys_per_split;
+  if (R == 0 || kb >= L) return;  // idle sequence or empty partition: skipped
+  const int ke = min(kb + p.keys_per_split, L);
+  const int C = L - R;
+  const int G = p.group;
+  const int P = G * R;
+  const int row_bytes_head = D * kEsz;
+
+  for (int pc0 = 0; pc0 < P; pc0 += kPairChunk) {
+    const int npc = min(kPairChunk, P - pc0);
+    // Q chunk, scaled by softmax_scale * log2(e) so scores are in log2 units
+    for (int e = tid; e < kPairChunk * D; e += kThreads) {
+      const int i = e / D, d = e - (e / D) * D;
+      float v = 0.f;
+      if (i < npc) {
+        const int pr = pc0 + i, r = pr / G, h = g * G + (pr - r * G);
+        v = p.q[((long long)(row0 + r) * p.n_q_heads + h) * D + d] * p.scale_log2;
+      }
+      Qs[e] = v;
+    }
+    if (tid < kPairChunk) {
+      unsigned long long m = 0;
+      if (tid < npc) {
+        const int r = (pc0 + tid) / G;
+        m = p.row_masks ? p.row_masks[row0 + r]
+                        : (r >= 63 ? ~0ull : ((1ull << (r + 1)) - 1ull));
+      }
+      mask_s[tid] = m;
+    }
+    // this warp's pairs (warp + 4k) keep running max / sum in registers
+    float m_run[kPairChunk / 4], l_run[kPairChunk / 4];
+#pragma unroll
+    for (int k = 0; k < kPairChunk / 4; ++k) {
+      m_run[k] = -INFINITY;
+      l_run[k] = 0.f;
+    }
+    const int dset = tid % Sh::kDimCover, pset = tid / Sh::kDimCover;
+    float acc[Sh::kPairsPerThread][Sh::kDimsPerThread];
+#pragma unroll
+    for (int a = 0; a < Sh::kPairsPerThread; ++a)
+#pragma unroll
+      for (int b = 0; b < Sh::kDimsPerThread; ++b) acc[a][b] = 0.f;
+    __syncthreads();
+
+    for (int t0 = kb; t0 < ke; t0 += kTileKeys) {
+      // load + convert this tile of K and V (one read per key row)
+      for (int v = tid; v < kTileKeys * kVecPerRow; v += kThreads) {
+        const int j = v / kVecPerRow, c = v - j * kVecPerRow;
+        const int key = t0 + j;
+        float kf[kElemPerVec], vf[kElemPerVec];
+        bool ok = key < ke;
+        const uint8_t *ka = nullptr, *va = nullptr;
+        if (ok) {
+          ka = kv_addr(p, p.k_pages, s, key, g, row_bytes_head);
+          va = kv_addr(p, p.v_pages, s, key, g, row_bytes_head);
+          ok = ka && va;
+        }
+        if (ok) {
+          const uint4 kr = __ldg(reinterpret_cast<const uint4 *>(ka) + c);
+          const uint4 vr = __ldg(reinterpret_cast<const uint4 *>(va) + c);
+          Fmt::to_float(kr, kf);
+          Fmt::to_float(vr, vf);
+        } else {
+#pragma unroll
+          for (int e = 0; e < kElemPerVec; ++e) kf[e] = vf[e] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < kElemPerVec; e += 4) {
+          *reinterpret_cast<float4 *>(&Ks[j * Sh::kRow + c * kElemPerVec + e]) =
+              make_float4(kf[e], kf[e + 1], kf[e + 2], kf[e + 3]);
+          *reinterpret_cast<float4 *>(&Vs[j * Sh::kRow + c * kElemPerVec + e]) =
+              make_float4(vf[e], vf[e + 1], vf[e + 2], vf[e + 3]);
+        }
+      }
+      __syncthreads();
+
+      // scores for key `lane` and pairs warp + 4k, then the online softmax
+      {
+        const int key = t0 + lane;
+        float x[kPairChunk / 4];
+#pragma unroll
+        for (int k = 0; k < kPairChunk / 4; ++k) x[k] = 0.f;
+        const float *krow = &Ks[lane * Sh::kRow];
+#pragma unroll 4
+        for (int d = 0; d < D; d += 4) {
+          const float4 kv = *reinterpret_cast<const float4 *>(krow + d);
+#pragma unroll
+          for (int k = 0; k < kPairChunk / 4; ++k) {
+            const float4 qv = *reinterpret_cast<const float4 *>(&Qs[(warp + 4 * k) * D + d]);
+            x[k] = fmaf(qv.x, kv.x, x[k]);
+            x[k] = fmaf(qv.y, kv.y, x[k]);
+            x[k] = fmaf(qv.z, kv.z, x[k]);
+            x[k] = fmaf(qv.w, kv.w, x[k]);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < kPairChunk / 4; ++k) {
+          const int i = warp + 4 * k;
+          const unsigned long long m = mask_s[i];
+          const bool vis = i < npc && key < ke && (key < C || ((m >> (key - C)) & 1ull));
+          const float xv = vis ? x[k] : -INFINITY;
+          const float m_new = fmaxf(m_run[k], warp_max(xv));
+          float pe = 0.f, alpha = 1.f;
+          if (m_new != -INFINITY) {
+            pe = vis ? exp2f(xv - m_new) : 0.f;
+            alpha = exp2f(m_run[k] - m_new);  // 0 when nothing was seen yet
+          }
+          l_run[k] = l_run[k] * alpha + warp_sum(pe);
+          m_run[k] = m_new;
+          Ps[i * kTileKeys + lane] = pe;
+          if (lane == 0) alpha_s[i] = alpha;
+        }
+      }
+      __syncthreads();
+
+      // O <- O * alpha + P . V for this thread's pairs and dims
+#pragma unroll
+      for (int a = 0; a < Sh::kPairsPerThread; ++a) {
+        const float al = alpha_s[pset + Sh::kPairSets * a];
+#pragma unroll
+        for (int b = 0; b < Sh::kDimsPerThread; ++b) acc[a][b] *= al;
+      }
+      for (int j = 0; j < kTileKeys; j += 4) {
+        float vv[4][Sh::kDimsPerThread];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+          for (int b = 0; b < Sh::kDimsPerThread; ++b)
+            vv[jj][b] = Vs[(j + jj) * Sh::kRow + dset + b * Sh::kDimCover];
+#pragma unroll
+        for (int a = 0; a < Sh::kPairsPerThread; ++a) {
+          const float4 pp =
+              *reinterpret_cast<const float4 *>(&Ps[(pset + Sh::kPairSets * a) * kTileKeys + j]);
+#pragma unroll
+          for (int b = 0; b < Sh::kDimsPerThread; ++b) {
+            acc[a][b] = fmaf(pp.x, vv[0][b], acc[a][b]);
+            acc[a][b] = fmaf(pp.y, vv[1][b], acc[a][b]);
+            acc[a][b] = fmaf(pp.z, vv[2][b], acc[a][b]);
+            acc[a][b] = fmaf(pp.w, vv[3][b], acc[a][b]);
+          }
+        }
+      }
+      __syncthreads();
+    }
+
+    // partial results: o / l and lse (log2 units); -inf for no visible key
+    if (lane == 0) {
+#pragma unroll
+      for (int k = 0; k < kPairChunk / 4; ++k) {
+        m_s[warp + 4 * k] = m_run[k];
+        l_s[warp + 4 * k] = l_run[k];
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int a = 0; a < Sh::kPairsPerThread; ++a) {
+      const int i = pset + Sh::kPairSets * a;
+      if (i >= npc) continue;
+      const int pr = pc0 + i, r = pr / G, h = g * G + (pr - r * G);
+      const long long ph = ((long long)(row0 + r) * p.n_q_heads + h) * p.n_splits + split;
+      const float l = l_s[i];
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+      for (int b = 0; b < Sh::kDimsPerThread; ++b)
+        p.o_part[ph * D + dset + b * Sh::kDimCover] = acc[a][b] * inv;
+      if (dset == 0) p.lse_part[ph] = l > 0.f ? m_s[i] + log2f(l) : -INFINITY;
+    }
+    __syncthreads();
+  }
+}
+
+// ---- merge pass -------------------------------------------------------------
+
+// grid (ceil(Hq / 4), max_rows, n_seqs), 4 warps; warp w -> head 4 * x + w.
+template <int D>
+__global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ LseKernelParams p) {
+  constexpr int kPerLane = D / 32;
+  const int s = blockIdx.z, r = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.x * 4 + warp;
+  int L, row0, R;
+  if (!seq_shape(p, s, L, row0, R)) return;
+  if (r >= R || h >= p.n_q_heads) return;
+  const int row = row0 + r;
+  const int n_live = min((L + p.keys_per_split - 1) / p.keys_per_split, p.n_splits);
+  const long long base = ((long long)row * p.n_q_heads + h) * p.n_splits;
+  const float *lse = p.lse_part + base;
+  const float *o = p.o_part + base * D;
+
+  float M = -INFINITY;
+  for (int i = lane; i < n_live; i += 32) M = fmaxf(M, lse[i]);
+  M = warp_max(M);
+  float acc[kPerLane];
+#pragma unroll
+  for (int k = 0; k < kPerLane; ++k) acc[k] = 0.f;
+  float wsum = 0.f;
+  if (M != -INFINITY) {
+    for (int i = 0; i < n_live; ++i) {
+      const float li = lse[i];
+      if (li == -INFINITY) continue;  // partition without a visible key
+      const float w = exp2f(li - M);
+      wsum += w;
+      const float *oi = o + (long long)i * D;
+#pragma unroll
+      for (int k = 0; k < kPerLane; ++k) acc[k] = fmaf(w, oi[lane + 32 * k], acc[k]);
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  float *out = p.out + ((long long)row * p.n_q_heads + h) * D;
+#pragma unroll
+  for (int k = 0; k < kPerLane; ++k) out[lane + 32 * k] = acc[k] * inv;
+  if (p.lse_out && lane == 0)
+    p.lse_out[(long long)row * p.n_q_heads + h] =
+        wsum > 0.f ? (M + log2f(wsum)) * 0.69314718055994530942f : -INFINITY;
+}
+
+template <int DT, int D>
+int launch_cc(const LseKernelParams &p, int gx, int gy, int gz, int smem, cudaStream_t st) {
+  auto k = partial_cuda_core_kernel<DT, D>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return (int)e;
+  k<<<dim3(gx, gy, gz), kThreads, smem, st>>>(p);
+  return (int)cudaGetLastError();
+}
+
+template <int DT>
+int launch_cc_d(const LseKernelParams &p, int D, int gx, int gy, int gz, int smem,
+                cudaStream_t st) {
+  switch (D) {
+    case 64: return launch_cc<DT, 64>(p, gx, gy, gz, smem, st);
+    case 128: return launch_cc<DT, 128>(p, gx, gy, gz, smem, st);
+    case 256: return launch_cc<DT, 256>(p, gx, gy, gz, smem, st);
+  }
+  return (int)cudaErrorInvalidValue;
+}
+
+template <int DT, int D>
+int occ_cc(int smem, int *n) {
+  auto k = partial_cuda_core_kernel<DT, D>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return (int)e;
+  return (int)cudaOccupancyMaxActiveBlocksPerMultiprocessor(n, k, kThreads, smem);
+}
+
+}  // namespace
+
+int lse_partial_cuda_core_smem(int head_dim) {
+  switch (head_dim) {
+    case 64: return CcShape<64>::kSmemBytes;
+    case 128: return CcShape<128>::kSmemBytes;
+    case 256: return CcShape<256>::kSmemBytes;
+  }
+  return -1;
+}
+
+int lse_partial_cuda_core_occupancy(int dtype, int head_dim, int smem, int *n) {
+  // occupancy depends on registers and shared memory, not on the format;
+  // the BF16 instance stands for all
+  (void)dtype;
+  switch (head_dim) {
+    case 64: return occ_cc<LSE_KV_BF16, 64>(smem, n);
+    case 128: return occ_cc<LSE_KV_BF16, 128>(smem, n);
+    case 256: return occ_cc<LSE_KV_BF16, 256>(smem, n);
+  }
+  return (int)cudaErrorInvalidValue;
+}
+
+int lse_launch_partial_cuda_core(const LseKernelParams &p, int dtype, int head_dim, int gx,
+                                 int gy, int gz, int smem, void *stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  switch (dtype) {
+    case LSE_KV_F32: return launch_cc_d<LSE_KV_F32>(p, head_dim, gx, gy, gz, smem, st);
+    case LSE_KV_F16: return launch_cc_d<LSE_KV_F16>(p, head_dim, gx, gy, gz, smem, st);
+    case LSE_KV_BF16: return launch_cc_d<LSE_KV_BF16>(p, head_dim, gx, gy, gz, smem, st);
+    case LSE_KV_FP8_E4M3:
+      return launch_cc_d<LSE_KV_FP8_E4M3>(p, head_dim, gx, gy, gz, smem, st);
+    case LSE_KV_FP8_E5M2:
+      return launch_cc_d<LSE_KV_FP8_E5M2>(p, head_dim, gx, gy, gz, smem, st);
+  }
+  return (int)cudaErrorInvalidValue;
+}
+
+int lse_launch_merge(const LseKernelParams &p, int head_dim, void *stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  dim3 grid((p.n_q_heads + 3) / 4, p.max_rows, p.n_seqs);
+  switch (head_dim) {
+    case 64: merge_kernel<64><<<grid, 128, 0, st>>>(p); break;
+    case 128: merge_kernel<128><<<grid, 128, 0, st>>>(p); break;
+    case 256: merge_kernel<256><<<grid, 128, 0, st>>>(p); break;
+    default: return (int)cudaErrorInvalidValue;
+  }
+  return (int)cudaGetLastError();
+}
+
+const char *lse_cuda_error_string(int code) { return cudaGetErrorString((cudaError_t)code); }
