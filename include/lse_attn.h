@@ -97,9 +97,11 @@ typedef enum {
 
 /* Bits of the device error word (lse_attn_read_error). */
 #define LSE_DEVERR_BAD_FRAGMENT 0x1u /* a page-table entry named no fragment   */
+#define LSE_DEVERR_TIMEOUT 0x4u      /* a pipeline wait ran out (~2 s); the call aborted */
 #define LSE_DEVERR_BAD_LENGTH 0x2u   /* L_s > capacity, R_s > L_s, R_s > max rows or rows past max_total_rows */
 
 #define LSE_MAX_CHUNKS 64     /* arena chunks a kernel can address          */
+#define LSE_MAX_TMA_CHUNKS 16 /* chunks the tensor-core kernel can address; more -> CUDA cores */
 #define LSE_MAX_ROWS_PER_SEQ 64
 
 typedef struct lse_kv_arena lse_kv_arena;
@@ -182,13 +184,22 @@ LSE_API int lse_attn_plan_ex(const lse_kv_arena *arena, int n_seqs, int max_rows
 #define LSE_KERNEL_CUDA_CORE 0 /* FP32 math on CUDA cores (any dtype, any P) */
 #define LSE_KERNEL_TCGEN05 1   /* tensor-core (tcgen05) partial pass           */
 
+/* For LSE_KERNEL_CUDA_CORE the partitions are fixed ranges of K_p keys,
+ * n_splits = ceil(capacity / K_p), and partitions past a sequence's live
+ * keys are skipped.  For LSE_KERNEL_TCGEN05 the partial pass is persistent
+ * (one CTA per SM): the live 128-key tiles of all (sequence, kv head) pairs
+ * are laid end to end and cut into equal contiguous ranges, one per CTA;
+ * n_splits = min(CTAs, capacity tiles) bounds the pieces of one (sequence,
+ * kv head), keys_per_split reports the tile (128), and capacity without
+ * live keys is never visited. */
 typedef struct {
-  int32_t n_splits;        /* partitions per (sequence, kv head)            */
-  int32_t keys_per_split;  /* K_p                                           */
+  int32_t n_splits;        /* partial slots per (row, head)                  */
+  int32_t keys_per_split;  /* K_p (CUDA-core) or the key tile (tcgen05)      */
   int32_t kernel;          /* LSE_KERNEL_*                                  */
   int32_t key_tile;        /* keys per pipeline stage                      */
   int32_t pairs;           /* (row, head) pairs per kv head: G * max rows   */
   int32_t smem_bytes;      /* dynamic shared memory of the partial kernel  */
+  int32_t ctas;            /* partial-pass CTAs when persistent, else 0     */
   int64_t workspace_bytes;
 } lse_attn_plan_info;
 

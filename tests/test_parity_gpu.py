@@ -157,3 +157,108 @@ def test_full_size_workload(binding, name):
         ref, ref_lse = orc.attention_one(pb, int(s), r, h, marshalled=m)
         assert_close(out[r0 + r, h], ref, w.dtype, what=f"{name} seq {s} row {r} head {h}")
         assert abs(lse[r0 + r, h] - ref_lse) <= lse_tol(w.dtype) * 4
+
+
+# ---- the tensor-core (tcgen05) partial pass --------------------------------------
+
+def _rewrite_k(w, fn):
+    """Rewrite every live K row of every sequence in place (test-side layout
+    writer): row j of sequence s becomes fn(s, j, old_row_as_float32)."""
+    from verify_attention_paged_b200.workloads import TORCH_DTYPES, ELEM_SIZE
+    chunks = [c.copy() for c in w.chunks]
+    T = w.tokens_per_fragment
+    fpc = w.chunk_bytes // w.fragment_bytes
+    row = w.n_kv_heads * w.head_dim * ELEM_SIZE[w.dtype]
+    tdt = TORCH_DTYPES[w.dtype]
+    for s in range(w.n_seqs):
+        L = int(w.seq_lens[s])
+        for j in range(L):
+            c, off = divmod(int(w.k_pages[s, j // T]), fpc)
+            b = off * w.fragment_bytes + (j % T) * row
+            old = torch.from_numpy(chunks[c][b:b + row].copy()).view(tdt).float()
+            new = fn(s, j, old).to(tdt).contiguous().view(torch.uint8).numpy()
+            chunks[c][b:b + row] = new
+    return wl.Workload(**{**w.__dict__, "chunks": chunks})
+
+
+def check_kernel(b, w, kernel):
+    (out, lse, info), err = gpu_run(b, w, kernel=kernel)
+    assert info["kernel_name"] == kernel
+    assert err == 0, f"device error word {err:#x}"
+    ref_out, ref_lse = orc.attention(to_problem(w))
+    assert_close(out, ref_out, w.dtype)
+    np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=lse_tol(w.dtype) * 4)
+    return out
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("tpf", [8, 16, 64, 128, 256, 512])
+def test_tcgen05_fragment_sizes(binding, dtype, tpf):
+    w = wl.small_case(dtype, [1, 127, 128, 129, 700, 2051], [1, 1, 2, 3, 4, 8],
+                      n_q_heads=24, n_kv_heads=4, head_dim=128, tokens_per_fragment=tpf,
+                      seed=200 + tpf)
+    check_kernel(binding, w, "tcgen05")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("heads,rows", [((24, 4), 8), ((32, 8), 12), ((8, 8), 1),
+                                        ((16, 1), 3), ((12, 4), 16)])
+def test_tcgen05_pairs_and_trees(binding, dtype, heads, rows):
+    hq, hkv = heads
+    lens = [300, 1000, rows, 4100, 64]
+    w = wl.small_case(dtype, lens, [rows] * 5, n_q_heads=hq, n_kv_heads=hkv, head_dim=128,
+                      tokens_per_fragment=64, tree=True, seed=210 + rows)
+    check_kernel(binding, w, "tcgen05")
+
+
+def test_tcgen05_many_segments_per_cta(binding):
+    # 70 short sequences: CTAs cross many (sequence, kv head) segments, so the
+    # Q ring, the two TMEM output slots and the piece numbering all rotate
+    rng = np.random.default_rng(5)
+    lens = [int(x) for x in rng.integers(1, 600, 70)]
+    rows = [int(min(L, r)) for L, r in zip(lens, rng.integers(0, 7, 70))]
+    w = wl.small_case("bf16", lens, rows, n_q_heads=24, n_kv_heads=4, head_dim=128,
+                      tokens_per_fragment=128, tree=True, seed=220)
+    out_tc = check_kernel(binding, w, "tcgen05")
+    out_cc = check_kernel(binding, w, "cuda_core")
+    assert_close(out_tc, out_cc, "bf16", what="tcgen05 vs cuda_core")
+
+
+def test_tcgen05_fewer_tiles_than_ctas(binding):
+    w = wl.small_case("f16", [200], [2], n_q_heads=8, n_kv_heads=2, head_dim=128,
+                      tokens_per_fragment=64, seed=221)
+    check_kernel(binding, w, "tcgen05")
+
+
+def test_tcgen05_growing_scores_trigger_rescale(binding):
+    # key rows grow with position, so the running maximum rises tile after
+    # tile by more than the lazy threshold: the TMEM output must be rescaled
+    w = wl.small_case("bf16", [3000, 900], [4, 1], n_q_heads=24, n_kv_heads=4, head_dim=128,
+                      tokens_per_fragment=256, seed=222)
+    w2 = _rewrite_k(w, lambda s, j, k: k * (0.25 + j / 150.0))
+    check_kernel(binding, w2, "tcgen05")
+
+
+def test_tcgen05_capacity_far_above_live(binding):
+    w = wl.small_case("bf16", [130, 5, 1000], [1, 1, 2], n_q_heads=24, n_kv_heads=4,
+                      head_dim=128, tokens_per_fragment=128, max_pages=300, seed=223)
+    check_kernel(binding, w, "tcgen05")
+
+
+def test_tcgen05_bad_page_sets_error_word(binding):
+    w = wl.small_case("bf16", [600], [2], n_q_heads=8, n_kv_heads=2, head_dim=128,
+                      tokens_per_fragment=128, seed=224)
+    kp = w.k_pages.copy()
+    kp[0, 1] = 10 ** 6
+    w2 = wl.Workload(**{**w.__dict__, "k_pages": kp})
+    (_, _, info), err = gpu_run(binding, w2, kernel="tcgen05")
+    assert err & binding.DEVERR_BAD_FRAGMENT and not err & binding.DEVERR_TIMEOUT
+
+
+def test_plan_picks_tensor_cores_for_the_bf16_workloads(binding):
+    for name, want in (("batched_decode", "tcgen05"), ("chain_verify", "tcgen05"),
+                       ("tiny_decode", "cuda_core")):
+        w = wl.BUILDERS[name]()
+        call = binding.DeviceCall(w)
+        assert call.info["kernel_name"] == want, name
+        call.close()

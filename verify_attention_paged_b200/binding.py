@@ -33,6 +33,7 @@ KV_DTYPES = {"f32": 0, "f16": 1, "bf16": 2, "e4m3": 3, "e5m2": 4}
 KERNELS = {0: "cuda_core", 1: "tcgen05"}
 DEVERR_BAD_FRAGMENT = 0x1
 DEVERR_BAD_LENGTH = 0x2
+DEVERR_TIMEOUT = 0x4
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
@@ -50,7 +51,7 @@ class PlanInfo(ctypes.Structure):
     _fields_ = [("n_splits", ctypes.c_int32), ("keys_per_split", ctypes.c_int32),
                 ("kernel", ctypes.c_int32), ("key_tile", ctypes.c_int32),
                 ("pairs", ctypes.c_int32), ("smem_bytes", ctypes.c_int32),
-                ("workspace_bytes", ctypes.c_int64)]
+                ("ctas", ctypes.c_int32), ("workspace_bytes", ctypes.c_int64)]
 
 
 class DeviceLimits(ctypes.Structure):
@@ -267,10 +268,17 @@ class DeviceCall:
     masks, Q, shapes, scale).
     """
 
-    def __init__(self, problem, max_total_rows=None, stream=None, plan_limits=None):
+    def __init__(self, problem, max_total_rows=None, stream=None, plan_limits=None,
+                 kernel="auto"):
         import torch
         self.torch = torch
         dev = torch.device("cuda", torch.cuda.current_device())
+        if kernel != "auto" and plan_limits is None:
+            props = torch.cuda.get_device_properties(dev)
+            plan_limits = dict(n_sms=props.multi_processor_count,
+                               smem_optin=getattr(props, "shared_memory_per_block_optin",
+                                                  232448),
+                               ctas_per_sm=0, allow_tcgen05=int(kernel == "tcgen05"))
         self.w = problem
         self.chunks = [torch.from_numpy(c).to(dev) for c in problem.chunks]
         self.k_pages = torch.from_numpy(np.ascontiguousarray(problem.k_pages)).to(dev)
@@ -297,6 +305,8 @@ class DeviceCall:
                                              problem.n_q_heads, problem.k_pages.shape[1],
                                              **plan_limits)
         self.info = lse_attn_plan_query(self.plan)
+        if kernel != "auto" and self.info["kernel_name"] != kernel:
+            raise LseError(2, f"plan chose {self.info['kernel_name']}, not {kernel}")
         self.workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
         self.stream = stream if stream is not None else torch.cuda.current_stream()
         lse_attn_workspace_init(self.plan, self.workspace, self.stream)

@@ -247,8 +247,11 @@ int lse_attn_plan_ex(const lse_kv_arena *a, int n_seqs, int max_rows, int max_to
     if (ce) return cuda_fail(err, ce, "cudaDeviceGetAttribute(SM count)");
     ce = (int)cudaDeviceGetAttribute(&smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (ce) return cuda_fail(err, ce, "cudaDeviceGetAttribute(shared memory)");
+    int major = 0;
+    ce = (int)cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (ce) return cuda_fail(err, ce, "cudaDeviceGetAttribute(compute capability)");
+    allow_tc = major == 10;  // tcgen05 needs sm_100
   }
-  (void)allow_tc;
 
   lse_attn_plan_t *pl = new (std::nothrow) lse_attn_plan_t;
   if (!pl) return fail(err, LSE_ERR_NO_MEMORY, "plan");
@@ -266,29 +269,50 @@ int lse_attn_plan_ex(const lse_kv_arena *a, int n_seqs, int max_rows, int max_to
   pl->pairs = pl->group * max_rows;
   pl->n_sms = n_sms;
 
-  // kernel choice and its on-chip memory check
-  pl->kernel = LSE_KERNEL_CUDA_CORE;
-  pl->key_tile = 32;
-  pl->smem_bytes = lse_partial_cuda_core_smem(a->head_dim);
-  if (pl->smem_bytes < 0 || pl->smem_bytes > smem_optin) {
-    delete pl;
-    return fail(err, LSE_ERR_UNSUPPORTED, "partial kernel needs %d bytes of shared memory, "
-                "device allows %d", pl->smem_bytes, smem_optin);
-  }
-  int ctas_per_sm = ctas_given;
-  if (ctas_per_sm == 0) {
-    ce = lse_partial_cuda_core_occupancy(a->dtype, a->head_dim, pl->smem_bytes, &ctas_per_sm);
-    if (ce) {
+  // kernel choice and its on-chip memory check.  The tensor-core kernel
+  // takes 16-bit K/V with head_dim 128, up to 48 (row, head) pairs per kv
+  // head, and fragments whose token count tiles evenly into 128-key tiles.
+  const int T = a->tokens_per_fragment;
+  const bool t_ok = (T % 128 == 0) || (T >= 8 && T % 8 == 0 && 128 % T == 0);
+  const int p8 = lse_tc_pairs_bucket(pl->pairs);
+  int tc_stages = 0;
+  const int tc_smem = p8 > 0 ? lse_tc_smem(p8, smem_optin, &tc_stages) : -1;
+  if (allow_tc && (a->dtype == LSE_KV_BF16 || a->dtype == LSE_KV_F16) && a->head_dim == 128 &&
+      t_ok && p8 > 0 && tc_smem > 0) {
+    const int tile = lse_tc_key_tile();
+    pl->kernel = LSE_KERNEL_TCGEN05;
+    pl->key_tile = tile;
+    pl->smem_bytes = tc_smem;
+    pl->stages = tc_stages;
+    pl->pairs_bucket = p8;
+    pl->box_tokens = T < tile ? T : tile;
+    pl->ctas = n_sms;
+    const int64_t cap_tiles = ceil_div(cap_keys, tile);
+    pl->n_splits = int(std::min<int64_t>(n_sms, cap_tiles));
+    pl->keys_per_split = tile;
+  } else {
+    pl->kernel = LSE_KERNEL_CUDA_CORE;
+    pl->key_tile = 32;
+    pl->smem_bytes = lse_partial_cuda_core_smem(a->head_dim);
+    if (pl->smem_bytes < 0 || pl->smem_bytes > smem_optin) {
       delete pl;
-      return cuda_fail(err, ce, "occupancy query");
+      return fail(err, LSE_ERR_UNSUPPORTED, "partial kernel needs %d bytes of shared memory, "
+                  "device allows %d", pl->smem_bytes, smem_optin);
     }
+    int ctas_per_sm = ctas_given;
+    if (ctas_per_sm == 0) {
+      ce = lse_partial_cuda_core_occupancy(a->dtype, a->head_dim, pl->smem_bytes, &ctas_per_sm);
+      if (ce) {
+        delete pl;
+        return cuda_fail(err, ce, "occupancy query");
+      }
+    }
+    ctas_per_sm = std::max(1, ctas_per_sm);
+    int32_t kp = 0;
+    pl->n_splits = lse_attn_split_rule(cap_keys, n_seqs * a->n_kv_heads, n_sms, ctas_per_sm,
+                                       pl->key_tile, &kp);
+    pl->keys_per_split = kp;
   }
-  ctas_per_sm = std::max(1, ctas_per_sm);
-
-  int32_t kp = 0;
-  pl->n_splits = lse_attn_split_rule(cap_keys, n_seqs * a->n_kv_heads, n_sms, ctas_per_sm,
-                                     pl->key_tile, &kp);
-  pl->keys_per_split = kp;
 
   const size_t n_part = size_t(max_total_rows) * n_q_heads * pl->n_splits;
   pl->ws_o_off = kWsHeader;
@@ -307,6 +331,7 @@ int lse_attn_plan_query(const lse_attn_plan_t *pl, lse_attn_plan_info *info) {
   info->key_tile = pl->key_tile;
   info->pairs = pl->pairs;
   info->smem_bytes = pl->smem_bytes;
+  info->ctas = pl->kernel == LSE_KERNEL_TCGEN05 ? pl->ctas : 0;
   info->workspace_bytes = int64_t(pl->ws_bytes);
   return LSE_OK;
 }
@@ -368,8 +393,30 @@ int lse_attn_run(const lse_attn_plan_t *pl, const float *q, const int32_t *k_pag
   p.seq_lens = seq_lens;
   p.row_offsets = row_offsets;
   p.row_masks = reinterpret_cast<const unsigned long long *>(row_masks);
-  int ce = lse_launch_partial_cuda_core(p, pl->dtype, pl->head_dim, pl->n_splits,
-                                        pl->n_kv_heads, pl->n_seqs, pl->smem_bytes, stream);
+  int ce = 0;
+  if (pl->kernel == LSE_KERNEL_TCGEN05) {
+    const lse_kv_arena *a = pl->arena;
+    const int nch = int(a->chunk_base.size());
+    if (nch > LSE_MAX_TMA_CHUNKS)
+      return fail(err, LSE_ERR_UNSUPPORTED, "arena has %d chunks; the tensor-core kernel "
+                  "addresses at most %d", nch, LSE_MAX_TMA_CHUNKS);
+    if (pl->maps_chunks != nch) {
+      pl->maps.assign(lse_tc_map_bytes() * nch, 0);
+      ce = lse_tc_build_maps(a->chunk_base.data(), nch, a->chunk_bytes, a->n_kv_heads,
+                             pl->box_tokens, pl->maps.data());
+      if (ce) {
+        pl->maps_chunks = 0;
+        return cuda_fail(err, ce, "building TMA descriptors");
+      }
+      pl->maps_chunks = nch;
+    }
+    ce = lse_launch_partial_tcgen05(p, pl->maps.data(), nch, pl->dtype, pl->pairs_bucket,
+                                    pl->ctas, pl->n_splits, pl->stages, pl->box_tokens,
+                                    pl->smem_bytes, stream);
+  } else {
+    ce = lse_launch_partial_cuda_core(p, pl->dtype, pl->head_dim, pl->n_splits, pl->n_kv_heads,
+                                      pl->n_seqs, pl->smem_bytes, stream);
+  }
   if (ce) return cuda_fail(err, ce, "partial kernel launch");
   return LSE_OK;
 }
@@ -384,6 +431,8 @@ int lse_attn_merge(const lse_attn_plan_t *pl, const int32_t *seq_lens, const int
   if (st) return st;
   p.seq_lens = seq_lens;
   p.row_offsets = row_offsets;
+  p.balanced = pl->kernel == LSE_KERNEL_TCGEN05;
+  p.n_ctas = pl->ctas;
   p.out = out;
   p.lse_out = lse_out;
   int ce = lse_launch_merge(p, pl->head_dim, stream);

@@ -44,6 +44,13 @@ struct lse_attn_plan_s {
   int pairs = 0;        // G * max_rows
   int smem_bytes = 0;
   int n_sms = 0;
+  int ctas = 0;          // persistent grid of the tensor-core kernel
+  int stages = 0;        // its pipeline depth
+  int pairs_bucket = 0;  // its compile-time pair count (P8)
+  int box_tokens = 0;    // its TMA box height
+  // tensor maps of the arena chunks (built on first run, rebuilt on growth)
+  mutable std::vector<uint8_t> maps;
+  mutable int maps_chunks = 0;
   size_t ws_bytes = 0;
   size_t ws_o_off = 0;   // partial outputs  FP32 [rows][Hq][n_splits][D]
   size_t ws_lse_off = 0; // partial lse (log2 units) FP32 [rows][Hq][n_splits]
@@ -81,6 +88,8 @@ struct LseKernelParams {
   unsigned int *err;
   float *out;
   float *lse_out;
+  int balanced;    // merge: 1 = slots are persistent-CTA pieces (tcgen05)
+  int n_ctas;      // persistent grid size when balanced
 };
 
 // Kernel entry points (lse_kernels.cu).  Return a cudaError_t value.
@@ -90,3 +99,14 @@ int lse_launch_merge(const LseKernelParams &p, int head_dim, void *stream);
 int lse_partial_cuda_core_smem(int head_dim);
 int lse_partial_cuda_core_occupancy(int dtype, int head_dim, int smem, int *ctas_per_sm);
 const char *lse_cuda_error_string(int code);
+
+// tensor-core partial pass (lse_tcgen05.cu)
+int lse_tc_pairs_bucket(int pairs);
+int lse_tc_smem(int p8, int smem_optin, int *stages);
+int lse_tc_key_tile();
+size_t lse_tc_map_bytes();
+int lse_tc_build_maps(const uint64_t *chunk_base, int n_chunks, size_t chunk_bytes,
+                      int n_kv_heads, int box_tokens, void *maps_out);
+int lse_launch_partial_tcgen05(const LseKernelParams &p, const void *maps, int n_maps,
+                               int dtype, int p8, int n_ctas, int n_slots, int stages,
+                               int box_tokens, int smem, void *stream);

@@ -349,6 +349,19 @@ __global__ void __launch_bounds__(kThreads)
 
 // ---- merge pass -------------------------------------------------------------
 
+// 128-key tiles of sequence s as the tensor-core pass counts them.
+__device__ __forceinline__ int seq_tiles_merge(const LseKernelParams &p, int s, int &L, int &row0,
+                                               int &R) {
+  L = p.seq_lens[s];
+  row0 = p.row_offsets[s];
+  R = p.row_offsets[s + 1] - row0;
+  const long long cap = (long long)p.max_pages * p.tokens_per_fragment;
+  if (row0 < 0 || R < 0 || R > p.max_rows || row0 + R > p.max_total_rows || R > L ||
+      (long long)L > cap || R == 0)
+    return 0;
+  return (L + 127) / 128;
+}
+
 // grid (ceil(Hq / 4), max_rows, n_seqs), 4 warps; warp w -> head 4 * x + w.
 template <int D>
 __global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ LseKernelParams p) {
@@ -360,7 +373,28 @@ __global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ LseK
   if (!seq_shape(p, s, L, row0, R)) return;
   if (r >= R || h >= p.n_q_heads) return;
   const int row = row0 + r;
-  const int n_live = min((L + p.keys_per_split - 1) / p.keys_per_split, p.n_splits);
+  int n_live;
+  if (p.balanced) {
+    // pieces of (s, kv head) written by the persistent tensor-core pass:
+    // tiles of all segments end to end, CTA c owning [c U / C, (c+1) U / C)
+    long long U = 0, before = 0;
+    int n_s = 0;
+    for (int q = 0; q < p.n_seqs; ++q) {
+      int Lq, r0q, Rq;
+      const int n = seq_tiles_merge(p, q, Lq, r0q, Rq);
+      if (q < s) before += n;
+      if (q == s) n_s = n;
+      U += n;
+    }
+    U *= p.n_kv_heads;
+    const int g = h / p.group;
+    const long long first = before * p.n_kv_heads + (long long)g * n_s;
+    const long long last = first + n_s - 1;
+    const long long C = U < p.n_ctas ? U : p.n_ctas;  // working CTAs of the partial pass
+    n_live = n_s > 0 ? int(((last + 1) * C - 1) / U - ((first + 1) * C - 1) / U) + 1 : 0;
+  } else {
+    n_live = min((L + p.keys_per_split - 1) / p.keys_per_split, p.n_splits);
+  }
   const long long base = ((long long)row * p.n_q_heads + h) * p.n_splits;
   const float *lse = p.lse_part + base;
   const float *o = p.o_part + base * D;
