@@ -189,9 +189,10 @@ LSE_API int lse_attn_plan_ex(const lse_kv_arena *arena, int n_seqs, int max_rows
  * keys are skipped.  For LSE_KERNEL_TCGEN05 the partial pass is persistent
  * (one CTA per SM): the live 128-key tiles of all (sequence, kv head) pairs
  * are laid end to end and cut into equal contiguous ranges, one per CTA;
- * n_splits = min(CTAs, capacity tiles) bounds the pieces of one (sequence,
- * kv head), keys_per_split reports the tile (128), and capacity without
- * live keys is never visited. */
+ * each piece yields one partial per softmax warpgroup, so n_splits =
+ * 2 * min(CTAs, capacity tiles) bounds the partials of one (sequence, kv
+ * head); keys_per_split reports the tile (128); capacity without live keys
+ * is never visited. */
 typedef struct {
   int32_t n_splits;        /* partial slots per (row, head)                  */
   int32_t keys_per_split;  /* K_p (CUDA-core) or the key tile (tcgen05)      */

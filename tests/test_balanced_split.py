@@ -39,5 +39,5 @@ def test_segment_pieces_fit_their_slots():
         for n in tiles:
             if n:
                 pieces = cta_of(first + n - 1, U, C) - cta_of(first, U, C) + 1
-                assert 1 <= pieces <= min(grid, n)
+                assert 1 <= pieces <= min(grid, n)  # x2 partials per piece in the workspace
             first += n

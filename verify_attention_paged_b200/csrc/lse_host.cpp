@@ -288,7 +288,9 @@ int lse_attn_plan_ex(const lse_kv_arena *a, int n_seqs, int max_rows, int max_to
     pl->box_tokens = T < tile ? T : tile;
     pl->ctas = n_sms;
     const int64_t cap_tiles = ceil_div(cap_keys, tile);
-    pl->n_splits = int(std::min<int64_t>(n_sms, cap_tiles));
+    // a (sequence, kv head) has at most min(CTAs, tiles) pieces, and each
+    // piece holds one partial per softmax group
+    pl->n_splits = 2 * int(std::min<int64_t>(n_sms, cap_tiles));
     pl->keys_per_split = tile;
   } else {
     pl->kernel = LSE_KERNEL_CUDA_CORE;

@@ -172,6 +172,7 @@ __global__ void __launch_bounds__(kThreads)
   unsigned long long *mask_s =
       reinterpret_cast<unsigned long long *>(l_s + 2 * kPairChunk);  // [PC]
 
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int split = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int L, row0, R;
@@ -362,16 +363,25 @@ __device__ __forceinline__ int seq_tiles_merge(const LseKernelParams &p, int s, 
   return (L + 127) / 128;
 }
 
-// grid (ceil(Hq / 4), max_rows, n_seqs), 4 warps; warp w -> head 4 * x + w.
+// One CTA (4 warps) per (query head, row of a sequence): grid (Hq, max_rows,
+// n_seqs).  The CTA first finds the live partials of its (sequence, kv head)
+// and their maximum lse; each warp then sums a quarter of the partials
+// (each lane a D/32 slice of the head dim, eight partial rows in flight at
+// a time) and the four sums are combined in shared memory.
 template <int D>
 __global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ LseKernelParams p) {
   constexpr int kPerLane = D / 32;
-  const int s = blockIdx.z, r = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.x * 4 + warp;
+  constexpr int kUnroll = 8;
+  __shared__ float s_red[4];
+  __shared__ float s_acc[4][D];
+  __shared__ float s_w[4];
+  // partials are written by the preceding partial pass (programmatic launch)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int h = blockIdx.x, r = blockIdx.y, s = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int L, row0, R;
   if (!seq_shape(p, s, L, row0, R)) return;
-  if (r >= R || h >= p.n_q_heads) return;
+  if (r >= R) return;
   const int row = row0 + r;
   int n_live;
   if (p.balanced) {
@@ -391,7 +401,8 @@ __global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ LseK
     const long long first = before * p.n_kv_heads + (long long)g * n_s;
     const long long last = first + n_s - 1;
     const long long C = U < p.n_ctas ? U : p.n_ctas;  // working CTAs of the partial pass
-    n_live = n_s > 0 ? int(((last + 1) * C - 1) / U - ((first + 1) * C - 1) / U) + 1 : 0;
+    // two partials (one per softmax group) per piece
+    n_live = n_s > 0 ? 2 * (int(((last + 1) * C - 1) / U - ((first + 1) * C - 1) / U) + 1) : 0;
   } else {
     n_live = min((L + p.keys_per_split - 1) / p.keys_per_split, p.n_splits);
   }
@@ -399,38 +410,64 @@ __global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ LseK
   const float *lse = p.lse_part + base;
   const float *o = p.o_part + base * D;
 
+  // maximum lse over the live partials (all 128 threads)
   float M = -INFINITY;
-  for (int i = lane; i < n_live; i += 32) M = fmaxf(M, lse[i]);
+  for (int i = tid; i < n_live; i += 128) M = fmaxf(M, lse[i]);
   M = warp_max(M);
+  if (lane == 0) s_red[warp] = M;
+  __syncthreads();
+  M = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
+
   float acc[kPerLane];
 #pragma unroll
   for (int k = 0; k < kPerLane; ++k) acc[k] = 0.f;
   float wsum = 0.f;
   if (M != -INFINITY) {
-    for (int i = 0; i < n_live; ++i) {
-      const float li = lse[i];
-      if (li == -INFINITY) continue;  // partition without a visible key
-      const float w = exp2f(li - M);
-      wsum += w;
-      const float *oi = o + (long long)i * D;
+    // warp w takes partials w, w + 4, w + 8, ...
+    for (int i0 = warp; i0 < n_live; i0 += 4 * kUnroll) {
+      float v[kUnroll][kPerLane];
+      float w[kUnroll];
 #pragma unroll
-      for (int k = 0; k < kPerLane; ++k) acc[k] = fmaf(w, oi[lane + 32 * k], acc[k]);
+      for (int u = 0; u < kUnroll; ++u) {
+        const int i = i0 + 4 * u;
+        const bool in = i < n_live;
+        const float li = in ? lse[i] : -INFINITY;
+        w[u] = li == -INFINITY ? 0.f : exp2f(li - M);  // empty partial: weight 0
+#pragma unroll
+        for (int k = 0; k < kPerLane; ++k)
+          v[u][k] = in ? o[(long long)i * D + lane + 32 * k] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        wsum += w[u];
+#pragma unroll
+        for (int k = 0; k < kPerLane; ++k) acc[k] = fmaf(w[u], v[u][k], acc[k]);
+      }
     }
   }
-  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-  float *out = p.out + ((long long)row * p.n_q_heads + h) * D;
 #pragma unroll
-  for (int k = 0; k < kPerLane; ++k) out[lane + 32 * k] = acc[k] * inv;
-  if (p.lse_out && lane == 0)
+  for (int k = 0; k < kPerLane; ++k) s_acc[warp][lane + 32 * k] = acc[k];
+  if (lane == 0) s_w[warp] = wsum;
+  __syncthreads();
+  const float wt = s_w[0] + s_w[1] + s_w[2] + s_w[3];
+  const float inv = wt > 0.f ? 1.f / wt : 0.f;
+  float *out = p.out + ((long long)row * p.n_q_heads + h) * D;
+  for (int d = tid; d < D; d += 128)
+    out[d] = (s_acc[0][d] + s_acc[1][d] + s_acc[2][d] + s_acc[3][d]) * inv;
+  if (p.lse_out && tid == 0)
     p.lse_out[(long long)row * p.n_q_heads + h] =
-        wsum > 0.f ? (M + log2f(wsum)) * 0.69314718055994530942f : -INFINITY;
+        wt > 0.f ? (M + log2f(wt)) * 0.69314718055994530942f : -INFINITY;
 }
 
 template <int DT, int D>
 int launch_cc(const LseKernelParams &p, int gx, int gy, int gz, int smem, cudaStream_t st) {
   auto k = partial_cuda_core_kernel<DT, D>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return (int)e;
+  static int set_for = -1;
+  if (smem > set_for) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return (int)e;
+    set_for = smem;
+  }
   k<<<dim3(gx, gy, gz), kThreads, smem, st>>>(p);
   return (int)cudaGetLastError();
 }
@@ -492,16 +529,32 @@ int lse_launch_partial_cuda_core(const LseKernelParams &p, int dtype, int head_d
   return (int)cudaErrorInvalidValue;
 }
 
+// The merge is launched as a programmatic dependent of the partial pass on
+// the same stream: its CTAs may be scheduled while the partial pass drains
+// and wait in griddepcontrol.wait until the partial results are visible.
+template <int D>
+int launch_merge_d(const LseKernelParams &p, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.n_q_heads, p.max_rows, p.n_seqs);
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return (int)cudaLaunchKernelEx(&cfg, merge_kernel<D>, p);
+}
+
 int lse_launch_merge(const LseKernelParams &p, int head_dim, void *stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  dim3 grid((p.n_q_heads + 3) / 4, p.max_rows, p.n_seqs);
   switch (head_dim) {
-    case 64: merge_kernel<64><<<grid, 128, 0, st>>>(p); break;
-    case 128: merge_kernel<128><<<grid, 128, 0, st>>>(p); break;
-    case 256: merge_kernel<256><<<grid, 128, 0, st>>>(p); break;
-    default: return (int)cudaErrorInvalidValue;
+    case 64: return launch_merge_d<64>(p, st);
+    case 128: return launch_merge_d<128>(p, st);
+    case 256: return launch_merge_d<256>(p, st);
   }
-  return (int)cudaGetLastError();
+  return (int)cudaErrorInvalidValue;
 }
 
 const char *lse_cuda_error_string(int code) { return cudaGetErrorString((cudaError_t)code); }

@@ -26,15 +26,23 @@
 //    holds the value rounded to the storage's 16-bit format, the other the
 //    rounding error) so the products keep ~16 mantissa bits and only the
 //    K/V storage rounding remains.
-//  * Softmax: one thread per key reads its row of S from TMEM.  The running
-//    maximum is rescaled lazily: only when a score exceeds it by more than
-//    2^8 are the maxima recomputed and the TMEM output rescaled.
+//  * Softmax: two warpgroups take alternate tiles (ping-pong), each with
+//    its own score buffer in TMEM, its own P tile in shared memory and its
+//    own output accumulator, so one group's exponentials overlap the other
+//    group's tensor-core work; each group writes its own partial result per
+//    piece (the merge combines them like any other partials).  One thread
+//    per key reads its row of S from TMEM.  The running maximum is rescaled
+//    lazily: only when a score exceeds it by more than 2^8 are the maxima
+//    recomputed and the group's TMEM output rescaled.
+//  * K and V sit in separate rings, so a K slot is refilled as soon as its
+//    score product is done, and the score products run two tiles ahead of
+//    the output products.
 //
-// Roles (256 threads): warp 0 TMA producer, warp 1 MMA issuer (and TMEM
-// owner), warps 2-3 stage Q, warps 4-7 softmax and epilogue.  Every wait is
-// bounded: a wait that runs out sets LSE_DEVERR_TIMEOUT and every role
-// leaves its loop; TMEM is released and outstanding copies are drained
-// before the CTA exits.
+// Roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer (and TMEM
+// owner), warps 2-3 stage Q, warps 4-7 and 8-11 the two softmax groups.
+// Every wait is bounded: a wait that runs out sets LSE_DEVERR_TIMEOUT and
+// every role leaves its loop; TMEM is released and outstanding copies are
+// drained before the CTA exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -42,6 +50,7 @@
 #include <cudaTypedefs.h>
 
 #include <cstdint>
+#include <cfloat>
 #include <cstring>
 #include <mutex>
 
@@ -51,11 +60,10 @@ namespace {
 
 constexpr int kTK = 128;           // keys per tile = M of the score product
 constexpr int kD = 128;            // head dim = M of the output product
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr float kTau = 8.f;        // lazy-rescale threshold (log2 units)
 constexpr long long kWaitCycles = 4000000000ll;  // ~2 s at 2 GHz
 constexpr int kRegionBytes = kTK * 128;          // 128 rows x 128 B (64 dims)
-constexpr int kStageBytes = 4 * kRegionBytes;    // K (2 regions) + V (2 regions)
 
 struct __align__(64) TcParams {
   CUtensorMap maps[LSE_MAX_TMA_CHUNKS];
@@ -87,6 +95,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Non-blocking test of a phase.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
@@ -186,24 +207,6 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
       : "memory");
 }
 
-// 8 consecutive TMEM columns of this thread's lane; the wait is tied to the
-// destination registers so no use can be hoisted above it.
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float *v) {
-  uint32_t r[8];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7])
-      : "r"(taddr)
-      : "memory");
-  asm volatile("tcgen05.wait::ld.sync.aligned;"
-               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
-                 "+r"(r[6]), "+r"(r[7])
-               :
-               : "memory");
-#pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
-}
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const float *v) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
@@ -242,16 +245,6 @@ struct Op16<LSE_KV_F16> {
   }
 };
 
-__device__ __forceinline__ float warp_max(float x) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-  return x;
-}
-__device__ __forceinline__ float warp_sum(float x) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-  return x;
-}
 
 // ---- work decomposition ---------------------------------------------------------
 
@@ -275,7 +268,7 @@ struct TileIter {
   long long seg_first;       // global index of the segment's first tile
   long long t, t_end;        // current / end global tile
 
-  __device__ void next_seq(const LseKernelParams &p) {
+  __device__ __noinline__ void next_seq(const LseKernelParams &p) {
     // advance to the next sequence with tiles, starting at s
     while (s < p.n_seqs) {
       const int n = seq_tiles(p, s, L, row0, R);
@@ -286,7 +279,8 @@ struct TileIter {
       ++s;
     }
   }
-  __device__ void init(const LseKernelParams &p, long long t_begin, long long t_stop) {
+  __device__ __noinline__ void init(const LseKernelParams &p, long long t_begin,
+                                    long long t_stop) {
     t = t_begin;
     t_end = t_stop;
     s = 0;
@@ -326,44 +320,224 @@ __device__ __forceinline__ int cta_of_tile(long long t, long long U, int C) {
   return int(((t + 1) * (long long)C - 1) / U);
 }
 
-// ---- shared-memory layout --------------------------------------------------------
+
+// Fragment ids of the boxes of one tile (-1: past the sequence, -2: names
+// no fragment, flagged).
+__device__ __noinline__ void load_page_ids(const LseKernelParams &p, const TileIter &it, int nbox,
+                                           int box_t, int *pk, int *pv) {
+  const int key0 = it.tile * kTK;
+  const int T = p.tokens_per_fragment;
+#pragma unroll 1
+  for (int b = 0; b < nbox; ++b) {
+    const int kb = key0 + b * box_t;
+    int fk = -1, fv = -1;
+    if (kb < it.L) {
+      const long long e = (long long)it.s * p.max_pages + kb / T;
+      fk = p.k_pages[e];
+      fv = p.v_pages[e];
+      const bool bk = fk < 0 || fk >= p.n_fragments, bv = fv < 0 || fv >= p.n_fragments;
+      if (bk || bv) atomicOr(p.err, LSE_DEVERR_BAD_FRAGMENT);
+      if (bk) fk = -2;
+      if (bv) fv = -2;
+    }
+    pk[b] = fk;
+    pv[b] = fv;
+  }
+}
+
+// TMA boxes of one tile (K or V): fragment ids ids[0..nbox), into dst.
+__device__ __noinline__ void load_boxes(const TcParams &tp, int nbox, int box_t, int g, int key0,
+                                        const int *ids, uint32_t dst, uint32_t full_bar) {
+  const LseKernelParams &p = tp.p;
+  const int T = p.tokens_per_fragment;
+#pragma unroll 1
+  for (int b = 0; b < nbox; ++b) {
+    const int f = ids[b];
+    if (f < 0) continue;
+    const int kb = key0 + b * box_t;
+    const int c = f / p.frags_per_chunk;
+    const int z = (f - c * p.frags_per_chunk) * T + kb % T;
+    const uint32_t d = dst + b * box_t * 128;
+    tma_load_3d(d, &tp.maps[c], full_bar, 0, g * 2, z);
+    tma_load_3d(d + kRegionBytes, &tp.maps[c], full_bar, 0, g * 2 + 1, z);
+  }
+}
+
+// Producer work for tile n: K slot, tile record, K boxes, V slot, V boxes.
+// Returns 0 when a wait gave up.
+__device__ __noinline__ int produce_tile(const TcParams &tp, int n, int NS, int nbox, int box_t,
+                                         int g, int tile, int L, const int *pk, const int *pv,
+                                         uint32_t kdst, uint32_t vdst, const uint32_t *bars_k,
+                                         const uint32_t *bars_v, uint32_t info_bar,
+                                         uint4 *info, volatile int *abort_flag) {
+  const LseKernelParams &p = tp.p;
+  const uint32_t ph = ((n / NS) & 1) ^ 1;
+  const int key0 = tile * kTK;
+  uint32_t kmask = 0, vmask = 0;
+#pragma unroll 1
+  for (int b = 0; b < nbox; ++b) {
+    if (pk[b] >= 0) kmask |= 1u << b;
+    if (pv[b] >= 0) vmask |= 1u << b;
+  }
+  const int live = L - key0 < kTK ? L - key0 : kTK;
+  const uint32_t box_bytes = 2u * (uint32_t)box_t * 128u;
+  if (!mbar_wait(bars_k[0], ph, abort_flag, p.err)) return 0;
+  // the record slot was last read by the softmax of tile n - 8, which has
+  // finished: this producer passed its K slot wait for tile n, which
+  // follows the output product of tile n + 6 - NS >= n - 6
+  *info = make_uint4(kmask, vmask, (uint32_t)live, 0u);
+  mbar_arrive(info_bar);  // publishes the record
+  mbar_expect_tx(bars_k[1], (uint32_t)__popc(kmask) * box_bytes);
+  load_boxes(tp, nbox, box_t, g, key0, pk, kdst, bars_k[1]);
+  if (!mbar_wait(bars_v[0], ph, abort_flag, p.err)) return 0;
+  mbar_expect_tx(bars_v[1], (uint32_t)__popc(vmask) * box_bytes);
+  load_boxes(tp, nbox, box_t, g, key0, pv, vdst, bars_v[1]);
+  return 1;
+}
+
+
+// Column reduction of a [128 keys][P8 pairs] FP32 tile in shared memory by
+// the 128 threads of a softmax group: out[q] = max (or sum) over keys of
+// tile[key][q].  Each pair gets kSplit = max(2, 128 / P8) threads, each
+// folding a contiguous share of the keys; the shares are combined through
+// out[64 ...] (out holds 4 x 64 floats).
+template <int P8, bool kSum>
+__device__ __forceinline__ void column_reduce(const float *tile, int t, float *out, int bar_id) {
+  constexpr int kSplit = 128 / P8 >= 2 ? 128 / P8 : 2;
+  constexpr int kRows = (128 + kSplit - 1) / kSplit;
+  static_assert(kSplit * P8 <= 192, "shares must fit out[64 .. 256)");
+  const int q = t % P8, part = t / P8;
+  float a = kSum ? 0.f : -INFINITY;
+  if (part < kSplit) {
+#pragma unroll 8
+    for (int k = 0; k < kRows; ++k) {
+      const int row = part * kRows + k;
+      if (row < 128) {
+        const float v = tile[row * P8 + q];
+        a = kSum ? a + v : fmaxf(a, v);
+      }
+    }
+  }
+  float *shares = out + 64;
+  if (part < kSplit) shares[part * P8 + q] = a;
+  named_sync(bar_id, 128);
+  if (t < P8) {
+    float r = kSum ? 0.f : -INFINITY;
+#pragma unroll 1
+    for (int k = 0; k < kSplit; ++k)
+      r = kSum ? r + shares[k * P8 + t] : fmaxf(r, shares[k * P8 + t]);
+    out[t] = r;
+  }
+}
+
+// ---- shared-memory and TMEM layout ------------------------------------------------
 
 template <int P8>
 struct TcLayout {
-  static constexpr int kN = 2 * P8;                  // hi + lo columns
-  static constexpr int kQRegion = kN * 128;          // one 64-dim region of Q rows
-  static constexpr int kQBytes = 2 * kQRegion;
-  static constexpr int kPLbo = (kN / 8) * 128;       // P: stride between 8-key groups
-  static constexpr int kPBytes = kTK * kN * 2;
-  static constexpr int kTmemCols = (3 * kN <= 64) ? 64 : (3 * kN <= 128) ? 128
-                                 : (3 * kN <= 256) ? 256 : 512;
-  // misc block
-  static constexpr int kBars = 24;
-  static constexpr int kMiscBytes = kBars * 8 + 16 + 64 * 4 * 2 + 4 * 64 * 4 + 64 * 8 + 64 * 4;
+  static constexpr int kNQ = (P8 + 15) / 16 * 16;       // score columns (N of S^T)
+  static constexpr int kN = 2 * P8;                      // output columns: hi | lo pairs
+  static constexpr int kQSlots = P8 >= 48 ? 1 : 2;       // Q ring depth
+  static constexpr int kQRegion = kNQ * 128;             // 64 dims of kNQ rows
+  static constexpr int kQBytes = 4 * kQRegion;           // hi (2 regions) + lo (2 regions)
+  static constexpr int kPLbo = (kN / 8) * 128;           // P: stride of 8-key groups
+  static constexpr int kPBytes = kTK * kN * 2;           // one warpgroup's P tile
+  static constexpr int kOnesBytes = 4096;                // ones operand: 128 rows x 16
+  // TMEM: S per group, then per group and output slot the output O^T and the
+  // row sums L (both kN columns); two output slots when they fit
+  static constexpr int kOSlots = (2 * kNQ + 8 * kN <= 512) ? 2 : 1;
+  static constexpr int kTmemNeed = 2 * kNQ + 4 * kOSlots * kN;
+  static constexpr int kTmemCols = kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
+                                 : kTmemNeed <= 256 ? 256 : 512;
+  static constexpr int kBars = 48;
+  static constexpr int kMiscBytes = kBars * 8 + 16 + 2 * 64 * 4 * 2 + 2 * 4 * 64 * 4 +
+                                    2 * 64 * 8 + 64 * 4 + 8 * 16 + 2 * 32 * 16 * 4;
+  static constexpr int kHalfStage = 2 * kRegionBytes;    // one K or V tile
   static int smem_bytes(int stages) {
-    return 1024 + stages * kStageBytes + 2 * kQBytes + kPBytes + kMiscBytes;
+    return 1024 + stages * 2 * kHalfStage + kQSlots * kQBytes + 2 * kPBytes + kOnesBytes +
+           kMiscBytes;
   }
 };
 
 // barrier indices in the misc block
 enum {
-  kBarFull = 0,    // [4]
-  kBarEmpty = 4,   // [4]
-  kBarSFull = 8,
-  kBarPFull = 9,
-  kBarQFull = 10,  // [2]
-  kBarQEmpty = 12, // [2]
-  kBarOFull = 14,  // [2]
-  kBarOEmpty = 16, // [2]
-  kBarDone = 18,
+  kBarFullK = 0,    // [4]
+  kBarEmptyK = 4,   // [4]
+  kBarFullV = 8,    // [4]
+  kBarEmptyV = 12,  // [4]
+  kBarSFull = 16,   // [2] per softmax group
+  kBarPFull = 18,   // [2]
+  kBarQFull = 20,   // [2]
+  kBarQEmpty = 22,  // [2]
+  kBarOFull = 24,   // [4] = group * 2 + slot
+  kBarOEmpty = 28,  // [4]
+  kBarDone = 32,
+  kBarInfo = 33,    // [8] one per tile record
 };
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Two FP32 values -> packed hi (nearest 16-bit) and lo (its rounding error).
+template <int DT>
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t &hi, uint32_t &lo);
+template <>
+__device__ __forceinline__ void split2<LSE_KV_BF16>(float x0, float x1, uint32_t &hi,
+                                                    uint32_t &lo) {
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(hi) : "f"(x1), "f"(x0));
+  const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xffff0000u);
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(lo) : "f"(x1 - h1), "f"(x0 - h0));
+}
+template <>
+__device__ __forceinline__ void split2<LSE_KV_F16>(float x0, float x1, uint32_t &hi,
+                                                   uint32_t &lo) {
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(hi) : "f"(x1), "f"(x0));
+  const float2 h = __half22float2(*reinterpret_cast<const __half2 *>(&hi));
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(lo) : "f"(x1 - h.y), "f"(x0 - h.x));
+}
+
+// TMEM: this thread's lane, N consecutive 32-bit columns (N a multiple of 8),
+// one wait for all of them.
+template <int N>
+__device__ __forceinline__ void tmem_load(uint32_t taddr, float *v) {
+  static_assert(N % 8 == 0, "columns in groups of 8");
+  uint32_t r[N];
+#pragma unroll
+  for (int c = 0; c < N; c += 8)
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+        : "=r"(r[c]), "=r"(r[c + 1]), "=r"(r[c + 2]), "=r"(r[c + 3]), "=r"(r[c + 4]),
+          "=r"(r[c + 5]), "=r"(r[c + 6]), "=r"(r[c + 7])
+        : "r"(taddr + c)
+        : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  // tie every register to the wait so no use is scheduled above it
+#pragma unroll
+  for (int c = 0; c < N; ++c) {
+    asm volatile("" : "+r"(r[c]) :: "memory");
+    v[c] = __uint_as_float(r[c]);
+  }
+}
 
 template <int DT, int P8>
 __global__ void __launch_bounds__(kThreads, 1)
     partial_tcgen05_kernel(const __grid_constant__ TcParams tp) {
   using Lay = TcLayout<P8>;
-  using Op = Op16<DT>;
+  constexpr int kNQ = Lay::kNQ;
   constexpr int kN = Lay::kN;
+  constexpr int kQS = Lay::kQSlots;
   const LseKernelParams &p = tp.p;
   const int NS = tp.stages;
   const int cta = blockIdx.x;
@@ -373,21 +547,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t *smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t stage_base = sbase;
-  const uint32_t q_base = sbase + NS * kStageBytes;
-  const uint32_t p_base = q_base + 2 * Lay::kQBytes;
-  uint8_t *misc = smem + NS * kStageBytes + 2 * Lay::kQBytes + Lay::kPBytes;
+  const uint32_t k_base = sbase;                                // K ring
+  const uint32_t v_base = k_base + NS * Lay::kHalfStage;        // V ring
+  const uint32_t q_base = v_base + NS * Lay::kHalfStage;        // Q slots
+  const uint32_t p_base = q_base + kQS * Lay::kQBytes;          // P tiles (one per group)
+  const uint32_t ones_base = p_base + 2 * Lay::kPBytes;         // ones operand of the sums
+  uint8_t *misc = smem + (ones_base - sbase) + Lay::kOnesBytes;
   uint64_t *bars = reinterpret_cast<uint64_t *>(misc);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + Lay::kBars * 8);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + Lay::kBars * 8 + 4);
   long long *shared_u = reinterpret_cast<long long *>(misc + Lay::kBars * 8 + 8);
-  float *m_run = reinterpret_cast<float *>(misc + Lay::kBars * 8 + 16);  // [64]
-  float *alpha = m_run + 64;                                             // [64]
-  float *red = alpha + 64;                                               // [4][64]
-  unsigned long long *masks = reinterpret_cast<unsigned long long *>(red + 4 * 64);  // [64]
-  int *pair_row = reinterpret_cast<int *>(masks + 64);                   // [64]
+  float *m_run_all = reinterpret_cast<float *>(misc + Lay::kBars * 8 + 16);  // [2][64]
+  float *alpha_all = m_run_all + 2 * 64;                                     // [2][64]
+  float *red_all = alpha_all + 2 * 64;                                       // [2][4][64]
+  unsigned long long *masks_all =
+      reinterpret_cast<unsigned long long *>(red_all + 2 * 4 * 64);          // [2][64]
+  int *pair_row = reinterpret_cast<int *>(masks_all + 2 * 64);               // [64]
+  // ring of 8 per-tile records written by the producer before its arrival on
+  // the tile's K barrier: {K box mask, V box mask, keys of the tile below L}
+  uint4 *tile_info = reinterpret_cast<uint4 *>(pair_row + 64);               // [8]
+  // fragment ids of a batch of 32 tiles (up to 16 boxes each), K then V
+  int *page_buf = reinterpret_cast<int *>(tile_info + 8);                    // [2][32][16]
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
+  // the merge pass may be scheduled now; it waits for this grid to finish
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // ---- prologue: total live tiles, barriers, TMEM -------------------------------
   if (tid == 0) {
     long long U = 0;
@@ -402,21 +586,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     *shared_u = U * p.n_kv_heads;
     *abort_flag = 0;
     for (int i = 0; i < 4; ++i) {
-      mbar_init(bar(kBarFull + i), 1);
-      mbar_init(bar(kBarEmpty + i), 1);
-    }
-    mbar_init(bar(kBarSFull), 1);
-    mbar_init(bar(kBarPFull), 128);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(kBarQFull + i), 64);
-      mbar_init(bar(kBarQEmpty + i), 1);
+      mbar_init(bar(kBarFullK + i), 1);
+      mbar_init(bar(kBarEmptyK + i), 1);
+      mbar_init(bar(kBarFullV + i), 1);
+      mbar_init(bar(kBarEmptyV + i), 1);
       mbar_init(bar(kBarOFull + i), 1);
       mbar_init(bar(kBarOEmpty + i), 128);
     }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(kBarSFull + i), 1);
+      mbar_init(bar(kBarPFull + i), 128);
+      mbar_init(bar(kBarQFull + i), 64);
+      mbar_init(bar(kBarQEmpty + i), 1);
+    }
     mbar_init(bar(kBarDone), 1);
+    for (int i = 0; i < 8; ++i) mbar_init(bar(kBarInfo + i), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (tid < 64) pair_row[tid] = tid / p.group;
+  {
+    // the ones operand (16-bit 1.0 in the storage's operand format)
+    const uint32_t one2 = Op16<DT>::kFmt == 1 ? 0x3F803F80u : 0x3C003C00u;
+    uint4 *ones = reinterpret_cast<uint4 *>(smem + (ones_base - sbase));
+    for (int i = tid; i < Lay::kOnesBytes / 16; i += kThreads)
+      ones[i] = make_uint4(one2, one2, one2, one2);
+    fence_proxy_async();
+  }
   __syncthreads();
   const long long U = *shared_u;
   // working CTAs: never more than tiles, so no working range is empty and a
@@ -436,113 +631,177 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_s = tmem;                 // S^T: lanes = keys, cols [0, N)
-  auto tmem_o = [&](int slot) { return tmem + (uint32_t)(kN * (1 + slot)); };
+  auto tmem_s = [&](int grp) { return tmem + (uint32_t)(grp * kNQ); };
+  constexpr int kOS = Lay::kOSlots;
+  auto tmem_o = [&](int grp, int slot) {
+    return tmem + (uint32_t)(2 * kNQ + (2 * (grp * kOS + slot)) * kN);
+  };
+  auto tmem_l = [&](int grp, int slot) { return tmem_o(grp, slot) + (uint32_t)kN; };
 
-  const int T = p.tokens_per_fragment;
   const int box_t = tp.box_tokens;
+  const int nbox = box_t >= kTK ? 1 : kTK / box_t;
+  const uint32_t full_boxes = nbox >= 32 ? 0xffffffffu : ((1u << nbox) - 1u);
   const int G = p.group;
 
   if (warp == 0) {
     // ============================ TMA producer ============================
-    if (lane == 0) {
-      TileIter it;
-      it.init(p, t_begin, t_stop);
-      int n = 0;
-      for (; it.valid(); it.advance(p), ++n) {
-        const int st = n % NS;
-        if (!mbar_wait(bar(kBarEmpty + st), ((n / NS) & 1) ^ 1, abort_flag, p.err)) break;
-        const int key0 = it.tile * kTK;
-        const int nbox = box_t >= kTK ? 1 : kTK / box_t;
-        // which boxes exist (live and naming a fragment), K and V separately
-        uint32_t kmask = 0, vmask = 0;
-        for (int b = 0; b < nbox; ++b) {
-          const int kb = key0 + b * box_t;
-          if (kb >= it.L) break;
-          const long long e = (long long)it.s * p.max_pages + kb / T;
-          const int fk = p.k_pages[e], fv = p.v_pages[e];
-          if (fk >= 0 && fk < p.n_fragments) kmask |= 1u << b;
-          else atomicOr(p.err, LSE_DEVERR_BAD_FRAGMENT);
-          if (fv >= 0 && fv < p.n_fragments) vmask |= 1u << b;
-          else atomicOr(p.err, LSE_DEVERR_BAD_FRAGMENT);
+    // The warp reads the fragment ids of 32 tiles at once (one lane per
+    // tile), then lane 0 streams the tiles: K then V of each, each into its
+    // ring.
+    const int n_total = (int)(t_stop - t_begin);
+    int *pk = page_buf, *pv = page_buf + 32 * 16;
+    int n = 0;
+    bool ok = true;
+#pragma unroll 1
+    for (int b0 = 0; b0 < n_total && ok; b0 += 32) {
+      const int cnt = n_total - b0 < 32 ? n_total - b0 : 32;
+      TileIter mine;
+      mine.init(p, t_begin + b0 + (lane < cnt ? lane : 0), t_stop);
+      if (lane < cnt) load_page_ids(p, mine, nbox, box_t, pk + lane * 16, pv + lane * 16);
+      __syncwarp();
+#pragma unroll 1
+      for (int i = 0; i < cnt; ++i, ++n) {
+        const int tg = __shfl_sync(0xffffffffu, mine.g, i);
+        const int tt = __shfl_sync(0xffffffffu, mine.tile, i);
+        const int tl = __shfl_sync(0xffffffffu, mine.L, i);
+        int go = 1;
+        if (lane == 0) {
+          const uint32_t bars_k[2] = {bar(kBarEmptyK + n % NS), bar(kBarFullK + n % NS)};
+          const uint32_t bars_v[2] = {bar(kBarEmptyV + n % NS), bar(kBarFullV + n % NS)};
+          go = produce_tile(tp, n, NS, nbox, box_t, tg, tt, tl, pk + i * 16, pv + i * 16,
+                            k_base + (n % NS) * Lay::kHalfStage,
+                            v_base + (n % NS) * Lay::kHalfStage, bars_k, bars_v,
+                            bar(kBarInfo + (n & 7)), tile_info + (n & 7), abort_flag);
         }
-        const uint32_t bytes =
-            (uint32_t)(__popc(kmask) + __popc(vmask)) * 2u * (uint32_t)box_t * 128u;
-        const uint32_t fb = bar(kBarFull + st);
-        mbar_expect_tx(fb, bytes);
-        const uint32_t kdst = stage_base + st * kStageBytes;
-        const uint32_t vdst = kdst + 2 * kRegionBytes;
-        for (int b = 0; b < nbox; ++b) {
-          const int kb = key0 + b * box_t;
-          const long long e = (long long)it.s * p.max_pages + kb / T;
-          const int off = kb % T;
-          if (kmask >> b & 1u) {
-            const int f = p.k_pages[e];
-            const int c = f / p.frags_per_chunk;
-            const int z = (f - c * p.frags_per_chunk) * T + off;
-            for (int h = 0; h < 2; ++h)
-              tma_load_3d(kdst + h * kRegionBytes + b * box_t * 128, &tp.maps[c], fb, 0,
-                          it.g * 2 + h, z);
-          }
-          if (vmask >> b & 1u) {
-            const int f = p.v_pages[e];
-            const int c = f / p.frags_per_chunk;
-            const int z = (f - c * p.frags_per_chunk) * T + off;
-            for (int h = 0; h < 2; ++h)
-              tma_load_3d(vdst + h * kRegionBytes + b * box_t * 128, &tp.maps[c], fb, 0,
-                          it.g * 2 + h, z);
-          }
+        go = __shfl_sync(0xffffffffu, go, 0);
+        if (!go) {
+          ok = false;
+          break;
         }
       }
-      // drain: every stage issued must have landed before the CTA exits
-      for (int k = (n > NS ? n - NS : 0); k < n; ++k) mbar_drain(bar(kBarFull + k % NS), (k / NS) & 1);
+      __syncwarp();
     }
+    // drain: every copy issued must have landed before the CTA exits
+    if (lane == 0)
+#pragma unroll 1
+      for (int k = (n > NS ? n - NS : 0); k < n; ++k) {
+        mbar_drain(bar(kBarFullK + k % NS), (k / NS) & 1);
+        mbar_drain(bar(kBarFullV + k % NS), (k / NS) & 1);
+      }
   } else if (warp == 1) {
     // ============================ MMA issuer ==============================
+    // An event loop: the score product of tile n runs up to two tiles ahead
+    // of the output products, and whichever is ready is issued first.
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = instr_desc(Op::kFmt, 0, 0, kTK, kN);
-      constexpr uint32_t idesc_pv = instr_desc(Op::kFmt, 1, 1, kD, kN);
-      TileIter it;
-      it.init(p, t_begin, t_stop);
-      int n = 0, seg = -1;
-      for (; it.valid(); it.advance(p), ++n) {
-        const bool first = it.seg_start(t_begin), last = it.seg_end();
-        if (first) {
-          ++seg;
-          if (!mbar_wait(bar(kBarQFull + (seg & 1)), (seg >> 1) & 1, abort_flag, p.err)) break;
-          if (!mbar_wait(bar(kBarOEmpty + (seg & 1)), ((seg >> 1) & 1) ^ 1, abort_flag, p.err))
+      constexpr uint32_t fmt = Op16<DT>::kFmt;
+      constexpr uint32_t idesc_qk = instr_desc(fmt, 0, 0, kTK, kNQ);
+      constexpr uint32_t idesc_pv = instr_desc(fmt, 1, 1, kD, kN);
+      constexpr uint32_t idesc_l = instr_desc(fmt, 0, 1, kD, kN);
+      const int n_total = (int)(t_stop - t_begin);
+      TileIter iq, iv;
+      iq.init(p, t_begin, t_stop);
+      iv.init(p, t_begin, t_stop);
+      int nq = 0, seg_q = -1;   // score side: tiles issued, segment count
+      int nv = 0, seg_v = -1;   // output side
+      bool grp_started[2] = {false, false};
+      long long t_idle = clock64();
+      int idle = 0;
+      while (nv < n_total) {
+        bool did = false;
+        if (nq < n_total && nq < nv + 2) {
+          const bool first = iq.seg_start(t_begin);
+          const int sq = first ? seg_q + 1 : seg_q;
+          const int st = nq % NS;
+          if ((!first || mbar_test(bar(kBarQFull + sq % kQS), (sq / kQS) & 1)) &&
+              mbar_test(bar(kBarFullK + st), (nq / NS) & 1)) {
+            seg_q = sq;
+            tc_fence_after();
+            const bool last = iq.seg_end();
+            const uint32_t kaddr = k_base + st * Lay::kHalfStage;
+            const uint32_t qaddr = q_base + (seg_q % kQS) * Lay::kQBytes;
+            const uint32_t d = tmem_s(nq & 1);
+#pragma unroll
+            for (int k = 0; k < kD / 16; ++k) {
+              const uint64_t a = smem_desc(kaddr + (k >> 2) * kRegionBytes + (k & 3) * 32, 16,
+                                           1024, kLayoutSw128);
+              const uint32_t qoff = (k >> 2) * Lay::kQRegion + (k & 3) * 32;
+              const uint64_t bh = smem_desc(qaddr + qoff, 16, 1024, kLayoutSw128);
+              const uint64_t bl =
+                  smem_desc(qaddr + 2 * Lay::kQRegion + qoff, 16, 1024, kLayoutSw128);
+              mma_f16(d, a, bh, idesc_qk, k > 0);   // K Q_hi^T
+              mma_f16(d, a, bl, idesc_qk, 1u);      // + K Q_lo^T, same columns
+            }
+            mma_commit(bar(kBarEmptyK + st));
+            mma_commit(bar(kBarSFull + (nq & 1)));
+            if (last) mma_commit(bar(kBarQEmpty + seg_q % kQS));
+            iq.advance(p);
+            ++nq;
+            did = true;
+          }
+        }
+        if (nv < nq) {
+          const bool first = iv.seg_start(t_begin), last = iv.seg_end();
+          const int sv = first ? seg_v + 1 : seg_v;
+          const int grp = nv & 1, slot = sv % kOS;
+          const bool started = first ? false : grp_started[grp];
+          const bool other = first ? false : grp_started[grp ^ 1];
+          const uint32_t oe_par = ((sv / kOS) & 1) ^ 1;
+          const int st = nv % NS;
+          bool ready = mbar_test(bar(kBarPFull + grp), (nv >> 1) & 1) &&
+                       mbar_test(bar(kBarFullV + st), (nv / NS) & 1);
+          // a group's output slot must have been read out two segments ago
+          if (ready && !started) ready = mbar_test(bar(kBarOEmpty + 2 * grp + slot), oe_par);
+          if (ready && last && !other)
+            ready = mbar_test(bar(kBarOEmpty + 2 * (grp ^ 1) + slot), oe_par);
+          if (ready) {
+            if (first) {
+              seg_v = sv;
+              grp_started[0] = grp_started[1] = false;
+            }
+            tc_fence_after();
+            const uint32_t vaddr = v_base + st * Lay::kHalfStage;
+            const uint32_t paddr = p_base + grp * Lay::kPBytes;
+            const uint32_t d = tmem_o(grp, slot);
+            const uint32_t dl = tmem_l(grp, slot);
+            // the ones operand is K-major without swizzle: 8x16-byte core
+            // matrices, K blocks 128 B apart, row blocks 256 B apart
+            const uint64_t a1 = smem_desc(ones_base, 128, 256, kLayoutNone);
+#pragma unroll
+            for (int k = 0; k < kTK / 16; ++k) {
+              const uint64_t a = smem_desc(vaddr + k * 2048, kRegionBytes, 1024, kLayoutSw128);
+              const uint64_t b =
+                  smem_desc(paddr + k * 2 * Lay::kPLbo, Lay::kPLbo, 128, kLayoutNone);
+              const uint32_t acc = (grp_started[grp] || k > 0) ? 1u : 0u;
+              mma_f16(d, a, b, idesc_pv, acc);     // O^T += V^T P^T
+              mma_f16(dl, a1, b, idesc_l, acc);    // L += 1 P^T (row sums of P)
+            }
+            grp_started[grp] = true;
+            mma_commit(bar(kBarEmptyV + st));
+            // this group's last tile of the piece: the tile is the piece's
+            // last, or the next one (the other group's) is
+            const bool next_is_last =
+                !last && (iv.t + 1 == iv.t_end - 1 || iv.tile + 1 == iv.n_tiles - 1);
+            if (last || next_is_last) mma_commit(bar(kBarOFull + 2 * grp + slot));
+            // the other group had no tile in this piece: release its (empty)
+            // output slot all the same (its previous use was read out)
+            if (last && !grp_started[grp ^ 1]) mma_commit(bar(kBarOFull + 2 * (grp ^ 1) + slot));
+            iv.advance(p);
+            ++nv;
+            did = true;
+          }
+        }
+        if (did) {
+          idle = 0;
+          t_idle = clock64();
+        } else if (++idle >= 64) {
+          idle = 0;
+          if (*abort_flag) break;
+          if (clock64() - t_idle > kWaitCycles) {
+            *abort_flag = 1;
+            atomicOr(p.err, LSE_DEVERR_TIMEOUT);
             break;
+          }
         }
-        const int st = n % NS;
-        if (!mbar_wait(bar(kBarFull + st), (n / NS) & 1, abort_flag, p.err)) break;
-        tc_fence_after();
-        const uint32_t kaddr = stage_base + st * kStageBytes;
-        const uint32_t vaddr = kaddr + 2 * kRegionBytes;
-        const uint32_t qaddr = q_base + (seg & 1) * Lay::kQBytes;
-        // S^T = K Q^T : 8 steps of 16 dims
-#pragma unroll
-        for (int k = 0; k < kD / 16; ++k) {
-          const uint64_t a = smem_desc(kaddr + (k >> 2) * kRegionBytes + (k & 3) * 32, 16, 1024,
-                                       kLayoutSw128);
-          const uint64_t b = smem_desc(qaddr + (k >> 2) * Lay::kQRegion + (k & 3) * 32, 16,
-                                       1024, kLayoutSw128);
-          mma_f16(tmem_s, a, b, idesc_qk, k > 0);
-        }
-        mma_commit(bar(kBarSFull));
-        if (last) mma_commit(bar(kBarQEmpty + (seg & 1)));
-        if (!mbar_wait(bar(kBarPFull), n & 1, abort_flag, p.err)) break;
-        tc_fence_after();
-        // O^T (+)= V^T P^T : 8 steps of 16 keys
-#pragma unroll
-        for (int k = 0; k < kTK / 16; ++k) {
-          const uint64_t a =
-              smem_desc(vaddr + k * 2048, kRegionBytes, 1024, kLayoutSw128);  // MN-major
-          const uint64_t b =
-              smem_desc(p_base + k * 2 * Lay::kPLbo, Lay::kPLbo, 128, kLayoutNone);  // MN-major
-          mma_f16(tmem_o(seg & 1), a, b, idesc_pv, (!first || k > 0) ? 1u : 0u);
-        }
-        mma_commit(bar(kBarEmpty + st));
-        if (last) mma_commit(bar(kBarOFull + (seg & 1)));
       }
       // every MMA issued has completed before TMEM is released
       mma_commit(bar(kBarDone));
@@ -557,212 +816,247 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (; it.valid(); it.advance(p)) {
       if (!it.seg_start(t_begin)) continue;
       ++seg;
-      const int slot = seg & 1;
-      if (!mbar_wait(bar(kBarQEmpty + slot), ((seg >> 1) & 1) ^ 1, abort_flag, p.err)) break;
-      uint8_t *qs = smem + (q_base - sbase) + slot * Lay::kQBytes;
+      const int slot = seg % kQS;
       const int P = G * it.R;
-      // row n < P8 holds hi of pair n, row P8 + n its lo; 16 chunks of 8 dims
-      for (int item = qt; item < P8 * 16; item += 64) {
+      // items (row n, 8-dim chunk c): every load of the segment in flight at
+      // once, issued before waiting for the slot
+      constexpr int kItems = kNQ * 16 / 64;
+      float4 ld[kItems][2];
+#pragma unroll
+      for (int k = 0; k < kItems; ++k) {
+        const int item = qt + 64 * k;
         const int n = item >> 4, c = item & 15;
-        float x[8];
         if (n < P) {
           const int r = n / G, h = it.g * G + (n - r * G);
           const float4 *src = reinterpret_cast<const float4 *>(
               p.q + ((long long)(it.row0 + r) * p.n_q_heads + h) * kD + c * 8);
-          const float4 a = __ldg(src), b2 = __ldg(src + 1);
-          x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-          x[4] = b2.x; x[5] = b2.y; x[6] = b2.z; x[7] = b2.w;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) x[i] *= p.scale_log2;
+          ld[k][0] = __ldg(src);
+          ld[k][1] = __ldg(src + 1);
         } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) x[i] = 0.f;
+          ld[k][0] = ld[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        uint16_t hi[8], lo[8];
+      }
+      if (!mbar_wait(bar(kBarQEmpty + slot), ((seg / kQS) & 1) ^ 1, abort_flag, p.err)) break;
+      uint8_t *qs = smem + (q_base - sbase) + slot * Lay::kQBytes;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) Op::split(x[i], hi[i], lo[i]);
-        const int region = c >> 3, cc = c & 7;
-        const uint32_t rh = n, rl = P8 + n;
-        const uint32_t ohi = region * Lay::kQRegion + (rh >> 3) * 1024 + (rh & 7) * 128 +
-                             ((cc ^ (rh & 7)) << 4);
-        const uint32_t olo = region * Lay::kQRegion + (rl >> 3) * 1024 + (rl & 7) * 128 +
-                             ((cc ^ (rl & 7)) << 4);
+      for (int k = 0; k < kItems; ++k) {
+        const int item = qt + 64 * k;
+        const int n = item >> 4, c = item & 15;
+        const float sc = p.scale_log2;
         uint4 vh, vl;
-        vh.x = hi[0] | (uint32_t)hi[1] << 16; vh.y = hi[2] | (uint32_t)hi[3] << 16;
-        vh.z = hi[4] | (uint32_t)hi[5] << 16; vh.w = hi[6] | (uint32_t)hi[7] << 16;
-        vl.x = lo[0] | (uint32_t)lo[1] << 16; vl.y = lo[2] | (uint32_t)lo[3] << 16;
-        vl.z = lo[4] | (uint32_t)lo[5] << 16; vl.w = lo[6] | (uint32_t)lo[7] << 16;
-        *reinterpret_cast<uint4 *>(qs + ohi) = vh;
-        *reinterpret_cast<uint4 *>(qs + olo) = vl;
+        split2<DT>(ld[k][0].x * sc, ld[k][0].y * sc, vh.x, vl.x);
+        split2<DT>(ld[k][0].z * sc, ld[k][0].w * sc, vh.y, vl.y);
+        split2<DT>(ld[k][1].x * sc, ld[k][1].y * sc, vh.z, vl.z);
+        split2<DT>(ld[k][1].z * sc, ld[k][1].w * sc, vh.w, vl.w);
+        const int region = c >> 3, cc = c & 7;
+        const uint32_t off = region * Lay::kQRegion + (n >> 3) * 1024 + (n & 7) * 128 +
+                             ((cc ^ (n & 7)) << 4);
+        *reinterpret_cast<uint4 *>(qs + off) = vh;
+        *reinterpret_cast<uint4 *>(qs + 2 * Lay::kQRegion + off) = vl;
       }
       fence_proxy_async();
       mbar_arrive(bar(kBarQFull + slot));
     }
   } else {
-    // ===================== softmax and epilogue (128 threads) =====================
-    const int j = tid - 128;          // key within tile = TMEM lane (scores)
-    const int quarter = warp - 4;     // TMEM lane quarter of this warp
+    // ============== softmax and epilogue: two groups of 128 threads ==============
+    // Scores are read from TMEM eight pairs at a time in loops whose code does
+    // not grow with the pair count; the row sums of P come from the tensor
+    // core (L = 1 P^T), so no per-pair state lives in registers.
+    const int grp = (warp - 4) >> 2;           // tiles of this parity
+    const int j = tid - 128 - grp * 128;       // key of the tile = TMEM lane (scores)
+    const int quarter = warp & 3;              // TMEM lane quarter of this warp
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const int bar_id = 1 + grp;
+    float *m_run = m_run_all + grp * 64;
+    float *alpha = alpha_all + grp * 64;
+    float *red = red_all + grp * 4 * 64;
+    unsigned long long *masks = masks_all + grp * 64;
+    float *scr = reinterpret_cast<float *>(smem + (p_base - sbase) + grp * Lay::kPBytes);
     TileIter it;
     it.init(p, t_begin, t_stop);
     int n = 0, seg = -1;
-    float l[P8];
-    bool ok = true;
+    bool had_tile = false, ok = true;
+#pragma unroll 1
     for (; it.valid() && ok; it.advance(p), ++n) {
       const bool first = it.seg_start(t_begin), last = it.seg_end();
       const int P = G * it.R;
       const int Cctx = it.L - it.R;
+      const int oslot = (seg + (first ? 1 : 0)) % kOS;
       if (first) {
         ++seg;
-        if (j < P8) m_run[j] = -INFINITY;
+        // a finite floor keeps exp2(-inf - m) at 0 (never NaN) for pairs
+        // with no visible key yet
+        if (j < P8) m_run[j] = -FLT_MAX;
         if (j < it.R)
           masks[j] = p.row_masks ? p.row_masks[it.row0 + j]
                                  : (j >= 63 ? ~0ull : ((1ull << (j + 1)) - 1ull));
-#pragma unroll
-        for (int q = 0; q < P8; ++q) l[q] = 0.f;
-        named_sync(1, 128);
+        had_tile = false;
+        named_sync(bar_id, 128);
       }
-      if (!mbar_wait(bar(kBarSFull), n & 1, abort_flag, p.err)) { ok = false; break; }
-      tc_fence_after();
-      __syncwarp();
-      // scores of key j for every pair: hi + lo columns
-      float s[P8];
-#pragma unroll
-      for (int c = 0; c < P8; c += 8) {
-        float hi[8], lo[8];
-        tmem_ld8(tmem_s + lane_off + c, hi);
-        tmem_ld8(tmem_s + lane_off + P8 + c, lo);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) s[c + i] = hi[i] + lo[i];
-      }
-      const int key = it.tile * kTK + j;
-      bool kvalid = key < it.L;
-      if (kvalid) {
-        const long long e = (long long)it.s * p.max_pages + key / T;
-        const int fk = p.k_pages[e], fv = p.v_pages[e];
-        kvalid = fk >= 0 && fk < p.n_fragments && fv >= 0 && fv < p.n_fragments;
-      }
-#pragma unroll
-      for (int q = 0; q < P8; ++q) {
-        bool vis = kvalid && q < P;
-        if (vis && key >= Cctx) vis = (masks[pair_row[q]] >> (key - Cctx)) & 1ull;
-        if (!vis) s[q] = -INFINITY;
-      }
-      // lazy maximum: rescale only when some score passes the running max by 2^tau
-      bool need = false;
-#pragma unroll
-      for (int q = 0; q < P8; ++q) need |= s[q] > m_run[q] + kTau;
-      if (named_or(1, 128, need)) {
-#pragma unroll
-        for (int q = 0; q < P8; ++q) {
-          const float v = warp_max(s[q]);
-          if (lane == 0) red[quarter * 64 + q] = v;
+      if ((n & 1) == grp) {
+        if (!mbar_wait(bar(kBarSFull + grp), (n >> 1) & 1, abort_flag, p.err)) {
+          ok = false;
+          break;
         }
-        named_sync(1, 128);
-        if (j < P8) {
-          const float mo = m_run[j];
-          const float mt = fmaxf(fmaxf(red[j], red[64 + j]), fmaxf(red[128 + j], red[192 + j]));
-          const float mn = fmaxf(mo, mt);
-          alpha[j] = (mn == -INFINITY) ? 1.f : exp2f(mo - mn);
-          m_run[j] = mn;
+        tc_fence_after();
+        // tile record, published by the producer on its own barrier (the
+        // K ring may already hold a later tile)
+        if (!mbar_wait(bar(kBarInfo + (n & 7)), (n >> 3) & 1, abort_flag, p.err)) {
+          ok = false;
+          break;
         }
-        named_sync(1, 128);
-#pragma unroll
-        for (int q = 0; q < P8; ++q) l[q] *= alpha[q];
-        if (!first) {
-          __syncwarp();
-          // the previous tile's P.V has completed (the score commit covers it)
-          const uint32_t ob = tmem_o(seg & 1) + lane_off;
-#pragma unroll
-          for (int c = 0; c < P8; c += 8) {
-            float v[8], w[8];
-            tmem_ld8(ob + c, v);
-            tmem_ld8(ob + P8 + c, w);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              v[i] *= alpha[c + i];
-              w[i] *= alpha[c + i];
+        const uint4 inf = tile_info[n & 7];
+        const int key0 = it.tile * kTK;
+        const int key = key0 + j;
+        const uint32_t both = inf.x & inf.y;
+        const bool kvalid = j < (int)inf.z && (both >> (j / box_t) & 1u);
+        // visibility of this key to each pair, as a bit mask
+        unsigned long long vis;
+        if (key0 + kTK <= Cctx && inf.z == (uint32_t)kTK && both == full_boxes) {
+          vis = ~0ull;  // context tile (pairs past P have zero Q rows; never read)
+        } else {
+          vis = 0;
+          if (kvalid) {
+            if (key < Cctx) {
+              vis = P >= 64 ? ~0ull : ((1ull << P) - 1ull);
+            } else {
+#pragma unroll 1
+              for (int q = 0; q < P; ++q)
+                vis |= ((masks[pair_row[q]] >> (key - Cctx)) & 1ull) << q;
             }
-            tmem_st8(ob + c, v);
-            tmem_st8(ob + P8 + c, w);
           }
-          tmem_st_wait();
         }
-      }
-      // probabilities (hi + lo operand terms) into the P buffer, row j
-      uint8_t *prow = smem + (p_base - sbase) + (j >> 3) * Lay::kPLbo + (j & 7) * 16;
+        const uint32_t s_addr = tmem_s(grp) + lane_off;
+        __syncwarp();
+        // pass 1: does any score pass the running max by 2^tau?
+        float gap = -INFINITY;
+#pragma unroll 1
+        for (int c = 0; c < P8; c += 8) {
+          float v[8];
+          tmem_load<8>(s_addr + c, v);
 #pragma unroll
-      for (int c = 0; c < P8; c += 8) {
-        uint16_t hi[8], lo[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float x = s[c + i];
-          const float e = (x == -INFINITY) ? 0.f : exp2f(x - m_run[c + i]);
-          l[c + i] += e;
-          Op::split(e, hi[i], lo[i]);
+          for (int i = 0; i < 8; ++i)
+            if ((vis >> (c + i)) & 1ull) gap = fmaxf(gap, v[i] - m_run[c + i]);
         }
-        uint4 vh, vl;
-        vh.x = hi[0] | (uint32_t)hi[1] << 16; vh.y = hi[2] | (uint32_t)hi[3] << 16;
-        vh.z = hi[4] | (uint32_t)hi[5] << 16; vh.w = hi[6] | (uint32_t)hi[7] << 16;
-        vl.x = lo[0] | (uint32_t)lo[1] << 16; vl.y = lo[2] | (uint32_t)lo[3] << 16;
-        vl.z = lo[4] | (uint32_t)lo[5] << 16; vl.w = lo[6] | (uint32_t)lo[7] << 16;
-        *reinterpret_cast<uint4 *>(prow + (c >> 3) * 128) = vh;
-        *reinterpret_cast<uint4 *>(prow + ((P8 + c) >> 3) * 128) = vl;
-      }
-      if (!kvalid) {
-        // a dead slot may hold any bits: give it a zero V row (P is 0 there)
-        const int st = n % NS;
-        mbar_wait(bar(kBarFull + st), (n / NS) & 1, abort_flag, p.err);
-        uint8_t *v0 = smem + st * kStageBytes + 2 * kRegionBytes + j * 128;
+        if (named_or(bar_id, 128, gap > kTau)) {
+          // per-pair maximum over the tile's keys, through this group's P tile
+          // as FP32 scratch [key][pair] (free: the group's previous P.V and sums
+          // have completed, its score commit came later)
+#pragma unroll 1
+          for (int c = 0; c < P8; c += 8) {
+            float v[8];
+            tmem_load<8>(s_addr + c, v);
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
+            for (int i = 0; i < 8; ++i)
+              if (!((vis >> (c + i)) & 1ull)) v[i] = -INFINITY;
+            *reinterpret_cast<float4 *>(scr + j * P8 + c) = make_float4(v[0], v[1], v[2], v[3]);
+            *reinterpret_cast<float4 *>(scr + j * P8 + c + 4) =
+                make_float4(v[4], v[5], v[6], v[7]);
+          }
+          named_sync(bar_id, 128);
+          column_reduce<P8, false>(scr, j, red, bar_id);  // red[q] = max over keys
+          named_sync(bar_id, 128);
+          if (j < P8) {
+            const float mo = m_run[j];
+            const float mn = fmaxf(mo, red[j]);
+            alpha[j] = ex2(mo - mn);
+            m_run[j] = mn;
+          }
+          named_sync(bar_id, 128);
+          if (had_tile) {
+            // rescale this group's output and sums (the previous P.V and sums
+            // have completed)
+            __syncwarp();
+            const uint32_t ob = tmem_o(grp, oslot) + lane_off;
+#pragma unroll 1
+            for (int c = 0; c < 2 * kN; c += 8) {
+              float v[8];
+              tmem_load<8>(ob + c, v);
+              const int cc = c % kN;
+              const int q0 = cc < P8 ? cc : cc - P8;
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4 *>(v0 + h * kRegionBytes + c * 16) = make_uint4(0, 0, 0, 0);
+              for (int i = 0; i < 8; ++i) v[i] *= alpha[q0 + i];
+              tmem_st8(ob + c, v);
+            }
+            tmem_st_wait();
+          }
+        }
+        // pass 2: probabilities -> this group's P tile, row j: hi then lo columns
+        uint8_t *prow = smem + (p_base - sbase) + grp * Lay::kPBytes + (j >> 3) * Lay::kPLbo +
+                        (j & 7) * 16;
+#pragma unroll 1
+        for (int c = 0; c < P8; c += 8) {
+          float v[8];
+          tmem_load<8>(s_addr + c, v);
+          float e[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            e[i] = ((vis >> (c + i)) & 1ull) ? ex2(v[i] - m_run[c + i]) : 0.f;
+          uint4 vh, vl;
+          split2<DT>(e[0], e[1], vh.x, vl.x);
+          split2<DT>(e[2], e[3], vh.y, vl.y);
+          split2<DT>(e[4], e[5], vh.z, vl.z);
+          split2<DT>(e[6], e[7], vh.w, vl.w);
+          *reinterpret_cast<uint4 *>(prow + (c >> 3) * 128) = vh;
+          *reinterpret_cast<uint4 *>(prow + ((P8 + c) >> 3) * 128) = vl;
+        }
+        if (!kvalid) {
+          // a dead slot may hold any bits: give it a zero V row (P is 0 there)
+          mbar_wait(bar(kBarFullV + n % NS), (n / NS) & 1, abort_flag, p.err);
+          uint8_t *v0 = smem + (v_base - sbase) + (n % NS) * Lay::kHalfStage + j * 128;
+#pragma unroll 1
+          for (int c = 0; c < 16; ++c)
+            *reinterpret_cast<uint4 *>(v0 + (c >> 3) * kRegionBytes + (c & 7) * 16) =
+                make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        mbar_arrive(bar(kBarPFull + grp));
+        had_tile = true;
       }
-      fence_proxy_async();
-      tc_fence_before();
-      mbar_arrive(bar(kBarPFull));
 
       if (last) {
-        // ---- epilogue: normalised partial output and its log2-sum-exp ----
-#pragma unroll
-        for (int q = 0; q < P8; ++q) {
-          const float v = warp_sum(l[q]);
-          if (lane == 0) red[quarter * 64 + q] = v;
-        }
-        named_sync(1, 128);
-        if (!mbar_wait(bar(kBarOFull + (seg & 1)), (seg >> 1) & 1, abort_flag, p.err)) {
+        // ---- epilogue of this group's piece: normalised output and log2-sum-exp ----
+        if (!mbar_wait(bar(kBarOFull + 2 * grp + oslot), (seg / kOS) & 1, abort_flag, p.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
         __syncwarp();
         const int c_first = cta_of_tile(it.seg_first, U, C);
-        const int slot = cta - c_first;
-        const int d = j;  // output lane = head dim
-        const uint32_t ob = tmem_o(seg & 1) + lane_off;
-#pragma unroll
+        const int slot = 2 * (cta - c_first) + grp;
+        const int d = j;  // output lane = head dim; every lane holds the sums
+        const uint32_t ob = tmem_o(grp, oslot) + lane_off;
+        const uint32_t lb = tmem_l(grp, oslot) + lane_off;
+        const long long row_stride = (long long)p.n_q_heads * tp.n_slots * kD;
+        const long long base =
+            ((long long)it.row0 * p.n_q_heads + it.g * G) * tp.n_slots + slot;
+#pragma unroll 1
         for (int c = 0; c < P8; c += 8) {
-          float v[8], w[8];
-          tmem_ld8(ob + c, v);
-          tmem_ld8(ob + P8 + c, w);
+          float oh[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, ol[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          float lh[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, ll[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          if (had_tile) {
+            tmem_load<8>(ob + c, oh);
+            tmem_load<8>(ob + P8 + c, ol);
+            tmem_load<8>(lb + c, lh);
+            tmem_load<8>(lb + P8 + c, ll);
+          }
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int q = c + i;
             if (q < P) {
-              const float lt = red[q] + red[64 + q] + red[128 + q] + red[192 + q];
-              const int r = pair_row[q], h = it.g * G + (q - r * G);
+              const int r = pair_row[q];
               const long long idx =
-                  ((long long)(it.row0 + r) * p.n_q_heads + h) * tp.n_slots + slot;
-              p.o_part[idx * kD + d] = lt > 0.f ? (v[i] + w[i]) / lt : 0.f;
-              if (d == q) p.lse_part[idx] = lt > 0.f ? m_run[q] + log2f(lt) : -INFINITY;
+                  base + r * row_stride / kD + (long long)(q - r * G) * tp.n_slots;
+              const float lt = lh[i] + ll[i];
+              p.o_part[idx * kD + d] = lt > 0.f ? (oh[i] + ol[i]) * rcp(lt) : 0.f;
+              if (d == q) p.lse_part[idx] = lt > 0.f ? m_run[q] + lg2(lt) : -INFINITY;
             }
           }
         }
         tc_fence_before();
-        named_sync(1, 128);
-        mbar_arrive(bar(kBarOEmpty + (seg & 1)));
+        named_sync(bar_id, 128);
+        mbar_arrive(bar(kBarOEmpty + 2 * grp + oslot));
       }
     }
   }
@@ -797,8 +1091,12 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 template <int DT, int P8>
 int launch_tc(const TcParams &tp, int smem, cudaStream_t st) {
   auto k = partial_tcgen05_kernel<DT, P8>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return (int)e;
+  static int set_for = -1;  // largest dynamic smem already allowed (per device run)
+  if (smem > set_for) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return (int)e;
+    set_for = smem;
+  }
   k<<<tp.n_ctas, kThreads, smem, st>>>(tp);
   return (int)cudaGetLastError();
 }
