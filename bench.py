@@ -133,6 +133,21 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
+def reduce_max(value, dist, device):
+    """Max over ranks of a per-rank float (device time: the slowest rank)."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(world, bytes_per_call, calls, max_ms):
+    """Whole-job effective GB/s: every rank's bytes over the slowest rank's time."""
+    return world * bytes_per_call * calls / (max_ms * 1e-3) / 1e9
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -276,11 +291,7 @@ def run_ours(args, w, world, rank, local):
     assert call.device_error() == 0, "device error during the timed steps"
     steps_ms = [e[0].elapsed_time(e[1]) for e in ev]
     part = [e[0].elapsed_time(e[1]) for e in evp]
-    total_ms = sum(steps_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-    if dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = reduce_max(sum(steps_ms), dist, "cuda")
 
     # end to end: pinned host inputs -> device -> run -> result back to host
     e2e = None
@@ -294,7 +305,7 @@ def run_ours(args, w, world, rank, local):
     peak, peak_kind = measured_peaks()
     part_ms = statistics.mean(part)
     achieved = bytes_partial / (part_ms * 1e-3) / 1e9
-    value = world * bytes_call * args.steps / (total_ms * 1e-3) / 1e9
+    value = job_gbs(world, bytes_call, args.steps, total_ms)
     info = call.info
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
@@ -370,13 +381,9 @@ def measure_e2e(call, w, args, stream, flush, dist):
         step()
         evs[i][1].record(stream)
     torch.cuda.synchronize()
-    ms = sum(a.elapsed_time(b) for a, b in evs)
-    t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-    if dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = reduce_max(sum(a.elapsed_time(b) for a, b in evs), dist, "cuda")
     world = dist.get_world_size() if dist else 1
-    ms = float(t.item())
-    return {"value": world * w.call_bytes() * steps / (ms * 1e-3) / 1e9, "unit": "GB/s",
+    return {"value": job_gbs(world, w.call_bytes(), steps, ms), "unit": "GB/s",
             "us_per_call": ms / steps * 1e3, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h}
 
