@@ -271,6 +271,36 @@ LSE_API int lse_attn_validate(const lse_attn_plan_t *plan, const int32_t *k_page
 LSE_API int lse_attn_read_error(const lse_attn_plan_t *plan, void *workspace, void *stream,
                         uint32_t *device_error, char **err);
 
+/* ---------------------------------------------------------------------------
+ * No-allocation variant (the pages have no counterpart: it exists for
+ * callers that cannot allocate device memory when attention runs, such as
+ * plugin or custom-op hosts that hand a kernel only its inputs and outputs,
+ * serving loops that forbid allocation after warm-up, and code running under
+ * CUDA-graph stream capture, where a synchronising allocation is illegal).
+ * Runs lse_attn_run then lse_attn_merge on `stream` with the workspace taken
+ * from a static device array of LSE_STATIC_SCRATCH_BYTES that the library
+ * holds on every GPU that loads it until the process exits.  Arguments as
+ * lse_attn_run and lse_attn_merge (device pointers; out [total_rows][Hq][D],
+ * lse_out optional).  It calls no cudaMalloc, cudaFree or other allocating
+ * routine.
+ *   - A plan whose workspace_bytes exceed LSE_STATIC_SCRATCH_BYTES is
+ *     rejected with LSE_ERR_UNSUPPORTED and a message.
+ *   - The first call on each device looks the array's device address up
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - Every call shares the one array and leaves its contents behind; the
+ *     device error word is cleared at the start of each call.  Calls whose
+ *     GPU work overlaps (other streams, other threads) race on the array:
+ *     serialise them.
+ * ------------------------------------------------------------------------- */
+#define LSE_STATIC_SCRATCH_BYTES (32u << 20)
+
+LSE_API int lse_attn_forward_static(const lse_attn_plan_t *plan, const float *q,
+                                    const int32_t *k_pages, const int32_t *v_pages,
+                                    const int32_t *seq_lens, const int32_t *row_offsets,
+                                    const uint64_t *row_masks, float softmax_scale, float *out,
+                                    float *lse_out, void *stream, char **err);
+
 /* Release a string returned through an err argument. */
 LSE_API void lse_free(void *p);
 

@@ -88,6 +88,9 @@ _sig("lse_attn_merge", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _errp)
 _sig("lse_attn_validate", _i, _vp, _i32p, _i32p, _i32p, _i32p,
      ctypes.POINTER(ctypes.c_uint64), _errp)
 _sig("lse_attn_read_error", _i, _vp, _vp, _vp, ctypes.POINTER(ctypes.c_uint32), _errp)
+_sig("lse_attn_forward_static", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _vp,
+     _vp, _errp)
+STATIC_SCRATCH_BYTES = 32 << 20
 
 
 class LseError(RuntimeError):
@@ -248,6 +251,15 @@ def lse_attn_validate(plan, k_pages, v_pages, seq_lens, row_offsets, row_masks=N
         rm = np.ascontiguousarray(row_masks, dtype=np.uint64)
         mp = rm.ctypes.data_as(ctypes.POINTER(ctypes.c_uint64))
     _call(_lib.lse_attn_validate, plan, kpp, vpp, slp, rop, mp)
+
+
+def lse_attn_forward_static(plan, q, k_pages, v_pages, seq_lens, row_offsets, row_masks,
+                            softmax_scale, out, lse_out=None, stream=0) -> None:
+    """Partial and merge passes on the library's static scratch (no
+    device allocation; see include/lse_attn.h for the limits)."""
+    _call(_lib.lse_attn_forward_static, plan, _ptr(q), _ptr(k_pages), _ptr(v_pages),
+          _ptr(seq_lens), _ptr(row_offsets), _ptr(row_masks), float(softmax_scale), _ptr(out),
+          _ptr(lse_out), _ptr(stream))
 
 
 def lse_attn_read_error(plan, workspace, stream=0) -> int:
