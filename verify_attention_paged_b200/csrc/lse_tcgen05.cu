@@ -261,17 +261,38 @@ __device__ __forceinline__ int seq_tiles(const LseKernelParams &p, int s, int &L
   return R == 0 ? 0 : (L + kTK - 1) / kTK;
 }
 
-// Walks the CTA's contiguous range of global tiles, segment by segment.
+// Per-sequence record built once per CTA in shared memory (sequences up to
+// kSeqTab): tiles before the sequence (all kv heads counted once), its
+// tiles, L, first row, R.
+constexpr int kSeqTab = 256;
+struct SeqRec {
+  int prefix, n_tiles, L, row0, R;
+};
+
+// Walks the CTA's contiguous range of global tiles, segment by segment.  With
+// a sequence table it looks sequences up in shared memory; without one (more
+// sequences than the table holds) it reads them from global memory.
 struct TileIter {
   int s, g, tile, n_tiles;   // segment (sequence, kv head) and tile within it
   int L, row0, R;
   long long seg_first;       // global index of the segment's first tile
   long long t, t_end;        // current / end global tile
+  const SeqRec *tab;         // shared-memory sequence table or null
 
+  __device__ int tiles_of(const LseKernelParams &p, int q) {
+    if (tab) {
+      const SeqRec r = tab[q];
+      L = r.L;
+      row0 = r.row0;
+      R = r.R;
+      return r.n_tiles;
+    }
+    return seq_tiles(p, q, L, row0, R);
+  }
   __device__ __noinline__ void next_seq(const LseKernelParams &p) {
     // advance to the next sequence with tiles, starting at s
     while (s < p.n_seqs) {
-      const int n = seq_tiles(p, s, L, row0, R);
+      const int n = tiles_of(p, s);
       if (n > 0) {
         n_tiles = n;
         return;
@@ -280,18 +301,33 @@ struct TileIter {
     }
   }
   __device__ __noinline__ void init(const LseKernelParams &p, long long t_begin,
-                                    long long t_stop) {
+                                    long long t_stop, const SeqRec *table) {
     t = t_begin;
     t_end = t_stop;
+    tab = table;
     s = 0;
     long long base = 0;
     n_tiles = 0;
     if (t >= t_end) return;
-    next_seq(p);
-    while (base + (long long)p.n_kv_heads * n_tiles <= t) {
-      base += (long long)p.n_kv_heads * n_tiles;
-      ++s;
+    if (tab) {
+      // last sequence whose first tile is at or before t (idle sequences share
+      // the prefix of the next one, so the last such index has tiles)
+      int lo = 0, hi = p.n_seqs - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((long long)tab[mid].prefix * p.n_kv_heads <= t) lo = mid;
+        else hi = mid - 1;
+      }
+      s = lo;
+      base = (long long)tab[s].prefix * p.n_kv_heads;
       next_seq(p);
+    } else {
+      next_seq(p);
+      while (base + (long long)p.n_kv_heads * n_tiles <= t) {
+        base += (long long)p.n_kv_heads * n_tiles;
+        ++s;
+        next_seq(p);
+      }
     }
     g = int((t - base) / n_tiles);
     tile = int((t - base) - (long long)g * n_tiles);
@@ -450,7 +486,8 @@ struct TcLayout {
                                  : kTmemNeed <= 256 ? 256 : 512;
   static constexpr int kBars = 48;
   static constexpr int kMiscBytes = kBars * 8 + 16 + 2 * 64 * 4 * 2 + 2 * 4 * 64 * 4 +
-                                    2 * 64 * 8 + 64 * 4 + 8 * 16 + 2 * 32 * 16 * 4;
+                                    2 * 64 * 8 + 64 * 4 + 8 * 16 + 2 * 32 * 16 * 4 +
+                                    kSeqTab * (int)sizeof(SeqRec);
   static constexpr int kHalfStage = 2 * kRegionBytes;    // one K or V tile
   static int smem_bytes(int stages) {
     return 1024 + stages * 2 * kHalfStage + kQSlots * kQBytes + 2 * kPBytes + kOnesBytes +
@@ -568,22 +605,49 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint4 *tile_info = reinterpret_cast<uint4 *>(pair_row + 64);               // [8]
   // fragment ids of a batch of 32 tiles (up to 16 boxes each), K then V
   int *page_buf = reinterpret_cast<int *>(tile_info + 8);                    // [2][32][16]
+  SeqRec *seq_tab = reinterpret_cast<SeqRec *>(page_buf + 2 * 32 * 16);     // [kSeqTab]
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
   // the merge pass may be scheduled now; it waits for this grid to finish
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // ---- prologue: total live tiles, barriers, TMEM -------------------------------
-  if (tid == 0) {
-    long long U = 0;
+  const bool use_tab = p.n_seqs <= kSeqTab;
+  if (warp == 0) {
+    // every sequence's tiles, lanes taking contiguous blocks; then a warp
+    // exclusive scan gives each sequence its first tile
+    const int per = (p.n_seqs + 31) / 32;
+    const int s0 = lane * per, s1 = min(p.n_seqs, s0 + per);
+    long long mine = 0;
     bool bad = false;
-    for (int s = 0; s < p.n_seqs; ++s) {
+    for (int q = s0; q < s1; ++q) {
       int L, r0, R;
-      const int n = seq_tiles(p, s, L, r0, R);
-      if (n < 0) bad = true;
-      else U += n;
+      int n = seq_tiles(p, q, L, r0, R);
+      if (n < 0) {
+        bad = true;
+        n = 0;
+      }
+      if (use_tab) seq_tab[q] = SeqRec{0, n, L, r0, R};
+      mine += n;
     }
-    if (bad && cta == 0) atomicOr(p.err, LSE_DEVERR_BAD_LENGTH);
-    *shared_u = U * p.n_kv_heads;
+    long long incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (use_tab) {
+      long long run = incl - mine;
+      for (int q = s0; q < s1; ++q) {
+        seq_tab[q].prefix = (int)run;
+        run += seq_tab[q].n_tiles;
+      }
+    }
+    bad = __any_sync(0xffffffffu, bad);
+    if (lane == 31) *shared_u = incl * p.n_kv_heads;
+    if (lane == 0 && bad && cta == 0) atomicOr(p.err, LSE_DEVERR_BAD_LENGTH);
+  }
+  const SeqRec *tab = use_tab ? seq_tab : nullptr;
+  if (tid == 32) {
     *abort_flag = 0;
     for (int i = 0; i < 4; ++i) {
       mbar_init(bar(kBarFullK + i), 1);
@@ -656,7 +720,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int b0 = 0; b0 < n_total && ok; b0 += 32) {
       const int cnt = n_total - b0 < 32 ? n_total - b0 : 32;
       TileIter mine;
-      mine.init(p, t_begin + b0 + (lane < cnt ? lane : 0), t_stop);
+      mine.init(p, t_begin + b0 + (lane < cnt ? lane : 0), t_stop, tab);
       if (lane < cnt) load_page_ids(p, mine, nbox, box_t, pk + lane * 16, pv + lane * 16);
       __syncwarp();
 #pragma unroll 1
@@ -699,8 +763,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_l = instr_desc(fmt, 0, 1, kD, kN);
       const int n_total = (int)(t_stop - t_begin);
       TileIter iq, iv;
-      iq.init(p, t_begin, t_stop);
-      iv.init(p, t_begin, t_stop);
+      iq.init(p, t_begin, t_stop, tab);
+      iv.init(p, t_begin, t_stop, tab);
       int nq = 0, seg_q = -1;   // score side: tiles issued, segment count
       int nv = 0, seg_v = -1;   // output side
       bool grp_started[2] = {false, false};
@@ -811,7 +875,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ============================ Q staging ===============================
     const int qt = tid - 64;  // 0..63
     TileIter it;
-    it.init(p, t_begin, t_stop);
+    it.init(p, t_begin, t_stop, tab);
     int seg = -1;
     for (; it.valid(); it.advance(p)) {
       if (!it.seg_start(t_begin)) continue;
@@ -873,7 +937,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned long long *masks = masks_all + grp * 64;
     float *scr = reinterpret_cast<float *>(smem + (p_base - sbase) + grp * Lay::kPBytes);
     TileIter it;
-    it.init(p, t_begin, t_stop);
+    it.init(p, t_begin, t_stop, tab);
     int n = 0, seg = -1;
     bool had_tile = false, ok = true;
 #pragma unroll 1
