@@ -216,6 +216,13 @@ def run_reference(args, w, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def compute_dtype(kv_dtype, kernel):
+    """The arithmetic the partial pass runs in: the tensor-core kernel takes
+    16-bit K/V times 16-bit hi + lo terms of Q and P, or 8-bit K/V times 8-bit
+    terms, accumulating in FP32; the CUDA-core kernel is FP32 throughout."""
+    return f"{kv_dtype}-mma/f32" if kernel == 1 else "f32"
+
+
 def workload_config(w):
     return {"workload": w.name, "seqs": w.n_seqs, "keys_total": int(np.sum(w.seq_lens)),
             "query_rows": w.total_rows, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
@@ -317,7 +324,7 @@ def run_ours(args, w, world, rank, local):
         "pct_of_8tbs": value / world / 8000.0 * 100.0,
         "pct_of_measured_hbm": value / world / peak * 100.0,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16-mma/f32" if info["kernel"] == 1 else "f32",
+        "dtype": compute_dtype(w.dtype, info["kernel"]),
         "data": "synthetic", "config": {**workload_config(w), "parallelism": f"replicas{world}",
                                         "kernel": info["kernel_name"],
                                         "n_splits": info["n_splits"],

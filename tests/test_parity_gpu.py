@@ -191,7 +191,10 @@ def check_kernel(b, w, kernel):
     return out
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+TC_DTYPES = ["bf16", "f16", "e4m3", "e5m2"]
+
+
+@pytest.mark.parametrize("dtype", TC_DTYPES)
 @pytest.mark.parametrize("tpf", [8, 16, 64, 128, 256, 512])
 def test_tcgen05_fragment_sizes(binding, dtype, tpf):
     w = wl.small_case(dtype, [1, 127, 128, 129, 700, 2051], [1, 1, 2, 3, 4, 8],
@@ -200,7 +203,7 @@ def test_tcgen05_fragment_sizes(binding, dtype, tpf):
     check_kernel(binding, w, "tcgen05")
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("dtype", TC_DTYPES)
 @pytest.mark.parametrize("heads,rows", [((24, 4), 8), ((32, 8), 12), ((8, 8), 1),
                                         ((16, 1), 3), ((12, 4), 16)])
 def test_tcgen05_pairs_and_trees(binding, dtype, heads, rows):
@@ -211,42 +214,59 @@ def test_tcgen05_pairs_and_trees(binding, dtype, heads, rows):
     check_kernel(binding, w, "tcgen05")
 
 
-def test_tcgen05_many_segments_per_cta(binding):
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_tcgen05_many_segments_per_cta(binding, dtype):
     # 70 short sequences: CTAs cross many (sequence, kv head) segments, so the
     # Q ring, the two TMEM output slots and the piece numbering all rotate
     rng = np.random.default_rng(5)
     lens = [int(x) for x in rng.integers(1, 600, 70)]
     rows = [int(min(L, r)) for L, r in zip(lens, rng.integers(0, 7, 70))]
-    w = wl.small_case("bf16", lens, rows, n_q_heads=24, n_kv_heads=4, head_dim=128,
+    w = wl.small_case(dtype, lens, rows, n_q_heads=24, n_kv_heads=4, head_dim=128,
                       tokens_per_fragment=128, tree=True, seed=220)
     out_tc = check_kernel(binding, w, "tcgen05")
     out_cc = check_kernel(binding, w, "cuda_core")
-    assert_close(out_tc, out_cc, "bf16", what="tcgen05 vs cuda_core")
+    assert_close(out_tc, out_cc, dtype, what="tcgen05 vs cuda_core")
 
 
-def test_tcgen05_fewer_tiles_than_ctas(binding):
-    w = wl.small_case("f16", [200], [2], n_q_heads=8, n_kv_heads=2, head_dim=128,
+@pytest.mark.parametrize("dtype", ["f16", "e5m2"])
+def test_tcgen05_fewer_tiles_than_ctas(binding, dtype):
+    w = wl.small_case(dtype, [200], [2], n_q_heads=8, n_kv_heads=2, head_dim=128,
                       tokens_per_fragment=64, seed=221)
     check_kernel(binding, w, "tcgen05")
 
 
-def test_tcgen05_growing_scores_trigger_rescale(binding):
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_tcgen05_growing_scores_trigger_rescale(binding, dtype):
     # key rows grow with position, so the running maximum rises tile after
     # tile by more than the lazy threshold: the TMEM output must be rescaled
-    w = wl.small_case("bf16", [3000, 900], [4, 1], n_q_heads=24, n_kv_heads=4, head_dim=128,
+    w = wl.small_case(dtype, [3000, 900], [4, 1], n_q_heads=24, n_kv_heads=4, head_dim=128,
                       tokens_per_fragment=256, seed=222)
     w2 = _rewrite_k(w, lambda s, j, k: k * (0.25 + j / 150.0))
     check_kernel(binding, w2, "tcgen05")
 
 
-def test_tcgen05_capacity_far_above_live(binding):
-    w = wl.small_case("bf16", [130, 5, 1000], [1, 1, 2], n_q_heads=24, n_kv_heads=4,
+@pytest.mark.parametrize("dtype", ["e4m3", "e5m2"])
+@pytest.mark.parametrize("q_gain", [1e-3, 16.0])
+def test_tcgen05_fp8_query_scale_range(binding, dtype, q_gain):
+    # FP8 scores enter the tensor cores as scaled 8-bit terms of Q: tiny and
+    # large query magnitudes (near-uniform and sharply peaked softmax, where
+    # tiny probabilities must still count) stay within tolerance
+    w = wl.small_case(dtype, [2000, 700], [3, 1], n_q_heads=24, n_kv_heads=4, head_dim=128,
+                      tokens_per_fragment=128, seed=225)
+    w2 = wl.Workload(**{**w.__dict__, "q": (w.q * q_gain).astype(np.float32)})
+    check_kernel(binding, w2, "tcgen05")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_tcgen05_capacity_far_above_live(binding, dtype):
+    w = wl.small_case(dtype, [130, 5, 1000], [1, 1, 2], n_q_heads=24, n_kv_heads=4,
                       head_dim=128, tokens_per_fragment=128, max_pages=300, seed=223)
     check_kernel(binding, w, "tcgen05")
 
 
-def test_tcgen05_bad_page_sets_error_word(binding):
-    w = wl.small_case("bf16", [600], [2], n_q_heads=8, n_kv_heads=2, head_dim=128,
+@pytest.mark.parametrize("dtype", ["bf16", "e5m2"])
+def test_tcgen05_bad_page_sets_error_word(binding, dtype):
+    w = wl.small_case(dtype, [600], [2], n_q_heads=8, n_kv_heads=2, head_dim=128,
                       tokens_per_fragment=128, seed=224)
     kp = w.k_pages.copy()
     kp[0, 1] = 10 ** 6
@@ -255,9 +275,9 @@ def test_tcgen05_bad_page_sets_error_word(binding):
     assert err & binding.DEVERR_BAD_FRAGMENT and not err & binding.DEVERR_TIMEOUT
 
 
-def test_plan_picks_tensor_cores_for_the_bf16_workloads(binding):
+def test_plan_picks_tensor_cores_for_the_bf16_and_fp8_workloads(binding):
     for name, want in (("batched_decode", "tcgen05"), ("chain_verify", "tcgen05"),
-                       ("tiny_decode", "cuda_core")):
+                       ("long_fp8", "tcgen05"), ("tiny_decode", "cuda_core")):
         w = wl.BUILDERS[name]()
         call = binding.DeviceCall(w)
         assert call.info["kernel_name"] == want, name

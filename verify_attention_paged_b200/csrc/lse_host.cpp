@@ -270,20 +270,23 @@ int lse_attn_plan_ex(const lse_kv_arena *a, int n_seqs, int max_rows, int max_to
   pl->n_sms = n_sms;
 
   // kernel choice and its on-chip memory check.  The tensor-core kernel
-  // takes 16-bit K/V with head_dim 128, up to 48 (row, head) pairs per kv
-  // head, and fragments whose token count tiles evenly into 128-key tiles.
+  // takes 16-bit and FP8 K/V with head_dim 128, up to 48 (row, head) pairs
+  // per kv head, and fragments whose token count tiles evenly into 128-key
+  // tiles.
   const int T = a->tokens_per_fragment;
   const bool t_ok = (T % 128 == 0) || (T >= 8 && T % 8 == 0 && 128 % T == 0);
   const int p8 = lse_tc_pairs_bucket(pl->pairs);
-  int tc_stages = 0;
-  const int tc_smem = p8 > 0 ? lse_tc_smem(p8, smem_optin, &tc_stages) : -1;
-  if (allow_tc && (a->dtype == LSE_KV_BF16 || a->dtype == LSE_KV_F16) && a->head_dim == 128 &&
+  int tc_stages = 0, tc_q_slots = 0;
+  const int tc_smem =
+      p8 > 0 ? lse_tc_smem(a->dtype, p8, smem_optin, &tc_stages, &tc_q_slots) : -1;
+  if (allow_tc && a->dtype != LSE_KV_F32 && a->head_dim == 128 &&
       t_ok && p8 > 0 && tc_smem > 0) {
     const int tile = lse_tc_key_tile();
     pl->kernel = LSE_KERNEL_TCGEN05;
     pl->key_tile = tile;
     pl->smem_bytes = tc_smem;
     pl->stages = tc_stages;
+    pl->q_slots = tc_q_slots;
     pl->pairs_bucket = p8;
     pl->box_tokens = T < tile ? T : tile;
     pl->ctas = n_sms;
@@ -405,7 +408,7 @@ int lse_attn_run(const lse_attn_plan_t *pl, const float *q, const int32_t *k_pag
     if (pl->maps_chunks != nch) {
       pl->maps.assign(lse_tc_map_bytes() * nch, 0);
       ce = lse_tc_build_maps(a->chunk_base.data(), nch, a->chunk_bytes, a->n_kv_heads,
-                             pl->box_tokens, pl->maps.data());
+                             a->dtype, pl->box_tokens, pl->maps.data());
       if (ce) {
         pl->maps_chunks = 0;
         return cuda_fail(err, ce, "building TMA descriptors");
@@ -413,7 +416,8 @@ int lse_attn_run(const lse_attn_plan_t *pl, const float *q, const int32_t *k_pag
       pl->maps_chunks = nch;
     }
     ce = lse_launch_partial_tcgen05(p, pl->maps.data(), nch, pl->dtype, pl->pairs_bucket,
-                                    pl->ctas, pl->n_splits, pl->stages, pl->box_tokens,
+                                    pl->ctas, pl->n_splits, pl->stages, pl->q_slots,
+                                    pl->box_tokens,
                                     pl->smem_bytes, stream);
   } else {
     ce = lse_launch_partial_cuda_core(p, pl->dtype, pl->head_dim, pl->n_splits, pl->n_kv_heads,

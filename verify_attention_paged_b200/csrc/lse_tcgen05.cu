@@ -71,6 +71,7 @@ struct __align__(64) TcParams {
   int n_ctas;
   int n_slots;
   int stages;
+  int q_slots;
   int box_tokens;
 };
 
@@ -185,10 +186,12 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
 constexpr uint32_t kLayoutNone = 0;
 constexpr uint32_t kLayoutSw128 = 2;
 
-// Instruction descriptor, kind::f16, FP32 accumulation.
-__host__ __device__ constexpr uint32_t instr_desc(uint32_t ab_fmt, uint32_t a_mn, uint32_t b_mn,
-                                                  uint32_t M, uint32_t N) {
-  return (1u << 4) | (ab_fmt << 7) | (ab_fmt << 10) | (a_mn << 15) | (b_mn << 16) |
+// Instruction descriptor, FP32 accumulation.  Formats: kind::f16 takes
+// 0 = F16, 1 = BF16 (A and B alike); kind::f8f6f4 takes 0 = E4M3, 1 = E5M2
+// for A and B independently.  a_mn / b_mn: 1 = MN-major operand.
+__host__ __device__ constexpr uint32_t instr_desc(uint32_t a_fmt, uint32_t b_fmt, uint32_t a_mn,
+                                                  uint32_t b_mn, uint32_t M, uint32_t N) {
+  return (1u << 4) | (a_fmt << 7) | (b_fmt << 10) | (a_mn << 15) | (b_mn << 16) |
          ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
@@ -198,6 +201,16 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b,
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// 8-bit operands, K = 32 per instruction.
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -219,32 +232,6 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const float *v) {
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
-
-// Round an FP32 value to the 16-bit operand format: the nearest value plus
-// the rounding error in the same format (hi + lo carries ~16 mantissa bits).
-template <int DT>
-struct Op16;
-template <>
-struct Op16<LSE_KV_BF16> {
-  static constexpr uint32_t kFmt = 1;
-  static __device__ __forceinline__ void split(float x, uint16_t &hi, uint16_t &lo) {
-    const __nv_bfloat16 h = __float2bfloat16_rn(x);
-    const __nv_bfloat16 l = __float2bfloat16_rn(x - __bfloat162float(h));
-    hi = *reinterpret_cast<const uint16_t *>(&h);
-    lo = *reinterpret_cast<const uint16_t *>(&l);
-  }
-};
-template <>
-struct Op16<LSE_KV_F16> {
-  static constexpr uint32_t kFmt = 0;
-  static __device__ __forceinline__ void split(float x, uint16_t &hi, uint16_t &lo) {
-    const __half h = __float2half_rn(x);
-    const __half l = __float2half_rn(x - __half2float(h));
-    hi = *reinterpret_cast<const uint16_t *>(&h);
-    lo = *reinterpret_cast<const uint16_t *>(&l);
-  }
-};
-
 
 // ---- work decomposition ---------------------------------------------------------
 
@@ -381,9 +368,12 @@ __device__ __noinline__ void load_page_ids(const LseKernelParams &p, const TileI
   }
 }
 
-// TMA boxes of one tile (K or V): fragment ids ids[0..nbox), into dst.
-__device__ __noinline__ void load_boxes(const TcParams &tp, int nbox, int box_t, int g, int key0,
-                                        const int *ids, uint32_t dst, uint32_t full_bar) {
+// TMA boxes of one tile (K or V): fragment ids ids[0..nbox), into dst.  A
+// 16-bit tile is two regions of 64 dims (tensor rows 2g and 2g + 1); an
+// FP8 tile is one region of 128 dims (tensor row g).
+__device__ __noinline__ void load_boxes(const TcParams &tp, int nbox, int box_t, int regions,
+                                        int g, int key0, const int *ids, uint32_t dst,
+                                        uint32_t full_bar) {
   const LseKernelParams &p = tp.p;
   const int T = p.tokens_per_fragment;
 #pragma unroll 1
@@ -394,15 +384,17 @@ __device__ __noinline__ void load_boxes(const TcParams &tp, int nbox, int box_t,
     const int c = f / p.frags_per_chunk;
     const int z = (f - c * p.frags_per_chunk) * T + kb % T;
     const uint32_t d = dst + b * box_t * 128;
-    tma_load_3d(d, &tp.maps[c], full_bar, 0, g * 2, z);
-    tma_load_3d(d + kRegionBytes, &tp.maps[c], full_bar, 0, g * 2 + 1, z);
+#pragma unroll 1
+    for (int r = 0; r < regions; ++r)
+      tma_load_3d(d + r * kRegionBytes, &tp.maps[c], full_bar, 0, g * regions + r, z);
   }
 }
 
 // Producer work for tile n: K slot, tile record, K boxes, V slot, V boxes.
 // Returns 0 when a wait gave up.
 __device__ __noinline__ int produce_tile(const TcParams &tp, int n, int NS, int nbox, int box_t,
-                                         int g, int tile, int L, const int *pk, const int *pv,
+                                         int regions, int g, int tile, int L, const int *pk,
+                                         const int *pv,
                                          uint32_t kdst, uint32_t vdst, const uint32_t *bars_k,
                                          const uint32_t *bars_v, uint32_t info_bar,
                                          uint4 *info, volatile int *abort_flag) {
@@ -416,7 +408,7 @@ __device__ __noinline__ int produce_tile(const TcParams &tp, int n, int NS, int 
     if (pv[b] >= 0) vmask |= 1u << b;
   }
   const int live = L - key0 < kTK ? L - key0 : kTK;
-  const uint32_t box_bytes = 2u * (uint32_t)box_t * 128u;
+  const uint32_t box_bytes = (uint32_t)regions * (uint32_t)box_t * 128u;
   if (!mbar_wait(bars_k[0], ph, abort_flag, p.err)) return 0;
   // the record slot was last read by the softmax of tile n - 8, which has
   // finished: this producer passed its K slot wait for tile n, which
@@ -424,10 +416,10 @@ __device__ __noinline__ int produce_tile(const TcParams &tp, int n, int NS, int 
   *info = make_uint4(kmask, vmask, (uint32_t)live, 0u);
   mbar_arrive(info_bar);  // publishes the record
   mbar_expect_tx(bars_k[1], (uint32_t)__popc(kmask) * box_bytes);
-  load_boxes(tp, nbox, box_t, g, key0, pk, kdst, bars_k[1]);
+  load_boxes(tp, nbox, box_t, regions, g, key0, pk, kdst, bars_k[1]);
   if (!mbar_wait(bars_v[0], ph, abort_flag, p.err)) return 0;
   mbar_expect_tx(bars_v[1], (uint32_t)__popc(vmask) * box_bytes);
-  load_boxes(tp, nbox, box_t, g, key0, pv, vdst, bars_v[1]);
+  load_boxes(tp, nbox, box_t, regions, g, key0, pv, vdst, bars_v[1]);
   return 1;
 }
 
@@ -468,47 +460,66 @@ __device__ __forceinline__ void column_reduce(const float *tile, int t, float *o
 
 // ---- shared-memory and TMEM layout ------------------------------------------------
 
-template <int P8>
+constexpr bool is_f8(int dt) { return dt == LSE_KV_FP8_E4M3 || dt == LSE_KV_FP8_E5M2; }
+
+// FP8 operands: Q and P enter the 8-bit products as sums of kTerms 8-bit
+// values (each term holds the rounding error of the ones before it).
+constexpr int kQTerms = 4;         // E4M3 terms of Q (per-pair power-of-2 scale)
+constexpr int kPTerms = 4;         // E5M2 terms of P
+constexpr int kPScaleLog2 = 7;     // P enters the FP8 products times 2^7
+
+template <int DT, int P8>
 struct TcLayout {
+  static constexpr bool kF8 = is_f8(DT);
   static constexpr int kNQ = (P8 + 15) / 16 * 16;       // score columns (N of S^T)
-  static constexpr int kN = 2 * P8;                      // output columns: hi | lo pairs
-  static constexpr int kQSlots = P8 >= 48 ? 1 : 2;       // Q ring depth
-  static constexpr int kQRegion = kNQ * 128;             // 64 dims of kNQ rows
-  static constexpr int kQBytes = 4 * kQRegion;           // hi (2 regions) + lo (2 regions)
-  static constexpr int kPLbo = (kN / 8) * 128;           // P: stride of 8-key groups
-  static constexpr int kPBytes = kTK * kN * 2;           // one warpgroup's P tile
-  static constexpr int kOnesBytes = 4096;                // ones operand: 128 rows x 16
+  // output columns: 16-bit K/V keep hi | lo probability columns side by side;
+  // FP8 accumulates its probability terms into the same columns
+  static constexpr int kN = kF8 ? kNQ : 2 * P8;
+  static constexpr int kQRegion = kNQ * 128;             // kNQ rows of 128 bytes
+  // 16-bit: hi (2 regions of 64 dims) + lo (2 regions); FP8: kQTerms regions
+  static constexpr int kQBytes = 4 * kQRegion;
+  static_assert(!kF8 || kQTerms == 4, "Q slot holds four FP8 terms");
+  // P: 16-bit, 8x16-byte core matrices of 8 keys x 8 pairs; FP8, one
+  // block per term of 8 keys x 16 pairs core matrices
+  static constexpr int kPLbo = kF8 ? (kNQ / 16) * 128 : (kN / 8) * 128;  // 8-key group stride
+  static constexpr int kPTerm = kTK * kNQ;               // FP8: bytes of one P term
+  static constexpr int kPBytes = kF8 ? kPTerms * kPTerm : kTK * kN * 2;  // one group's P
+  static constexpr int kOnesBytes = 4096;                // ones operand: 128 rows x 32 bytes
   // TMEM: S per group, then per group and output slot the output O^T and the
   // row sums L (both kN columns); two output slots when they fit
   static constexpr int kOSlots = (2 * kNQ + 8 * kN <= 512) ? 2 : 1;
   static constexpr int kTmemNeed = 2 * kNQ + 4 * kOSlots * kN;
   static constexpr int kTmemCols = kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                  : kTmemNeed <= 256 ? 256 : 512;
-  static constexpr int kBars = 48;
+  static_assert(kTmemNeed <= 512, "TMEM holds at most 512 columns");
+  static constexpr int kBars = 64;
   static constexpr int kMiscBytes = kBars * 8 + 16 + 2 * 64 * 4 * 2 + 2 * 4 * 64 * 4 +
                                     2 * 64 * 8 + 64 * 4 + 8 * 16 + 2 * 32 * 16 * 4 +
-                                    kSeqTab * (int)sizeof(SeqRec);
-  static constexpr int kHalfStage = 2 * kRegionBytes;    // one K or V tile
-  static int smem_bytes(int stages) {
-    return 1024 + stages * 2 * kHalfStage + kQSlots * kQBytes + 2 * kPBytes + kOnesBytes +
+                                    (kF8 ? 4 * 64 * 4 : 0) + kSeqTab * (int)sizeof(SeqRec);
+  // one K or V tile: 128 keys of 128 dims (two 64-dim regions when 16-bit)
+  static constexpr int kHalfStage = kF8 ? kRegionBytes : 2 * kRegionBytes;
+  // stages: K/V ring depth; q_slots: Q ring depth (1 or 2)
+  static int smem_bytes(int stages, int q_slots) {
+    return 1024 + stages * 2 * kHalfStage + q_slots * kQBytes + 2 * kPBytes + kOnesBytes +
            kMiscBytes;
   }
 };
 
 // barrier indices in the misc block
+constexpr int kMaxStages = 6;  // K/V ring depth limit (tile records: ring of 8)
 enum {
-  kBarFullK = 0,    // [4]
-  kBarEmptyK = 4,   // [4]
-  kBarFullV = 8,    // [4]
-  kBarEmptyV = 12,  // [4]
-  kBarSFull = 16,   // [2] per softmax group
-  kBarPFull = 18,   // [2]
-  kBarQFull = 20,   // [2]
-  kBarQEmpty = 22,  // [2]
-  kBarOFull = 24,   // [4] = group * 2 + slot
-  kBarOEmpty = 28,  // [4]
-  kBarDone = 32,
-  kBarInfo = 33,    // [8] one per tile record
+  kBarFullK = 0,    // [8]
+  kBarEmptyK = 8,   // [8]
+  kBarFullV = 16,   // [8]
+  kBarEmptyV = 24,  // [8]
+  kBarSFull = 32,   // [2] per softmax group
+  kBarPFull = 34,   // [2]
+  kBarQFull = 36,   // [2]
+  kBarQEmpty = 38,  // [2]
+  kBarOFull = 40,   // [4] = group * 2 + slot
+  kBarOEmpty = 44,  // [4]
+  kBarDone = 48,
+  kBarInfo = 49,    // [8] one per tile record
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -545,6 +556,48 @@ __device__ __forceinline__ void split2<LSE_KV_F16>(float x0, float x1, uint32_t 
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(lo) : "f"(x1 - h.y), "f"(x0 - h.x));
 }
 
+// Two FP32 values -> the nearest 8-bit pair (x1 in the high byte, saturating
+// at the format's largest finite value), and the values that pair decodes
+// to (exactly, through F16, which holds every E4M3 and E5M2 value).
+template <bool kE5>
+__device__ __forceinline__ uint32_t f8x2(float x0, float x1, float &d0, float &d1) {
+  uint16_t r;
+  uint32_t h;
+  if (kE5) {
+    asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(x1), "f"(x0));
+    asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h) : "h"(r));
+  } else {
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(x1), "f"(x0));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(r));
+  }
+  const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h));
+  d0 = f.x;
+  d1 = f.y;
+  return r;
+}
+
+// Eight FP32 values -> kTerms 8-byte words of 8-bit values whose sum is the
+// input up to the last term's rounding (each term takes the remainder left
+// by the ones before it; the subtractions are exact).
+template <bool kE5, int kTerms>
+__device__ __forceinline__ void f8_terms(float *x, uint2 *out) {
+#pragma unroll
+  for (int t = 0; t < kTerms; ++t) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float d0, d1;
+      w[i] = f8x2<kE5>(x[2 * i], x[2 * i + 1], d0, d1);
+      x[2 * i] -= d0;
+      x[2 * i + 1] -= d1;
+    }
+    out[t] = make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+  }
+}
+
+// 2^e as a float, e in [-126, 127].
+__device__ __forceinline__ float exp2i(int e) { return __int_as_float((e + 127) << 23); }
+
 // TMEM: this thread's lane, N consecutive 32-bit columns (N a multiple of 8),
 // one wait for all of them.
 template <int N>
@@ -571,10 +624,12 @@ __device__ __forceinline__ void tmem_load(uint32_t taddr, float *v) {
 template <int DT, int P8>
 __global__ void __launch_bounds__(kThreads, 1)
     partial_tcgen05_kernel(const __grid_constant__ TcParams tp) {
-  using Lay = TcLayout<P8>;
+  using Lay = TcLayout<DT, P8>;
+  constexpr bool kF8 = Lay::kF8;
+  constexpr bool kE5 = DT == LSE_KV_FP8_E5M2;
   constexpr int kNQ = Lay::kNQ;
   constexpr int kN = Lay::kN;
-  constexpr int kQS = Lay::kQSlots;
+  const int QS = tp.q_slots;
   const LseKernelParams &p = tp.p;
   const int NS = tp.stages;
   const int cta = blockIdx.x;
@@ -587,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t k_base = sbase;                                // K ring
   const uint32_t v_base = k_base + NS * Lay::kHalfStage;        // V ring
   const uint32_t q_base = v_base + NS * Lay::kHalfStage;        // Q slots
-  const uint32_t p_base = q_base + kQS * Lay::kQBytes;          // P tiles (one per group)
+  const uint32_t p_base = q_base + QS * Lay::kQBytes;          // P tiles (one per group)
   const uint32_t ones_base = p_base + 2 * Lay::kPBytes;         // ones operand of the sums
   uint8_t *misc = smem + (ones_base - sbase) + Lay::kOnesBytes;
   uint64_t *bars = reinterpret_cast<uint64_t *>(misc);
@@ -605,7 +660,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint4 *tile_info = reinterpret_cast<uint4 *>(pair_row + 64);               // [8]
   // fragment ids of a batch of 32 tiles (up to 16 boxes each), K then V
   int *page_buf = reinterpret_cast<int *>(tile_info + 8);                    // [2][32][16]
-  SeqRec *seq_tab = reinterpret_cast<SeqRec *>(page_buf + 2 * 32 * 16);     // [kSeqTab]
+  // FP8: the inverse of Q's per-pair scale, per Q slot [0, 2) and the
+  // copy each softmax group keeps for its segment [2, 4)
+  float *isig_all = reinterpret_cast<float *>(page_buf + 2 * 32 * 16);       // [4][64]
+  SeqRec *seq_tab = reinterpret_cast<SeqRec *>(isig_all + (kF8 ? 4 * 64 : 0)); // [kSeqTab]
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
   // the merge pass may be scheduled now; it waits for this grid to finish
@@ -649,11 +707,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const SeqRec *tab = use_tab ? seq_tab : nullptr;
   if (tid == 32) {
     *abort_flag = 0;
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 8; ++i) {
       mbar_init(bar(kBarFullK + i), 1);
       mbar_init(bar(kBarEmptyK + i), 1);
       mbar_init(bar(kBarFullV + i), 1);
       mbar_init(bar(kBarEmptyV + i), 1);
+    }
+    for (int i = 0; i < 4; ++i) {
       mbar_init(bar(kBarOFull + i), 1);
       mbar_init(bar(kBarOEmpty + i), 128);
     }
@@ -661,7 +721,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(kBarSFull + i), 1);
       mbar_init(bar(kBarPFull + i), 128);
       mbar_init(bar(kBarQFull + i), 64);
-      mbar_init(bar(kBarQEmpty + i), 1);
+      // FP8: the softmax groups also hold the slot until they have copied
+      // the segment's Q scales
+      mbar_init(bar(kBarQEmpty + i), kF8 ? 3 : 1);
     }
     mbar_init(bar(kBarDone), 1);
     for (int i = 0; i < 8; ++i) mbar_init(bar(kBarInfo + i), 1);
@@ -669,8 +731,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid < 64) pair_row[tid] = tid / p.group;
   {
-    // the ones operand (16-bit 1.0 in the storage's operand format)
-    const uint32_t one2 = Op16<DT>::kFmt == 1 ? 0x3F803F80u : 0x3C003C00u;
+    // the ones operand: 1.0 in the format of P (E5M2 for FP8 K/V, else the
+    // storage's 16-bit format)
+    const uint32_t one2 = kF8 ? 0x3C3C3C3Cu : DT == LSE_KV_BF16 ? 0x3F803F80u : 0x3C003C00u;
     uint4 *ones = reinterpret_cast<uint4 *>(smem + (ones_base - sbase));
     for (int i = tid; i < Lay::kOnesBytes / 16; i += kThreads)
       ones[i] = make_uint4(one2, one2, one2, one2);
@@ -732,7 +795,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
           const uint32_t bars_k[2] = {bar(kBarEmptyK + n % NS), bar(kBarFullK + n % NS)};
           const uint32_t bars_v[2] = {bar(kBarEmptyV + n % NS), bar(kBarFullV + n % NS)};
-          go = produce_tile(tp, n, NS, nbox, box_t, tg, tt, tl, pk + i * 16, pv + i * 16,
+          go = produce_tile(tp, n, NS, nbox, box_t, kF8 ? 1 : 2, tg, tt, tl, pk + i * 16,
+                            pv + i * 16,
                             k_base + (n % NS) * Lay::kHalfStage,
                             v_base + (n % NS) * Lay::kHalfStage, bars_k, bars_v,
                             bar(kBarInfo + (n & 7)), tile_info + (n & 7), abort_flag);
@@ -757,10 +821,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // An event loop: the score product of tile n runs up to two tiles ahead
     // of the output products, and whichever is ready is issued first.
     if (lane == 0) {
-      constexpr uint32_t fmt = Op16<DT>::kFmt;
-      constexpr uint32_t idesc_qk = instr_desc(fmt, 0, 0, kTK, kNQ);
-      constexpr uint32_t idesc_pv = instr_desc(fmt, 1, 1, kD, kN);
-      constexpr uint32_t idesc_l = instr_desc(fmt, 0, 1, kD, kN);
+      // operand formats: 16-bit K/V use their own format for every operand;
+      // FP8 K/V meet E4M3 Q terms and E5M2 P terms (ones in E5M2)
+      constexpr uint32_t f16fmt = DT == LSE_KV_BF16 ? 1u : 0u;
+      constexpr uint32_t kvfmt = kF8 ? (kE5 ? 1u : 0u) : f16fmt;
+      constexpr uint32_t qfmt = kF8 ? 0u : f16fmt;
+      constexpr uint32_t pfmt = kF8 ? 1u : f16fmt;
+      constexpr uint32_t idesc_qk = instr_desc(kvfmt, qfmt, 0, 0, kTK, kNQ);
+      constexpr uint32_t idesc_pv = instr_desc(kvfmt, pfmt, 1, 1, kD, kN);
+      constexpr uint32_t idesc_l = instr_desc(pfmt, pfmt, 0, 1, kD, kN);
       const int n_total = (int)(t_stop - t_begin);
       TileIter iq, iv;
       iq.init(p, t_begin, t_stop, tab);
@@ -776,28 +845,43 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool first = iq.seg_start(t_begin);
           const int sq = first ? seg_q + 1 : seg_q;
           const int st = nq % NS;
-          if ((!first || mbar_test(bar(kBarQFull + sq % kQS), (sq / kQS) & 1)) &&
+          if ((!first || mbar_test(bar(kBarQFull + sq % QS), (sq / QS) & 1)) &&
               mbar_test(bar(kBarFullK + st), (nq / NS) & 1)) {
             seg_q = sq;
             tc_fence_after();
             const bool last = iq.seg_end();
             const uint32_t kaddr = k_base + st * Lay::kHalfStage;
-            const uint32_t qaddr = q_base + (seg_q % kQS) * Lay::kQBytes;
+            const uint32_t qaddr = q_base + (seg_q % QS) * Lay::kQBytes;
             const uint32_t d = tmem_s(nq & 1);
+            if constexpr (kF8) {
+              // one 128-dim region; K steps of 32 bytes; the Q terms add up
+              // in the same columns
 #pragma unroll
-            for (int k = 0; k < kD / 16; ++k) {
-              const uint64_t a = smem_desc(kaddr + (k >> 2) * kRegionBytes + (k & 3) * 32, 16,
-                                           1024, kLayoutSw128);
-              const uint32_t qoff = (k >> 2) * Lay::kQRegion + (k & 3) * 32;
-              const uint64_t bh = smem_desc(qaddr + qoff, 16, 1024, kLayoutSw128);
-              const uint64_t bl =
-                  smem_desc(qaddr + 2 * Lay::kQRegion + qoff, 16, 1024, kLayoutSw128);
-              mma_f16(d, a, bh, idesc_qk, k > 0);   // K Q_hi^T
-              mma_f16(d, a, bl, idesc_qk, 1u);      // + K Q_lo^T, same columns
+              for (int k = 0; k < kD / 32; ++k) {
+                const uint64_t a = smem_desc(kaddr + k * 32, 16, 1024, kLayoutSw128);
+#pragma unroll
+                for (int t = 0; t < kQTerms; ++t) {
+                  const uint64_t bq =
+                      smem_desc(qaddr + t * Lay::kQRegion + k * 32, 16, 1024, kLayoutSw128);
+                  mma_f8(d, a, bq, idesc_qk, (k | t) != 0);
+                }
+              }
+            } else {
+#pragma unroll
+              for (int k = 0; k < kD / 16; ++k) {
+                const uint64_t a = smem_desc(kaddr + (k >> 2) * kRegionBytes + (k & 3) * 32, 16,
+                                             1024, kLayoutSw128);
+                const uint32_t qoff = (k >> 2) * Lay::kQRegion + (k & 3) * 32;
+                const uint64_t bh = smem_desc(qaddr + qoff, 16, 1024, kLayoutSw128);
+                const uint64_t bl =
+                    smem_desc(qaddr + 2 * Lay::kQRegion + qoff, 16, 1024, kLayoutSw128);
+                mma_f16(d, a, bh, idesc_qk, k > 0);   // K Q_hi^T
+                mma_f16(d, a, bl, idesc_qk, 1u);      // + K Q_lo^T, same columns
+              }
             }
             mma_commit(bar(kBarEmptyK + st));
             mma_commit(bar(kBarSFull + (nq & 1)));
-            if (last) mma_commit(bar(kBarQEmpty + seg_q % kQS));
+            if (last) mma_commit(bar(kBarQEmpty + seg_q % QS));
             iq.advance(p);
             ++nq;
             did = true;
@@ -830,14 +914,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the ones operand is K-major without swizzle: 8x16-byte core
             // matrices, K blocks 128 B apart, row blocks 256 B apart
             const uint64_t a1 = smem_desc(ones_base, 128, 256, kLayoutNone);
+            if constexpr (kF8) {
+              // V^T is MN-major with one 128-byte swizzle atom across the
+              // dims; K steps of 32 keys; the P terms add up in the same
+              // columns
 #pragma unroll
-            for (int k = 0; k < kTK / 16; ++k) {
-              const uint64_t a = smem_desc(vaddr + k * 2048, kRegionBytes, 1024, kLayoutSw128);
-              const uint64_t b =
-                  smem_desc(paddr + k * 2 * Lay::kPLbo, Lay::kPLbo, 128, kLayoutNone);
-              const uint32_t acc = (grp_started[grp] || k > 0) ? 1u : 0u;
-              mma_f16(d, a, b, idesc_pv, acc);     // O^T += V^T P^T
-              mma_f16(dl, a1, b, idesc_l, acc);    // L += 1 P^T (row sums of P)
+              for (int k = 0; k < kTK / 32; ++k) {
+                const uint64_t a = smem_desc(vaddr + k * 4096, 0, 1024, kLayoutSw128);
+#pragma unroll
+                for (int t = 0; t < kPTerms; ++t) {
+                  const uint64_t b = smem_desc(paddr + t * Lay::kPTerm + k * 4 * Lay::kPLbo,
+                                               Lay::kPLbo, 128, kLayoutNone);
+                  const uint32_t acc = (grp_started[grp] || k > 0 || t > 0) ? 1u : 0u;
+                  mma_f8(d, a, b, idesc_pv, acc);     // O^T += V^T P_t^T
+                  mma_f8(dl, a1, b, idesc_l, acc);    // L += 1 P_t^T
+                }
+              }
+            } else {
+#pragma unroll
+              for (int k = 0; k < kTK / 16; ++k) {
+                const uint64_t a = smem_desc(vaddr + k * 2048, kRegionBytes, 1024, kLayoutSw128);
+                const uint64_t b =
+                    smem_desc(paddr + k * 2 * Lay::kPLbo, Lay::kPLbo, 128, kLayoutNone);
+                const uint32_t acc = (grp_started[grp] || k > 0) ? 1u : 0u;
+                mma_f16(d, a, b, idesc_pv, acc);     // O^T += V^T P^T
+                mma_f16(dl, a1, b, idesc_l, acc);    // L += 1 P^T (row sums of P)
+              }
             }
             grp_started[grp] = true;
             mma_commit(bar(kBarEmptyV + st));
@@ -880,7 +982,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (; it.valid(); it.advance(p)) {
       if (!it.seg_start(t_begin)) continue;
       ++seg;
-      const int slot = seg % kQS;
+      const int slot = seg % QS;
       const int P = G * it.R;
       // items (row n, 8-dim chunk c): every load of the segment in flight at
       // once, issued before waiting for the slot
@@ -900,23 +1002,58 @@ __global__ void __launch_bounds__(kThreads, 1)
           ld[k][0] = ld[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
-      if (!mbar_wait(bar(kBarQEmpty + slot), ((seg / kQS) & 1) ^ 1, abort_flag, p.err)) break;
+      if (!mbar_wait(bar(kBarQEmpty + slot), ((seg / QS) & 1) ^ 1, abort_flag, p.err)) break;
       uint8_t *qs = smem + (q_base - sbase) + slot * Lay::kQBytes;
+      const float sc = p.scale_log2;
+      if constexpr (kF8) {
+        // pair n's row scaled by 2^e (max |x| 2^e in [128, 256)), then
+        // written as kQTerms E4M3 terms, one 128-byte swizzled row per term;
+        // the 16 lanes holding a row find its maximum by shuffles
+        float *isig = isig_all + slot * 64;
 #pragma unroll
-      for (int k = 0; k < kItems; ++k) {
-        const int item = qt + 64 * k;
-        const int n = item >> 4, c = item & 15;
-        const float sc = p.scale_log2;
-        uint4 vh, vl;
-        split2<DT>(ld[k][0].x * sc, ld[k][0].y * sc, vh.x, vl.x);
-        split2<DT>(ld[k][0].z * sc, ld[k][0].w * sc, vh.y, vl.y);
-        split2<DT>(ld[k][1].x * sc, ld[k][1].y * sc, vh.z, vl.z);
-        split2<DT>(ld[k][1].z * sc, ld[k][1].w * sc, vh.w, vl.w);
-        const int region = c >> 3, cc = c & 7;
-        const uint32_t off = region * Lay::kQRegion + (n >> 3) * 1024 + (n & 7) * 128 +
-                             ((cc ^ (n & 7)) << 4);
-        *reinterpret_cast<uint4 *>(qs + off) = vh;
-        *reinterpret_cast<uint4 *>(qs + 2 * Lay::kQRegion + off) = vl;
+        for (int k = 0; k < kItems; ++k) {
+          const int item = qt + 64 * k;
+          const int n = item >> 4, c = item & 15;
+          float x[8] = {ld[k][0].x * sc, ld[k][0].y * sc, ld[k][0].z * sc, ld[k][0].w * sc,
+                        ld[k][1].x * sc, ld[k][1].y * sc, ld[k][1].z * sc, ld[k][1].w * sc};
+          float mx = 0.f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(x[i]));
+#pragma unroll
+          for (int o = 1; o < 16; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          int e = 0;
+          if (mx > 0.f && mx <= FLT_MAX) {
+            const int E = ((__float_as_int(mx) >> 23) & 0xff) - 127;
+            e = min(max(7 - E, -126), 126);
+          }
+          const float sg = exp2i(e);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) x[i] *= sg;
+          uint2 w[kQTerms];
+          f8_terms<false, kQTerms>(x, w);
+          const uint32_t off = (n >> 3) * 1024 + (n & 7) * 128 +
+                               ((((c >> 1) ^ (n & 7))) << 4) + (c & 1) * 8;
+#pragma unroll
+          for (int t = 0; t < kQTerms; ++t)
+            *reinterpret_cast<uint2 *>(qs + t * Lay::kQRegion + off) = w[t];
+          if (c == 0) isig[n] = exp2i(-e);
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < kItems; ++k) {
+          const int item = qt + 64 * k;
+          const int n = item >> 4, c = item & 15;
+          uint4 vh, vl;
+          split2<DT>(ld[k][0].x * sc, ld[k][0].y * sc, vh.x, vl.x);
+          split2<DT>(ld[k][0].z * sc, ld[k][0].w * sc, vh.y, vl.y);
+          split2<DT>(ld[k][1].x * sc, ld[k][1].y * sc, vh.z, vl.z);
+          split2<DT>(ld[k][1].z * sc, ld[k][1].w * sc, vh.w, vl.w);
+          const int region = c >> 3, cc = c & 7;
+          const uint32_t off = region * Lay::kQRegion + (n >> 3) * 1024 + (n & 7) * 128 +
+                               ((cc ^ (n & 7)) << 4);
+          *reinterpret_cast<uint4 *>(qs + off) = vh;
+          *reinterpret_cast<uint4 *>(qs + 2 * Lay::kQRegion + off) = vl;
+        }
       }
       fence_proxy_async();
       mbar_arrive(bar(kBarQFull + slot));
@@ -936,6 +1073,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *red = red_all + grp * 4 * 64;
     unsigned long long *masks = masks_all + grp * 64;
     float *scr = reinterpret_cast<float *>(smem + (p_base - sbase) + grp * Lay::kPBytes);
+    float *isg = isig_all + (2 + grp) * 64;    // FP8: the segment's inverse Q scales
+    // a score in log2 units from its TMEM value (FP8: undo Q's pair scale)
+    auto score = [&](float v, int q) { return kF8 ? v * isg[q] : v; };
     TileIter it;
     it.init(p, t_begin, t_stop, tab);
     int n = 0, seg = -1;
@@ -955,17 +1095,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           masks[j] = p.row_masks ? p.row_masks[it.row0 + j]
                                  : (j >= 63 ? ~0ull : ((1ull << (j + 1)) - 1ull));
         had_tile = false;
-        named_sync(bar_id, 128);
-      }
-      if ((n & 1) == grp) {
-        if (!mbar_wait(bar(kBarSFull + grp), (n >> 1) & 1, abort_flag, p.err)) {
+        bool w = true;
+        if constexpr (kF8) {
+          // the segment's Q scales: wait for its Q slot, keep a copy, then
+          // release the slot (with the score products)
+          const int qslot = seg % QS;
+          w = mbar_wait(bar(kBarQFull + qslot), (seg / QS) & 1, abort_flag, p.err);
+          if (w && j < P8) isg[j] = isig_all[qslot * 64 + j];
+        }
+        // every thread of the group leaves together when a wait gave up
+        if (named_or(bar_id, 128, !w)) {
           ok = false;
           break;
         }
+        if (kF8 && j == 0) mbar_arrive(bar(kBarQEmpty + seg % QS));
+      }
+      if ((n & 1) == grp) {
+        bool w = mbar_wait(bar(kBarSFull + grp), (n >> 1) & 1, abort_flag, p.err);
         tc_fence_after();
         // tile record, published by the producer on its own barrier (the
         // K ring may already hold a later tile)
-        if (!mbar_wait(bar(kBarInfo + (n & 7)), (n >> 3) & 1, abort_flag, p.err)) {
+        if (w) w = mbar_wait(bar(kBarInfo + (n & 7)), (n >> 3) & 1, abort_flag, p.err);
+        if (named_or(bar_id, 128, !w)) {
           ok = false;
           break;
         }
@@ -1000,7 +1151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_load<8>(s_addr + c, v);
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            if ((vis >> (c + i)) & 1ull) gap = fmaxf(gap, v[i] - m_run[c + i]);
+            if ((vis >> (c + i)) & 1ull) gap = fmaxf(gap, score(v[i], c + i) - m_run[c + i]);
         }
         if (named_or(bar_id, 128, gap > kTau)) {
           // per-pair maximum over the tile's keys, through this group's P tile
@@ -1012,7 +1163,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_load<8>(s_addr + c, v);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-              if (!((vis >> (c + i)) & 1ull)) v[i] = -INFINITY;
+              v[i] = ((vis >> (c + i)) & 1ull) ? score(v[i], c + i) : -INFINITY;
             *reinterpret_cast<float4 *>(scr + j * P8 + c) = make_float4(v[0], v[1], v[2], v[3]);
             *reinterpret_cast<float4 *>(scr + j * P8 + c + 4) =
                 make_float4(v[4], v[5], v[6], v[7]);
@@ -1034,10 +1185,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t ob = tmem_o(grp, oslot) + lane_off;
 #pragma unroll 1
             for (int c = 0; c < 2 * kN; c += 8) {
+              const int cc = c % kN;
+              if (kF8 && cc >= P8) continue;  // padding columns
               float v[8];
               tmem_load<8>(ob + c, v);
-              const int cc = c % kN;
-              const int q0 = cc < P8 ? cc : cc - P8;
+              const int q0 = kF8 ? cc : cc < P8 ? cc : cc - P8;
 #pragma unroll
               for (int i = 0; i < 8; ++i) v[i] *= alpha[q0 + i];
               tmem_st8(ob + c, v);
@@ -1045,7 +1197,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st_wait();
           }
         }
-        // pass 2: probabilities -> this group's P tile, row j: hi then lo columns
+        // pass 2: probabilities -> this group's P tile, row j (16-bit: hi then
+        // lo columns; FP8: P 2^7 as kPTerms E5M2 terms, one block per term)
         uint8_t *prow = smem + (p_base - sbase) + grp * Lay::kPBytes + (j >> 3) * Lay::kPLbo +
                         (j & 7) * 16;
 #pragma unroll 1
@@ -1055,21 +1208,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           float e[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            e[i] = ((vis >> (c + i)) & 1ull) ? ex2(v[i] - m_run[c + i]) : 0.f;
-          uint4 vh, vl;
-          split2<DT>(e[0], e[1], vh.x, vl.x);
-          split2<DT>(e[2], e[3], vh.y, vl.y);
-          split2<DT>(e[4], e[5], vh.z, vl.z);
-          split2<DT>(e[6], e[7], vh.w, vl.w);
-          *reinterpret_cast<uint4 *>(prow + (c >> 3) * 128) = vh;
-          *reinterpret_cast<uint4 *>(prow + ((P8 + c) >> 3) * 128) = vl;
+            e[i] = ((vis >> (c + i)) & 1ull) ? ex2(score(v[i], c + i) - m_run[c + i]) : 0.f;
+          if constexpr (kF8) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) e[i] *= (float)(1 << kPScaleLog2);
+            uint2 w[kPTerms];
+            f8_terms<true, kPTerms>(e, w);
+            uint8_t *dst = prow + (c >> 4) * 128 + ((c >> 3) & 1) * 8;
+#pragma unroll
+            for (int t = 0; t < kPTerms; ++t)
+              *reinterpret_cast<uint2 *>(dst + t * Lay::kPTerm) = w[t];
+          } else {
+            uint4 vh, vl;
+            split2<DT>(e[0], e[1], vh.x, vl.x);
+            split2<DT>(e[2], e[3], vh.y, vl.y);
+            split2<DT>(e[4], e[5], vh.z, vl.z);
+            split2<DT>(e[6], e[7], vh.w, vl.w);
+            *reinterpret_cast<uint4 *>(prow + (c >> 3) * 128) = vh;
+            *reinterpret_cast<uint4 *>(prow + ((P8 + c) >> 3) * 128) = vl;
+          }
         }
         if (!kvalid) {
           // a dead slot may hold any bits: give it a zero V row (P is 0 there)
           mbar_wait(bar(kBarFullV + n % NS), (n / NS) & 1, abort_flag, p.err);
           uint8_t *v0 = smem + (v_base - sbase) + (n % NS) * Lay::kHalfStage + j * 128;
+          constexpr int kChunks = kF8 ? 8 : 16;  // 16-byte chunks of the row
 #pragma unroll 1
-          for (int c = 0; c < 16; ++c)
+          for (int c = 0; c < kChunks; ++c)
             *reinterpret_cast<uint4 *>(v0 + (c >> 3) * kRegionBytes + (c & 7) * 16) =
                 make_uint4(0, 0, 0, 0);
         }
@@ -1081,7 +1246,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       if (last) {
         // ---- epilogue of this group's piece: normalised output and log2-sum-exp ----
-        if (!mbar_wait(bar(kBarOFull + 2 * grp + oslot), (seg / kOS) & 1, abort_flag, p.err)) {
+        const bool w = mbar_wait(bar(kBarOFull + 2 * grp + oslot), (seg / kOS) & 1, abort_flag,
+                                 p.err);
+        if (named_or(bar_id, 128, !w)) {
           ok = false;
           break;
         }
@@ -1101,9 +1268,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           float lh[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, ll[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
           if (had_tile) {
             tmem_load<8>(ob + c, oh);
-            tmem_load<8>(ob + P8 + c, ol);
             tmem_load<8>(lb + c, lh);
-            tmem_load<8>(lb + P8 + c, ll);
+            if constexpr (!kF8) {
+              tmem_load<8>(ob + P8 + c, ol);
+              tmem_load<8>(lb + P8 + c, ll);
+            }
           }
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
@@ -1114,7 +1283,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                   base + r * row_stride / kD + (long long)(q - r * G) * tp.n_slots;
               const float lt = lh[i] + ll[i];
               p.o_part[idx * kD + d] = lt > 0.f ? (oh[i] + ol[i]) * rcp(lt) : 0.f;
-              if (d == q) p.lse_part[idx] = lt > 0.f ? m_run[q] + lg2(lt) : -INFINITY;
+              // (FP8 sums carry P's factor 2^7)
+              if (d == q)
+                p.lse_part[idx] = lt > 0.f ? m_run[q] + lg2(lt) - (kF8 ? kPScaleLog2 : 0)
+                                           : -INFINITY;
             }
           }
         }
@@ -1177,15 +1349,22 @@ int launch_tc_p(const TcParams &tp, int p8, int smem, cudaStream_t st) {
   return (int)cudaErrorInvalidValue;
 }
 
-int smem_for(int p8, int stages) {
+template <int DT>
+int smem_for_p(int p8, int stages, int q_slots) {
   switch (p8) {
-    case 8: return TcLayout<8>::smem_bytes(stages);
-    case 16: return TcLayout<16>::smem_bytes(stages);
-    case 24: return TcLayout<24>::smem_bytes(stages);
-    case 32: return TcLayout<32>::smem_bytes(stages);
-    case 48: return TcLayout<48>::smem_bytes(stages);
+    case 8: return TcLayout<DT, 8>::smem_bytes(stages, q_slots);
+    case 16: return TcLayout<DT, 16>::smem_bytes(stages, q_slots);
+    case 24: return TcLayout<DT, 24>::smem_bytes(stages, q_slots);
+    case 32: return TcLayout<DT, 32>::smem_bytes(stages, q_slots);
+    case 48: return TcLayout<DT, 48>::smem_bytes(stages, q_slots);
   }
   return -1;
+}
+
+int smem_for(int dtype, int p8, int stages, int q_slots) {
+  // the two 16-bit formats share a layout, and so do the two 8-bit ones
+  return is_f8(dtype) ? smem_for_p<LSE_KV_FP8_E4M3>(p8, stages, q_slots)
+                      : smem_for_p<LSE_KV_BF16>(p8, stages, q_slots);
 }
 
 }  // namespace
@@ -1199,34 +1378,43 @@ int lse_tc_pairs_bucket(int pairs) {
   return -1;
 }
 
-int lse_tc_smem(int p8, int smem_optin, int *stages) {
-  int best = -1;
-  for (int ns = 2; ns <= 4; ++ns) {
-    const int b = smem_for(p8, ns);
-    if (b > 0 && b <= smem_optin) {
-      best = b;
-      *stages = ns;
+// The deepest K/V ring that fits (stages count more than a second Q slot,
+// which only overlaps Q staging with the end of the previous segment).
+int lse_tc_smem(int dtype, int p8, int smem_optin, int *stages, int *q_slots) {
+  for (int ns = kMaxStages; ns >= 2; --ns)
+    for (int qs = 2; qs >= 1; --qs) {
+      const int b = smem_for(dtype, p8, ns, qs);
+      if (b > 0 && b <= smem_optin) {
+        *stages = ns;
+        *q_slots = qs;
+        return b;
+      }
     }
-  }
-  return best;
+  return -1;
 }
 
 int lse_tc_key_tile() { return kTK; }
 
 int lse_tc_build_maps(const uint64_t *chunk_base, int n_chunks, size_t chunk_bytes,
-                      int n_kv_heads, int box_tokens, void *maps_out) {
+                      int n_kv_heads, int dtype, int box_tokens, void *maps_out) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode();
   if (!enc) return (int)cudaErrorNotSupported;
   if (n_chunks > LSE_MAX_TMA_CHUNKS) return (int)cudaErrorInvalidValue;
   CUtensorMap *maps = static_cast<CUtensorMap *>(maps_out);
-  const uint64_t row = (uint64_t)n_kv_heads * kD * 2;  // bytes per token, all kv heads
+  // a chunk as [tokens][rows][128 bytes]: 16-bit K/V give two 64-dim rows
+  // per kv head, FP8 one 128-dim row
+  const bool f8 = is_f8(dtype);
+  const int esize = f8 ? 1 : 2;
+  const int rows_per_head = f8 ? 1 : 2;
+  const uint64_t row = (uint64_t)n_kv_heads * kD * esize;  // bytes per token, all kv heads
   for (int c = 0; c < n_chunks; ++c) {
-    cuuint64_t dims[3] = {64, (cuuint64_t)n_kv_heads * 2, (cuuint64_t)(chunk_bytes / row)};
+    cuuint64_t dims[3] = {(cuuint64_t)(128 / esize), (cuuint64_t)n_kv_heads * rows_per_head,
+                          (cuuint64_t)(chunk_bytes / row)};
     cuuint64_t strides[2] = {128, row};
-    cuuint32_t box[3] = {64, 1, (cuuint32_t)box_tokens};
+    cuuint32_t box[3] = {(cuuint32_t)(128 / esize), 1, (cuuint32_t)box_tokens};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = enc(&maps[c], CU_TENSOR_MAP_DATA_TYPE_UINT16, 3,
-                     reinterpret_cast<void *>(chunk_base[c]), dims, strides, box, estr,
+    CUresult r = enc(&maps[c], f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16,
+                     3, reinterpret_cast<void *>(chunk_base[c]), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return (int)cudaErrorInvalidValue;
@@ -1238,7 +1426,7 @@ size_t lse_tc_map_bytes() { return sizeof(CUtensorMap); }
 
 int lse_launch_partial_tcgen05(const LseKernelParams &p, const void *maps, int n_maps,
                                int dtype, int p8, int n_ctas, int n_slots, int stages,
-                               int box_tokens, int smem, void *stream) {
+                               int q_slots, int box_tokens, int smem, void *stream) {
   static_assert(sizeof(TcParams) < 30000, "kernel parameter block too large");
   TcParams tp;
   memset(&tp, 0, sizeof tp);
@@ -1247,11 +1435,14 @@ int lse_launch_partial_tcgen05(const LseKernelParams &p, const void *maps, int n
   tp.n_ctas = n_ctas;
   tp.n_slots = n_slots;
   tp.stages = stages;
+  tp.q_slots = q_slots;
   tp.box_tokens = box_tokens;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   switch (dtype) {
     case LSE_KV_BF16: return launch_tc_p<LSE_KV_BF16>(tp, p8, smem, st);
     case LSE_KV_F16: return launch_tc_p<LSE_KV_F16>(tp, p8, smem, st);
+    case LSE_KV_FP8_E4M3: return launch_tc_p<LSE_KV_FP8_E4M3>(tp, p8, smem, st);
+    case LSE_KV_FP8_E5M2: return launch_tc_p<LSE_KV_FP8_E5M2>(tp, p8, smem, st);
   }
   return (int)cudaErrorInvalidValue;
 }
