@@ -22,10 +22,13 @@
 //  * Scores are computed transposed, S^T = K Q^T (M = 128 keys, N = pairs),
 //    so the tile's keys fill the 128-row MMA whatever the number of query
 //    rows; the output is O^T = V^T P^T (M = 128 dims).  Both accumulate in
-//    TMEM in FP32.  Q and P carry a hi + lo pair of 16-bit terms (one term
-//    holds the value rounded to the storage's 16-bit format, the other the
-//    rounding error) so the products keep ~16 mantissa bits and only the
-//    K/V storage rounding remains.
+//    TMEM in FP32.  With 16-bit K/V, Q and P carry a hi + lo pair of 16-bit
+//    terms (one term holds the value rounded to the storage's 16-bit format,
+//    the other the rounding error) so the products keep ~16 mantissa bits
+//    and only the K/V storage rounding remains.  With FP8 K/V the tiles
+//    enter kind::f8f6f4 products as loaded: Q as four E4M3 terms under a
+//    per-pair power-of-2 scale, P (times 2^7) as four E5M2 terms, each term
+//    holding the rounding error of the ones before it.
 //  * Softmax: two warpgroups take alternate tiles (ping-pong), each with
 //    its own score buffer in TMEM, its own P tile in shared memory and its
 //    own output accumulator, so one group's exponentials overlap the other
@@ -35,11 +38,17 @@
 //    lazily: only when a score exceeds it by more than 2^8 are the maxima
 //    recomputed and the group's TMEM output rescaled.
 //  * K and V sit in separate rings, so a K slot is refilled as soon as its
-//    score product is done, and the score products run two tiles ahead of
-//    the output products.
+//    score product is done.  A group's next score product waits only for
+//    the group's softmax to finish reading its score buffer, and its next
+//    softmax pass only for the output product that read its P tile.
+//  * Each product issues one MMA per K step with all operand terms side by
+//    side along N (an MMA costs its issuing thread the same whatever its
+//    N), and the two products are issued by two threads; the row sums of P
+//    are summed by the softmax warps.
 //
-// Roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer (and TMEM
-// owner), warps 2-3 stage Q, warps 4-7 and 8-11 the two softmax groups.
+// Roles (384 threads): warp 0 TMA producer, warp 1 score-product issuer
+// (and TMEM owner), warp 2 output-product issuer, warp 3 stages Q, warps 4-7
+// and 8-11 the two softmax groups.
 // Every wait is bounded: a wait that runs out sets LSE_DEVERR_TIMEOUT and
 // every role leaves its loop; TMEM is released and outstanding copies are
 // drained before the CTA exits.
@@ -116,11 +125,10 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase of `bar` with the given parity; false when the wait ran
-// out (then the CTA-wide abort flag is set) or another role aborted.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                       unsigned int *err) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Slow path of mbar_wait (out of line: it runs only when the phase is not
+// complete at the first test).
+__device__ __noinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity,
+                                            volatile int *abort_flag, unsigned int *err) {
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -133,6 +141,13 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile i
       }
     }
   }
+}
+
+// Wait for the phase of `bar` with the given parity; false when the wait ran
+// out (then the CTA-wide abort flag is set) or another role aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                          unsigned int *err) {
+  return mbar_try_wait(bar, parity) || mbar_wait_spin(bar, parity, abort_flag, err);
 }
 
 // Time-bounded wait that ignores the abort flag: used to drain copies and
@@ -276,7 +291,7 @@ struct TileIter {
     }
     return seq_tiles(p, q, L, row0, R);
   }
-  __device__ __noinline__ void next_seq(const LseKernelParams &p) {
+  __device__ __forceinline__ void next_seq(const LseKernelParams &p) {
     // advance to the next sequence with tiles, starting at s
     while (s < p.n_seqs) {
       const int n = tiles_of(p, s);
@@ -287,8 +302,8 @@ struct TileIter {
       ++s;
     }
   }
-  __device__ __noinline__ void init(const LseKernelParams &p, long long t_begin,
-                                    long long t_stop, const SeqRec *table) {
+  __device__ __forceinline__ void init(const LseKernelParams &p, long long t_begin,
+                                       long long t_stop, const SeqRec *table) {
     t = t_begin;
     t_end = t_stop;
     tab = table;
@@ -346,16 +361,16 @@ __device__ __forceinline__ int cta_of_tile(long long t, long long U, int C) {
 
 // Fragment ids of the boxes of one tile (-1: past the sequence, -2: names
 // no fragment, flagged).
-__device__ __noinline__ void load_page_ids(const LseKernelParams &p, const TileIter &it, int nbox,
-                                           int box_t, int *pk, int *pv) {
-  const int key0 = it.tile * kTK;
+__device__ __noinline__ void load_page_ids(const LseKernelParams &p, int seq, int tile, int L,
+                                           int nbox, int box_t, int *pk, int *pv) {
+  const int key0 = tile * kTK;
   const int T = p.tokens_per_fragment;
 #pragma unroll 1
   for (int b = 0; b < nbox; ++b) {
     const int kb = key0 + b * box_t;
     int fk = -1, fv = -1;
-    if (kb < it.L) {
-      const long long e = (long long)it.s * p.max_pages + kb / T;
+    if (kb < L) {
+      const long long e = (long long)seq * p.max_pages + kb / T;
       fk = p.k_pages[e];
       fv = p.v_pages[e];
       const bool bk = fk < 0 || fk >= p.n_fragments, bv = fv < 0 || fv >= p.n_fragments;
@@ -371,7 +386,7 @@ __device__ __noinline__ void load_page_ids(const LseKernelParams &p, const TileI
 // TMA boxes of one tile (K or V): fragment ids ids[0..nbox), into dst.  A
 // 16-bit tile is two regions of 64 dims (tensor rows 2g and 2g + 1); an
 // FP8 tile is one region of 128 dims (tensor row g).
-__device__ __noinline__ void load_boxes(const TcParams &tp, int nbox, int box_t, int regions,
+__device__ __forceinline__ void load_boxes(const TcParams &tp, int nbox, int box_t, int regions,
                                         int g, int key0, const int *ids, uint32_t dst,
                                         uint32_t full_bar) {
   const LseKernelParams &p = tp.p;
@@ -392,12 +407,12 @@ __device__ __noinline__ void load_boxes(const TcParams &tp, int nbox, int box_t,
 
 // Producer work for tile n: K slot, tile record, K boxes, V slot, V boxes.
 // Returns 0 when a wait gave up.
-__device__ __noinline__ int produce_tile(const TcParams &tp, int n, int NS, int nbox, int box_t,
-                                         int regions, int g, int tile, int L, const int *pk,
-                                         const int *pv,
-                                         uint32_t kdst, uint32_t vdst, const uint32_t *bars_k,
-                                         const uint32_t *bars_v, uint32_t info_bar,
-                                         uint4 *info, volatile int *abort_flag) {
+__device__ __forceinline__ int produce_tile(const TcParams &tp, int n, int NS, int nbox,
+                                            int box_t, int regions, int g, int tile, int L,
+                                            const int *pk, const int *pv, uint32_t kdst,
+                                            uint32_t vdst, const uint32_t *bars_k,
+                                            const uint32_t *bars_v, uint32_t info_bar,
+                                            uint4 *info, volatile int *abort_flag) {
   const LseKernelParams &p = tp.p;
   const uint32_t ph = ((n / NS) & 1) ^ 1;
   const int key0 = tile * kTK;
@@ -411,8 +426,9 @@ __device__ __noinline__ int produce_tile(const TcParams &tp, int n, int NS, int 
   const uint32_t box_bytes = (uint32_t)regions * (uint32_t)box_t * 128u;
   if (!mbar_wait(bars_k[0], ph, abort_flag, p.err)) return 0;
   // the record slot was last read by the softmax of tile n - 8, which has
-  // finished: this producer passed its K slot wait for tile n, which
-  // follows the output product of tile n + 6 - NS >= n - 6
+  // finished: the K slot of tile n was freed by the score product of tile
+  // n - NS, issued in order after the softmax of tiles up to n - NS - 2
+  // (>= n - 8 for NS <= 6) released their score buffers
   *info = make_uint4(kmask, vmask, (uint32_t)live, 0u);
   mbar_arrive(info_bar);  // publishes the record
   mbar_expect_tx(bars_k[1], (uint32_t)__popc(kmask) * box_bytes);
@@ -471,37 +487,50 @@ constexpr int kPScaleLog2 = 7;     // P enters the FP8 products times 2^7
 template <int DT, int P8>
 struct TcLayout {
   static constexpr bool kF8 = is_f8(DT);
-  static constexpr int kNQ = (P8 + 15) / 16 * 16;       // score columns (N of S^T)
-  // output columns: 16-bit K/V keep hi | lo probability columns side by side;
-  // FP8 accumulates its probability terms into the same columns
-  static constexpr int kN = kF8 ? kNQ : 2 * P8;
+  static constexpr int kNQ = (P8 + 15) / 16 * 16;       // pairs rounded to 16 (MMA N step)
+  // Every product carries its operand terms side by side along N, so one
+  // MMA per K step covers them all (the issue of an MMA costs the same
+  // whatever its N).  Score columns per group: 16-bit, Q hi | Q lo blocks of
+  // kNQ; FP8, four Q-term blocks of kNQ.
+  static constexpr int kSW = kF8 ? kQTerms * kNQ : 2 * kNQ;
+  // Output columns per group and slot: 16-bit, P hi | P lo blocks of P8;
+  // FP8, four P-term blocks of kNQ when they fit in TMEM, else one block
+  // that the four terms accumulate into (four MMAs per K step)
+  static constexpr bool kPSide = !kF8 || 4 * kSW <= 256;
+  static constexpr int kOBlk = kF8 ? kNQ : P8;            // width of one output block
+  static constexpr int kN = kF8 ? (kPSide ? kPTerms * kNQ : kNQ) : 2 * P8;
   static constexpr int kQRegion = kNQ * 128;             // kNQ rows of 128 bytes
-  // 16-bit: hi (2 regions of 64 dims) + lo (2 regions); FP8: kQTerms regions
+  // 16-bit: two 64-dim regions, each [hi rows | lo rows]; FP8: one 128-dim
+  // region of kQTerms x kNQ rows
   static constexpr int kQBytes = 4 * kQRegion;
   static_assert(!kF8 || kQTerms == 4, "Q slot holds four FP8 terms");
-  // P: 16-bit, 8x16-byte core matrices of 8 keys x 8 pairs; FP8, one
-  // block per term of 8 keys x 16 pairs core matrices
-  static constexpr int kPLbo = kF8 ? (kNQ / 16) * 128 : (kN / 8) * 128;  // 8-key group stride
-  static constexpr int kPTerm = kTK * kNQ;               // FP8: bytes of one P term
-  static constexpr int kPBytes = kF8 ? kPTerms * kPTerm : kTK * kN * 2;  // one group's P
-  static constexpr int kOnesBytes = 4096;                // ones operand: 128 rows x 32 bytes
-  // TMEM: S per group, then per group and output slot the output O^T and the
-  // row sums L (both kN columns); two output slots when they fit
-  static constexpr int kOSlots = (2 * kNQ + 8 * kN <= 512) ? 2 : 1;
-  static constexpr int kTmemNeed = 2 * kNQ + 4 * kOSlots * kN;
+  // P^T operand, MN-major without swizzle: core matrices of 8 keys x 16
+  // bytes (8 16-bit or 16 FP8 columns); 8-key groups kPLbo apart; columns
+  // hi block then lo block (16-bit) or term blocks of kNQ (FP8)
+  static constexpr int kPCols = kF8 ? kPTerms * kNQ : 2 * P8;
+  static constexpr int kPLbo = (kF8 ? kPCols / 16 : kPCols / 8) * 128;
+  static constexpr int kPBytes = kTK / 8 * kPLbo;        // one group's P tile
+  // TMEM: S per group, then per group and output slot O^T (kN columns);
+  // two output slots when they fit
+  static constexpr int kOSlots = (2 * kSW + 4 * kN <= 512) ? 2 : 1;
+  static constexpr int kTmemNeed = 2 * kSW + 2 * kOSlots * kN;
   static constexpr int kTmemCols = kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                  : kTmemNeed <= 256 ? 256 : 512;
   static_assert(kTmemNeed <= 512, "TMEM holds at most 512 columns");
+  static_assert(kSW <= 256 && kN <= 256, "MMA N is at most 256");
   static constexpr int kBars = 64;
+  // row sums of P per group [2][64] and their per-warp partials
+  // [2 groups][2 buffers][4 warps][P8]
+  static constexpr int kLBytes = 2 * 64 * 4 + 2 * 2 * 4 * P8 * 4;
   static constexpr int kMiscBytes = kBars * 8 + 16 + 2 * 64 * 4 * 2 + 2 * 4 * 64 * 4 +
                                     2 * 64 * 8 + 64 * 4 + 8 * 16 + 2 * 32 * 16 * 4 +
-                                    (kF8 ? 4 * 64 * 4 : 0) + kSeqTab * (int)sizeof(SeqRec);
+                                    (kF8 ? 4 * 64 * 4 : 0) + kLBytes +
+                                    kSeqTab * (int)sizeof(SeqRec);
   // one K or V tile: 128 keys of 128 dims (two 64-dim regions when 16-bit)
   static constexpr int kHalfStage = kF8 ? kRegionBytes : 2 * kRegionBytes;
   // stages: K/V ring depth; q_slots: Q ring depth (1 or 2)
   static int smem_bytes(int stages, int q_slots) {
-    return 1024 + stages * 2 * kHalfStage + q_slots * kQBytes + 2 * kPBytes + kOnesBytes +
-           kMiscBytes;
+    return 1024 + stages * 2 * kHalfStage + q_slots * kQBytes + 2 * kPBytes + kMiscBytes;
   }
 };
 
@@ -518,8 +547,10 @@ enum {
   kBarQEmpty = 38,  // [2]
   kBarOFull = 40,   // [4] = group * 2 + slot
   kBarOEmpty = 44,  // [4]
-  kBarDone = 48,
+  kBarDone = 48,     // the score issuer's MMAs have completed
   kBarInfo = 49,    // [8] one per tile record
+  kBarPEmpty = 57,  // [2] per softmax group: its P tile has been read
+  kBarDoneV = 59,   // the output issuer's MMAs have completed
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -595,6 +626,38 @@ __device__ __forceinline__ void f8_terms(float *x, uint2 *out) {
   }
 }
 
+// Eight FP32 values -> F16 (round to nearest), then kTerms E5M2 terms of
+// the F16 values: every E5M2 value is an F16 value, so each remainder is an
+// exact F16 subtraction, and four terms of 3 significant bits hold all 11
+// bits of an F16.  Also returns the F16-rounded values as FP32.
+template <int kTerms>
+__device__ __forceinline__ void e5_terms_f16(const float *x, uint2 *out, float *rounded) {
+  uint32_t h[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h[i]) : "f"(x[2 * i + 1]), "f"(x[2 * i]));
+    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h[i]));
+    rounded[2 * i] = f.x;
+    rounded[2 * i + 1] = f.y;
+  }
+#pragma unroll
+  for (int t = 0; t < kTerms; ++t) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint16_t r;
+      asm("cvt.rn.satfinite.e5m2x2.f16x2 %0, %1;" : "=h"(r) : "r"(h[i]));
+      w[i] = r;
+      if (t + 1 < kTerms) {
+        uint32_t d;
+        asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(d) : "h"(r));
+        asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(h[i]) : "r"(h[i]), "r"(d));
+      }
+    }
+    out[t] = make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+  }
+}
+
 // 2^e as a float, e in [-126, 127].
 __device__ __forceinline__ float exp2i(int e) { return __int_as_float((e + 127) << 23); }
 
@@ -621,6 +684,139 @@ __device__ __forceinline__ void tmem_load(uint32_t taddr, float *v) {
   }
 }
 
+// TMEM: this thread's lane, 8 columns from each of T blocks `stride`
+// columns apart, summed in block order; one wait for all loads.
+template <int T>
+__device__ __forceinline__ void tmem_load_sum8(uint32_t taddr, int stride, float *v) {
+  uint32_t r[T][8];
+#pragma unroll
+  for (int t = 0; t < T; ++t)
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+        : "=r"(r[t][0]), "=r"(r[t][1]), "=r"(r[t][2]), "=r"(r[t][3]), "=r"(r[t][4]),
+          "=r"(r[t][5]), "=r"(r[t][6]), "=r"(r[t][7])
+        : "r"(taddr + (uint32_t)(t * stride))
+        : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int t = 0; t < T; ++t)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) asm volatile("" : "+r"(r[t][c]) :: "memory");
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float a = __uint_as_float(r[0][c]);
+#pragma unroll
+    for (int t = 1; t < T; ++t) a += __uint_as_float(r[t][c]);
+    v[c] = a;
+  }
+}
+
+// Sum of eight per-lane values over the 32 lanes of a warp, by a fixed
+// butterfly (halving the values each lane keeps, then full sums): every
+// lane returns the warp sum of value (lane >> 2).
+__device__ __forceinline__ float warp_sum8(const float *e, int lane) {
+  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+  float w4[4], w2[2];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float keep = b4 ? e[4 + i] : e[i], give = b4 ? e[i] : e[4 + i];
+    w4[i] = keep + __shfl_xor_sync(0xffffffffu, give, 16);
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float keep = b3 ? w4[2 + i] : w4[i], give = b3 ? w4[i] : w4[2 + i];
+    w2[i] = keep + __shfl_xor_sync(0xffffffffu, give, 8);
+  }
+  float x = (b2 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? w2[0] : w2[1], 4);
+  x += __shfl_xor_sync(0xffffffffu, x, 2);
+  x += __shfl_xor_sync(0xffffffffu, x, 1);
+  return x;
+}
+
+// Stage one segment's Q into a Q slot, by T threads (t = 0 .. T-1): each
+// (pair row n, 8-dim chunk c) item is scaled by the softmax scale (log2
+// units) and written in the operand layout of the score product.  Item
+// t + T k goes to thread t, so the 16 lanes of a half warp hold one row.
+// Items go in rounds of up to 8 per thread; the first round's loads are
+// issued before `before_store` (the wait for the slot) runs.  FP8: each row
+// is scaled by 2^e (max |x| 2^e in [128, 256)) and written as kQTerms E4M3
+// terms; 2^-e goes to isig[n].
+template <int DT, int P8, int T, class Wait>
+__device__ __forceinline__ bool stage_q(const LseKernelParams &p, int t, int g, int row0, int P,
+                                        uint8_t *qs, float *isig, Wait before_store) {
+  using Lay = TcLayout<DT, P8>;
+  constexpr int kNQ = Lay::kNQ;
+  constexpr int kItems = kNQ * 16 / T;
+  constexpr int kRound = kItems < 8 ? kItems : 8;
+  static_assert(kItems * T == kNQ * 16, "items split evenly");
+  const int G = p.group;
+  const float sc = p.scale_log2;
+#pragma unroll 1
+  for (int r0 = 0; r0 < kItems; r0 += kRound) {
+    float4 ld[kRound][2];
+#pragma unroll
+    for (int k = 0; k < kRound; ++k) {
+      const int item = t + T * (r0 + k);
+      const int n = item >> 4, c = item & 15;
+      if (n < P) {
+        const int r = n / G, h = g * G + (n - r * G);
+        const float4 *src = reinterpret_cast<const float4 *>(
+            p.q + ((long long)(row0 + r) * p.n_q_heads + h) * kD + c * 8);
+        ld[k][0] = __ldg(src);
+        ld[k][1] = __ldg(src + 1);
+      } else {
+        ld[k][0] = ld[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    if (r0 == 0 && !before_store()) return false;
+#pragma unroll
+    for (int k = 0; k < kRound; ++k) {
+      const int item = t + T * (r0 + k);
+      const int n = item >> 4, c = item & 15;
+      float x[8] = {ld[k][0].x * sc, ld[k][0].y * sc, ld[k][0].z * sc, ld[k][0].w * sc,
+                    ld[k][1].x * sc, ld[k][1].y * sc, ld[k][1].z * sc, ld[k][1].w * sc};
+      if constexpr (Lay::kF8) {
+        float mx = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(x[i]));
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        int e = 0;
+        if (mx > 0.f && mx <= FLT_MAX) {
+          const int E = ((__float_as_int(mx) >> 23) & 0xff) - 127;
+          e = min(max(7 - E, -126), 126);
+        }
+        const float sg = exp2i(e);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] *= sg;
+        uint2 w[kQTerms];
+        f8_terms<false, kQTerms>(x, w);
+        // one 128-byte swizzled row per term
+        const uint32_t off =
+            (n >> 3) * 1024 + (n & 7) * 128 + ((((c >> 1) ^ (n & 7))) << 4) + (c & 1) * 8;
+#pragma unroll
+        for (int tt = 0; tt < kQTerms; ++tt)
+          *reinterpret_cast<uint2 *>(qs + tt * Lay::kQRegion + off) = w[tt];
+        if (c == 0) isig[n] = exp2i(-e);
+      } else {
+        uint4 vh, vl;
+        split2<DT>(x[0], x[1], vh.x, vl.x);
+        split2<DT>(x[2], x[3], vh.y, vl.y);
+        split2<DT>(x[4], x[5], vh.z, vl.z);
+        split2<DT>(x[6], x[7], vh.w, vl.w);
+        // region (64 dims) of 2 kNQ rows: hi rows, then lo rows
+        const int region = c >> 3, cc = c & 7;
+        const uint32_t off = region * 2 * Lay::kQRegion + (n >> 3) * 1024 + (n & 7) * 128 +
+                             ((cc ^ (n & 7)) << 4);
+        *reinterpret_cast<uint4 *>(qs + off) = vh;
+        *reinterpret_cast<uint4 *>(qs + Lay::kQRegion + off) = vl;
+      }
+    }
+  }
+  fence_proxy_async();  // the score product reads Q through the async proxy
+  return true;
+}
+
 template <int DT, int P8>
 __global__ void __launch_bounds__(kThreads, 1)
     partial_tcgen05_kernel(const __grid_constant__ TcParams tp) {
@@ -643,8 +839,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t v_base = k_base + NS * Lay::kHalfStage;        // V ring
   const uint32_t q_base = v_base + NS * Lay::kHalfStage;        // Q slots
   const uint32_t p_base = q_base + QS * Lay::kQBytes;          // P tiles (one per group)
-  const uint32_t ones_base = p_base + 2 * Lay::kPBytes;         // ones operand of the sums
-  uint8_t *misc = smem + (ones_base - sbase) + Lay::kOnesBytes;
+  uint8_t *misc = smem + (p_base - sbase) + 2 * Lay::kPBytes;
   uint64_t *bars = reinterpret_cast<uint64_t *>(misc);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + Lay::kBars * 8);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + Lay::kBars * 8 + 4);
@@ -663,7 +858,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // FP8: the inverse of Q's per-pair scale, per Q slot [0, 2) and the
   // copy each softmax group keeps for its segment [2, 4)
   float *isig_all = reinterpret_cast<float *>(page_buf + 2 * 32 * 16);       // [4][64]
-  SeqRec *seq_tab = reinterpret_cast<SeqRec *>(isig_all + (kF8 ? 4 * 64 : 0)); // [kSeqTab]
+  // row sums of P per softmax group, and each warp's partial sums of the
+  // group's latest tile (double buffered)
+  float *lsum_all = isig_all + (kF8 ? 4 * 64 : 0);                           // [2][64]
+  float *lpart_all = lsum_all + 2 * 64;                                      // [2][2][4][P8]
+  SeqRec *seq_tab = reinterpret_cast<SeqRec *>(lpart_all + 2 * 2 * 4 * P8);  // [kSeqTab]
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
   // the merge pass may be scheduled now; it waits for this grid to finish
@@ -720,25 +919,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarSFull + i), 1);
       mbar_init(bar(kBarPFull + i), 128);
-      mbar_init(bar(kBarQFull + i), 64);
+      mbar_init(bar(kBarQFull + i), 1);
       // FP8: the softmax groups also hold the slot until they have copied
       // the segment's Q scales
       mbar_init(bar(kBarQEmpty + i), kF8 ? 3 : 1);
     }
     mbar_init(bar(kBarDone), 1);
+    mbar_init(bar(kBarDoneV), 1);
     for (int i = 0; i < 8; ++i) mbar_init(bar(kBarInfo + i), 1);
+    for (int i = 0; i < 2; ++i) mbar_init(bar(kBarPEmpty + i), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (tid < 64) pair_row[tid] = tid / p.group;
-  {
-    // the ones operand: 1.0 in the format of P (E5M2 for FP8 K/V, else the
-    // storage's 16-bit format)
-    const uint32_t one2 = kF8 ? 0x3C3C3C3Cu : DT == LSE_KV_BF16 ? 0x3F803F80u : 0x3C003C00u;
-    uint4 *ones = reinterpret_cast<uint4 *>(smem + (ones_base - sbase));
-    for (int i = tid; i < Lay::kOnesBytes / 16; i += kThreads)
-      ones[i] = make_uint4(one2, one2, one2, one2);
-    fence_proxy_async();
-  }
   __syncthreads();
   const long long U = *shared_u;
   // working CTAs: never more than tiles, so no working range is empty and a
@@ -758,12 +950,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  auto tmem_s = [&](int grp) { return tmem + (uint32_t)(grp * kNQ); };
+  constexpr int kSW = Lay::kSW;
+  auto tmem_s = [&](int grp) { return tmem + (uint32_t)(grp * kSW); };
   constexpr int kOS = Lay::kOSlots;
   auto tmem_o = [&](int grp, int slot) {
-    return tmem + (uint32_t)(2 * kNQ + (2 * (grp * kOS + slot)) * kN);
+    return tmem + (uint32_t)(2 * kSW + (grp * kOS + slot) * kN);
   };
-  auto tmem_l = [&](int grp, int slot) { return tmem_o(grp, slot) + (uint32_t)kN; };
 
   const int box_t = tp.box_tokens;
   const int nbox = box_t >= kTK ? 1 : kTK / box_t;
@@ -784,7 +976,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int cnt = n_total - b0 < 32 ? n_total - b0 : 32;
       TileIter mine;
       mine.init(p, t_begin + b0 + (lane < cnt ? lane : 0), t_stop, tab);
-      if (lane < cnt) load_page_ids(p, mine, nbox, box_t, pk + lane * 16, pv + lane * 16);
+      if (lane < cnt)
+        load_page_ids(p, mine.s, mine.tile, mine.L, nbox, box_t, pk + lane * 16, pv + lane * 16);
       __syncwarp();
 #pragma unroll 1
       for (int i = 0; i < cnt; ++i, ++n) {
@@ -816,253 +1009,169 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_drain(bar(kBarFullK + k % NS), (k / NS) & 1);
         mbar_drain(bar(kBarFullV + k % NS), (k / NS) & 1);
       }
-  } else if (warp == 1) {
-    // ============================ MMA issuer ==============================
-    // An event loop: the score product of tile n runs up to two tiles ahead
-    // of the output products, and whichever is ready is issued first.
-    if (lane == 0) {
-      // operand formats: 16-bit K/V use their own format for every operand;
-      // FP8 K/V meet E4M3 Q terms and E5M2 P terms (ones in E5M2)
-      constexpr uint32_t f16fmt = DT == LSE_KV_BF16 ? 1u : 0u;
-      constexpr uint32_t kvfmt = kF8 ? (kE5 ? 1u : 0u) : f16fmt;
-      constexpr uint32_t qfmt = kF8 ? 0u : f16fmt;
-      constexpr uint32_t pfmt = kF8 ? 1u : f16fmt;
-      constexpr uint32_t idesc_qk = instr_desc(kvfmt, qfmt, 0, 0, kTK, kNQ);
-      constexpr uint32_t idesc_pv = instr_desc(kvfmt, pfmt, 1, 1, kD, kN);
-      constexpr uint32_t idesc_l = instr_desc(pfmt, pfmt, 0, 1, kD, kN);
-      const int n_total = (int)(t_stop - t_begin);
-      TileIter iq, iv;
+  } else if (warp == 1 || warp == 2) {
+    // ====================== MMA issuers (one thread each) ======================
+    // Warp 1 issues the score products, warp 2 the output products: a
+    // thread waits ~120 cycles per tcgen05.mma issue whatever its N, so two
+    // issuing threads double the rate.  Every product carries its operand
+    // terms side by side along N, one MMA per K step.
+    // Operand formats: 16-bit K/V use their own format for every operand;
+    // FP8 K/V meet E4M3 Q terms and E5M2 P terms.
+    constexpr uint32_t f16fmt = DT == LSE_KV_BF16 ? 1u : 0u;
+    constexpr uint32_t kvfmt = kF8 ? (kE5 ? 1u : 0u) : f16fmt;
+    constexpr uint32_t qfmt = kF8 ? 0u : f16fmt;
+    constexpr uint32_t pfmt = kF8 ? 1u : f16fmt;
+    const int n_total = (int)(t_stop - t_begin);
+    if (warp == 1 && lane == 0) {
+      // ---- S^T = K Q^T into the group's score buffer ----
+      constexpr uint32_t idesc_qk = instr_desc(kvfmt, qfmt, 0, 0, kTK, kSW);
+      TileIter iq;
       iq.init(p, t_begin, t_stop, tab);
-      iv.init(p, t_begin, t_stop, tab);
-      int nq = 0, seg_q = -1;   // score side: tiles issued, segment count
-      int nv = 0, seg_v = -1;   // output side
-      bool grp_started[2] = {false, false};
-      long long t_idle = clock64();
-      int idle = 0;
-      while (nv < n_total) {
-        bool did = false;
-        if (nq < n_total && nq < nv + 2) {
-          const bool first = iq.seg_start(t_begin);
-          const int sq = first ? seg_q + 1 : seg_q;
-          const int st = nq % NS;
-          if ((!first || mbar_test(bar(kBarQFull + sq % QS), (sq / QS) & 1)) &&
-              mbar_test(bar(kBarFullK + st), (nq / NS) & 1)) {
-            seg_q = sq;
-            tc_fence_after();
-            const bool last = iq.seg_end();
-            const uint32_t kaddr = k_base + st * Lay::kHalfStage;
-            const uint32_t qaddr = q_base + (seg_q % QS) * Lay::kQBytes;
-            const uint32_t d = tmem_s(nq & 1);
-            if constexpr (kF8) {
-              // one 128-dim region; K steps of 32 bytes; the Q terms add up
-              // in the same columns
+      int seg_q = -1;
+#pragma unroll 1
+      for (int nq = 0; nq < n_total; ++nq, iq.advance(p)) {
+        const bool first = iq.seg_start(t_begin), last = iq.seg_end();
+        if (first) ++seg_q;
+        const int st = nq % NS;
+        // the segment's Q, the K tile, and the group's score buffer, which
+        // its softmax finished reading with tile nq - 2
+        bool go = !first || mbar_wait(bar(kBarQFull + seg_q % QS), (seg_q / QS) & 1, abort_flag,
+                                      p.err);
+        go = go && mbar_wait(bar(kBarFullK + st), (nq / NS) & 1, abort_flag, p.err);
+        go = go && (nq < 2 ||
+                    mbar_wait(bar(kBarPFull + (nq & 1)), ((nq - 2) >> 1) & 1, abort_flag, p.err));
+        if (!go) break;
+        tc_fence_after();
+        const uint32_t kaddr = k_base + st * Lay::kHalfStage;
+        const uint32_t qaddr = q_base + (seg_q % QS) * Lay::kQBytes;
+        const uint32_t d = tmem_s(nq & 1);
+        // descriptors advance by adding the byte offset / 16 to the start
+        // address field
+        const uint64_t a0 = smem_desc(kaddr, 16, 1024, kLayoutSw128);
+        const uint64_t b0 = smem_desc(qaddr, 16, 1024, kLayoutSw128);
+        if constexpr (kF8) {
+          // K: one 128-dim region, K steps of 32 bytes
 #pragma unroll
-              for (int k = 0; k < kD / 32; ++k) {
-                const uint64_t a = smem_desc(kaddr + k * 32, 16, 1024, kLayoutSw128);
+          for (int k = 0; k < kD / 32; ++k)
+            mma_f8(d, a0 + (uint64_t)(k * 2), b0 + (uint64_t)(k * 2), idesc_qk, k > 0);
+        } else {
+          // two 64-dim regions of K and of Q; K steps of 32 bytes
 #pragma unroll
-                for (int t = 0; t < kQTerms; ++t) {
-                  const uint64_t bq =
-                      smem_desc(qaddr + t * Lay::kQRegion + k * 32, 16, 1024, kLayoutSw128);
-                  mma_f8(d, a, bq, idesc_qk, (k | t) != 0);
-                }
-              }
-            } else {
-#pragma unroll
-              for (int k = 0; k < kD / 16; ++k) {
-                const uint64_t a = smem_desc(kaddr + (k >> 2) * kRegionBytes + (k & 3) * 32, 16,
-                                             1024, kLayoutSw128);
-                const uint32_t qoff = (k >> 2) * Lay::kQRegion + (k & 3) * 32;
-                const uint64_t bh = smem_desc(qaddr + qoff, 16, 1024, kLayoutSw128);
-                const uint64_t bl =
-                    smem_desc(qaddr + 2 * Lay::kQRegion + qoff, 16, 1024, kLayoutSw128);
-                mma_f16(d, a, bh, idesc_qk, k > 0);   // K Q_hi^T
-                mma_f16(d, a, bl, idesc_qk, 1u);      // + K Q_lo^T, same columns
-              }
-            }
-            mma_commit(bar(kBarEmptyK + st));
-            mma_commit(bar(kBarSFull + (nq & 1)));
-            if (last) mma_commit(bar(kBarQEmpty + seg_q % QS));
-            iq.advance(p);
-            ++nq;
-            did = true;
+          for (int k = 0; k < kD / 16; ++k) {
+            const uint32_t ka = ((k >> 2) * kRegionBytes + (k & 3) * 32) >> 4;
+            const uint32_t kb = ((k >> 2) * 2 * Lay::kQRegion + (k & 3) * 32) >> 4;
+            mma_f16(d, a0 + ka, b0 + kb, idesc_qk, k > 0);
           }
         }
-        if (nv < nq) {
-          const bool first = iv.seg_start(t_begin), last = iv.seg_end();
-          const int sv = first ? seg_v + 1 : seg_v;
-          const int grp = nv & 1, slot = sv % kOS;
-          const bool started = first ? false : grp_started[grp];
-          const bool other = first ? false : grp_started[grp ^ 1];
-          const uint32_t oe_par = ((sv / kOS) & 1) ^ 1;
-          const int st = nv % NS;
-          bool ready = mbar_test(bar(kBarPFull + grp), (nv >> 1) & 1) &&
-                       mbar_test(bar(kBarFullV + st), (nv / NS) & 1);
-          // a group's output slot must have been read out two segments ago
-          if (ready && !started) ready = mbar_test(bar(kBarOEmpty + 2 * grp + slot), oe_par);
-          if (ready && last && !other)
-            ready = mbar_test(bar(kBarOEmpty + 2 * (grp ^ 1) + slot), oe_par);
-          if (ready) {
-            if (first) {
-              seg_v = sv;
-              grp_started[0] = grp_started[1] = false;
-            }
-            tc_fence_after();
-            const uint32_t vaddr = v_base + st * Lay::kHalfStage;
-            const uint32_t paddr = p_base + grp * Lay::kPBytes;
-            const uint32_t d = tmem_o(grp, slot);
-            const uint32_t dl = tmem_l(grp, slot);
-            // the ones operand is K-major without swizzle: 8x16-byte core
-            // matrices, K blocks 128 B apart, row blocks 256 B apart
-            const uint64_t a1 = smem_desc(ones_base, 128, 256, kLayoutNone);
-            if constexpr (kF8) {
-              // V^T is MN-major with one 128-byte swizzle atom across the
-              // dims; K steps of 32 keys; the P terms add up in the same
-              // columns
-#pragma unroll
-              for (int k = 0; k < kTK / 32; ++k) {
-                const uint64_t a = smem_desc(vaddr + k * 4096, 0, 1024, kLayoutSw128);
-#pragma unroll
-                for (int t = 0; t < kPTerms; ++t) {
-                  const uint64_t b = smem_desc(paddr + t * Lay::kPTerm + k * 4 * Lay::kPLbo,
-                                               Lay::kPLbo, 128, kLayoutNone);
-                  const uint32_t acc = (grp_started[grp] || k > 0 || t > 0) ? 1u : 0u;
-                  mma_f8(d, a, b, idesc_pv, acc);     // O^T += V^T P_t^T
-                  mma_f8(dl, a1, b, idesc_l, acc);    // L += 1 P_t^T
-                }
-              }
-            } else {
-#pragma unroll
-              for (int k = 0; k < kTK / 16; ++k) {
-                const uint64_t a = smem_desc(vaddr + k * 2048, kRegionBytes, 1024, kLayoutSw128);
-                const uint64_t b =
-                    smem_desc(paddr + k * 2 * Lay::kPLbo, Lay::kPLbo, 128, kLayoutNone);
-                const uint32_t acc = (grp_started[grp] || k > 0) ? 1u : 0u;
-                mma_f16(d, a, b, idesc_pv, acc);     // O^T += V^T P^T
-                mma_f16(dl, a1, b, idesc_l, acc);    // L += 1 P^T (row sums of P)
-              }
-            }
-            grp_started[grp] = true;
-            mma_commit(bar(kBarEmptyV + st));
-            // this group's last tile of the piece: the tile is the piece's
-            // last, or the next one (the other group's) is
-            const bool next_is_last =
-                !last && (iv.t + 1 == iv.t_end - 1 || iv.tile + 1 == iv.n_tiles - 1);
-            if (last || next_is_last) mma_commit(bar(kBarOFull + 2 * grp + slot));
-            // the other group had no tile in this piece: release its (empty)
-            // output slot all the same (its previous use was read out)
-            if (last && !grp_started[grp ^ 1]) mma_commit(bar(kBarOFull + 2 * (grp ^ 1) + slot));
-            iv.advance(p);
-            ++nv;
-            did = true;
-          }
-        }
-        if (did) {
-          idle = 0;
-          t_idle = clock64();
-        } else if (++idle >= 64) {
-          idle = 0;
-          if (*abort_flag) break;
-          if (clock64() - t_idle > kWaitCycles) {
-            *abort_flag = 1;
-            atomicOr(p.err, LSE_DEVERR_TIMEOUT);
-            break;
-          }
-        }
+        mma_commit(bar(kBarEmptyK + st));
+        mma_commit(bar(kBarSFull + (nq & 1)));
+        if (last) mma_commit(bar(kBarQEmpty + seg_q % QS));
       }
       // every MMA issued has completed before TMEM is released
       mma_commit(bar(kBarDone));
       mbar_drain(bar(kBarDone), 0);
+    } else if (warp == 2 && lane == 0) {
+      // ---- O^T += V^T P^T into the group's output slot ----
+      constexpr uint32_t idesc_pv =
+          instr_desc(kvfmt, pfmt, 1, 1, kD, (kF8 && !Lay::kPSide) ? kNQ : kN);
+      TileIter iv;
+      iv.init(p, t_begin, t_stop, tab);
+      int seg_v = -1;
+      uint32_t started = 0;  // bit g: group g has an output product in this piece
+#pragma unroll 1
+      for (int nv = 0; nv < n_total; ++nv, iv.advance(p)) {
+        const bool first = iv.seg_start(t_begin), last = iv.seg_end();
+        if (first) {
+          ++seg_v;
+          started = 0;
+        }
+        const int grp = nv & 1, slot = seg_v % kOS;
+        const uint32_t oe_par = ((seg_v / kOS) & 1) ^ 1;
+        const int st = nv % NS;
+        bool go = mbar_wait(bar(kBarPFull + grp), (nv >> 1) & 1, abort_flag, p.err);
+        go = go && mbar_wait(bar(kBarFullV + st), (nv / NS) & 1, abort_flag, p.err);
+        // a group's output slot must have been read out kOS segments ago
+        const bool mine = (started >> grp) & 1u, other = (started >> (grp ^ 1)) & 1u;
+        if (!mine)
+          go = go && mbar_wait(bar(kBarOEmpty + 2 * grp + slot), oe_par, abort_flag, p.err);
+        if (last && !other)
+          go = go && mbar_wait(bar(kBarOEmpty + 2 * (grp ^ 1) + slot), oe_par, abort_flag, p.err);
+        if (!go) break;
+        tc_fence_after();
+        const uint32_t vaddr = v_base + st * Lay::kHalfStage;
+        const uint32_t paddr = p_base + grp * Lay::kPBytes;
+        const uint32_t d = tmem_o(grp, slot);
+        const uint64_t b0 = smem_desc(paddr, Lay::kPLbo, 128, kLayoutNone);
+        if constexpr (kF8) {
+          // V^T is MN-major with one 128-byte swizzle atom across the dims
+          // (LBO unused); K steps of 32 keys
+          const uint64_t a0 = smem_desc(vaddr, 0, 1024, kLayoutSw128);
+#pragma unroll
+          for (int k = 0; k < kTK / 32; ++k) {
+            const uint64_t a = a0 + (uint64_t)(k * 4096 / 16);
+            const uint64_t b = b0 + (uint64_t)(k * 4 * Lay::kPLbo / 16);
+            if constexpr (Lay::kPSide) {
+              // the P terms side by side along N
+              mma_f8(d, a, b, idesc_pv, (mine || k > 0) ? 1u : 0u);
+            } else {
+              // the P terms accumulate into the same columns
+#pragma unroll
+              for (int t = 0; t < kPTerms; ++t)
+                mma_f8(d, a, b + (uint64_t)(t * (kNQ / 16) * 128 / 16), idesc_pv,
+                       (mine || k > 0 || t > 0) ? 1u : 0u);
+            }
+          }
+        } else {
+          // V^T is MN-major: two 64-dim atoms (LBO), K steps of 16 keys
+          const uint64_t a0 = smem_desc(vaddr, kRegionBytes, 1024, kLayoutSw128);
+#pragma unroll
+          for (int k = 0; k < kTK / 16; ++k)
+            mma_f16(d, a0 + (uint64_t)(k * 2048 / 16), b0 + (uint64_t)(k * 2 * Lay::kPLbo / 16),
+                    idesc_pv, (mine || k > 0) ? 1u : 0u);
+        }
+        started |= 1u << grp;
+        mma_commit(bar(kBarEmptyV + st));
+        mma_commit(bar(kBarPEmpty + grp));
+        // this group's last tile of the piece: the tile is the piece's
+        // last, or the next one (the other group's) is
+        const bool next_is_last =
+            !last && (iv.t + 1 == iv.t_end - 1 || iv.tile + 1 == iv.n_tiles - 1);
+        if (last || next_is_last) mma_commit(bar(kBarOFull + 2 * grp + slot));
+        // the other group had no tile in this piece: release its (empty)
+        // output slot all the same (its previous use was read out)
+        if (last && !other) mma_commit(bar(kBarOFull + 2 * (grp ^ 1) + slot));
+      }
+      mma_commit(bar(kBarDoneV));
+      mbar_drain(bar(kBarDoneV), 0);
     }
-  } else if (warp < 4) {
+  } else if (warp == 3) {
     // ============================ Q staging ===============================
-    const int qt = tid - 64;  // 0..63
+    // Every segment after the first, ahead of the score products (softmax
+    // group 0 stages the first: it is idle until the first scores arrive,
+    // and 128 threads do it faster than one warp).
     TileIter it;
     it.init(p, t_begin, t_stop, tab);
     int seg = -1;
     for (; it.valid(); it.advance(p)) {
       if (!it.seg_start(t_begin)) continue;
-      ++seg;
+      if (++seg == 0) continue;
       const int slot = seg % QS;
-      const int P = G * it.R;
-      // items (row n, 8-dim chunk c): every load of the segment in flight at
-      // once, issued before waiting for the slot
-      constexpr int kItems = kNQ * 16 / 64;
-      float4 ld[kItems][2];
-#pragma unroll
-      for (int k = 0; k < kItems; ++k) {
-        const int item = qt + 64 * k;
-        const int n = item >> 4, c = item & 15;
-        if (n < P) {
-          const int r = n / G, h = it.g * G + (n - r * G);
-          const float4 *src = reinterpret_cast<const float4 *>(
-              p.q + ((long long)(it.row0 + r) * p.n_q_heads + h) * kD + c * 8);
-          ld[k][0] = __ldg(src);
-          ld[k][1] = __ldg(src + 1);
-        } else {
-          ld[k][0] = ld[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-      }
-      if (!mbar_wait(bar(kBarQEmpty + slot), ((seg / QS) & 1) ^ 1, abort_flag, p.err)) break;
       uint8_t *qs = smem + (q_base - sbase) + slot * Lay::kQBytes;
-      const float sc = p.scale_log2;
-      if constexpr (kF8) {
-        // pair n's row scaled by 2^e (max |x| 2^e in [128, 256)), then
-        // written as kQTerms E4M3 terms, one 128-byte swizzled row per term;
-        // the 16 lanes holding a row find its maximum by shuffles
-        float *isig = isig_all + slot * 64;
-#pragma unroll
-        for (int k = 0; k < kItems; ++k) {
-          const int item = qt + 64 * k;
-          const int n = item >> 4, c = item & 15;
-          float x[8] = {ld[k][0].x * sc, ld[k][0].y * sc, ld[k][0].z * sc, ld[k][0].w * sc,
-                        ld[k][1].x * sc, ld[k][1].y * sc, ld[k][1].z * sc, ld[k][1].w * sc};
-          float mx = 0.f;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(x[i]));
-#pragma unroll
-          for (int o = 1; o < 16; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-          int e = 0;
-          if (mx > 0.f && mx <= FLT_MAX) {
-            const int E = ((__float_as_int(mx) >> 23) & 0xff) - 127;
-            e = min(max(7 - E, -126), 126);
-          }
-          const float sg = exp2i(e);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) x[i] *= sg;
-          uint2 w[kQTerms];
-          f8_terms<false, kQTerms>(x, w);
-          const uint32_t off = (n >> 3) * 1024 + (n & 7) * 128 +
-                               ((((c >> 1) ^ (n & 7))) << 4) + (c & 1) * 8;
-#pragma unroll
-          for (int t = 0; t < kQTerms; ++t)
-            *reinterpret_cast<uint2 *>(qs + t * Lay::kQRegion + off) = w[t];
-          if (c == 0) isig[n] = exp2i(-e);
-        }
-      } else {
-#pragma unroll
-        for (int k = 0; k < kItems; ++k) {
-          const int item = qt + 64 * k;
-          const int n = item >> 4, c = item & 15;
-          uint4 vh, vl;
-          split2<DT>(ld[k][0].x * sc, ld[k][0].y * sc, vh.x, vl.x);
-          split2<DT>(ld[k][0].z * sc, ld[k][0].w * sc, vh.y, vl.y);
-          split2<DT>(ld[k][1].x * sc, ld[k][1].y * sc, vh.z, vl.z);
-          split2<DT>(ld[k][1].z * sc, ld[k][1].w * sc, vh.w, vl.w);
-          const int region = c >> 3, cc = c & 7;
-          const uint32_t off = region * Lay::kQRegion + (n >> 3) * 1024 + (n & 7) * 128 +
-                               ((cc ^ (n & 7)) << 4);
-          *reinterpret_cast<uint4 *>(qs + off) = vh;
-          *reinterpret_cast<uint4 *>(qs + 2 * Lay::kQRegion + off) = vl;
-        }
-      }
-      fence_proxy_async();
-      mbar_arrive(bar(kBarQFull + slot));
+      const bool okq = stage_q<DT, P8, 32>(
+          p, lane, it.g, it.row0, G * it.R, qs, isig_all + slot * 64, [&]() {
+            return mbar_wait(bar(kBarQEmpty + slot), ((seg / QS) & 1) ^ 1, abort_flag, p.err);
+          });
+      if (!okq) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kBarQFull + slot));
     }
   } else {
     // ============== softmax and epilogue: two groups of 128 threads ==============
     // Scores are read from TMEM eight pairs at a time in loops whose code does
-    // not grow with the pair count; the row sums of P come from the tensor
-    // core (L = 1 P^T), so no per-pair state lives in registers.
+    // not grow with the pair count.  The row sums of P are summed here: each
+    // warp reduces its 32 keys per pair, and the four warps' partials are
+    // folded into the group's sums after the next group barrier, in a fixed
+    // order (so results repeat bit for bit).
     const int grp = (warp - 4) >> 2;           // tiles of this parity
     const int j = tid - 128 - grp * 128;       // key of the tile = TMEM lane (scores)
     const int quarter = warp & 3;              // TMEM lane quarter of this warp
@@ -1074,8 +1183,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned long long *masks = masks_all + grp * 64;
     float *scr = reinterpret_cast<float *>(smem + (p_base - sbase) + grp * Lay::kPBytes);
     float *isg = isig_all + (2 + grp) * 64;    // FP8: the segment's inverse Q scales
-    // a score in log2 units from its TMEM value (FP8: undo Q's pair scale)
-    auto score = [&](float v, int q) { return kF8 ? v * isg[q] : v; };
+    float *lsum = lsum_all + grp * 64;         // row sums of P of the segment so far
+    float *lpart = lpart_all + grp * 2 * 4 * P8;  // [buffer][warp][pair] partials
+    bool pend = false;                         // partials of buffer pbuf not yet folded
+    int pbuf = 0;
+    auto fold = [&]() {
+      if (pend && j < P8) {
+        const float *pp = lpart + pbuf * 4 * P8 + j;
+        lsum[j] += ((pp[0] + pp[P8]) + pp[2 * P8]) + pp[3 * P8];
+      }
+      pend = false;
+    };
+    // Up to 32 pairs each thread keeps its key's sums of P over the segment
+    // in registers (one column reduction per segment); beyond that, each
+    // tile's sums are reduced across the warp and folded into lsum.
+    constexpr bool kLAcc = P8 <= 32;
+    float lacc[kLAcc ? P8 : 1];
     TileIter it;
     it.init(p, t_begin, t_stop, tab);
     int n = 0, seg = -1;
@@ -1090,11 +1213,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++seg;
         // a finite floor keeps exp2(-inf - m) at 0 (never NaN) for pairs
         // with no visible key yet
-        if (j < P8) m_run[j] = -FLT_MAX;
+        if (j < P8) {
+          m_run[j] = -FLT_MAX;
+          lsum[j] = 0.f;
+        }
+        if constexpr (kLAcc) {
+#pragma unroll
+          for (int q = 0; q < P8; ++q) lacc[q] = 0.f;
+        }
         if (j < it.R)
           masks[j] = p.row_masks ? p.row_masks[it.row0 + j]
                                  : (j >= 63 ? ~0ull : ((1ull << (j + 1)) - 1ull));
         had_tile = false;
+        if (seg == 0 && grp == 0) {
+          // the first segment's Q (slot 0, never used before)
+          stage_q<DT, P8, 128>(p, j, it.g, it.row0, P, smem + (q_base - sbase), isig_all,
+                               [] { return true; });
+          named_sync(bar_id, 128);
+          if (j == 0) mbar_arrive(bar(kBarQFull));
+        }
         bool w = true;
         if constexpr (kF8) {
           // the segment's Q scales: wait for its Q slot, keep a copy, then
@@ -1116,6 +1253,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // tile record, published by the producer on its own barrier (the
         // K ring may already hold a later tile)
         if (w) w = mbar_wait(bar(kBarInfo + (n & 7)), (n >> 3) & 1, abort_flag, p.err);
+        // the group's P tile and output are free once its previous P.V (tile
+        // n - 2) has completed
+        if (w && n >= 2) w = mbar_wait(bar(kBarPEmpty + grp), ((n - 2) >> 1) & 1, abort_flag, p.err);
         if (named_or(bar_id, 128, !w)) {
           ok = false;
           break;
@@ -1143,27 +1283,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const uint32_t s_addr = tmem_s(grp) + lane_off;
         __syncwarp();
-        // pass 1: does any score pass the running max by 2^tau?
+        if constexpr (!kLAcc) fold();  // the previous tile's partials (written before the barrier above)
+        // pass 1: the score terms (16-bit: Q hi and lo blocks; FP8: four Q-term
+        // blocks, times the pair's inverse Q scale) summed into the first
+        // block; does any score pass the running max by 2^tau?
         float gap = -INFINITY;
 #pragma unroll 1
         for (int c = 0; c < P8; c += 8) {
           float v[8];
-          tmem_load<8>(s_addr + c, v);
+          tmem_load_sum8<kSW / kNQ>(s_addr + c, kNQ, v);
+          if constexpr (kF8) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] *= isg[c + i];
+          }
+          tmem_st8(s_addr + c, v);
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            if ((vis >> (c + i)) & 1ull) gap = fmaxf(gap, score(v[i], c + i) - m_run[c + i]);
+            if ((vis >> (c + i)) & 1ull) gap = fmaxf(gap, v[i] - m_run[c + i]);
         }
+        tmem_st_wait();
         if (named_or(bar_id, 128, gap > kTau)) {
           // per-pair maximum over the tile's keys, through this group's P tile
-          // as FP32 scratch [key][pair] (free: the group's previous P.V and sums
-          // have completed, its score commit came later)
+          // as FP32 scratch [key][pair] (free: the group's previous P.V has
+          // completed)
 #pragma unroll 1
           for (int c = 0; c < P8; c += 8) {
             float v[8];
             tmem_load<8>(s_addr + c, v);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-              v[i] = ((vis >> (c + i)) & 1ull) ? score(v[i], c + i) : -INFINITY;
+              if (!((vis >> (c + i)) & 1ull)) v[i] = -INFINITY;
             *reinterpret_cast<float4 *>(scr + j * P8 + c) = make_float4(v[0], v[1], v[2], v[3]);
             *reinterpret_cast<float4 *>(scr + j * P8 + c + 4) =
                 make_float4(v[4], v[5], v[6], v[7]);
@@ -1174,50 +1323,64 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (j < P8) {
             const float mo = m_run[j];
             const float mn = fmaxf(mo, red[j]);
-            alpha[j] = ex2(mo - mn);
+            const float al = ex2(mo - mn);
+            alpha[j] = al;
             m_run[j] = mn;
+            lsum[j] *= al;  // (this thread folded pair j's partials above)
           }
           named_sync(bar_id, 128);
+          if constexpr (kLAcc) {
+#pragma unroll
+            for (int q = 0; q < P8; ++q) lacc[q] *= alpha[q];
+          }
           if (had_tile) {
-            // rescale this group's output and sums (the previous P.V and sums
-            // have completed)
+            // rescale this group's output (the previous P.V has completed)
             __syncwarp();
             const uint32_t ob = tmem_o(grp, oslot) + lane_off;
 #pragma unroll 1
-            for (int c = 0; c < 2 * kN; c += 8) {
-              const int cc = c % kN;
-              if (kF8 && cc >= P8) continue;  // padding columns
+            for (int c = 0; c < kN; c += 8) {
+              const int cc = c % Lay::kOBlk;
+              if (cc >= P8) continue;  // padding columns
               float v[8];
               tmem_load<8>(ob + c, v);
-              const int q0 = kF8 ? cc : cc < P8 ? cc : cc - P8;
 #pragma unroll
-              for (int i = 0; i < 8; ++i) v[i] *= alpha[q0 + i];
+              for (int i = 0; i < 8; ++i) v[i] *= alpha[cc + i];
               tmem_st8(ob + c, v);
             }
             tmem_st_wait();
           }
         }
-        // pass 2: probabilities -> this group's P tile, row j (16-bit: hi then
-        // lo columns; FP8: P 2^7 as kPTerms E5M2 terms, one block per term)
+        // pass 2: probabilities -> this group's P tile, row j (16-bit: hi block
+        // then lo block; FP8: P 2^7 as kPTerms E5M2 terms, a block each), and
+        // this warp's sums of them per pair
         uint8_t *prow = smem + (p_base - sbase) + grp * Lay::kPBytes + (j >> 3) * Lay::kPLbo +
                         (j & 7) * 16;
-#pragma unroll 1
+        const int buf = (n >> 1) & 1;
+        float *lp = lpart + buf * 4 * P8 + quarter * P8;
+#pragma unroll
         for (int c = 0; c < P8; c += 8) {
           float v[8];
           tmem_load<8>(s_addr + c, v);
           float e[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            e[i] = ((vis >> (c + i)) & 1ull) ? ex2(score(v[i], c + i) - m_run[c + i]) : 0.f;
+            e[i] = ((vis >> (c + i)) & 1ull) ? ex2(v[i] - m_run[c + i]) : 0.f;
           if constexpr (kF8) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) e[i] *= (float)(1 << kPScaleLog2);
             uint2 w[kPTerms];
-            f8_terms<true, kPTerms>(e, w);
-            uint8_t *dst = prow + (c >> 4) * 128 + ((c >> 3) & 1) * 8;
+            float er[8];
+            e5_terms_f16<kPTerms>(e, w, er);
+            // the sums take P as the products see it (rounded to F16)
 #pragma unroll
-            for (int t = 0; t < kPTerms; ++t)
-              *reinterpret_cast<uint2 *>(dst + t * Lay::kPTerm) = w[t];
+            for (int i = 0; i < 8; ++i) e[i] = er[i];
+            // 16 FP8 columns per core matrix: term t's pair c sits in column
+            // t kNQ + c
+#pragma unroll
+            for (int t = 0; t < kPTerms; ++t) {
+              const int col = t * kNQ + c;
+              *reinterpret_cast<uint2 *>(prow + (col >> 4) * 128 + ((col >> 3) & 1) * 8) = w[t];
+            }
           } else {
             uint4 vh, vl;
             split2<DT>(e[0], e[1], vh.x, vl.x);
@@ -1227,7 +1390,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint4 *>(prow + (c >> 3) * 128) = vh;
             *reinterpret_cast<uint4 *>(prow + ((P8 + c) >> 3) * 128) = vl;
           }
+          if constexpr (kLAcc) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) lacc[c + i] += e[i];
+          } else {
+            const float ws = warp_sum8(e, lane);
+            if ((lane & 3) == 0) lp[c + (lane >> 2)] = ws;
+          }
         }
+        pend = !kLAcc;
+        pbuf = buf;
         if (!kvalid) {
           // a dead slot may hold any bits: give it a zero V row (P is 0 there)
           mbar_wait(bar(kBarFullV + n % NS), (n / NS) & 1, abort_flag, p.err);
@@ -1252,28 +1424,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
+        const float *lt_of = lsum;  // the group's row sums of P, per pair
+        if constexpr (kLAcc) {
+          // column sums of the threads' sums, through the group's P tile as
+          // FP32 scratch [key][pair] (free: the piece's last P.V has completed)
+#pragma unroll
+          for (int c = 0; c < P8; c += 4)
+            *reinterpret_cast<float4 *>(scr + j * P8 + c) =
+                make_float4(lacc[c], lacc[c + 1], lacc[c + 2], lacc[c + 3]);
+          named_sync(bar_id, 128);
+          column_reduce<P8, true>(scr, j, red, bar_id);  // red[q] = sum over keys
+          lt_of = red;
+        } else {
+          fold();  // the group's last tile's partials
+        }
+        named_sync(bar_id, 128);
         tc_fence_after();
         __syncwarp();
         const int c_first = cta_of_tile(it.seg_first, U, C);
         const int slot = 2 * (cta - c_first) + grp;
-        const int d = j;  // output lane = head dim; every lane holds the sums
+        const int d = j;  // output lane = head dim
         const uint32_t ob = tmem_o(grp, oslot) + lane_off;
-        const uint32_t lb = tmem_l(grp, oslot) + lane_off;
         const long long row_stride = (long long)p.n_q_heads * tp.n_slots * kD;
         const long long base =
             ((long long)it.row0 * p.n_q_heads + it.g * G) * tp.n_slots + slot;
 #pragma unroll 1
         for (int c = 0; c < P8; c += 8) {
-          float oh[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, ol[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-          float lh[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, ll[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-          if (had_tile) {
-            tmem_load<8>(ob + c, oh);
-            tmem_load<8>(lb + c, lh);
-            if constexpr (!kF8) {
-              tmem_load<8>(ob + P8 + c, ol);
-              tmem_load<8>(lb + P8 + c, ll);
-            }
-          }
+          float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          // the output blocks (hi and lo, or the P terms) summed
+          if (had_tile) tmem_load_sum8<kN / Lay::kOBlk>(ob + c, Lay::kOBlk, o);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int q = c + i;
@@ -1281,8 +1460,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int r = pair_row[q];
               const long long idx =
                   base + r * row_stride / kD + (long long)(q - r * G) * tp.n_slots;
-              const float lt = lh[i] + ll[i];
-              p.o_part[idx * kD + d] = lt > 0.f ? (oh[i] + ol[i]) * rcp(lt) : 0.f;
+              const float lt = lt_of[q];
+              p.o_part[idx * kD + d] = lt > 0.f ? o[i] * rcp(lt) : 0.f;
               // (FP8 sums carry P's factor 2^7)
               if (d == q)
                 p.lse_part[idx] = lt > 0.f ? m_run[q] + lg2(lt) - (kF8 ? kPScaleLog2 : 0)
@@ -1402,21 +1581,28 @@ int lse_tc_build_maps(const uint64_t *chunk_base, int n_chunks, size_t chunk_byt
   if (n_chunks > LSE_MAX_TMA_CHUNKS) return (int)cudaErrorInvalidValue;
   CUtensorMap *maps = static_cast<CUtensorMap *>(maps_out);
   // a chunk as [tokens][rows][128 bytes]: 16-bit K/V give two 64-dim rows
-  // per kv head, FP8 one 128-dim row
+  // per kv head, FP8 one 128-dim row.  The bytes are described to the TMA
+  // unit as 8-byte elements (16 per row) whatever the storage format: the
+  // 128-byte swizzle moves 16-byte pieces, so shared memory receives the same
+  // layout, and the copy engine handles far fewer elements per byte.
   const bool f8 = is_f8(dtype);
   const int esize = f8 ? 1 : 2;
   const int rows_per_head = f8 ? 1 : 2;
   const uint64_t row = (uint64_t)n_kv_heads * kD * esize;  // bytes per token, all kv heads
   for (int c = 0; c < n_chunks; ++c) {
-    cuuint64_t dims[3] = {(cuuint64_t)(128 / esize), (cuuint64_t)n_kv_heads * rows_per_head,
+    cuuint64_t dims[3] = {16, (cuuint64_t)n_kv_heads * rows_per_head,
                           (cuuint64_t)(chunk_bytes / row)};
     cuuint64_t strides[2] = {128, row};
-    cuuint32_t box[3] = {(cuuint32_t)(128 / esize), 1, (cuuint32_t)box_tokens};
+    cuuint32_t box[3] = {16, 1, (cuuint32_t)box_tokens};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = enc(&maps[c], f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16,
-                     3, reinterpret_cast<void *>(chunk_base[c]), dims, strides, box, estr,
+    CUresult r = enc(&maps[c], CU_TENSOR_MAP_DATA_TYPE_UINT64, 3,
+                     reinterpret_cast<void *>(chunk_base[c]), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                     // L2 fills no wider than one kv head's row (128 bytes
+                     // for FP8, 256 for 16-bit), so no fill drags in a
+                     // neighbouring head's bytes
+                     f8 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B : CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return (int)cudaErrorInvalidValue;
   }
   return 0;
