@@ -202,6 +202,9 @@ typedef struct {
   int32_t smem_bytes;      /* dynamic shared memory of the partial kernel  */
   int32_t ctas;            /* partial-pass CTAs when persistent, else 0     */
   int64_t workspace_bytes;
+  int32_t stages;          /* tensor-core kernel: K/V ring depth, else 0      */
+  int32_t q_slots;         /* tensor-core kernel: Q ring depth, else 0        */
+  int32_t p_bufs;          /* tensor-core kernel: P tiles per softmax group   */
 } lse_attn_plan_info;
 
 LSE_API int lse_attn_plan_query(const lse_attn_plan_t *plan, lse_attn_plan_info *info);

@@ -258,6 +258,28 @@ def test_tcgen05_fp8_query_scale_range(binding, dtype, q_gain):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+@pytest.mark.parametrize("smem", [232448, 200000, 185000, 160000])
+def test_tcgen05_pipeline_configurations(binding, dtype, smem):
+    # smaller shared-memory limits make the plan pick shallower K/V rings,
+    # one Q slot and one P tile per softmax group: every configuration gives
+    # the same results
+    lens = [4000, 300, 2500, 129, 1]
+    w = wl.small_case(dtype, lens, [3, 1, 2, 1, 1], n_q_heads=24, n_kv_heads=4, head_dim=128,
+                      tokens_per_fragment=128, seed=226)
+    props = torch.cuda.get_device_properties(0)
+    limits = dict(n_sms=props.multi_processor_count, smem_optin=smem, ctas_per_sm=0,
+                  allow_tcgen05=1)
+    (out, lse, info), err = gpu_run(binding, w, plan_limits=limits)
+    if info["kernel_name"] != "tcgen05":
+        pytest.skip(f"no tensor-core configuration fits in {smem} bytes")
+    assert err == 0
+    ref_out, ref_lse = orc.attention(to_problem(w))
+    assert_close(out, ref_out, w.dtype, what=f"stages {info['stages']} q_slots "
+                 f"{info['q_slots']} p_bufs {info['p_bufs']}")
+    np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=lse_tol(w.dtype) * 4)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
 def test_tcgen05_capacity_far_above_live(binding, dtype):
     w = wl.small_case(dtype, [130, 5, 1000], [1, 1, 2], n_q_heads=24, n_kv_heads=4,
                       head_dim=128, tokens_per_fragment=128, max_pages=300, seed=223)

@@ -51,7 +51,9 @@ class PlanInfo(ctypes.Structure):
     _fields_ = [("n_splits", ctypes.c_int32), ("keys_per_split", ctypes.c_int32),
                 ("kernel", ctypes.c_int32), ("key_tile", ctypes.c_int32),
                 ("pairs", ctypes.c_int32), ("smem_bytes", ctypes.c_int32),
-                ("ctas", ctypes.c_int32), ("workspace_bytes", ctypes.c_int64)]
+                ("ctas", ctypes.c_int32), ("workspace_bytes", ctypes.c_int64),
+                ("stages", ctypes.c_int32), ("q_slots", ctypes.c_int32),
+                ("p_bufs", ctypes.c_int32)]
 
 
 class DeviceLimits(ctypes.Structure):

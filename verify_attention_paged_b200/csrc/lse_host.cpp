@@ -276,9 +276,9 @@ int lse_attn_plan_ex(const lse_kv_arena *a, int n_seqs, int max_rows, int max_to
   const int T = a->tokens_per_fragment;
   const bool t_ok = (T % 128 == 0) || (T >= 8 && T % 8 == 0 && 128 % T == 0);
   const int p8 = lse_tc_pairs_bucket(pl->pairs);
-  int tc_stages = 0, tc_q_slots = 0;
+  int tc_stages = 0, tc_q_slots = 0, tc_p_bufs = 0;
   const int tc_smem =
-      p8 > 0 ? lse_tc_smem(a->dtype, p8, smem_optin, &tc_stages, &tc_q_slots) : -1;
+      p8 > 0 ? lse_tc_smem(a->dtype, p8, smem_optin, &tc_stages, &tc_q_slots, &tc_p_bufs) : -1;
   if (allow_tc && a->dtype != LSE_KV_F32 && a->head_dim == 128 &&
       t_ok && p8 > 0 && tc_smem > 0) {
     const int tile = lse_tc_key_tile();
@@ -287,6 +287,7 @@ int lse_attn_plan_ex(const lse_kv_arena *a, int n_seqs, int max_rows, int max_to
     pl->smem_bytes = tc_smem;
     pl->stages = tc_stages;
     pl->q_slots = tc_q_slots;
+    pl->p_bufs = tc_p_bufs;
     pl->pairs_bucket = p8;
     pl->box_tokens = T < tile ? T : tile;
     pl->ctas = n_sms;
@@ -338,6 +339,10 @@ int lse_attn_plan_query(const lse_attn_plan_t *pl, lse_attn_plan_info *info) {
   info->smem_bytes = pl->smem_bytes;
   info->ctas = pl->kernel == LSE_KERNEL_TCGEN05 ? pl->ctas : 0;
   info->workspace_bytes = int64_t(pl->ws_bytes);
+  const bool tc = pl->kernel == LSE_KERNEL_TCGEN05;
+  info->stages = tc ? pl->stages : 0;
+  info->q_slots = tc ? pl->q_slots : 0;
+  info->p_bufs = tc ? pl->p_bufs : 0;
   return LSE_OK;
 }
 
@@ -417,7 +422,7 @@ int lse_attn_run(const lse_attn_plan_t *pl, const float *q, const int32_t *k_pag
     }
     ce = lse_launch_partial_tcgen05(p, pl->maps.data(), nch, pl->dtype, pl->pairs_bucket,
                                     pl->ctas, pl->n_splits, pl->stages, pl->q_slots,
-                                    pl->box_tokens,
+                                    pl->p_bufs, pl->box_tokens,
                                     pl->smem_bytes, stream);
   } else {
     ce = lse_launch_partial_cuda_core(p, pl->dtype, pl->head_dim, pl->n_splits, pl->n_kv_heads,

@@ -47,6 +47,7 @@ struct lse_attn_plan_s {
   int ctas = 0;          // persistent grid of the tensor-core kernel
   int stages = 0;        // its pipeline depth
   int q_slots = 0;       // and its Q ring depth
+  int p_bufs = 0;        // and its P tiles per softmax group
   int pairs_bucket = 0;  // its compile-time pair count (P8)
   int box_tokens = 0;    // its TMA box height
   // tensor maps of the arena chunks (built on first run, rebuilt on growth)
@@ -103,11 +104,12 @@ const char *lse_cuda_error_string(int code);
 
 // tensor-core partial pass (lse_tcgen05.cu)
 int lse_tc_pairs_bucket(int pairs);
-int lse_tc_smem(int dtype, int p8, int smem_optin, int *stages, int *q_slots);
+int lse_tc_smem(int dtype, int p8, int smem_optin, int *stages, int *q_slots, int *p_bufs);
 int lse_tc_key_tile();
 size_t lse_tc_map_bytes();
 int lse_tc_build_maps(const uint64_t *chunk_base, int n_chunks, size_t chunk_bytes,
                       int n_kv_heads, int dtype, int box_tokens, void *maps_out);
 int lse_launch_partial_tcgen05(const LseKernelParams &p, const void *maps, int n_maps,
                                int dtype, int p8, int n_ctas, int n_slots, int stages,
-                               int q_slots, int box_tokens, int smem, void *stream);
+                               int q_slots, int p_bufs, int box_tokens, int smem,
+                               void *stream);

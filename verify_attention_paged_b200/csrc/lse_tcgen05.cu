@@ -81,6 +81,7 @@ struct __align__(64) TcParams {
   int n_slots;
   int stages;
   int q_slots;
+  int p_bufs;
   int box_tokens;
 };
 
@@ -112,6 +113,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but a thread whose phase is not complete is suspended
+// (until the phase completes, or for at most about a microsecond) instead of
+// returning at once, so waiting warps leave their issue slots to the warps
+// doing work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "n"(1000)
+      : "memory");
+  return ok != 0;
+}
+
 // Non-blocking test of a phase.
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -131,8 +148,8 @@ __device__ __noinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity,
                                             volatile int *abort_flag, unsigned int *err) {
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 31u) == 0) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if ((i & 3u) == 0) {
       if (*abort_flag) return false;
       if (clock64() - t0 > kWaitCycles) {
         *abort_flag = 1;
@@ -154,7 +171,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // MMAs already in flight before the CTA releases TMEM and exits.
 __device__ __noinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
   const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity))
+  while (!mbar_try_wait_sleep(bar, parity))
     if (clock64() - t0 > kWaitCycles) return;
 }
 
@@ -210,28 +227,46 @@ __host__ __device__ constexpr uint32_t instr_desc(uint32_t a_fmt, uint32_t b_fmt
          ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
-__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                        uint32_t accumulate) {
+// One lane of the warp (elect.sync): 1 in that lane, 0 in the others.
+__device__ __forceinline__ uint32_t elect_one() {
+  uint32_t r;
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred e;\n\t.reg .b32 x;\n\t"
+      "elect.sync x|e, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, e;\n\t}\n"
+      : "=r"(r));
+  return r;
+}
+
+// The MMA issue helpers run in all lanes of a converged warp with the same
+// operands; only the lane with `leader` set issues.
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                        uint32_t accumulate, uint32_t leader) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      "setp.ne.b32 e, %5, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(leader)
       : "memory");
 }
 // 8-bit operands, K = 32 per instruction.
 __device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                       uint32_t accumulate) {
+                                       uint32_t accumulate, uint32_t leader) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      "setp.ne.b32 e, %5, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(leader)
       : "memory");
 }
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
+__device__ __forceinline__ void mma_commit(uint32_t bar, uint32_t leader) {
   asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      "{\n\t.reg .pred e;\n\t"
+      "setp.ne.b32 e, %1, 0;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(bar),
+      "r"(leader)
       : "memory");
 }
 
@@ -528,9 +563,11 @@ struct TcLayout {
                                     kSeqTab * (int)sizeof(SeqRec);
   // one K or V tile: 128 keys of 128 dims (two 64-dim regions when 16-bit)
   static constexpr int kHalfStage = kF8 ? kRegionBytes : 2 * kRegionBytes;
-  // stages: K/V ring depth; q_slots: Q ring depth (1 or 2)
-  static int smem_bytes(int stages, int q_slots) {
-    return 1024 + stages * 2 * kHalfStage + q_slots * kQBytes + 2 * kPBytes + kMiscBytes;
+  // stages: K/V ring depth; q_slots: Q ring depth (1 or 2); p_bufs: P tiles
+  // per softmax group (1 or 2)
+  static int smem_bytes(int stages, int q_slots, int p_bufs) {
+    return 1024 + stages * 2 * kHalfStage + q_slots * kQBytes + 2 * p_bufs * kPBytes +
+           kMiscBytes;
   }
 };
 
@@ -549,8 +586,8 @@ enum {
   kBarOEmpty = 44,  // [4]
   kBarDone = 48,     // the score issuer's MMAs have completed
   kBarInfo = 49,    // [8] one per tile record
-  kBarPEmpty = 57,  // [2] per softmax group: its P tile has been read
-  kBarDoneV = 59,   // the output issuer's MMAs have completed
+  kBarPEmpty = 57,  // [4] = group * 2 + P buffer: the P tile has been read
+  kBarDoneV = 61,   // the output issuer's MMAs have completed
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -627,32 +664,28 @@ __device__ __forceinline__ void f8_terms(float *x, uint2 *out) {
 }
 
 // Eight FP32 values -> F16 (round to nearest), then kTerms E5M2 terms of
-// the F16 values: every E5M2 value is an F16 value, so each remainder is an
-// exact F16 subtraction, and four terms of 3 significant bits hold all 11
-// bits of an F16.  Also returns the F16-rounded values as FP32.
+// the F16 values.  E5M2 is the upper byte of F16 (same sign and exponent
+// fields), so the nearest E5M2 of each half of a packed F16 pair is its bit
+// pattern with the low byte rounded away (ties to even; a carry out of the
+// mantissa raises the exponent), done for both halves in integer arithmetic
+// (a half stays far below 0xFF80 here, so no carry crosses halves).  Each
+// remainder is an exact F16 subtraction, and four terms of 3 significant
+// bits hold all 11 bits of an F16.
 template <int kTerms>
-__device__ __forceinline__ void e5_terms_f16(const float *x, uint2 *out, float *rounded) {
+__device__ __forceinline__ void e5_terms_f16(const float *x, uint2 *out) {
   uint32_t h[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < 4; ++i)
     asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h[i]) : "f"(x[2 * i + 1]), "f"(x[2 * i]));
-    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h[i]));
-    rounded[2 * i] = f.x;
-    rounded[2 * i + 1] = f.y;
-  }
 #pragma unroll
   for (int t = 0; t < kTerms; ++t) {
     uint32_t w[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      uint16_t r;
-      asm("cvt.rn.satfinite.e5m2x2.f16x2 %0, %1;" : "=h"(r) : "r"(h[i]));
-      w[i] = r;
-      if (t + 1 < kTerms) {
-        uint32_t d;
-        asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(d) : "h"(r));
-        asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(h[i]) : "r"(h[i]), "r"(d));
-      }
+      const uint32_t r = (h[i] + 0x007F007Fu + ((h[i] >> 8) & 0x00010001u)) & 0xFF00FF00u;
+      // bytes 1 and 3 of r: the lower value's E5M2 in the low byte
+      asm("prmt.b32 %0, %1, 0, 0x0031;" : "=r"(w[i]) : "r"(r));
+      if (t + 1 < kTerms) asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(h[i]) : "r"(h[i]), "r"(r));
     }
     out[t] = make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
   }
@@ -662,7 +695,9 @@ __device__ __forceinline__ void e5_terms_f16(const float *x, uint2 *out, float *
 __device__ __forceinline__ float exp2i(int e) { return __int_as_float((e + 127) << 23); }
 
 // TMEM: this thread's lane, N consecutive 32-bit columns (N a multiple of 8),
-// one wait for all of them.
+// one wait for all of them.  The TMEM loads carry no memory clobber (TMEM is
+// not memory the compiler tracks): volatile keeps them in order with the
+// barrier waits and fences, and shared-memory traffic may overlap them.
 template <int N>
 __device__ __forceinline__ void tmem_load(uint32_t taddr, float *v) {
   static_assert(N % 8 == 0, "columns in groups of 8");
@@ -673,13 +708,12 @@ __device__ __forceinline__ void tmem_load(uint32_t taddr, float *v) {
         "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
         : "=r"(r[c]), "=r"(r[c + 1]), "=r"(r[c + 2]), "=r"(r[c + 3]), "=r"(r[c + 4]),
           "=r"(r[c + 5]), "=r"(r[c + 6]), "=r"(r[c + 7])
-        : "r"(taddr + c)
-        : "memory");
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        : "r"(taddr + c));
+  asm volatile("tcgen05.wait::ld.sync.aligned;");
   // tie every register to the wait so no use is scheduled above it
 #pragma unroll
   for (int c = 0; c < N; ++c) {
-    asm volatile("" : "+r"(r[c]) :: "memory");
+    asm volatile("" : "+r"(r[c]));
     v[c] = __uint_as_float(r[c]);
   }
 }
@@ -695,13 +729,12 @@ __device__ __forceinline__ void tmem_load_sum8(uint32_t taddr, int stride, float
         "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
         : "=r"(r[t][0]), "=r"(r[t][1]), "=r"(r[t][2]), "=r"(r[t][3]), "=r"(r[t][4]),
           "=r"(r[t][5]), "=r"(r[t][6]), "=r"(r[t][7])
-        : "r"(taddr + (uint32_t)(t * stride))
-        : "memory");
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        : "r"(taddr + (uint32_t)(t * stride)));
+  asm volatile("tcgen05.wait::ld.sync.aligned;");
 #pragma unroll
   for (int t = 0; t < T; ++t)
 #pragma unroll
-    for (int c = 0; c < 8; ++c) asm volatile("" : "+r"(r[t][c]) :: "memory");
+    for (int c = 0; c < 8; ++c) asm volatile("" : "+r"(r[t][c]));
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     float a = __uint_as_float(r[0][c]);
@@ -826,6 +859,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kNQ = Lay::kNQ;
   constexpr int kN = Lay::kN;
   const int QS = tp.q_slots;
+  const int PB = tp.p_bufs;
   const LseKernelParams &p = tp.p;
   const int NS = tp.stages;
   const int cta = blockIdx.x;
@@ -838,8 +872,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t k_base = sbase;                                // K ring
   const uint32_t v_base = k_base + NS * Lay::kHalfStage;        // V ring
   const uint32_t q_base = v_base + NS * Lay::kHalfStage;        // Q slots
-  const uint32_t p_base = q_base + QS * Lay::kQBytes;          // P tiles (one per group)
-  uint8_t *misc = smem + (p_base - sbase) + 2 * Lay::kPBytes;
+  const uint32_t p_base = q_base + QS * Lay::kQBytes;          // P tiles [group][buffer]
+  uint8_t *misc = smem + (p_base - sbase) + 2 * PB * Lay::kPBytes;
+  // the P tile of group grp used with its tile of index n (n & 1 == grp)
+  auto p_tile = [&](int grp, int n) {
+    return p_base + (uint32_t)((grp * PB + ((n >> 1) % PB)) * Lay::kPBytes);
+  };
   uint64_t *bars = reinterpret_cast<uint64_t *>(misc);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + Lay::kBars * 8);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + Lay::kBars * 8 + 4);
@@ -927,7 +965,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(kBarDone), 1);
     mbar_init(bar(kBarDoneV), 1);
     for (int i = 0; i < 8; ++i) mbar_init(bar(kBarInfo + i), 1);
-    for (int i = 0; i < 2; ++i) mbar_init(bar(kBarPEmpty + i), 1);
+    for (int i = 0; i < 4; ++i) mbar_init(bar(kBarPEmpty + i), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (tid < 64) pair_row[tid] = tid / p.group;
@@ -1022,7 +1060,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t qfmt = kF8 ? 0u : f16fmt;
     constexpr uint32_t pfmt = kF8 ? 1u : f16fmt;
     const int n_total = (int)(t_stop - t_begin);
-    if (warp == 1 && lane == 0) {
+    // the whole warp runs the loop (uniform operands); one elected lane issues
+    const uint32_t leader = elect_one();
+    if (warp == 1) {
       // ---- S^T = K Q^T into the group's score buffer ----
       constexpr uint32_t idesc_qk = instr_desc(kvfmt, qfmt, 0, 0, kTK, kSW);
       TileIter iq;
@@ -1040,7 +1080,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         go = go && mbar_wait(bar(kBarFullK + st), (nq / NS) & 1, abort_flag, p.err);
         go = go && (nq < 2 ||
                     mbar_wait(bar(kBarPFull + (nq & 1)), ((nq - 2) >> 1) & 1, abort_flag, p.err));
-        if (!go) break;
+        if (!__all_sync(0xffffffffu, go)) break;
         tc_fence_after();
         const uint32_t kaddr = k_base + st * Lay::kHalfStage;
         const uint32_t qaddr = q_base + (seg_q % QS) * Lay::kQBytes;
@@ -1053,24 +1093,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           // K: one 128-dim region, K steps of 32 bytes
 #pragma unroll
           for (int k = 0; k < kD / 32; ++k)
-            mma_f8(d, a0 + (uint64_t)(k * 2), b0 + (uint64_t)(k * 2), idesc_qk, k > 0);
+            mma_f8(d, a0 + (uint64_t)(k * 2), b0 + (uint64_t)(k * 2), idesc_qk, k > 0, leader);
         } else {
           // two 64-dim regions of K and of Q; K steps of 32 bytes
 #pragma unroll
           for (int k = 0; k < kD / 16; ++k) {
             const uint32_t ka = ((k >> 2) * kRegionBytes + (k & 3) * 32) >> 4;
             const uint32_t kb = ((k >> 2) * 2 * Lay::kQRegion + (k & 3) * 32) >> 4;
-            mma_f16(d, a0 + ka, b0 + kb, idesc_qk, k > 0);
+            mma_f16(d, a0 + ka, b0 + kb, idesc_qk, k > 0, leader);
           }
         }
-        mma_commit(bar(kBarEmptyK + st));
-        mma_commit(bar(kBarSFull + (nq & 1)));
-        if (last) mma_commit(bar(kBarQEmpty + seg_q % QS));
+        mma_commit(bar(kBarEmptyK + st), leader);
+        mma_commit(bar(kBarSFull + (nq & 1)), leader);
+        if (last) mma_commit(bar(kBarQEmpty + seg_q % QS), leader);
       }
       // every MMA issued has completed before TMEM is released
-      mma_commit(bar(kBarDone));
+      mma_commit(bar(kBarDone), leader);
       mbar_drain(bar(kBarDone), 0);
-    } else if (warp == 2 && lane == 0) {
+    } else {
       // ---- O^T += V^T P^T into the group's output slot ----
       constexpr uint32_t idesc_pv =
           instr_desc(kvfmt, pfmt, 1, 1, kD, (kF8 && !Lay::kPSide) ? kNQ : kN);
@@ -1096,10 +1136,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           go = go && mbar_wait(bar(kBarOEmpty + 2 * grp + slot), oe_par, abort_flag, p.err);
         if (last && !other)
           go = go && mbar_wait(bar(kBarOEmpty + 2 * (grp ^ 1) + slot), oe_par, abort_flag, p.err);
-        if (!go) break;
+        if (!__all_sync(0xffffffffu, go)) break;
         tc_fence_after();
         const uint32_t vaddr = v_base + st * Lay::kHalfStage;
-        const uint32_t paddr = p_base + grp * Lay::kPBytes;
+        const uint32_t paddr = p_tile(grp, nv);
         const uint32_t d = tmem_o(grp, slot);
         const uint64_t b0 = smem_desc(paddr, Lay::kPLbo, 128, kLayoutNone);
         if constexpr (kF8) {
@@ -1112,13 +1152,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t b = b0 + (uint64_t)(k * 4 * Lay::kPLbo / 16);
             if constexpr (Lay::kPSide) {
               // the P terms side by side along N
-              mma_f8(d, a, b, idesc_pv, (mine || k > 0) ? 1u : 0u);
+              mma_f8(d, a, b, idesc_pv, (mine || k > 0) ? 1u : 0u, leader);
             } else {
               // the P terms accumulate into the same columns
 #pragma unroll
               for (int t = 0; t < kPTerms; ++t)
                 mma_f8(d, a, b + (uint64_t)(t * (kNQ / 16) * 128 / 16), idesc_pv,
-                       (mine || k > 0 || t > 0) ? 1u : 0u);
+                       (mine || k > 0 || t > 0) ? 1u : 0u, leader);
             }
           }
         } else {
@@ -1127,21 +1167,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < kTK / 16; ++k)
             mma_f16(d, a0 + (uint64_t)(k * 2048 / 16), b0 + (uint64_t)(k * 2 * Lay::kPLbo / 16),
-                    idesc_pv, (mine || k > 0) ? 1u : 0u);
+                    idesc_pv, (mine || k > 0) ? 1u : 0u, leader);
         }
         started |= 1u << grp;
-        mma_commit(bar(kBarEmptyV + st));
-        mma_commit(bar(kBarPEmpty + grp));
+        mma_commit(bar(kBarEmptyV + st), leader);
+        mma_commit(bar(kBarPEmpty + 2 * grp + ((nv >> 1) % PB)), leader);
         // this group's last tile of the piece: the tile is the piece's
         // last, or the next one (the other group's) is
         const bool next_is_last =
             !last && (iv.t + 1 == iv.t_end - 1 || iv.tile + 1 == iv.n_tiles - 1);
-        if (last || next_is_last) mma_commit(bar(kBarOFull + 2 * grp + slot));
+        if (last || next_is_last) mma_commit(bar(kBarOFull + 2 * grp + slot), leader);
         // the other group had no tile in this piece: release its (empty)
         // output slot all the same (its previous use was read out)
-        if (last && !other) mma_commit(bar(kBarOFull + 2 * (grp ^ 1) + slot));
+        if (last && !other) mma_commit(bar(kBarOFull + 2 * (grp ^ 1) + slot), leader);
       }
-      mma_commit(bar(kBarDoneV));
+      mma_commit(bar(kBarDoneV), leader);
       mbar_drain(bar(kBarDoneV), 0);
     }
   } else if (warp == 3) {
@@ -1181,7 +1221,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *alpha = alpha_all + grp * 64;
     float *red = red_all + grp * 4 * 64;
     unsigned long long *masks = masks_all + grp * 64;
-    float *scr = reinterpret_cast<float *>(smem + (p_base - sbase) + grp * Lay::kPBytes);
+    // FP32 scratch [key][pair] in one of the group's P tiles
+    auto scratch = [&](int tile_n) {
+      return reinterpret_cast<float *>(smem + (p_tile(grp, tile_n) - sbase));
+    };
     float *isg = isig_all + (2 + grp) * 64;    // FP8: the segment's inverse Q scales
     float *lsum = lsum_all + grp * 64;         // row sums of P of the segment so far
     float *lpart = lpart_all + grp * 2 * 4 * P8;  // [buffer][warp][pair] partials
@@ -1253,9 +1296,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // tile record, published by the producer on its own barrier (the
         // K ring may already hold a later tile)
         if (w) w = mbar_wait(bar(kBarInfo + (n & 7)), (n >> 3) & 1, abort_flag, p.err);
-        // the group's P tile and output are free once its previous P.V (tile
-        // n - 2) has completed
-        if (w && n >= 2) w = mbar_wait(bar(kBarPEmpty + grp), ((n - 2) >> 1) & 1, abort_flag, p.err);
+        // this tile's P buffer is free once the output product that last
+        // read it (the group's tile n - 2 PB) has completed
+        const int pbuf_n = (n >> 1) % PB, use = (n >> 1) / PB;
+        if (w && use >= 1)
+          w = mbar_wait(bar(kBarPEmpty + 2 * grp + pbuf_n), (use - 1) & 1, abort_flag, p.err);
         if (named_or(bar_id, 128, !w)) {
           ok = false;
           break;
@@ -1284,39 +1329,43 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t s_addr = tmem_s(grp) + lane_off;
         __syncwarp();
         if constexpr (!kLAcc) fold();  // the previous tile's partials (written before the barrier above)
-        // pass 1: the score terms (16-bit: Q hi and lo blocks; FP8: four Q-term
-        // blocks, times the pair's inverse Q scale) summed into the first
-        // block; does any score pass the running max by 2^tau?
-        float gap = -INFINITY;
-#pragma unroll 1
+        // pass 1: the key's scores into registers, the score terms summed
+        // (16-bit: Q hi and lo blocks; FP8: four Q-term blocks, times the
+        // pair's inverse Q scale), -inf where not visible; does any score pass
+        // the running max by 2^tau?
+        float sv[P8], mr[P8];
+#pragma unroll
         for (int c = 0; c < P8; c += 8) {
-          float v[8];
-          tmem_load_sum8<kSW / kNQ>(s_addr + c, kNQ, v);
+          tmem_load_sum8<kSW / kNQ>(s_addr + c, kNQ, sv + c);
           if constexpr (kF8) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] *= isg[c + i];
+            for (int i = 0; i < 8; ++i) sv[c + i] *= isg[c + i];
           }
-          tmem_st8(s_addr + c, v);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            if ((vis >> (c + i)) & 1ull) gap = fmaxf(gap, v[i] - m_run[c + i]);
         }
-        tmem_st_wait();
-        if (named_or(bar_id, 128, gap > kTau)) {
-          // per-pair maximum over the tile's keys, through this group's P tile
-          // as FP32 scratch [key][pair] (free: the group's previous P.V has
-          // completed)
-#pragma unroll 1
-          for (int c = 0; c < P8; c += 8) {
-            float v[8];
-            tmem_load<8>(s_addr + c, v);
+        if (vis != ~0ull) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              if (!((vis >> (c + i)) & 1ull)) v[i] = -INFINITY;
-            *reinterpret_cast<float4 *>(scr + j * P8 + c) = make_float4(v[0], v[1], v[2], v[3]);
-            *reinterpret_cast<float4 *>(scr + j * P8 + c + 4) =
-                make_float4(v[4], v[5], v[6], v[7]);
-          }
+          for (int q = 0; q < P8; ++q)
+            if (!((vis >> q) & 1ull)) sv[q] = -INFINITY;
+        }
+#pragma unroll
+        for (int q = 0; q < P8; q += 4) {
+          const float4 m4 = *reinterpret_cast<const float4 *>(m_run + q);
+          mr[q] = m4.x;
+          mr[q + 1] = m4.y;
+          mr[q + 2] = m4.z;
+          mr[q + 3] = m4.w;
+        }
+        float gap = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < P8; ++q) gap = fmaxf(gap, sv[q] - mr[q]);
+        float *scr = scratch(n);
+        if (named_or(bar_id, 128, gap > kTau)) {
+          // per-pair maximum over the tile's keys, through this tile's P
+          // buffer as FP32 scratch [key][pair] (free: waited for above)
+#pragma unroll
+          for (int c = 0; c < P8; c += 4)
+            *reinterpret_cast<float4 *>(scr + j * P8 + c) =
+                make_float4(sv[c], sv[c + 1], sv[c + 2], sv[c + 3]);
           named_sync(bar_id, 128);
           column_reduce<P8, false>(scr, j, red, bar_id);  // red[q] = max over keys
           named_sync(bar_id, 128);
@@ -1329,12 +1378,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             lsum[j] *= al;  // (this thread folded pair j's partials above)
           }
           named_sync(bar_id, 128);
+#pragma unroll
+          for (int q = 0; q < P8; q += 4) {
+            const float4 m4 = *reinterpret_cast<const float4 *>(m_run + q);
+            mr[q] = m4.x;
+            mr[q + 1] = m4.y;
+            mr[q + 2] = m4.z;
+            mr[q + 3] = m4.w;
+          }
           if constexpr (kLAcc) {
 #pragma unroll
             for (int q = 0; q < P8; ++q) lacc[q] *= alpha[q];
           }
           if (had_tile) {
-            // rescale this group's output (the previous P.V has completed)
+            // rescale this group's output once every earlier P.V of the group
+            // has completed (with two P buffers, tile n - 2's used the other)
+            bool wo = true;
+            if (PB == 2 && n >= 2)
+              wo = mbar_wait(bar(kBarPEmpty + 2 * grp + (pbuf_n ^ 1)), (((n >> 1) - 1) >> 1) & 1,
+                             abort_flag, p.err);
+            if (named_or(bar_id, 128, !wo)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
             __syncwarp();
             const uint32_t ob = tmem_o(grp, oslot) + lane_off;
 #pragma unroll 1
@@ -1353,27 +1420,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         // pass 2: probabilities -> this group's P tile, row j (16-bit: hi block
         // then lo block; FP8: P 2^7 as kPTerms E5M2 terms, a block each), and
         // this warp's sums of them per pair
-        uint8_t *prow = smem + (p_base - sbase) + grp * Lay::kPBytes + (j >> 3) * Lay::kPLbo +
-                        (j & 7) * 16;
+        uint8_t *prow = smem + (p_tile(grp, n) - sbase) + (j >> 3) * Lay::kPLbo + (j & 7) * 16;
         const int buf = (n >> 1) & 1;
         float *lp = lpart + buf * 4 * P8 + quarter * P8;
 #pragma unroll
         for (int c = 0; c < P8; c += 8) {
-          float v[8];
-          tmem_load<8>(s_addr + c, v);
           float e[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            e[i] = ((vis >> (c + i)) & 1ull) ? ex2(v[i] - m_run[c + i]) : 0.f;
+          for (int i = 0; i < 8; ++i) e[i] = ex2(sv[c + i] - mr[c + i]);  // 0 where not visible
           if constexpr (kF8) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) e[i] *= (float)(1 << kPScaleLog2);
             uint2 w[kPTerms];
-            float er[8];
-            e5_terms_f16<kPTerms>(e, w, er);
-            // the sums take P as the products see it (rounded to F16)
-#pragma unroll
-            for (int i = 0; i < 8; ++i) e[i] = er[i];
+            e5_terms_f16<kPTerms>(e, w);
             // 16 FP8 columns per core matrix: term t's pair c sits in column
             // t kNQ + c
 #pragma unroll
@@ -1426,8 +1485,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float *lt_of = lsum;  // the group's row sums of P, per pair
         if constexpr (kLAcc) {
-          // column sums of the threads' sums, through the group's P tile as
-          // FP32 scratch [key][pair] (free: the piece's last P.V has completed)
+          // column sums of the threads' sums, through one of the group's P
+          // tiles as FP32 scratch [key][pair] (free: the piece's last P.V has
+          // completed)
+          float *scr = scratch(grp);
 #pragma unroll
           for (int c = 0; c < P8; c += 4)
             *reinterpret_cast<float4 *>(scr + j * P8 + c) =
@@ -1529,21 +1590,21 @@ int launch_tc_p(const TcParams &tp, int p8, int smem, cudaStream_t st) {
 }
 
 template <int DT>
-int smem_for_p(int p8, int stages, int q_slots) {
+int smem_for_p(int p8, int stages, int q_slots, int p_bufs) {
   switch (p8) {
-    case 8: return TcLayout<DT, 8>::smem_bytes(stages, q_slots);
-    case 16: return TcLayout<DT, 16>::smem_bytes(stages, q_slots);
-    case 24: return TcLayout<DT, 24>::smem_bytes(stages, q_slots);
-    case 32: return TcLayout<DT, 32>::smem_bytes(stages, q_slots);
-    case 48: return TcLayout<DT, 48>::smem_bytes(stages, q_slots);
+    case 8: return TcLayout<DT, 8>::smem_bytes(stages, q_slots, p_bufs);
+    case 16: return TcLayout<DT, 16>::smem_bytes(stages, q_slots, p_bufs);
+    case 24: return TcLayout<DT, 24>::smem_bytes(stages, q_slots, p_bufs);
+    case 32: return TcLayout<DT, 32>::smem_bytes(stages, q_slots, p_bufs);
+    case 48: return TcLayout<DT, 48>::smem_bytes(stages, q_slots, p_bufs);
   }
   return -1;
 }
 
-int smem_for(int dtype, int p8, int stages, int q_slots) {
+int smem_for(int dtype, int p8, int stages, int q_slots, int p_bufs) {
   // the two 16-bit formats share a layout, and so do the two 8-bit ones
-  return is_f8(dtype) ? smem_for_p<LSE_KV_FP8_E4M3>(p8, stages, q_slots)
-                      : smem_for_p<LSE_KV_BF16>(p8, stages, q_slots);
+  return is_f8(dtype) ? smem_for_p<LSE_KV_FP8_E4M3>(p8, stages, q_slots, p_bufs)
+                      : smem_for_p<LSE_KV_BF16>(p8, stages, q_slots, p_bufs);
 }
 
 }  // namespace
@@ -1557,18 +1618,24 @@ int lse_tc_pairs_bucket(int pairs) {
   return -1;
 }
 
-// The deepest K/V ring that fits (stages count more than a second Q slot,
-// which only overlaps Q staging with the end of the previous segment).
-int lse_tc_smem(int dtype, int p8, int smem_optin, int *stages, int *q_slots) {
-  for (int ns = kMaxStages; ns >= 2; --ns)
-    for (int qs = 2; qs >= 1; --qs) {
-      const int b = smem_for(dtype, p8, ns, qs);
-      if (b > 0 && b <= smem_optin) {
-        *stages = ns;
-        *q_slots = qs;
-        return b;
+// Shared-memory configuration: the deepest K/V ring with one P tile per
+// softmax group (the groups then alternate on the SM's pipes, which their
+// exponentials and conversions keep busy), a second Q slot (overlapping Q
+// staging with the end of the previous segment) when it fits as well.  The
+// kernel also runs with two P tiles per group (p_bufs = 2), which the planner
+// does not pick.
+int lse_tc_smem(int dtype, int p8, int smem_optin, int *stages, int *q_slots, int *p_bufs) {
+  for (int pb = 1; pb >= 1; --pb)
+    for (int ns = kMaxStages; ns >= 2; --ns)
+      for (int qs = 2; qs >= 1; --qs) {
+        const int b = smem_for(dtype, p8, ns, qs, pb);
+        if (b > 0 && b <= smem_optin) {
+          *stages = ns;
+          *q_slots = qs;
+          *p_bufs = pb;
+          return b;
+        }
       }
-    }
   return -1;
 }
 
@@ -1612,7 +1679,8 @@ size_t lse_tc_map_bytes() { return sizeof(CUtensorMap); }
 
 int lse_launch_partial_tcgen05(const LseKernelParams &p, const void *maps, int n_maps,
                                int dtype, int p8, int n_ctas, int n_slots, int stages,
-                               int q_slots, int box_tokens, int smem, void *stream) {
+                               int q_slots, int p_bufs, int box_tokens, int smem,
+                               void *stream) {
   static_assert(sizeof(TcParams) < 30000, "kernel parameter block too large");
   TcParams tp;
   memset(&tp, 0, sizeof tp);
@@ -1622,6 +1690,7 @@ int lse_launch_partial_tcgen05(const LseKernelParams &p, const void *maps, int n
   tp.n_slots = n_slots;
   tp.stages = stages;
   tp.q_slots = q_slots;
+  tp.p_bufs = p_bufs;
   tp.box_tokens = box_tokens;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   switch (dtype) {
