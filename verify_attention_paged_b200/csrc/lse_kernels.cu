@@ -363,39 +363,59 @@ __device__ __forceinline__ int seq_tiles_merge(const LseKernelParams &p, int s, 
   return (L + 127) / 128;
 }
 
-// One CTA (4 warps) per (query head, row of a sequence): grid (Hq, max_rows,
-// n_seqs).  The CTA first finds the live partials of its (sequence, kv head)
-// and their maximum lse; each warp then sums a quarter of the partials
-// (each lane a D/32 slice of the head dim, eight partial rows in flight at
-// a time) and the four sums are combined in shared memory.
+constexpr int kMergeWarps = 16;
+constexpr int kMergeThreads = kMergeWarps * 32;
+
+// One CTA (16 warps) per (query head, row of a sequence): grid (Hq, max_rows,
+// n_seqs).  Before waiting for the partial pass the CTA works out which
+// partials of its (sequence, kv head) are live (the sequence scan reads only
+// call inputs, so it overlaps the partial pass's tail).  Each warp then loads
+// its share of the partials (warp w: partials w, w + 16, ..., eight in
+// flight per lane, each lane a D/32 slice of the head dim) and keeps a
+// running maximum of their lse; the warps' sums are rescaled to the common
+// maximum and added in warp order in shared memory.
 template <int D>
-__global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ LseKernelParams p) {
+__global__ void __launch_bounds__(kMergeThreads) merge_kernel(
+    const __grid_constant__ LseKernelParams p) {
   constexpr int kPerLane = D / 32;
   constexpr int kUnroll = 8;
-  __shared__ float s_red[4];
-  __shared__ float s_acc[4][D];
-  __shared__ float s_w[4];
-  // partials are written by the preceding partial pass (programmatic launch)
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ float s_m[kMergeWarps], s_w[kMergeWarps];
+  __shared__ float s_acc[kMergeWarps][D];
+  __shared__ long long s_cnt[kMergeWarps][2];
   const int h = blockIdx.x, r = blockIdx.y, s = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int L, row0, R;
-  if (!seq_shape(p, s, L, row0, R)) return;
-  if (r >= R) return;
-  const int row = row0 + r;
-  int n_live;
+  const bool live_row = seq_shape(p, s, L, row0, R) && r < R;
+  int n_live = 0;
   if (p.balanced) {
     // pieces of (s, kv head) written by the persistent tensor-core pass:
-    // tiles of all segments end to end, CTA c owning [c U / C, (c+1) U / C)
-    long long U = 0, before = 0;
-    int n_s = 0;
-    for (int q = 0; q < p.n_seqs; ++q) {
+    // tiles of all segments end to end, CTA c owning [c U / C, (c+1) U / C);
+    // the tiles before sequence s and in all, summed over the CTA
+    long long mine_before = 0, mine_all = 0;
+    for (int q = tid; q < p.n_seqs; q += kMergeThreads) {
       int Lq, r0q, Rq;
       const int n = seq_tiles_merge(p, q, Lq, r0q, Rq);
-      if (q < s) before += n;
-      if (q == s) n_s = n;
-      U += n;
+      mine_all += n;
+      if (q < s) mine_before += n;
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mine_before += __shfl_xor_sync(0xffffffffu, mine_before, o);
+      mine_all += __shfl_xor_sync(0xffffffffu, mine_all, o);
+    }
+    if (lane == 0) {
+      s_cnt[warp][0] = mine_before;
+      s_cnt[warp][1] = mine_all;
+    }
+    __syncthreads();
+    long long before = 0, U = 0;
+#pragma unroll
+    for (int w = 0; w < kMergeWarps; ++w) {
+      before += s_cnt[w][0];
+      U += s_cnt[w][1];
+    }
+    int Ls, r0s, Rs;
+    const int n_s = seq_tiles_merge(p, s, Ls, r0s, Rs);
     U *= p.n_kv_heads;
     const int g = h / p.group;
     const long long first = before * p.n_kv_heads + (long long)g * n_s;
@@ -403,57 +423,75 @@ __global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ LseK
     const long long C = U < p.n_ctas ? U : p.n_ctas;  // working CTAs of the partial pass
     // two partials (one per softmax group) per piece
     n_live = n_s > 0 ? 2 * (int(((last + 1) * C - 1) / U - ((first + 1) * C - 1) / U) + 1) : 0;
-  } else {
+  } else if (live_row) {
     n_live = min((L + p.keys_per_split - 1) / p.keys_per_split, p.n_splits);
   }
+  // partials are written by the preceding partial pass (programmatic launch)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (!live_row) return;  // uniform over the CTA
+  const int row = row0 + r;
   const long long base = ((long long)row * p.n_q_heads + h) * p.n_splits;
   const float *lse = p.lse_part + base;
   const float *o = p.o_part + base * D;
 
-  // maximum lse over the live partials (all 128 threads)
-  float M = -INFINITY;
-  for (int i = tid; i < n_live; i += 128) M = fmaxf(M, lse[i]);
-  M = warp_max(M);
-  if (lane == 0) s_red[warp] = M;
-  __syncthreads();
-  M = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
-
+  // this warp's partials, kUnroll at a time, with a running maximum
+  float m = -INFINITY, wsum = 0.f;
   float acc[kPerLane];
 #pragma unroll
   for (int k = 0; k < kPerLane; ++k) acc[k] = 0.f;
-  float wsum = 0.f;
-  if (M != -INFINITY) {
-    // warp w takes partials w, w + 4, w + 8, ...
-    for (int i0 = warp; i0 < n_live; i0 += 4 * kUnroll) {
-      float v[kUnroll][kPerLane];
-      float w[kUnroll];
+  for (int i0 = warp; i0 < n_live; i0 += kMergeWarps * kUnroll) {
+    float li[kUnroll], v[kUnroll][kPerLane];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int i = i0 + 4 * u;
-        const bool in = i < n_live;
-        const float li = in ? lse[i] : -INFINITY;
-        w[u] = li == -INFINITY ? 0.f : exp2f(li - M);  // empty partial: weight 0
+    for (int u = 0; u < kUnroll; ++u) {
+      const int i = i0 + kMergeWarps * u;
+      const bool in = i < n_live;
+      li[u] = in ? lse[i] : -INFINITY;
 #pragma unroll
-        for (int k = 0; k < kPerLane; ++k)
-          v[u][k] = in ? o[(long long)i * D + lane + 32 * k] : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        wsum += w[u];
-#pragma unroll
-        for (int k = 0; k < kPerLane; ++k) acc[k] = fmaf(w[u], v[u][k], acc[k]);
-      }
+      for (int k = 0; k < kPerLane; ++k)
+        v[u][k] = in ? o[(long long)i * D + lane + 32 * k] : 0.f;
     }
+    float mc = m;
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) mc = fmaxf(mc, li[u]);
+    if (mc == -INFINITY) continue;  // nothing live yet
+    const float sc = exp2f(m - mc);  // 0 when m = -inf
+    wsum *= sc;
+#pragma unroll
+    for (int k = 0; k < kPerLane; ++k) acc[k] *= sc;
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const float w = li[u] == -INFINITY ? 0.f : exp2f(li[u] - mc);  // empty partial: 0
+      wsum += w;
+#pragma unroll
+      for (int k = 0; k < kPerLane; ++k) acc[k] = fmaf(w, v[u][k], acc[k]);
+    }
+    m = mc;
   }
 #pragma unroll
   for (int k = 0; k < kPerLane; ++k) s_acc[warp][lane + 32 * k] = acc[k];
-  if (lane == 0) s_w[warp] = wsum;
+  if (lane == 0) {
+    s_m[warp] = m;
+    s_w[warp] = wsum;
+  }
   __syncthreads();
-  const float wt = s_w[0] + s_w[1] + s_w[2] + s_w[3];
+  float M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kMergeWarps; ++w) M = fmaxf(M, s_m[w]);
+  float scale[kMergeWarps];
+  float wt = 0.f;
+#pragma unroll
+  for (int w = 0; w < kMergeWarps; ++w) {
+    scale[w] = s_m[w] == -INFINITY ? 0.f : exp2f(s_m[w] - M);
+    wt += s_w[w] * scale[w];
+  }
   const float inv = wt > 0.f ? 1.f / wt : 0.f;
   float *out = p.out + ((long long)row * p.n_q_heads + h) * D;
-  for (int d = tid; d < D; d += 128)
-    out[d] = (s_acc[0][d] + s_acc[1][d] + s_acc[2][d] + s_acc[3][d]) * inv;
+  for (int d = tid; d < D; d += kMergeThreads) {
+    float a = 0.f;
+#pragma unroll
+    for (int w = 0; w < kMergeWarps; ++w) a += s_acc[w][d] * scale[w];
+    out[d] = a * inv;
+  }
   if (p.lse_out && tid == 0)
     p.lse_out[(long long)row * p.n_q_heads + h] =
         wt > 0.f ? (M + log2f(wt)) * 0.69314718055994530942f : -INFINITY;
@@ -536,7 +574,7 @@ template <int D>
 int launch_merge_d(const LseKernelParams &p, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.n_q_heads, p.max_rows, p.n_seqs);
-  cfg.blockDim = dim3(128, 1, 1);
+  cfg.blockDim = dim3(kMergeThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
