@@ -214,6 +214,28 @@ def test_tcgen05_pairs_and_trees(binding, dtype, heads, rows):
     check_kernel(binding, w, "tcgen05")
 
 
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "e4m3"])
+@pytest.mark.parametrize("heads,rows", [((24, 4), 16), ((32, 4), 12), ((16, 1), 8),
+                                        ((24, 4), 9)])
+def test_tcgen05_row_chunks(binding, dtype, heads, rows):
+    # more (row, head) pairs per kv head than one score tile holds: the rows
+    # are cut into chunks of floor(48 / G), each a segment of its own over
+    # all of the sequence's keys (trees, ragged chunks, idle and short
+    # sequences)
+    hq, hkv = heads
+    lens = [3000, rows, 700, 4100, 64, 1]
+    rws = [rows, rows, max(1, rows // 2), rows, min(rows, 64), 1]
+    w = wl.small_case(dtype, lens, rws, n_q_heads=hq, n_kv_heads=hkv, head_dim=128,
+                      tokens_per_fragment=128, tree=True, seed=230 + rows + hq)
+    (out, lse, info), err = gpu_run(binding, w, kernel="tcgen05")
+    G = hq // hkv
+    assert info["rows_per_chunk"] == (rows if G * rows <= 48 else 48 // G)
+    assert err == 0
+    ref_out, ref_lse = orc.attention(to_problem(w))
+    assert_close(out, ref_out, w.dtype)
+    np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=lse_tol(w.dtype) * 4)
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
 def test_tcgen05_many_segments_per_cta(binding, dtype):
     # 70 short sequences: CTAs cross many (sequence, kv head) segments, so the
@@ -297,9 +319,10 @@ def test_tcgen05_bad_page_sets_error_word(binding, dtype):
     assert err & binding.DEVERR_BAD_FRAGMENT and not err & binding.DEVERR_TIMEOUT
 
 
-def test_plan_picks_tensor_cores_for_the_bf16_and_fp8_workloads(binding):
+def test_plan_picks_tensor_cores_for_the_16_bit_and_fp8_workloads(binding):
     for name, want in (("batched_decode", "tcgen05"), ("chain_verify", "tcgen05"),
-                       ("long_fp8", "tcgen05"), ("tiny_decode", "cuda_core")):
+                       ("long_fp8", "tcgen05"), ("tree_verify", "tcgen05"),
+                       ("tiny_decode", "cuda_core")):
         w = wl.BUILDERS[name]()
         call = binding.DeviceCall(w)
         assert call.info["kernel_name"] == want, name

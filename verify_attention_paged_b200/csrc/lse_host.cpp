@@ -270,12 +270,16 @@ int lse_attn_plan_ex(const lse_kv_arena *a, int n_seqs, int max_rows, int max_to
   pl->n_sms = n_sms;
 
   // kernel choice and its on-chip memory check.  The tensor-core kernel
-  // takes 16-bit and FP8 K/V with head_dim 128, up to 48 (row, head) pairs
-  // per kv head, and fragments whose token count tiles evenly into 128-key
-  // tiles.
+  // takes 16-bit and FP8 K/V with head_dim 128 and fragments whose token
+  // count tiles evenly into 128-key tiles.  A kv head's (row, head) pairs
+  // must fit one score tile (48); more rows are cut into row chunks of
+  // floor(48 / G) rows, each reading the sequence's keys again.
   const int T = a->tokens_per_fragment;
   const bool t_ok = (T % 128 == 0) || (T >= 8 && T % 8 == 0 && 128 % T == 0);
-  const int p8 = lse_tc_pairs_bucket(pl->pairs);
+  const int max_tile_pairs = 48;
+  const int rows_per_chunk =
+      pl->pairs <= max_tile_pairs ? max_rows : max_tile_pairs / pl->group;
+  const int p8 = rows_per_chunk > 0 ? lse_tc_pairs_bucket(pl->group * rows_per_chunk) : -1;
   int tc_stages = 0, tc_q_slots = 0, tc_p_bufs = 0;
   const int tc_smem =
       p8 > 0 ? lse_tc_smem(a->dtype, p8, smem_optin, &tc_stages, &tc_q_slots, &tc_p_bufs) : -1;
@@ -289,6 +293,7 @@ int lse_attn_plan_ex(const lse_kv_arena *a, int n_seqs, int max_rows, int max_to
     pl->q_slots = tc_q_slots;
     pl->p_bufs = tc_p_bufs;
     pl->pairs_bucket = p8;
+    pl->rows_per_chunk = rows_per_chunk;
     pl->box_tokens = T < tile ? T : tile;
     pl->ctas = n_sms;
     const int64_t cap_tiles = ceil_div(cap_keys, tile);
@@ -343,6 +348,7 @@ int lse_attn_plan_query(const lse_attn_plan_t *pl, lse_attn_plan_info *info) {
   info->stages = tc ? pl->stages : 0;
   info->q_slots = tc ? pl->q_slots : 0;
   info->p_bufs = tc ? pl->p_bufs : 0;
+  info->rows_per_chunk = tc ? pl->rows_per_chunk : 0;
   return LSE_OK;
 }
 
@@ -377,6 +383,7 @@ static int fill_params(const lse_attn_plan_t *pl, void *ws, LseKernelParams &p, 
   p.max_rows = pl->max_rows;
   p.max_total_rows = pl->max_total_rows;
   p.n_seqs = pl->n_seqs;
+  p.rows_per_chunk = pl->rows_per_chunk > 0 ? pl->rows_per_chunk : 1;
   char *base = static_cast<char *>(ws);
   p.err = reinterpret_cast<unsigned int *>(base);
   p.o_part = reinterpret_cast<float *>(base + pl->ws_o_off);

@@ -49,6 +49,7 @@ struct lse_attn_plan_s {
   int q_slots = 0;       // and its Q ring depth
   int p_bufs = 0;        // and its P tiles per softmax group
   int pairs_bucket = 0;  // its compile-time pair count (P8)
+  int rows_per_chunk = 0;  // tensor-core kernel: query rows per segment
   int box_tokens = 0;    // its TMA box height
   // tensor maps of the arena chunks (built on first run, rebuilt on growth)
   mutable std::vector<uint8_t> maps;
@@ -90,6 +91,7 @@ struct LseKernelParams {
   unsigned int *err;
   float *out;
   float *lse_out;
+  int rows_per_chunk;  // tcgen05: query rows per segment (row chunk)
   int balanced;    // merge: 1 = slots are persistent-CTA pieces (tcgen05)
   int n_ctas;      // persistent grid size when balanced
 };

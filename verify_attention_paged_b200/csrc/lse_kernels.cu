@@ -388,15 +388,19 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
   const bool live_row = seq_shape(p, s, L, row0, R) && r < R;
   int n_live = 0;
   if (p.balanced) {
-    // pieces of (s, kv head) written by the persistent tensor-core pass:
-    // tiles of all segments end to end, CTA c owning [c U / C, (c+1) U / C);
-    // the tiles before sequence s and in all, summed over the CTA
+    // pieces of the row's segment (sequence, row chunk, kv head) written by
+    // the persistent tensor-core pass: the tiles of all segments end to end
+    // (per sequence: row chunks x kv heads segments of its tiles), CTA c
+    // owning [c U / C, (c+1) U / C); the tiles before sequence s and in all,
+    // summed over the CTA
+    const int Rc = p.rows_per_chunk;
     long long mine_before = 0, mine_all = 0;
     for (int q = tid; q < p.n_seqs; q += kMergeThreads) {
       int Lq, r0q, Rq;
       const int n = seq_tiles_merge(p, q, Lq, r0q, Rq);
-      mine_all += n;
-      if (q < s) mine_before += n;
+      const long long tq = (long long)n * ((Rq + Rc - 1) / Rc) * p.n_kv_heads;
+      mine_all += tq;
+      if (q < s) mine_before += tq;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -416,9 +420,8 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
     }
     int Ls, r0s, Rs;
     const int n_s = seq_tiles_merge(p, s, Ls, r0s, Rs);
-    U *= p.n_kv_heads;
     const int g = h / p.group;
-    const long long first = before * p.n_kv_heads + (long long)g * n_s;
+    const long long first = before + ((long long)(r / Rc) * p.n_kv_heads + g) * n_s;
     const long long last = first + n_s - 1;
     const long long C = U < p.n_ctas ? U : p.n_ctas;  // working CTAs of the partial pass
     // two partials (one per softmax group) per piece

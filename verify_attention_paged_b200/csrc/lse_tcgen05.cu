@@ -298,23 +298,33 @@ __device__ __forceinline__ int seq_tiles(const LseKernelParams &p, int s, int &L
   return R == 0 ? 0 : (L + kTK - 1) / kTK;
 }
 
+// Row chunks of a sequence: its R query rows are cut into chunks of at most
+// rows_per_chunk rows (so a chunk's (row, head) pairs fit one score tile);
+// each chunk reads all of the sequence's keys.
+__device__ __forceinline__ int seq_chunks(const LseKernelParams &p, int R) {
+  return (R + p.rows_per_chunk - 1) / p.rows_per_chunk;
+}
+
 // Per-sequence record built once per CTA in shared memory (sequences up to
-// kSeqTab): tiles before the sequence (all kv heads counted once), its
-// tiles, L, first row, R.
+// kSeqTab): tiles of all segments before the sequence, its 128-key tiles,
+// L, first row, R.
 constexpr int kSeqTab = 256;
 struct SeqRec {
   int prefix, n_tiles, L, row0, R;
 };
 
-// Walks the CTA's contiguous range of global tiles, segment by segment.  With
-// a sequence table it looks sequences up in shared memory; without one (more
-// sequences than the table holds) it reads them from global memory.
+// Walks the CTA's contiguous range of global tiles, segment by segment.  The
+// segments of a sequence are (row chunk, kv head), chunk-major, each of
+// n_tiles tiles.  With a sequence table it looks sequences up in shared
+// memory; without one (more sequences than the table holds) it reads them
+// from global memory.
 struct TileIter {
-  int s, g, tile, n_tiles;   // segment (sequence, kv head) and tile within it
-  int L, row0, R;
-  long long seg_first;       // global index of the segment's first tile
-  long long t, t_end;        // current / end global tile
-  const SeqRec *tab;         // shared-memory sequence table or null
+  int s, c, g, tile, n_tiles;  // segment (sequence, row chunk, kv head), tile within it
+  int n_chunks;
+  int L, row0, R;              // the sequence
+  long long seg_first;         // global index of the segment's first tile
+  long long t, t_end;          // current / end global tile
+  const SeqRec *tab;           // shared-memory sequence table or null
 
   __device__ int tiles_of(const LseKernelParams &p, int q) {
     if (tab) {
@@ -332,6 +342,7 @@ struct TileIter {
       const int n = tiles_of(p, s);
       if (n > 0) {
         n_tiles = n;
+        n_chunks = seq_chunks(p, R);
         return;
       }
       ++s;
@@ -352,27 +363,35 @@ struct TileIter {
       int lo = 0, hi = p.n_seqs - 1;
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if ((long long)tab[mid].prefix * p.n_kv_heads <= t) lo = mid;
+        if ((long long)tab[mid].prefix <= t) lo = mid;
         else hi = mid - 1;
       }
       s = lo;
-      base = (long long)tab[s].prefix * p.n_kv_heads;
+      base = tab[s].prefix;
       next_seq(p);
     } else {
       next_seq(p);
-      while (base + (long long)p.n_kv_heads * n_tiles <= t) {
-        base += (long long)p.n_kv_heads * n_tiles;
+      while (base + (long long)n_chunks * p.n_kv_heads * n_tiles <= t) {
+        base += (long long)n_chunks * p.n_kv_heads * n_tiles;
         ++s;
         next_seq(p);
       }
     }
-    g = int((t - base) / n_tiles);
-    tile = int((t - base) - (long long)g * n_tiles);
-    seg_first = base + (long long)g * n_tiles;
+    const int sg = int((t - base) / n_tiles);  // segment within the sequence
+    c = sg / p.n_kv_heads;
+    g = sg - c * p.n_kv_heads;
+    tile = int((t - base) - (long long)sg * n_tiles);
+    seg_first = base + (long long)sg * n_tiles;
   }
   __device__ bool valid() const { return t < t_end; }
   __device__ bool seg_start(long long t_begin) const { return t == t_begin || tile == 0; }
   __device__ bool seg_end() const { return t == t_end - 1 || tile == n_tiles - 1; }
+  // the segment's rows: global index of the first, count, and offset of the
+  // first within the sequence
+  __device__ int crow0(const LseKernelParams &p) const { return row0 + c * p.rows_per_chunk; }
+  __device__ int crows(const LseKernelParams &p) const {
+    return min(p.rows_per_chunk, R - c * p.rows_per_chunk);
+  }
   __device__ void advance(const LseKernelParams &p) {
     ++t;
     if (t >= t_end) return;
@@ -381,8 +400,11 @@ struct TileIter {
       seg_first += n_tiles;
       if (++g == p.n_kv_heads) {
         g = 0;
-        ++s;
-        next_seq(p);
+        if (++c == n_chunks) {
+          c = 0;
+          ++s;
+          next_seq(p);
+        }
       }
     }
   }
@@ -922,7 +944,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         n = 0;
       }
       if (use_tab) seq_tab[q] = SeqRec{0, n, L, r0, R};
-      mine += n;
+      // all segments of the sequence: row chunks x kv heads
+      mine += (long long)n * (n > 0 ? seq_chunks(p, R) : 0) * p.n_kv_heads;
     }
     long long incl = mine;
 #pragma unroll
@@ -934,11 +957,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       long long run = incl - mine;
       for (int q = s0; q < s1; ++q) {
         seq_tab[q].prefix = (int)run;
-        run += seq_tab[q].n_tiles;
+        const int n = seq_tab[q].n_tiles;
+        run += (long long)n * (n > 0 ? seq_chunks(p, seq_tab[q].R) : 0) * p.n_kv_heads;
       }
     }
     bad = __any_sync(0xffffffffu, bad);
-    if (lane == 31) *shared_u = incl * p.n_kv_heads;
+    if (lane == 31) *shared_u = incl;
     if (lane == 0 && bad && cta == 0) atomicOr(p.err, LSE_DEVERR_BAD_LENGTH);
   }
   const SeqRec *tab = use_tab ? seq_tab : nullptr;
@@ -1198,7 +1222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int slot = seg % QS;
       uint8_t *qs = smem + (q_base - sbase) + slot * Lay::kQBytes;
       const bool okq = stage_q<DT, P8, 32>(
-          p, lane, it.g, it.row0, G * it.R, qs, isig_all + slot * 64, [&]() {
+          p, lane, it.g, it.crow0(p), G * it.crows(p), qs, isig_all + slot * 64, [&]() {
             return mbar_wait(bar(kBarQEmpty + slot), ((seg / QS) & 1) ^ 1, abort_flag, p.err);
           });
       if (!okq) break;
@@ -1249,8 +1273,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
     for (; it.valid() && ok; it.advance(p), ++n) {
       const bool first = it.seg_start(t_begin), last = it.seg_end();
-      const int P = G * it.R;
-      const int Cctx = it.L - it.R;
+      const int P = G * it.crows(p);     // (row, head) pairs of the segment
+      const int Cctx = it.L - it.R;      // context keys (all rows are drafts)
       const int oslot = (seg + (first ? 1 : 0)) % kOS;
       if (first) {
         ++seg;
@@ -1264,13 +1288,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int q = 0; q < P8; ++q) lacc[q] = 0.f;
         }
-        if (j < it.R)
-          masks[j] = p.row_masks ? p.row_masks[it.row0 + j]
-                                 : (j >= 63 ? ~0ull : ((1ull << (j + 1)) - 1ull));
+        if (j < it.crows(p)) {
+          // the chunk's rows; the default mask is the chain (row r sees drafts
+          // 0 .. r of its sequence)
+          const int r = it.c * p.rows_per_chunk + j;
+          masks[j] = p.row_masks ? p.row_masks[it.row0 + r]
+                                 : (r >= 63 ? ~0ull : ((1ull << (r + 1)) - 1ull));
+        }
         had_tile = false;
         if (seg == 0 && grp == 0) {
           // the first segment's Q (slot 0, never used before)
-          stage_q<DT, P8, 128>(p, j, it.g, it.row0, P, smem + (q_base - sbase), isig_all,
+          stage_q<DT, P8, 128>(p, j, it.g, it.crow0(p), P, smem + (q_base - sbase), isig_all,
                                [] { return true; });
           named_sync(bar_id, 128);
           if (j == 0) mbar_arrive(bar(kBarQFull));
@@ -1508,7 +1536,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ob = tmem_o(grp, oslot) + lane_off;
         const long long row_stride = (long long)p.n_q_heads * tp.n_slots * kD;
         const long long base =
-            ((long long)it.row0 * p.n_q_heads + it.g * G) * tp.n_slots + slot;
+            ((long long)it.crow0(p) * p.n_q_heads + it.g * G) * tp.n_slots + slot;
 #pragma unroll 1
         for (int c = 0; c < P8; c += 8) {
           float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
