@@ -19,6 +19,7 @@
 #include <cuda_runtime.h>
 
 #include <cfloat>
+#include <climits>
 #include <cstdint>
 
 #include "lse_internal.h"
@@ -363,17 +364,18 @@ __device__ __forceinline__ int seq_tiles_merge(const LseKernelParams &p, int s, 
   return (L + 127) / 128;
 }
 
-constexpr int kMergeWarps = 16;
+constexpr int kMergeWarps = 8;
 constexpr int kMergeThreads = kMergeWarps * 32;
 
-// One CTA (16 warps) per (query head, row of a sequence): grid (Hq, max_rows,
-// n_seqs).  Before waiting for the partial pass the CTA works out which
-// partials of its (sequence, kv head) are live (the sequence scan reads only
-// call inputs, so it overlaps the partial pass's tail).  Each warp then loads
-// its share of the partials (warp w: partials w, w + 16, ..., eight in
-// flight per lane, each lane a D/32 slice of the head dim) and keeps a
-// running maximum of their lse; the warps' sums are rescaled to the common
-// maximum and added in warp order in shared memory.
+// One CTA (8 warps) per (row, query head) of the call's rows: blockIdx.x =
+// row * Hq + head.  Before waiting for the partial pass the CTA finds the
+// row's sequence and which partials of its segment are live (the scan over
+// the sequences reads only call inputs, all threads at once, so it overlaps
+// the partial pass's tail).  Each warp then loads its share of the partials
+// (warp w: partials w, w + 8, ..., eight in flight per lane, each lane a D/32
+// slice of the head dim) and keeps a running maximum of their lse; the
+// warps' sums are rescaled to the common maximum and added in warp order in
+// shared memory.
 template <int D>
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
     const __grid_constant__ LseKernelParams p) {
@@ -382,12 +384,22 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
   __shared__ float s_m[kMergeWarps], s_w[kMergeWarps];
   __shared__ float s_acc[kMergeWarps][D];
   __shared__ long long s_cnt[kMergeWarps][2];
-  const int h = blockIdx.x, r = blockIdx.y, s = blockIdx.z;
+  __shared__ int s_seq;
+  const int h = blockIdx.x % p.n_q_heads;
+  const int grow = blockIdx.x / p.n_q_heads;  // the row, over all sequences
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  int L, row0, R;
-  const bool live_row = seq_shape(p, s, L, row0, R) && r < R;
+  // the sequence holding the row: every thread tests its share of them
+  if (tid == 0) s_seq = INT_MAX;
+  __syncthreads();
+  for (int q = tid; q < p.n_seqs; q += kMergeThreads)
+    if (p.row_offsets[q] <= grow && grow < p.row_offsets[q + 1]) atomicMin(&s_seq, q);
+  __syncthreads();
+  const int s = s_seq;
+  int L = 0, row0 = 0, R = 0;
+  const bool live_row = s != INT_MAX && seq_shape(p, s, L, row0, R);
+  const int r = grow - row0;  // row within the sequence
   int n_live = 0;
-  if (p.balanced) {
+  if (p.balanced && live_row) {
     // pieces of the row's segment (sequence, row chunk, kv head) written by
     // the persistent tensor-core pass: the tiles of all segments end to end
     // (per sequence: row chunks x kv heads segments of its tiles), CTA c
@@ -432,7 +444,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
   // partials are written by the preceding partial pass (programmatic launch)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   if (!live_row) return;  // uniform over the CTA
-  const int row = row0 + r;
+  const int row = grow;
   const long long base = ((long long)row * p.n_q_heads + h) * p.n_splits;
   const float *lse = p.lse_part + base;
   const float *o = p.o_part + base * D;
@@ -576,7 +588,7 @@ int lse_launch_partial_cuda_core(const LseKernelParams &p, int dtype, int head_d
 template <int D>
 int launch_merge_d(const LseKernelParams &p, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.n_q_heads, p.max_rows, p.n_seqs);
+  cfg.gridDim = dim3((unsigned)p.max_total_rows * (unsigned)p.n_q_heads, 1, 1);
   cfg.blockDim = dim3(kMergeThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
