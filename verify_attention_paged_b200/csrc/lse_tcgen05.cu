@@ -580,7 +580,7 @@ struct TcLayout {
   // [2 groups][2 buffers][4 warps][P8]
   static constexpr int kLBytes = 2 * 64 * 4 + 2 * 2 * 4 * P8 * 4;
   static constexpr int kMiscBytes = kBars * 8 + 16 + 2 * 64 * 4 * 2 + 2 * 4 * 64 * 4 +
-                                    2 * 64 * 8 + 64 * 4 + 8 * 16 + 2 * 32 * 16 * 4 +
+                                    2 * 64 * 8 * 2 + 64 * 4 + 8 * 16 + 2 * 32 * 16 * 4 +
                                     (kF8 ? 4 * 64 * 4 : 0) + kLBytes +
                                     kSeqTab * (int)sizeof(SeqRec);
   // one K or V tile: 128 keys of 128 dims (two 64-dim regions when 16-bit)
@@ -909,7 +909,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   float *red_all = alpha_all + 2 * 64;                                       // [2][4][64]
   unsigned long long *masks_all =
       reinterpret_cast<unsigned long long *>(red_all + 2 * 4 * 64);          // [2][64]
-  int *pair_row = reinterpret_cast<int *>(masks_all + 2 * 64);               // [64]
+  // per softmax group and draft key k of the sequence: the pairs that see it
+  unsigned long long *visk_all = masks_all + 2 * 64;                         // [2][64]
+  int *pair_row = reinterpret_cast<int *>(visk_all + 2 * 64);                // [64]
   // ring of 8 per-tile records written by the producer before its arrival on
   // the tile's K barrier: {K box mask, V box mask, keys of the tile below L}
   uint4 *tile_info = reinterpret_cast<uint4 *>(pair_row + 64);               // [8]
@@ -1245,6 +1247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *alpha = alpha_all + grp * 64;
     float *red = red_all + grp * 4 * 64;
     unsigned long long *masks = masks_all + grp * 64;
+    unsigned long long *visk = visk_all + grp * 64;
     // FP32 scratch [key][pair] in one of the group's P tiles
     auto scratch = [&](int tile_n) {
       return reinterpret_cast<float *>(smem + (p_tile(grp, tile_n) - sbase));
@@ -1317,6 +1320,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         if (kF8 && j == 0) mbar_arrive(bar(kBarQEmpty + seg % QS));
+        if (j < it.R) {
+          // draft key j of the sequence: the pairs (G per row) whose row's
+          // mask has bit j (read at the next group barrier)
+          unsigned long long v = 0;
+          const int cr = it.crows(p);
+          const unsigned long long row_pairs = G >= 64 ? ~0ull : ((1ull << G) - 1ull);
+#pragma unroll 1
+          for (int r = 0; r < cr; ++r)
+            if ((masks[r] >> j) & 1ull) v |= row_pairs << (r * G);
+          visk[j] = v;
+        }
       }
       if ((n & 1) == grp) {
         bool w = mbar_wait(bar(kBarSFull + grp), (n >> 1) & 1, abort_flag, p.err);
@@ -1345,13 +1359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           vis = 0;
           if (kvalid) {
-            if (key < Cctx) {
-              vis = P >= 64 ? ~0ull : ((1ull << P) - 1ull);
-            } else {
-#pragma unroll 1
-              for (int q = 0; q < P; ++q)
-                vis |= ((masks[pair_row[q]] >> (key - Cctx)) & 1ull) << q;
-            }
+            vis = key < Cctx ? (P >= 64 ? ~0ull : ((1ull << P) - 1ull)) : visk[key - Cctx];
           }
         }
         const uint32_t s_addr = tmem_s(grp) + lane_off;
