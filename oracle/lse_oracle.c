@@ -39,6 +39,15 @@
  *    lse  = m + ln sum_j exp(x_j - m)
  * GQA grouping (query head h reads kv head h / G, contiguous groups) is the
  * plain reading where the pages are silent.
+ *
+ * K/V append (the write of a verify step's new tokens into their fragments,
+ * FP32 cast to the storage format: LSE releases, v0.4.20, K/V memory
+ * management): each new token's K and V vectors go to position
+ * L_before + i of their sequence through its page tables.  The cast is the
+ * nearest value of the format, ties to even, from the format's bit layout;
+ * FP16/BF16 overflow to infinity as IEEE formats do; the FP8 formats
+ * saturate to their largest finite value (E4M3 has no infinity; the pages
+ * fix no overflow rule for E5M2, and saturating keeps a cache finite).
  */
 #include <math.h>
 #include <stddef.h>
@@ -140,6 +149,67 @@ double orc_decode(int dtype, uint32_t bits) {
   b[2] = (uint8_t)((bits >> 16) & 0xff);
   b[3] = (uint8_t)((bits >> 24) & 0xff);
   return decode_elem(dtype, b);
+}
+
+/* ---- encoding of one double to a format's bits (nearest, ties to even) --- */
+
+/* Generic sign/exponent/fraction encoder: ebits/mbits field widths; max_e /
+ * max_m the fields of the largest finite value; sat: overflow saturates to
+ * it (else it becomes infinity, exponent all ones and fraction 0); nan_bits:
+ * the encoding used for NaN input. */
+static uint32_t encode_minifloat(double x, int ebits, int mbits, uint32_t max_e, uint32_t max_m,
+                                 int sat, uint32_t nan_bits) {
+  if (isnan(x)) return nan_bits;
+  const uint32_t sign = signbit(x) ? 1u << (ebits + mbits) : 0u;
+  double a = fabs(x);
+  const int bias = (1 << (ebits - 1)) - 1;
+  const int emin = 1 - bias;  /* exponent of the smallest normal */
+  const double maxv = (1.0 + (double)max_m * pow2(-mbits)) * pow2((int)max_e - bias);
+  const double half_ulp_max = pow2((int)max_e - bias - mbits - 1);
+  if (a >= maxv + half_ulp_max) {  /* rounds past the largest finite value */
+    if (sat) return sign | (max_e << mbits) | max_m;
+    return sign | (((1u << ebits) - 1u) << mbits);
+  }
+  if (a == 0.0) return sign;
+  /* quantum of the binade of a (subnormals share the smallest normal's) */
+  int e;
+  frexp(a, &e);  /* a = f 2^e, f in [0.5, 1): binade exponent e - 1 */
+  int be = e - 1 < emin ? emin : e - 1;
+  const double q = pow2(be - mbits);
+  const double n = a / q;  /* exact: a carries 24 significant bits at most */
+  double r = floor(n);
+  const double frac = n - r;
+  if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+  const double v = r * q;  /* the rounded magnitude, exactly */
+  if (v == 0.0) return sign;
+  frexp(v, &e);
+  be = e - 1;
+  if (be < emin) /* subnormal: exponent field 0 */
+    return sign | (uint32_t)(v / pow2(emin - mbits));
+  const uint32_t ef = (uint32_t)(be + bias);
+  const uint32_t mf = (uint32_t)((v / pow2(be) - 1.0) * pow2(mbits));
+  return sign | (ef << mbits) | mf;
+}
+
+static uint32_t encode_elem(int dtype, double x) {
+  switch (dtype) {
+    case ORC_F16: return encode_minifloat(x, 5, 10, 30, 1023, 0, 0x7E00u);
+    case ORC_BF16: return encode_minifloat(x, 8, 7, 254, 127, 0, 0x7FC0u);
+    case ORC_E4M3: return encode_minifloat(x, 4, 3, 15, 6, 1, 0x7Fu);
+    case ORC_E5M2: return encode_minifloat(x, 5, 2, 30, 3, 1, 0x7Fu);
+  }
+  return 0;
+}
+
+/* Exported so tests can compare the encoder with library conversions. */
+uint32_t orc_encode(int dtype, double x) {
+  if (dtype == ORC_F32) {
+    float f = (float)x;
+    uint32_t b;
+    memcpy(&b, &f, 4);
+    return b;
+  }
+  return encode_elem(dtype, x);
 }
 
 /* ---- fragment addressing ---------------------------------------------- */
@@ -345,4 +415,53 @@ int64_t orc_kv_bytes_per_token(int dtype, int n_layers, int n_kv_heads, int head
   int64_t per = (int64_t)n_layers * 2 * n_kv_heads * head_dim * elem_size(dtype);
   if (with_scales) per += (int64_t)n_layers * 2 * n_kv_heads * 4;
   return per;
+}
+
+/* K/V append: new tokens i in [new_offsets[s], new_offsets[s+1]) of
+ * sequence s go to key position seq_lens_before[s] + (i - new_offsets[s]);
+ * k_new / v_new are [total_new][n_kv_heads][head_dim] FP32.  Writes the
+ * encoded elements into the (writable) host copies of the arena chunks.
+ * A position past the page table or a page naming no fragment is skipped
+ * and reported (ORC_BAD_PAGE); everything else is still written. */
+int orc_kv_append(uint8_t *const *chunks, int n_chunks, int64_t chunk_bytes,
+                  int64_t fragment_bytes, int dtype, int n_kv_heads, int head_dim, int n_seqs,
+                  int max_pages, const int32_t *k_pages, const int32_t *v_pages,
+                  const int32_t *seq_lens_before, const int32_t *new_offsets,
+                  const float *k_new, const float *v_new) {
+  const int es = elem_size(dtype);
+  if (es == 0) return ORC_BAD_DTYPE;
+  if (n_kv_heads < 1 || head_dim < 1 || fragment_bytes < (int64_t)n_kv_heads * head_dim * es)
+    return ORC_BAD_SHAPE;
+  const int64_t T = fragment_bytes / ((int64_t)n_kv_heads * head_dim * es);
+  const int64_t per_chunk = chunk_bytes / fragment_bytes;
+  int status = ORC_OK;
+  for (int s = 0; s < n_seqs; ++s) {
+    for (int32_t i = new_offsets[s]; i < new_offsets[s + 1]; ++i) {
+      const int64_t pos = (int64_t)seq_lens_before[s] + (i - new_offsets[s]);
+      const int64_t page = pos / T, off = pos % T;
+      for (int kv = 0; kv < 2; ++kv) {
+        const int32_t *table = kv ? v_pages : k_pages;
+        const float *src = kv ? v_new : k_new;
+        if (pos < 0 || page >= max_pages) {
+          status = ORC_BAD_PAGE;
+          continue;
+        }
+        const int32_t frag = table[(int64_t)s * max_pages + page];
+        if (frag < 0 || frag >= per_chunk * n_chunks) {
+          status = ORC_BAD_PAGE;
+          continue;
+        }
+        uint8_t *dst = chunks[frag / per_chunk] + (frag % per_chunk) * fragment_bytes +
+                       off * (int64_t)n_kv_heads * head_dim * es;
+        for (int g = 0; g < n_kv_heads; ++g)
+          for (int d = 0; d < head_dim; ++d) {
+            const int64_t e = ((int64_t)i * n_kv_heads + g) * head_dim + d;
+            const uint32_t bits = orc_encode(dtype, (double)src[e]);
+            uint8_t *o = dst + ((int64_t)g * head_dim + d) * es;
+            for (int b = 0; b < es; ++b) o[b] = (uint8_t)((bits >> (8 * b)) & 0xffu);
+          }
+      }
+    }
+  }
+  return status;
 }

@@ -82,6 +82,14 @@ def _load():
         lib.orc_decode.restype = ctypes.c_double
         lib.orc_kv_bytes_per_token.argtypes = [ctypes.c_int] * 5
         lib.orc_kv_bytes_per_token.restype = ctypes.c_int64
+        lib.orc_encode.argtypes = [ctypes.c_int, ctypes.c_double]
+        lib.orc_encode.restype = ctypes.c_uint32
+        vp = ctypes.c_void_p
+        lib.orc_kv_append.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int,
+                                      ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                                      ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                      vp, vp, vp, vp, vp, vp]
+        lib.orc_kv_append.restype = ctypes.c_int
         for f in (lib.orc_attention, lib.orc_attention_one, lib.orc_attention_split):
             f.restype = ctypes.c_int
         _lib = lib
@@ -187,3 +195,29 @@ def kv_bytes_per_token(dtype: str, n_layers: int, n_kv_heads: int, head_dim: int
                        with_scales: bool) -> int:
     return int(_load().orc_kv_bytes_per_token(DTYPE_CODES[dtype], n_layers, n_kv_heads,
                                               head_dim, int(with_scales)))
+
+
+def encode(dtype: str, x: float) -> int:
+    """The stored bits of x in a format: nearest value, ties to even (FP8
+    saturates at its largest finite value, F16/BF16 overflow to infinity)."""
+    return int(_load().orc_encode(DTYPE_CODES[dtype], float(x)))
+
+
+def kv_append(chunks, chunk_bytes, fragment_bytes, dtype, n_kv_heads, head_dim, k_pages,
+              v_pages, seq_lens_before, new_offsets, k_new, v_new):
+    """Write new tokens' K/V into host copies of the arena chunks (modified in
+    place): token i of sequence s (new_offsets[s] <= i < new_offsets[s+1])
+    goes to key position seq_lens_before[s] + i - new_offsets[s].  Returns
+    the oracle status (0, or 2 when some position has no fragment; the
+    others are written)."""
+    for c in chunks:
+        assert c.dtype == np.uint8 and c.flags["C_CONTIGUOUS"]
+    kp, vp_ = _as(k_pages, np.int32), _as(v_pages, np.int32)
+    sl, no = _as(seq_lens_before, np.int32), _as(new_offsets, np.int32)
+    kn, vn = _as(k_new, np.float32), _as(v_new, np.float32)
+    ptrs = (ctypes.c_void_p * max(1, len(chunks)))(*[c.ctypes.data for c in chunks])
+    return int(_load().orc_kv_append(
+        ctypes.cast(ptrs, ctypes.POINTER(ctypes.c_void_p)), len(chunks), int(chunk_bytes),
+        int(fragment_bytes), DTYPE_CODES[dtype], int(n_kv_heads), int(head_dim), len(sl),
+        kp.shape[1], kp.ctypes.data, vp_.ctypes.data, sl.ctypes.data, no.ctypes.data,
+        kn.ctypes.data, vn.ctypes.data))

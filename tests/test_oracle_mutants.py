@@ -18,6 +18,7 @@ from oracle import oracle as orc
 from verify_attention_paged_b200 import workloads as wl
 from conftest import to_problem
 from test_oracle_pins import sdpa_reference
+import test_oracle_append_pins as pins_append
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(__file__)), "oracle", "lse_oracle.c")
 
@@ -36,6 +37,16 @@ MUTANTS = {
     "merge_weight_sign": ("double w = exp(lp - M);", "double w = exp(M - lp);"),
     "bf16_no_specials": ("8, 7, 1, 0)", "8, 7, 0, 0)"),
     "f16_read_as_bf16": ("5, 10, 1, 0)", "8, 7, 1, 0)"),
+    # encoder and K/V append
+    "encode_ties_away": ("if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;",
+                         "if (frac >= 0.5) r += 1.0;"),
+    "encode_subnormal_quantum": ("int be = e - 1 < emin ? emin : e - 1;", "int be = e - 1;"),
+    "append_position_off": ("const int64_t pos = (int64_t)seq_lens_before[s] + (i - new_offsets[s]);",
+                            "const int64_t pos = (int64_t)seq_lens_before[s] + (i - new_offsets[s]) + 1;"),
+    "append_v_through_k_table": ("const int32_t *table = kv ? v_pages : k_pages;",
+                                 "const int32_t *table = k_pages;"),
+    "e4m3_overflow_not_saturated": ("encode_minifloat(x, 4, 3, 15, 6, 1, 0x7Fu)",
+                                    "encode_minifloat(x, 4, 3, 15, 6, 0, 0x7Fu)"),
 }
 
 
@@ -59,7 +70,7 @@ def _pins_fail(lib) -> list:
         real = orc._load()  # set argtypes on a fresh handle, then swap the library
         m = ctypes.CDLL(lib)
         for fn in ("orc_attention", "orc_attention_one", "orc_attention_split", "orc_decode",
-                   "orc_kv_bytes_per_token"):
+                   "orc_kv_bytes_per_token", "orc_encode", "orc_kv_append"):
             f = getattr(m, fn)
             f.argtypes = getattr(real, fn).argtypes
             f.restype = getattr(real, fn).restype
@@ -102,6 +113,24 @@ def _pins_fail(lib) -> list:
             assert np.array_equal(np.isnan(want), np.isnan(got))
             assert np.array_equal(want[~np.isnan(want)], got[~np.isnan(got)])
 
+        def encoder(dtype):
+            x = pins_append.sample_values(dtype, 3000, seed=12)
+            assert np.array_equal(pins_append.encode_all(dtype, x),
+                                  pins_append.torch_bits(dtype, x))
+
+        def append(dtype):
+            w = wl.small_case(dtype, [40, 9, 1], [1, 2, 1], n_q_heads=4, n_kv_heads=2,
+                              head_dim=8, tokens_per_fragment=8, seed=43)
+            chunks, st, *_ = pins_append._append_from_logical(w, 11)
+            assert st == 0
+            for a, b in zip(chunks, w.chunks):
+                assert np.array_equal(a, b)
+
+        check("encoder_e4m3", lambda: encoder("e4m3"))
+        check("encoder_f16", lambda: encoder("f16"))
+        check("encoder_overflow_e4m3", lambda: pins_append.test_overflow_and_nan_rules("e4m3"))
+        check("encoder_ties_e5m2", lambda: pins_append.test_encoder_rounds_ties_to_even("e5m2"))
+        check("append_bf16", lambda: append("bf16"))
         check("sdpa_bf16_tree", lambda: sdpa("bf16", True))
         check("sdpa_e4m3_chain", lambda: sdpa("e4m3", False))
         check("split", split)
