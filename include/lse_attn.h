@@ -278,6 +278,41 @@ LSE_API int lse_attn_read_error(const lse_attn_plan_t *plan, void *workspace, vo
                         uint32_t *device_error, char **err);
 
 /* ---------------------------------------------------------------------------
+ * K/V append (LSE releases, v0.4.20 "K/V memory management and automatic
+ * split attention": K/V tensors live in fragments reached through each
+ * sequence's page tables; a decode or verify step writes its new tokens'
+ * K/V there before attending).  Writes the K and V vectors of new tokens into
+ * their fragments, cast from FP32 to the arena's storage format: the nearest
+ * value of the format, ties to even; F16 and BF16 overflow to infinity,
+ * E4M3 and E5M2 saturate at their largest finite value (448, 57344).
+ *
+ * Token i of sequence s, new_offsets[s] <= i < new_offsets[s+1], goes to key
+ * position seq_lens_before[s] + i - new_offsets[s] of s (page = position / T,
+ * slot = position % T, T the fragment's tokens), the same element layout the
+ * attention passes read ([token][kv_head][dim] inside a fragment).
+ *   k_new, v_new      device, FP32 [total_new][n_kv_heads][head_dim]
+ *   k_pages, v_pages  device, int32 [n_seqs][max_pages]; the pages holding
+ *                     the new positions must already name fragments
+ *   seq_lens_before   device, int32 [n_seqs]: keys stored before this append
+ *   new_offsets       device, int32 [n_seqs + 1], ascending, new_offsets[0] = 0
+ *   total_new         host: new_offsets[n_seqs] (sizes the launch)
+ *   err_word          device uint32, or NULL: LSE_DEVERR_BAD_FRAGMENT is ORed
+ *                     in when a position is past its page table or a page
+ *                     names no fragment (that vector is not written),
+ *                     LSE_DEVERR_BAD_LENGTH when a token belongs to no
+ *                     sequence (new_offsets not ascending)
+ * Head dims 64, 128 and 256.  Asynchronous on `stream`; allocates nothing;
+ * the caller owns every buffer.  Returns LSE_OK, LSE_ERR_INVALID_ARG (NULL
+ * or out-of-range arguments), LSE_ERR_UNSUPPORTED (head dim) or
+ * LSE_ERR_CUDA (launch failure).
+ * ------------------------------------------------------------------------- */
+LSE_API int lse_kv_append(const lse_kv_arena *arena, int n_seqs, int max_pages,
+                          const float *k_new, const float *v_new, const int32_t *k_pages,
+                          const int32_t *v_pages, const int32_t *seq_lens_before,
+                          const int32_t *new_offsets, int total_new, uint32_t *err_word,
+                          void *stream, char **err);
+
+/* ---------------------------------------------------------------------------
  * No-allocation variant (the pages have no counterpart: it exists for
  * callers that cannot allocate device memory when attention runs, such as
  * plugin or custom-op hosts that hand a kernel only its inputs and outputs,

@@ -92,6 +92,7 @@ _sig("lse_attn_validate", _i, _vp, _i32p, _i32p, _i32p, _i32p,
 _sig("lse_attn_read_error", _i, _vp, _vp, _vp, ctypes.POINTER(ctypes.c_uint32), _errp)
 _sig("lse_attn_forward_static", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _vp,
      _vp, _errp)
+_sig("lse_kv_append", _i, _vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _errp)
 STATIC_SCRATCH_BYTES = 32 << 20
 
 
@@ -229,6 +230,15 @@ def lse_attn_plan_destroy(plan) -> None:
 
 
 # ---- run / merge / checks ---------------------------------------------------------
+
+def lse_kv_append(arena, n_seqs, max_pages, k_new, v_new, k_pages, v_pages, seq_lens_before,
+                  new_offsets, total_new, err_word=None, stream=0) -> None:
+    """Write new tokens' FP32 K/V into their fragments, cast to the arena's
+    format (device tensors; see include/lse_attn.h)."""
+    _call(_lib.lse_kv_append, arena, int(n_seqs), int(max_pages), _ptr(k_new), _ptr(v_new),
+          _ptr(k_pages), _ptr(v_pages), _ptr(seq_lens_before), _ptr(new_offsets),
+          int(total_new), _ptr(err_word), _ptr(stream))
+
 
 def lse_attn_run(plan, q, k_pages, v_pages, seq_lens, row_offsets, row_masks, softmax_scale,
                  workspace, stream=0) -> None:

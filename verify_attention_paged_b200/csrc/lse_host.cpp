@@ -391,6 +391,46 @@ static int fill_params(const lse_attn_plan_t *pl, void *ws, LseKernelParams &p, 
   return LSE_OK;
 }
 
+int lse_kv_append(const lse_kv_arena *a, int n_seqs, int max_pages, const float *k_new,
+                  const float *v_new, const int32_t *k_pages, const int32_t *v_pages,
+                  const int32_t *seq_lens_before, const int32_t *new_offsets, int total_new,
+                  uint32_t *err_word, void *stream, char **err) {
+  if (!a) return fail(err, LSE_ERR_INVALID_ARG, "arena is NULL");
+  if (n_seqs < 1 || max_pages < 1 || total_new < 0)
+    return fail(err, LSE_ERR_INVALID_ARG, "n_seqs %d, max_pages %d, total_new %d", n_seqs,
+                max_pages, total_new);
+  if (a->head_dim != 64 && a->head_dim != 128 && a->head_dim != 256)
+    return fail(err, LSE_ERR_UNSUPPORTED, "head_dim %d (append takes 64, 128, 256)",
+                a->head_dim);
+  if (!k_pages || !v_pages || !seq_lens_before || !new_offsets ||
+      (total_new > 0 && (!k_new || !v_new)))
+    return fail(err, LSE_ERR_INVALID_ARG, "a required device pointer is NULL");
+  if (int64_t(n_seqs) * max_pages > INT32_MAX || int64_t(total_new) * a->n_kv_heads > INT32_MAX)
+    return fail(err, LSE_ERR_INVALID_ARG, "too many pages or tokens");
+  if (total_new == 0) return LSE_OK;
+  AppendParams p;
+  memset(&p, 0, sizeof p);
+  for (size_t c = 0; c < a->chunk_base.size(); ++c) p.chunk_base[c] = a->chunk_base[c];
+  p.fragment_bytes = (long long)a->fragment_bytes;
+  p.frags_per_chunk = a->frags_per_chunk;
+  p.n_fragments = int(a->used.size());
+  p.tokens_per_fragment = a->tokens_per_fragment;
+  p.n_kv_heads = a->n_kv_heads;
+  p.n_seqs = n_seqs;
+  p.max_pages = max_pages;
+  p.total_new = total_new;
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.k_pages = k_pages;
+  p.v_pages = v_pages;
+  p.seq_lens_before = seq_lens_before;
+  p.new_offsets = new_offsets;
+  p.err = err_word;
+  const int ce = lse_launch_kv_append(p, a->dtype, a->head_dim, stream);
+  if (ce) return cuda_fail(err, ce, "append kernel launch");
+  return LSE_OK;
+}
+
 int lse_attn_run(const lse_attn_plan_t *pl, const float *q, const int32_t *k_pages,
                  const int32_t *v_pages, const int32_t *seq_lens, const int32_t *row_offsets,
                  const uint64_t *row_masks, float softmax_scale, void *ws, void *stream,

@@ -96,6 +96,27 @@ struct LseKernelParams {
   int n_ctas;      // persistent grid size when balanced
 };
 
+// Arguments of the K/V append kernel (lse_append.cu).
+struct AppendParams {
+  unsigned long long chunk_base[LSE_MAX_CHUNKS];
+  long long fragment_bytes;
+  int frags_per_chunk;
+  int n_fragments;
+  int tokens_per_fragment;
+  int n_kv_heads;
+  int n_seqs;
+  int max_pages;
+  int total_new;
+  const float *k_new;
+  const float *v_new;
+  const int32_t *k_pages;
+  const int32_t *v_pages;
+  const int32_t *seq_lens_before;
+  const int32_t *new_offsets;
+  unsigned int *err;
+};
+int lse_launch_kv_append(const AppendParams &a, int dtype, int head_dim, void *stream);
+
 // Kernel entry points (lse_kernels.cu).  Return a cudaError_t value.
 int lse_launch_partial_cuda_core(const LseKernelParams &p, int dtype, int head_dim, int grid_x,
                                  int grid_y, int grid_z, int smem, void *stream);
