@@ -11,6 +11,8 @@ every timed step, outside the step's CUDA-event interval.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--impl ours|reference]
 
+--workload append times the K/V append kernel instead (see run_append).
+
 Prints one JSON line.  ``value`` is effective GB/s: (K + V + Q + out bytes of
 every call on every rank) / (max over ranks of the summed step times).
 ``--impl reference`` times the float64 CPU oracle on a bounded sample of
@@ -395,9 +397,102 @@ def measure_e2e(call, w, args, stream, flush, dist):
             "d2h_bytes_per_step": d2h}
 
 
+APPEND_METRIC = "K/V append us/call and GB/s (FP32 read + stored bytes)"
+
+
+def run_append(args, world, rank, local):
+    """The K/V append (lse_kv_append) of a verify step's drafts: 256
+    sequences x 16 new tokens, 24/4 heads, head_dim 128, into a BF16 arena of
+    256 KiB fragments.  One step = one append call, captured in a CUDA graph,
+    L2 flushed before each step outside the interval."""
+    import torch
+    torch.cuda.set_device(local)
+    from verify_attention_paged_b200 import binding as b
+    n_seqs, new, hkv, d = 256, 16, 4, 128
+    dtype, esize, frag = "bf16", 2, 256 << 10
+    T = frag // (hkv * d * esize)
+    rng = np.random.default_rng(1240)
+    before = rng.integers(1024, 16384, n_seqs).astype(np.int32)
+    pages = (before + new + T - 1) // T
+    max_pages = int(pages.max())
+    n_frags = int(2 * pages.sum())
+    chunk = 256 << 20
+    n_chunks = (n_frags * frag + chunk - 1) // chunk
+    chunks = [torch.empty(chunk, dtype=torch.uint8, device="cuda") for _ in range(n_chunks)]
+    arena = b.lse_kv_arena_create(chunks, chunk, frag, dtype, hkv, d)
+    ids = rng.permutation(b.lse_kv_arena_alloc(arena, n_frags)).astype(np.int32)
+    kp = np.full((n_seqs, max_pages), -1, np.int32)
+    vp = np.full((n_seqs, max_pages), -1, np.int32)
+    at = 0
+    for s_ in range(n_seqs):
+        kp[s_, :pages[s_]] = ids[at:at + pages[s_]]
+        vp[s_, :pages[s_]] = ids[at + pages[s_]:at + 2 * pages[s_]]
+        at += 2 * pages[s_]
+    dev = lambda a: torch.from_numpy(a).cuda()  # noqa: E731
+    total = n_seqs * new
+    k_new = torch.randn((total, hkv, d), device="cuda")
+    v_new = torch.randn((total, hkv, d), device="cuda")
+    offs = dev(np.arange(0, total + 1, new, dtype=np.int32))
+    kp_d, vp_d, before_d = dev(kp), dev(vp), dev(before)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def step(stream):
+        b.lse_kv_append(arena, n_seqs, max_pages, k_new, v_new, kp_d, vp_d, before_d, offs,
+                        total, err, stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step(torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xff)
+            ev[i][0].record()
+            g.replay()
+            ev[i][1].record()
+        torch.cuda.synchronize()
+    assert int(err.item()) == 0, "device error during the append"
+    ms = [e[0].elapsed_time(e[1]) for e in ev]
+    total_ms = sum(ms)
+    nbytes = 2 * total * hkv * d * (4 + esize)  # K and V: FP32 read, BF16 written
+    gbs = nbytes * args.steps / (total_ms * 1e-3) / 1e9
+    peak, kind = measured_peaks()
+    line = {
+        "metric": APPEND_METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "us_per_call": total_ms / args.steps * 1e3,
+        "us_per_call_median": statistics.median(ms) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32->bf16",
+        "data": "synthetic",
+        "config": {"workload": "append", "seqs": n_seqs, "new_tokens_per_seq": new,
+                   "kv_heads": hkv, "head_dim": d, "kv_dtype": dtype, "fragment_bytes": frag,
+                   "bytes_per_call": nbytes, "l2": "flushed before every step (256 MiB write)",
+                   "timing": "CUDA events around a CUDA-graph replay of each step"},
+        "roofline": {"bound": "hbm", "kernel": "kv_append", "achieved": gbs, "peak": peak,
+                     "peak_kind": f"{kind} (copy, burst)", "unit": "GB/s", "frac": gbs / peak,
+                     "traffic": None, "algorithmic_bytes_per_launch": nbytes},
+        "gpu_launches": args.steps, "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line))
+    b.lse_kv_arena_destroy(arena)
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
+    if args.workload == "append":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the append has no separate reference arm"}))
+            return
+        run_append(args, world, rank, local)
+        return
     from verify_attention_paged_b200 import workloads as wl
     w = wl.BUILDERS[args.workload]()
     if args.impl == "reference":
