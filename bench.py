@@ -23,7 +23,6 @@ from __future__ import annotations
 
 import argparse
 import hashlib
-import glob
 import json
 import os
 import statistics
@@ -62,24 +61,32 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def kernel_source_hash():
+# the sources each measured kernel (and its launch plan) is built from
+KERNEL_SOURCES = {
+    "partial": ("lse_host.cpp", "lse_internal.h", "lse_kernels.cu", "lse_static.cu",
+                "lse_tcgen05.cu"),
+    "append": ("lse_append.cu", "lse_host.cpp", "lse_internal.h"),
+}
+
+
+def kernel_source_hash(kernel="partial"):
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "verify_attention_paged_b200", "csrc", "*"))):
-        with open(f, "rb") as fh:
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "verify_attention_paged_b200", "csrc", name), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(workload):
-    """DRAM bytes per launch of the partial kernel from the committed ncu
-    summary, when it was taken on the current kernel source."""
+def ncu_traffic(workload, kernel="partial"):
+    """DRAM bytes per launch of the workload's dominant kernel from the
+    committed ncu summary, when it was taken on the current kernel source."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(workload)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -475,7 +482,8 @@ def run_append(args, world, rank, local):
                    "timing": "CUDA events around a CUDA-graph replay of each step"},
         "roofline": {"bound": "hbm", "kernel": "kv_append", "achieved": gbs, "peak": peak,
                      "peak_kind": f"{kind} (copy, burst)", "unit": "GB/s", "frac": gbs / peak,
-                     "traffic": None, "algorithmic_bytes_per_launch": nbytes},
+                     "traffic": ncu_traffic("append", "append"),
+                     "algorithmic_bytes_per_launch": nbytes},
         "gpu_launches": args.steps, "clocks": clk.summary(),
     }
     if rank == 0:
@@ -483,9 +491,111 @@ def run_append(args, world, rank, local):
     b.lse_kv_arena_destroy(arena)
 
 
+FRAG_METRIC = "fragment-addressing overhead, % of the contiguous-cache time (worst case)"
+
+
+def _step_times(call, steps, flush):
+    """Device times (ms) of `steps` graph replays of one partial + merge
+    step, L2 flushed before each outside the interval."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    saved = call.stream
+    with torch.cuda.graph(g):
+        call.stream = torch.cuda.current_stream()
+        call.run_partial()
+        call.run_merge()
+    call.stream = saved
+    for i in range(3):
+        flush.fill_(i)
+        g.replay()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.fill_(i & 0xff)
+        ev[i][0].record()
+        g.replay()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    assert call.device_error() == 0, "device error during the timed steps"
+    return [e[0].elapsed_time(e[1]) for e in ev]
+
+
+def run_frag_ab(args, world, rank, local):
+    """The releases page's fragment-addressing measurements on this kernel:
+    the same keys through a shuffled page table (256 KiB fragments in random
+    order) and through an identity table over a contiguous cache, at 16K
+    context with one query row and at 68K with eight; and split attention
+    against a forced-unsplit plan (one CTA per kv head) at 65,656 keys with
+    four query rows.  Outputs of each pair are compared bit for bit."""
+    import torch
+    torch.cuda.set_device(local)
+    from verify_attention_paged_b200 import binding as b
+    from verify_attention_paged_b200 import workloads as wl
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    props = torch.cuda.get_device_properties(local)
+    optin = getattr(props, "shared_memory_per_block_optin", 232448)
+    cases = []
+    with ClockSampler(local) as clk:
+        for w in wl.fragment_ab_cases():
+            if w.name.startswith("split"):
+                variants = [("split", w, None),
+                            ("unsplit", w, dict(n_sms=w.n_kv_heads, smem_optin=optin,
+                                                ctas_per_sm=0, allow_tcgen05=1))]
+            else:
+                variants = [("shuffled", w, None), ("contiguous", wl.contiguous_copy(w), None)]
+            res = {}
+            for tag, wv, limits in variants:
+                call = b.DeviceCall(wv, plan_limits=limits)
+                for _ in range(args.warmup):
+                    flush.fill_(1)
+                    call.run()
+                t = _step_times(call, args.steps, flush)
+                out, lse = call.run()
+                torch.cuda.synchronize()
+                res[tag] = dict(us=statistics.median(t) * 1e3, kernel=call.info["kernel_name"],
+                                ctas=call.info["ctas"], out=out[:wv.total_rows].cpu(),
+                                lse=lse[:wv.total_rows].cpu())
+                call.close()
+            (ta, ra), (tb, rb) = res.items()
+            same = bool(torch.equal(ra["out"], rb["out"]) and torch.equal(ra["lse"], rb["lse"]))
+            diff = float((ra["out"] - rb["out"]).abs().max())
+            case = {"case": w.name, "keys": int(w.seq_lens.sum()), "rows": w.total_rows,
+                    "kv_bytes": w.kv_bytes(), "outputs_identical": same,
+                    "max_abs_diff": diff}
+            for tag, r in res.items():
+                case[f"{tag}_us"] = r["us"]
+                case[f"{tag}_ctas"] = r["ctas"]
+                case["kernel"] = r["kernel"]
+            if tb == "contiguous":
+                case["overhead_pct"] = (ra["us"] / rb["us"] - 1.0) * 100.0
+            else:
+                case["unsplit_over_split"] = rb["us"] / ra["us"]
+            cases.append(case)
+            del res
+    worst = max(c["overhead_pct"] for c in cases if "overhead_pct" in c)
+    if rank == 0:
+        print(json.dumps({
+            "metric": FRAG_METRIC, "value": worst, "unit": "%", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "fragment_ab", "fragment_bytes": 256 << 10,
+                       "heads": "24/4", "head_dim": 128,
+                       "l2": "flushed before every step (256 MiB write)",
+                       "timing": "median of CUDA events around graph replays of partial + merge"},
+            "cases": cases, "gpu_launches": 2 * args.steps * 2 * len(cases),
+            "clocks": clk.summary()}), flush=True)
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args)
+    if args.workload == "fragment_ab":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the fragment-addressing A/B has no separate reference arm"}))
+            return
+        run_frag_ab(args, world, rank, local)
+        return
     if args.workload == "append":
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable":

@@ -168,6 +168,22 @@ def test_fragment_placement_invariance_is_bitwise(dtype):
     assert np.array_equal(out, out2) and np.array_equal(lse, lse2)
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "e5m2"])
+def test_contiguous_cache_is_bitwise_equal(dtype):
+    # the identity page table over a contiguous cache (the fragment-addressing
+    # A/B's other arm) holds the same problem: identical oracle bits
+    w = wl.small_case(dtype, [70, 33, 8], [2, 4, 1], n_q_heads=6, n_kv_heads=3, head_dim=16,
+                      tokens_per_fragment=8, tree=True, seed=4)
+    c = wl.contiguous_copy(w)
+    nk = int(sum((w.seq_lens + 7) // 8))
+    live = c.k_pages >= 0
+    assert np.array_equal(np.sort(c.k_pages[live]), np.arange(nk))
+    assert np.array_equal(np.sort(c.v_pages[live]), np.arange(nk, 2 * nk))
+    out, lse = orc.attention(to_problem(w))
+    out2, lse2 = orc.attention(to_problem(c))
+    assert np.array_equal(out, out2) and np.array_equal(lse, lse2)
+
+
 @pytest.mark.parametrize("dtype", DTYPES)
 @pytest.mark.parametrize("kp", [1, 3, 8, 16, 1000])
 def test_split_equals_unsplit(dtype, kp):

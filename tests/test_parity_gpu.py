@@ -106,6 +106,30 @@ def test_fragment_placement_does_not_change_output(binding):
     assert np.array_equal(out1, out2) and np.array_equal(lse1, lse2)
 
 
+def test_contiguous_cache_gives_identical_bits(binding):
+    # the releases page reports that fragment addressing left outputs exactly
+    # unchanged; here the identity table over a contiguous cache and the
+    # shuffled table give the same bits on the tensor-core path
+    w = wl.small_case("bf16", [3000, 1500, 77], [1, 4, 2], n_q_heads=24, n_kv_heads=4,
+                      head_dim=128, tokens_per_fragment=128, seed=131)
+    (out1, lse1, info), e1 = gpu_run(binding, w)
+    (out2, lse2, _), e2 = gpu_run(binding, wl.contiguous_copy(w))
+    assert e1 == 0 and e2 == 0 and info["kernel_name"] == "tcgen05"
+    assert np.array_equal(out1, out2) and np.array_equal(lse1, lse2)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "e4m3"])
+def test_forced_unsplit_plan_matches_oracle(binding, dtype):
+    # one CTA per kv head (no split of the key range) against the oracle
+    w = wl.small_case(dtype, [2900, 1100], [4, 1], n_q_heads=24, n_kv_heads=4, head_dim=128,
+                      tokens_per_fragment=128, seed=132)
+    props = torch.cuda.get_device_properties(0)
+    limits = dict(n_sms=w.n_kv_heads, smem_optin=props.shared_memory_per_block_optin,
+                  ctas_per_sm=0, allow_tcgen05=1)
+    info = check_full(binding, w, plan_limits=limits)
+    assert info["kernel_name"] == "tcgen05" and info["ctas"] == w.n_kv_heads
+
+
 def test_bad_page_entry_sets_error_word_without_faulting(binding):
     w = wl.small_case("bf16", [100], [2], n_q_heads=4, n_kv_heads=2, head_dim=64,
                       tokens_per_fragment=16, seed=108)
@@ -129,10 +153,10 @@ def test_bad_length_sets_error_word(binding):
 # ---- the five full-size workloads, in the benchmark's launch configuration ----
 
 SAMPLES = {"tiny_decode": None, "batched_decode": 24, "chain_verify": 24, "long_fp8": 16,
-           "tree_verify": 24}
+           "tree_verify": 24, "long_e5m2": 16}
 
 
-@pytest.mark.parametrize("name", wl.NAMES)
+@pytest.mark.parametrize("name", wl.NAMES + wl.EXTRA_NAMES)
 def test_full_size_workload(binding, name):
     w = wl.BUILDERS[name]()
     (out, lse, info), err = gpu_run(binding, w)
@@ -322,6 +346,7 @@ def test_tcgen05_bad_page_sets_error_word(binding, dtype):
 def test_plan_picks_tensor_cores_for_the_16_bit_and_fp8_workloads(binding):
     for name, want in (("batched_decode", "tcgen05"), ("chain_verify", "tcgen05"),
                        ("long_fp8", "tcgen05"), ("tree_verify", "tcgen05"),
+                       ("long_e5m2", "tcgen05"),
                        ("tiny_decode", "cuda_core")):
         w = wl.BUILDERS[name]()
         call = binding.DeviceCall(w)

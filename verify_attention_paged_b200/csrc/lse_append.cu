@@ -3,10 +3,11 @@
 // management and automatic split attention"), cast from FP32 to the storage
 // format.
 //
-// One warp per (new token, kv head): it finds the token's sequence by a
-// binary search over new_offsets, the fragment through the page table, and
-// each lane converts and stores a contiguous D/32 slice of the head's K and
-// V vectors (coalesced across the warp).  Casts: nearest value, ties to
+// One warp per (new token, kv head): each lane loads a contiguous D/32
+// slice of the head's K and V vectors, the warp finds the token's sequence
+// by a 32-way search over new_offsets and the fragment through the page
+// table, and each lane stores its converted slices (coalesced across the
+// warp).  Casts: nearest value, ties to
 // even (cvt.rn); FP8 through cvt.rn.satfinite (saturating at the largest
 // finite value); F16 and BF16 overflow to infinity.
 #include <cuda_bf16.h>
@@ -49,16 +50,10 @@ __device__ __forceinline__ uint32_t pack2<LSE_KV_FP8_E5M2>(float x0, float x1) {
   return r;
 }
 
-// This lane's kPer consecutive FP32 elements -> stored bytes at dst.
+// This lane's kPer consecutive FP32 elements (already loaded) -> stored
+// bytes at dst.
 template <int DT, int kPer>
-__device__ __forceinline__ void store_slice(const float *src, uint8_t *dst) {
-  float x[kPer];
-#pragma unroll
-  for (int k = 0; k < kPer; k += 2) {
-    const float2 f = *reinterpret_cast<const float2 *>(src + k);
-    x[k] = f.x;
-    x[k + 1] = f.y;
-  }
+__device__ __forceinline__ void store_slice(const float *x, uint8_t *dst) {
   if constexpr (DT == LSE_KV_F32) {
 #pragma unroll
     for (int k = 0; k < kPer; k += 2)
@@ -83,12 +78,30 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) kv_append_kernel(const Ap
   const long long v = (long long)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5);
   if (v >= (long long)a.total_new * a.n_kv_heads) return;  // uniform per warp
   const int i = (int)(v / a.n_kv_heads), g = (int)(v - (long long)i * a.n_kv_heads);
-  // the token's sequence: the last s with new_offsets[s] <= i
-  int lo = 0, hi = a.n_seqs - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (a.new_offsets[mid] <= i) lo = mid;
-    else hi = mid - 1;
+  // the lane's slices of K and V first: their address does not depend on
+  // the sequence, so the loads overlap the search below
+  const long long src = ((long long)i * a.n_kv_heads + g) * D + lane * kPer;
+  float xk[kPer], xv[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; k += 2) {
+    const float2 fk = *reinterpret_cast<const float2 *>(a.k_new + src + k);
+    const float2 fv = *reinterpret_cast<const float2 *>(a.v_new + src + k);
+    xk[k] = fk.x;
+    xk[k + 1] = fk.y;
+    xv[k] = fv.x;
+    xv[k + 1] = fv.y;
+  }
+  // the token's sequence, the last s with new_offsets[s] <= i: each round the
+  // 32 lanes test 32 evenly spaced offsets of the remaining range
+  int lo = 0, span = a.n_seqs;  // s in [lo, lo + span)
+  while (span > 1) {
+    const int step = (span + 31) / 32;
+    const int idx = lo + lane * step;
+    const bool le = idx < lo + span && a.new_offsets[idx] <= i;
+    const unsigned m = __ballot_sync(0xffffffffu, le);
+    const int top = m ? 31 - __clz(m) : 0;  // the last lane whose offset is <= i
+    lo += top * step;
+    span = min(step, span - top * step);
   }
   const int s = lo;
   const int first = a.new_offsets[s];
@@ -99,7 +112,6 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) kv_append_kernel(const Ap
   const long long pos = (long long)a.seq_lens_before[s] + (i - first);
   const long long page = pos / a.tokens_per_fragment;
   const long long slot = pos - page * a.tokens_per_fragment;
-  const long long src = ((long long)i * a.n_kv_heads + g) * D + lane * kPer;
 #pragma unroll
   for (int kv = 0; kv < 2; ++kv) {
     const int32_t *table = kv ? a.v_pages : a.k_pages;
@@ -113,7 +125,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) kv_append_kernel(const Ap
     uint8_t *dst = reinterpret_cast<uint8_t *>(a.chunk_base[c]) +
                    (long long)(frag - c * a.frags_per_chunk) * a.fragment_bytes +
                    ((slot * a.n_kv_heads + g) * D + lane * kPer) * kEs;
-    store_slice<DT, kPer>((kv ? a.v_new : a.k_new) + src, dst);
+    store_slice<DT, kPer>(kv ? xv : xk, dst);
   }
 }
 

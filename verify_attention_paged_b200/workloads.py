@@ -262,13 +262,73 @@ def tree_verify(keep_logical=False) -> Workload:
                  keep_logical=keep_logical)
 
 
+def long_e5m2(keep_logical=False) -> Workload:
+    """The long-context FP8 workload with E5M2 storage (the releases page's
+    second 8-bit format, "BF8"): 68173 keys incl. 4 chained rows, 24/4 heads,
+    head_dim 128, cast from N(0, 0.5^2), 512-token fragments, capacity 256
+    pages."""
+    return build("long_e5m2", "e5m2", [68173], [4], 24, 4, 128, fragment_bytes=512 * 4 * 128,
+                 chunk_bytes=256 * MIB, max_pages=256, seed=1239, kv_std=0.5, n_chunks=1,
+                 keep_logical=keep_logical)
+
+
 BUILDERS = {
     "tiny_decode": tiny_decode,
     "batched_decode": batched_decode,
     "chain_verify": chain_verify,
     "long_fp8": long_fp8,
     "tree_verify": tree_verify,
+    "long_e5m2": long_e5m2,
 }
+# workloads beyond the five benchmark configurations
+EXTRA_NAMES = ["long_e5m2"]
+
+
+# ---------------------------------------------------------------------------
+# Fragment-addressing A/B (LSE releases, v0.4.20, "Validation and
+# performance"): the same keys reached through a shuffled page table and
+# through an identity one, and split against forced-unsplit attention.
+# ---------------------------------------------------------------------------
+
+def contiguous_copy(w: Workload) -> Workload:
+    """The same problem with its fragments moved so that every page table is
+    the identity on a contiguous run: the K pages of sequence 0, 1, ... come
+    first in fragment order, then the V pages, as in an unpaged cache."""
+    T = w.tokens_per_fragment
+    fpc = w.chunk_bytes // w.fragment_bytes
+    n_pages = [math.ceil(int(L) / T) for L in w.seq_lens]
+    k_pages = np.full_like(w.k_pages, -1)
+    v_pages = np.full_like(w.v_pages, -1)
+    nk = sum(n_pages)
+    chunks = [np.full(w.chunk_bytes, DEAD_BYTE, np.uint8) for _ in w.chunks]
+    fb = w.fragment_bytes
+    cursor = 0
+    for s, n in enumerate(n_pages):
+        for p in range(n):
+            for old_table, new_table, new_id in ((w.k_pages, k_pages, cursor + p),
+                                                 (w.v_pages, v_pages, nk + cursor + p)):
+                oc, oo = divmod(int(old_table[s, p]), fpc)
+                nc, no = divmod(new_id, fpc)
+                chunks[nc][no * fb:(no + 1) * fb] = w.chunks[oc][oo * fb:(oo + 1) * fb]
+                new_table[s, p] = new_id
+        cursor += n
+    return Workload(**{**w.__dict__, "name": w.name + "_contiguous", "chunks": chunks,
+                       "k_pages": k_pages, "v_pages": v_pages})
+
+
+def fragment_ab_cases() -> list[Workload]:
+    """The releases page's fragment-addressing measurements, as BF16 problems
+    with 24/4 heads, head_dim 128 and 256 KiB fragments: one query row at 16K
+    context; eight chained query rows at 68K (68,173 keys in total); and
+    65,656 live keys with four chained query rows, the split-vs-unsplit
+    check."""
+    common = dict(n_q_heads=24, n_kv_heads=4, head_dim=128, fragment_bytes=256 * KIB,
+                  chunk_bytes=256 * MIB)
+    return [
+        build("frag_16k_decode", "bf16", [16384], [1], max_pages=64, seed=1240, **common),
+        build("frag_68k_8rows", "bf16", [68173], [8], max_pages=267, seed=1241, **common),
+        build("split_65656_4rows", "bf16", [65656], [4], max_pages=257, seed=1242, **common),
+    ]
 
 
 def small_case(dtype: str, seq_lens, rows, n_q_heads=8, n_kv_heads=2, head_dim=64,
