@@ -173,7 +173,7 @@ def cpu_baseline(w, budget_s):
                      dtype=w.dtype, n_kv_heads=w.n_kv_heads, head_dim=w.head_dim,
                      n_q_heads=w.n_q_heads, k_pages=w.k_pages, v_pages=w.v_pages,
                      seq_lens=w.seq_lens, row_offsets=w.row_offsets, row_masks=w.row_masks,
-                     q=w.q, scale=w.scale)
+                     q=w.q, scale=w.scale, scales=w.scales)
     m = orc.marshal(pb)
     outputs = [(s, r, h) for s in range(w.n_seqs)
                for r in range(int(w.row_offsets[s + 1] - w.row_offsets[s]))

@@ -40,6 +40,17 @@
  * GQA grouping (query head h reads kv head h / G, contiguous groups) is the
  * plain reading where the pages are silent.
  *
+ * Per-vector scales (LSE README, "KV cache formats": fp8 and bf8 "with
+ * scales", 33,280 bytes per token where the 8-bit elements take 32,768, so
+ * one FP32 scale per (token, kv head) of K and one of V): the stored vector
+ * times its scale is the key or value,
+ *    K[j][g][d] = decode(stored K) * sK[j][g],  V likewise with sV.
+ * The pages do not place the scales; the reading here is that they are paged
+ * like the vectors: every fragment owns a block of T * Hkv FP32 scales,
+ * kv-head-major [kv_head][token], at index fragment_id * Hkv * T of one scale
+ * array, so K scales sit in the blocks of K fragments and V scales in those
+ * of V fragments.  Without a scale array every scale is 1.
+ *
  * K/V append (the write of a verify step's new tokens into their fragments,
  * FP32 cast to the storage format: LSE releases, v0.4.20, K/V memory
  * management): each new token's K and V vectors go to position
@@ -86,6 +97,8 @@ typedef struct {
   const uint64_t *row_masks;  /* [total_rows] or NULL for the chain        */
   const float *q;           /* [total_rows][n_q_heads][head_dim]           */
   double scale;
+  const float *scales;      /* per-vector scales by fragment, or NULL      */
+  int64_t n_scales;         /* floats in scales                            */
 } orc_problem;
 
 /* ---- decoding of one stored element to double, from each format's bit
@@ -237,6 +250,21 @@ static const uint8_t *kv_row(const orc_problem *pb, const int32_t *table, int s,
   return pb->chunks[chunk] + byte;
 }
 
+/* Per-vector scale of key j, kv head g, through a page table: entry
+ * (g, j % T) of the block of the fragment holding key j (1 without scales). */
+static double vec_scale(const orc_problem *pb, const int32_t *table, int s, int64_t j, int g,
+                        int *status) {
+  if (!pb->scales) return 1.0;
+  int64_t T = tokens_per_fragment(pb);
+  int32_t frag = table[(int64_t)s * pb->max_pages + j / T];
+  int64_t at = ((int64_t)frag * pb->n_kv_heads + g) * T + j % T;
+  if (frag < 0 || at >= pb->n_scales) {
+    *status = ORC_BAD_PAGE;
+    return 0.0;
+  }
+  return (double)pb->scales[at];
+}
+
 /* ---- visibility --------------------------------------------------------- */
 
 static uint64_t row_mask(const orc_problem *pb, int s, int r) {
@@ -261,6 +289,9 @@ static int check_problem(const orc_problem *pb) {
   if (pb->fragment_bytes % ((int64_t)pb->n_kv_heads * pb->head_dim * elem_size(pb->dtype)))
     return ORC_BAD_SHAPE;
   int64_t T = tokens_per_fragment(pb);
+  if (pb->scales && pb->n_scales < pb->n_chunks * (pb->chunk_bytes / pb->fragment_bytes) *
+                                       pb->n_kv_heads * T)
+    return ORC_BAD_SHAPE;  /* a block for every fragment of the arena */
   for (int s = 0; s < pb->n_seqs; ++s) {
     int64_t L = pb->seq_lens[s];
     int R = pb->row_offsets[s + 1] - pb->row_offsets[s];
@@ -298,9 +329,10 @@ static int attend_range(const orc_problem *pb, int s, int r, int h, int64_t key_
   for (int64_t j = key_begin; j < key_end; ++j) {
     if (!visible(j, C, mask)) continue;
     const uint8_t *k = kv_row(pb, pb->k_pages, s, j, g, &status);
+    const double sk = vec_scale(pb, pb->k_pages, s, j, g, &status);
     if (status) return status;
     double x = 0.0;
-    for (int d = 0; d < D; ++d) x += (double)q[d] * decode_elem(pb->dtype, k + d * es);
+    for (int d = 0; d < D; ++d) x += (double)q[d] * (decode_elem(pb->dtype, k + d * es) * sk);
     x *= pb->scale;
     if (x > m) m = x;
   }
@@ -315,13 +347,15 @@ static int attend_range(const orc_problem *pb, int s, int r, int h, int64_t key_
     if (!visible(j, C, mask)) continue;
     const uint8_t *k = kv_row(pb, pb->k_pages, s, j, g, &status);
     const uint8_t *v = kv_row(pb, pb->v_pages, s, j, g, &status);
+    const double sk = vec_scale(pb, pb->k_pages, s, j, g, &status);
+    const double sv = vec_scale(pb, pb->v_pages, s, j, g, &status);
     if (status) return status;
     double x = 0.0;
-    for (int d = 0; d < D; ++d) x += (double)q[d] * decode_elem(pb->dtype, k + d * es);
+    for (int d = 0; d < D; ++d) x += (double)q[d] * (decode_elem(pb->dtype, k + d * es) * sk);
     x *= pb->scale;
     double p = exp(x - m);
     l += p;
-    for (int d = 0; d < D; ++d) out[d] += p * decode_elem(pb->dtype, v + d * es);
+    for (int d = 0; d < D; ++d) out[d] += p * (decode_elem(pb->dtype, v + d * es) * sv);
   }
   for (int d = 0; d < D; ++d) out[d] /= l;
   *lse = m + log(l);

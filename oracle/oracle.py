@@ -63,6 +63,8 @@ class _Problem(ctypes.Structure):
         ("row_masks", ctypes.c_void_p),
         ("q", ctypes.c_void_p),
         ("scale", ctypes.c_double),
+        ("scales", ctypes.c_void_p),
+        ("n_scales", ctypes.c_int64),
     ]
 
 
@@ -113,6 +115,9 @@ class Problem:
     row_masks: np.ndarray | None  # uint64 [total_rows] or None (chain)
     q: np.ndarray           # float32 [total_rows, Hq, D]
     scale: float
+    # per-vector scales: float32, a block of T * Hkv per fragment id,
+    # [kv_head][token] inside it; None means every scale is 1
+    scales: np.ndarray | None = None
 
 
 def _as(a, dt):
@@ -130,6 +135,7 @@ class _Marshalled:
         self.row_offsets = _as(pb.row_offsets, np.int32)
         self.row_masks = None if pb.row_masks is None else _as(pb.row_masks, np.uint64)
         self.q = _as(pb.q, np.float32)
+        self.scales = None if pb.scales is None else _as(pb.scales, np.float32).reshape(-1)
         self.chunk_ptrs = (ctypes.c_void_p * max(1, len(self.chunks)))(
             *[c.ctypes.data for c in self.chunks])
         ptr = lambda a: None if a is None else a.ctypes.data  # noqa: E731
@@ -138,7 +144,8 @@ class _Marshalled:
             pb.chunk_bytes, pb.fragment_bytes, DTYPE_CODES[pb.dtype], pb.n_kv_heads,
             pb.head_dim, pb.n_q_heads, len(self.seq_lens), self.k_pages.shape[1],
             ptr(self.k_pages), ptr(self.v_pages), ptr(self.seq_lens), ptr(self.row_offsets),
-            ptr(self.row_masks), ptr(self.q), float(pb.scale))
+            ptr(self.row_masks), ptr(self.q), float(pb.scale), ptr(self.scales),
+            0 if self.scales is None else self.scales.size)
 
 
 def _check(st):

@@ -24,7 +24,7 @@ def to_problem(w, q=None, row_masks="keep", chunks=None, k_pages=None, v_pages=N
         v_pages=w.v_pages if v_pages is None else v_pages,
         seq_lens=w.seq_lens, row_offsets=w.row_offsets,
         row_masks=w.row_masks if isinstance(row_masks, str) else row_masks,
-        q=w.q if q is None else q, scale=w.scale)
+        q=w.q if q is None else q, scale=w.scale, scales=w.scales)
 
 
 @pytest.fixture

@@ -2,7 +2,8 @@
 
 Each case compiles a copy of the oracle source with one plausible slip
 (dropped scale, wrong kv head, off-by-one visibility, wrong fragment offset,
-wrong decoder field, dropped max in lse, flipped merge weight, ...) and runs a
+wrong decoder field, dropped max in lse, flipped merge weight, per-vector
+scales dropped, misplaced or misapplied, ...) and runs a
 compact subset of the pins against it; at least one must fail.  Mistakes are
 planted only in the CPU oracle.
 """
@@ -19,6 +20,7 @@ from verify_attention_paged_b200 import workloads as wl
 from conftest import to_problem
 from test_oracle_pins import sdpa_reference
 import test_oracle_append_pins as pins_append
+import test_oracle_scale_pins as pins_scale
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(__file__)), "oracle", "lse_oracle.c")
 
@@ -47,6 +49,15 @@ MUTANTS = {
                                  "const int32_t *table = k_pages;"),
     "e4m3_overflow_not_saturated": ("encode_minifloat(x, 4, 3, 15, 6, 1, 0x7Fu)",
                                     "encode_minifloat(x, 4, 3, 15, 6, 0, 0x7Fu)"),
+    # per-vector scales
+    "k_scale_dropped": ("(decode_elem(pb->dtype, k + d * es) * sk)",
+                        "decode_elem(pb->dtype, k + d * es)"),
+    "v_scale_dropped": ("(decode_elem(pb->dtype, v + d * es) * sv)",
+                        "decode_elem(pb->dtype, v + d * es)"),
+    "scale_block_token_major": ("int64_t at = ((int64_t)frag * pb->n_kv_heads + g) * T + j % T;",
+                                "int64_t at = ((int64_t)frag * T + j % T) * pb->n_kv_heads + g;"),
+    "v_scale_through_k_table": ("vec_scale(pb, pb->v_pages", "vec_scale(pb, pb->k_pages"),
+    "v_scale_in_denominator": ("    l += p;\n", "    l += p * sv;\n"),
 }
 
 
@@ -131,6 +142,7 @@ def _pins_fail(lib) -> list:
         check("encoder_overflow_e4m3", lambda: pins_append.test_overflow_and_nan_rules("e4m3"))
         check("encoder_ties_e5m2", lambda: pins_append.test_encoder_rounds_ties_to_even("e5m2"))
         check("append_bf16", lambda: append("bf16"))
+        check("scaled_sdpa_e4m3", lambda: pins_scale.test_scaled_matches_library_sdpa("e4m3", True))
         check("sdpa_bf16_tree", lambda: sdpa("bf16", True))
         check("sdpa_e4m3_chain", lambda: sdpa("e4m3", False))
         check("split", split)

@@ -40,8 +40,13 @@ def sdpa_reference(w):
         r0, r1 = int(w.row_offsets[s]), int(w.row_offsets[s + 1])
         R = r1 - r0
         C = L - R
-        k = w.logical_k[s].to(torch.float64).repeat_interleave(G, dim=1).permute(1, 0, 2)
-        v = w.logical_v[s].to(torch.float64).repeat_interleave(G, dim=1).permute(1, 0, 2)
+        k = w.logical_k[s].to(torch.float64)
+        v = w.logical_v[s].to(torch.float64)
+        if w.scales is not None:  # per-vector scales, as the generator drew them
+            k = k * torch.from_numpy(w.logical_k_scale[s]).to(torch.float64)[:, :, None]
+            v = v * torch.from_numpy(w.logical_v_scale[s]).to(torch.float64)[:, :, None]
+        k = k.repeat_interleave(G, dim=1).permute(1, 0, 2)
+        v = v.repeat_interleave(G, dim=1).permute(1, 0, 2)
         q = torch.from_numpy(w.q[r0:r1].astype(np.float64)).permute(1, 0, 2)
         mask = torch.zeros((R, L), dtype=torch.bool)
         mask[:, :C] = True

@@ -62,6 +62,11 @@ class Workload:
     logical_k: list = field(default_factory=list)  # per seq torch [L, Hkv, D] storage dtype
     logical_v: list = field(default_factory=list)
     parents: list = field(default_factory=list)    # per seq list of draft parents (-1 = root)
+    # per-vector FP32 scales, a block of T * Hkv per fragment id ([kv_head]
+    # [token] inside it; NaN where no live vector); None means unit scales
+    scales: np.ndarray | None = None
+    logical_k_scale: list = field(default_factory=list)  # per seq float32 [L, Hkv]
+    logical_v_scale: list = field(default_factory=list)
 
     @property
     def n_seqs(self) -> int:
@@ -84,9 +89,10 @@ class Workload:
         return int(np.max(np.diff(self.row_offsets))) if self.n_seqs else 0
 
     def kv_bytes(self) -> int:
-        """Bytes of live K and V (every key of every sequence, all kv heads)."""
-        return int(np.sum(self.seq_lens.astype(np.int64))) * 2 * self.n_kv_heads * \
-            self.head_dim * ELEM_SIZE[self.dtype]
+        """Bytes of live K and V (every key of every sequence, all kv heads),
+        their per-vector scales included."""
+        per_vec = self.head_dim * ELEM_SIZE[self.dtype] + (4 if self.scales is not None else 0)
+        return int(np.sum(self.seq_lens.astype(np.int64))) * 2 * self.n_kv_heads * per_vec
 
     def call_bytes(self) -> int:
         """K + V + Q + out bytes of one call (Q and out in FP32)."""
@@ -127,12 +133,20 @@ def build(
     keep_logical: bool = False,
     n_chunks: int | None = None,
     gen: torch.Generator | None = None,
+    scaled: bool = False,
+    scale_spread: float = 0.0,
 ) -> Workload:
     """Lay out one seeded problem.
 
     ``rows[s]`` query rows are the last positions of sequence ``s``;
     ``parents[s]`` (optional) gives each draft row's parent row, -1 for a row
     hanging off the cached context; without it the rows form a chain.
+
+    ``scaled`` (8-bit formats) stores every K and V vector with a per-vector
+    FP32 scale, amax / (largest finite value of the format), the stored
+    elements being the vector divided by it and cast; ``scale_spread``
+    first multiplies each vector by 2^u, u uniform in [-spread, spread], so
+    the scales span a range of magnitudes.
     """
     g = gen if gen is not None else torch.Generator().manual_seed(seed)
     es = ELEM_SIZE[dtype]
@@ -176,12 +190,26 @@ def build(
 
     chunks = [np.full(chunk_bytes, DEAD_BYTE, np.uint8) for _ in range(n_chunks)]
     tdt = TORCH_DTYPES[dtype]
+    assert not scaled or es == 1, "per-vector scales go with the 8-bit formats"
+    scales = np.full(n_chunks * fpc * n_kv_heads * T, np.nan, np.float32) if scaled else None
     logical_k, logical_v = [], []
+    logical_ks, logical_vs = [], []
     for s in range(S):
         L = seq_lens[s]
         for which, table in (("k", k_pages), ("v", v_pages)):
             x = torch.randn((L, n_kv_heads, head_dim), generator=g, dtype=torch.float32)
-            x = (x * kv_std).to(tdt)
+            x = x * kv_std
+            if scaled:
+                if scale_spread > 0:
+                    u = (torch.rand((L, n_kv_heads, 1), generator=g) * 2 - 1) * scale_spread
+                    x = x * torch.exp2(u)
+                sc = x.abs().amax(dim=2) / torch.finfo(tdt).max      # [L, Hkv]
+                sc = torch.where(sc > 0, sc, torch.ones_like(sc))
+                x = x / sc[:, :, None]
+                sc = sc.numpy()
+                if keep_logical:
+                    (logical_ks if which == "k" else logical_vs).append(sc)
+            x = x.to(tdt)
             if keep_logical:
                 (logical_k if which == "k" else logical_v).append(x)
             raw = x.contiguous().view(torch.uint8).reshape(L, row_bytes).numpy()
@@ -191,6 +219,9 @@ def build(
                 t0, t1 = p * T, min((p + 1) * T, L)
                 base = off * fragment_bytes
                 chunks[c][base:base + (t1 - t0) * row_bytes] = raw[t0:t1].reshape(-1)
+                if scaled:
+                    blk = scales[f * n_kv_heads * T:(f + 1) * n_kv_heads * T].reshape(n_kv_heads, T)
+                    blk[:, :t1 - t0] = sc[t0:t1].T
 
     return Workload(
         name=name, dtype=dtype, n_q_heads=n_q_heads, n_kv_heads=n_kv_heads, head_dim=head_dim,
@@ -198,7 +229,8 @@ def build(
         k_pages=k_pages, v_pages=v_pages, seq_lens=np.array(seq_lens, np.int32),
         row_offsets=row_offsets, row_masks=row_masks, q=q, scale=1.0 / math.sqrt(head_dim),
         seed=seed, logical_k=logical_k, logical_v=logical_v,
-        parents=parents if parents is not None else [])
+        parents=parents if parents is not None else [], scales=scales,
+        logical_k_scale=logical_ks, logical_v_scale=logical_vs)
 
 
 # ---------------------------------------------------------------------------
@@ -302,6 +334,8 @@ def contiguous_copy(w: Workload) -> Workload:
     nk = sum(n_pages)
     chunks = [np.full(w.chunk_bytes, DEAD_BYTE, np.uint8) for _ in w.chunks]
     fb = w.fragment_bytes
+    blk = w.n_kv_heads * T
+    scales = None if w.scales is None else np.full_like(w.scales, np.nan)
     cursor = 0
     for s, n in enumerate(n_pages):
         for p in range(n):
@@ -310,10 +344,13 @@ def contiguous_copy(w: Workload) -> Workload:
                 oc, oo = divmod(int(old_table[s, p]), fpc)
                 nc, no = divmod(new_id, fpc)
                 chunks[nc][no * fb:(no + 1) * fb] = w.chunks[oc][oo * fb:(oo + 1) * fb]
+                if scales is not None:
+                    old_id = int(old_table[s, p])
+                    scales[new_id * blk:(new_id + 1) * blk] = w.scales[old_id * blk:(old_id + 1) * blk]
                 new_table[s, p] = new_id
         cursor += n
     return Workload(**{**w.__dict__, "name": w.name + "_contiguous", "chunks": chunks,
-                       "k_pages": k_pages, "v_pages": v_pages})
+                       "k_pages": k_pages, "v_pages": v_pages, "scales": scales})
 
 
 def fragment_ab_cases() -> list[Workload]:
@@ -333,7 +370,7 @@ def fragment_ab_cases() -> list[Workload]:
 
 def small_case(dtype: str, seq_lens, rows, n_q_heads=8, n_kv_heads=2, head_dim=64,
                tokens_per_fragment=16, max_pages=None, seed=7, tree=False, kv_std=1.0,
-               keep_logical=True, n_chunks=None) -> Workload:
+               keep_logical=True, n_chunks=None, scaled=False, scale_spread=0.0) -> Workload:
     """A small seeded problem of any shape, for parity and pin tests."""
     g = torch.Generator().manual_seed(seed)
     es = ELEM_SIZE[dtype]
@@ -348,4 +385,4 @@ def small_case(dtype: str, seq_lens, rows, n_q_heads=8, n_kv_heads=2, head_dim=6
     return build(f"small_{dtype}", dtype, list(seq_lens), list(rows), n_q_heads, n_kv_heads,
                  head_dim, fragment_bytes=fb, chunk_bytes=fb * fpc, max_pages=max_pages,
                  seed=seed, parents=parents, kv_std=kv_std, keep_logical=keep_logical,
-                 n_chunks=n_chunks, gen=g)
+                 n_chunks=n_chunks, gen=g, scaled=scaled, scale_spread=scale_spread)
