@@ -146,6 +146,27 @@ typedef struct {
 
 LSE_API int lse_kv_arena_query(const lse_kv_arena *arena, lse_kv_arena_info *info);
 
+/* Per-vector FP32 scales of an 8-bit arena (LSE README, "KV cache formats":
+ * fp8 and bf8 "with scales", 33,280 bytes per token where the elements take
+ * 32,768: one FP32 scale per (token, kv head) of K and of V).  A stored
+ * vector times its scale is the key or value: K[j][g][:] =
+ * decode(stored K[j][g][:]) * sK[j][g], and V likewise.
+ *   scales: device FP32 array, 16-byte aligned, caller-owned, paged like
+ *           the vectors: fragment id f owns the block of T * Hkv floats at
+ *           scales + f * Hkv * T, laid out [kv_head][token], so K scales sit
+ *           in the blocks of K fragments and V scales in those of V
+ *           fragments.  n_floats >= n_fragments * Hkv * T (a chunk added
+ *           later needs a larger array, set again).  Scales are finite and
+ *           non-negative; a V scale below 2^-64 may be read as 2^-64 (the
+ *           value it weights changes by less than 2^-64 of the output).
+ *   scales = NULL removes them (unit scales).
+ * Plans record whether the arena had scales when they were made; running a
+ * plan after the arena's scales were added or removed is LSE_ERR_INVALID_ARG.
+ * Errors: LSE_ERR_UNSUPPORTED for 16-bit or FP32 arenas, LSE_ERR_INVALID_ARG
+ * for a misaligned or short array. */
+LSE_API int lse_kv_arena_set_scales(lse_kv_arena *arena, const float *scales, int64_t n_floats,
+                                    char **err);
+
 LSE_API void lse_kv_arena_destroy(lse_kv_arena *arena);
 
 /* ---------------------------------------------------------------------------
@@ -208,6 +229,7 @@ typedef struct {
   int32_t rows_per_chunk;  /* tensor-core kernel: query rows per segment (a
                               sequence with more rows is split into row
                               chunks, each reading its keys), else 0       */
+  int32_t scaled;          /* 1: made for an arena with per-vector scales  */
 } lse_attn_plan_info;
 
 LSE_API int lse_attn_plan_query(const lse_attn_plan_t *plan, lse_attn_plan_info *info);

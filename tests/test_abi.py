@@ -142,3 +142,44 @@ def test_run_rejects_null_pointers_without_launching():
         b.lse_attn_run(p, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0.1, FAKE + 8)
     with pytest.raises(b.LseError, match="finite"):
         b.lse_attn_run(p, FAKE, FAKE, FAKE, FAKE, FAKE, None, float("nan"), FAKE)
+
+
+def test_per_vector_scales_attach_and_plan():
+    a = b.lse_kv_arena_create([FAKE], 1 << 20, 256 << 10, "e4m3", 4, 128)  # T = 512, 4 frags
+    need = 4 * 4 * 512
+    with pytest.raises(b.LseError, match="need"):
+        b.lse_kv_arena_set_scales(a, FAKE, need - 1)
+    with pytest.raises(b.LseError, match="aligned"):
+        b.lse_kv_arena_set_scales(a, FAKE + 4, need)
+    b.lse_kv_arena_set_scales(a, FAKE, need)
+    args = (a, 1, 4, 4, 24, 4, 148, 232448)
+    p, _ = b.lse_attn_plan_ex(*args)
+    info = b.lse_attn_plan_query(p)
+    assert info["scaled"] == 1 and info["kernel_name"] == "tcgen05"
+    b.lse_kv_arena_set_scales(a, None)
+    p0, _ = b.lse_attn_plan_ex(*args)
+    info0 = b.lse_attn_plan_query(p0)
+    assert info0["scaled"] == 0
+    # the scale rows take shared memory from the same ring
+    assert info["smem_bytes"] > info0["smem_bytes"] or info["stages"] < info0["stages"]
+    # a plan runs only on an arena in the state it was made for (checked
+    # before any launch)
+    with pytest.raises(b.LseError, match="scales"):
+        b.lse_attn_run(p, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0.1, FAKE)
+    b.lse_kv_arena_set_scales(a, FAKE, need)
+    with pytest.raises(b.LseError, match="scales"):
+        b.lse_attn_run(p0, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0.1, FAKE)
+    # growth past the scale array is refused at run time
+    b.lse_kv_arena_add_chunk(a, FAKE * 2)
+    with pytest.raises(b.LseError, match="grew"):
+        b.lse_attn_run(p, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0.1, FAKE)
+    b.lse_attn_plan_destroy(p)
+    b.lse_attn_plan_destroy(p0)
+    b.lse_kv_arena_destroy(a)
+
+
+def test_per_vector_scales_only_for_8_bit_arenas():
+    a = b.lse_kv_arena_create([FAKE], 1 << 20, 256 << 10, "bf16", 4, 128)
+    with pytest.raises(b.LseError, match="8-bit"):
+        b.lse_kv_arena_set_scales(a, FAKE, 1 << 20)
+    b.lse_kv_arena_destroy(a)

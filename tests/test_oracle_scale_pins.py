@@ -30,7 +30,7 @@ FP8 = ["e4m3", "e5m2"]
 def scaled_case(dtype, seed, spread=6.0, tree=True, tpf=8):
     return wl.small_case(dtype, [37, 64, 5, 16], [3, 1, 5, 2], n_q_heads=8, n_kv_heads=2,
                          head_dim=16, tokens_per_fragment=tpf, tree=tree, seed=seed,
-                         scaled=True, scale_spread=spread)
+                         scaled=True, scale_spread=spread, magnitude_spread=spread)
 
 
 def with_scales(w, scales):

@@ -153,7 +153,7 @@ def test_bad_length_sets_error_word(binding):
 # ---- the five full-size workloads, in the benchmark's launch configuration ----
 
 SAMPLES = {"tiny_decode": None, "batched_decode": 24, "chain_verify": 24, "long_fp8": 16,
-           "tree_verify": 24, "long_e5m2": 16}
+           "tree_verify": 24, "long_e5m2": 16, "long_fp8_scaled": 16}
 
 
 @pytest.mark.parametrize("name", wl.NAMES + wl.EXTRA_NAMES)
@@ -346,7 +346,7 @@ def test_tcgen05_bad_page_sets_error_word(binding, dtype):
 def test_plan_picks_tensor_cores_for_the_16_bit_and_fp8_workloads(binding):
     for name, want in (("batched_decode", "tcgen05"), ("chain_verify", "tcgen05"),
                        ("long_fp8", "tcgen05"), ("tree_verify", "tcgen05"),
-                       ("long_e5m2", "tcgen05"),
+                       ("long_e5m2", "tcgen05"), ("long_fp8_scaled", "tcgen05"),
                        ("tiny_decode", "cuda_core")):
         w = wl.BUILDERS[name]()
         call = binding.DeviceCall(w)

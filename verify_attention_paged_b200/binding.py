@@ -53,7 +53,8 @@ class PlanInfo(ctypes.Structure):
                 ("pairs", ctypes.c_int32), ("smem_bytes", ctypes.c_int32),
                 ("ctas", ctypes.c_int32), ("workspace_bytes", ctypes.c_int64),
                 ("stages", ctypes.c_int32), ("q_slots", ctypes.c_int32),
-                ("p_bufs", ctypes.c_int32), ("rows_per_chunk", ctypes.c_int32)]
+                ("p_bufs", ctypes.c_int32), ("rows_per_chunk", ctypes.c_int32),
+                ("scaled", ctypes.c_int32)]
 
 
 class DeviceLimits(ctypes.Structure):
@@ -77,6 +78,7 @@ _sig("lse_kv_arena_alloc", _i, _vp, _i, _i32p, _errp)
 _sig("lse_kv_arena_free", _i, _vp, _i, _i32p, _errp)
 _sig("lse_kv_arena_query", _i, _vp, ctypes.POINTER(ArenaInfo))
 _sig("lse_kv_arena_destroy", None, _vp)
+_sig("lse_kv_arena_set_scales", _i, _vp, _vp, ctypes.c_int64, _errp)
 _sig("lse_attn_plan", _i, _vp, _i, _i, _i, _i, _i, ctypes.POINTER(_vp),
      ctypes.POINTER(ctypes.c_size_t), _errp)
 _sig("lse_attn_plan_ex", _i, _vp, _i, _i, _i, _i, _i, ctypes.POINTER(DeviceLimits),
@@ -183,6 +185,15 @@ def lse_kv_arena_query(arena) -> dict:
 
 def lse_kv_arena_destroy(arena) -> None:
     _lib.lse_kv_arena_destroy(arena)
+
+
+def lse_kv_arena_set_scales(arena, scales, n_floats: int | None = None) -> None:
+    """Attach a device FP32 per-vector scale array (None removes it)."""
+    if scales is None:
+        _call(_lib.lse_kv_arena_set_scales, arena, None, 0)
+        return
+    n = int(n_floats if n_floats is not None else scales.numel())
+    _call(_lib.lse_kv_arena_set_scales, arena, _ptr(scales), n)
 
 
 # ---- plan --------------------------------------------------------------------
@@ -320,6 +331,11 @@ class DeviceCall:
         self.arena = lse_kv_arena_create(self.chunks, problem.chunk_bytes,
                                          problem.fragment_bytes, problem.dtype,
                                          problem.n_kv_heads, problem.head_dim)
+        self.scales = None
+        if getattr(problem, "scales", None) is not None:
+            self.scales = torch.from_numpy(np.ascontiguousarray(problem.scales,
+                                                                dtype=np.float32)).to(dev)
+            lse_kv_arena_set_scales(self.arena, self.scales)
         mtr = max(1, max_total_rows or rows)
         if plan_limits is None:
             self.plan, ws = lse_attn_plan(self.arena, len(problem.seq_lens), max_rows, mtr,

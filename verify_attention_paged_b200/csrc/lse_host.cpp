@@ -134,6 +134,28 @@ int lse_kv_arena_add_chunk(lse_kv_arena *a, void *chunk_base, int32_t *first_id,
   return LSE_OK;
 }
 
+int lse_kv_arena_set_scales(lse_kv_arena *a, const float *scales, int64_t n_floats,
+                            char **err) {
+  if (!a) return fail(err, LSE_ERR_INVALID_ARG, "arena is NULL");
+  if (!scales) {
+    a->scales = nullptr;
+    a->n_scales = 0;
+    return LSE_OK;
+  }
+  if (a->dtype != LSE_KV_FP8_E4M3 && a->dtype != LSE_KV_FP8_E5M2)
+    return fail(err, LSE_ERR_UNSUPPORTED, "per-vector scales go with the 8-bit formats");
+  if (reinterpret_cast<uintptr_t>(scales) & 15u)
+    return fail(err, LSE_ERR_INVALID_ARG, "scale array is not 16-byte aligned");
+  const int64_t need = int64_t(a->used.size()) * a->n_kv_heads * a->tokens_per_fragment;
+  if (n_floats < need)
+    return fail(err, LSE_ERR_INVALID_ARG, "scale array holds %lld floats; the arena's %d "
+                "fragments need %lld", (long long)n_floats, int(a->used.size()),
+                (long long)need);
+  a->scales = scales;
+  a->n_scales = n_floats;
+  return LSE_OK;
+}
+
 int lse_kv_arena_alloc(lse_kv_arena *a, int n, int32_t *ids, char **err) {
   if (!a || n < 0 || (n > 0 && !ids)) return fail(err, LSE_ERR_INVALID_ARG, "bad arguments");
   if (n > a->n_free)
@@ -268,6 +290,7 @@ int lse_attn_plan_ex(const lse_kv_arena *a, int n_seqs, int max_rows, int max_to
   pl->tokens_per_fragment = a->tokens_per_fragment;
   pl->pairs = pl->group * max_rows;
   pl->n_sms = n_sms;
+  pl->scaled = a->scales != nullptr;
 
   // kernel choice and its on-chip memory check.  The tensor-core kernel
   // takes 16-bit and FP8 K/V with head_dim 128 and fragments whose token
@@ -282,7 +305,9 @@ int lse_attn_plan_ex(const lse_kv_arena *a, int n_seqs, int max_rows, int max_to
   const int p8 = rows_per_chunk > 0 ? lse_tc_pairs_bucket(pl->group * rows_per_chunk) : -1;
   int tc_stages = 0, tc_q_slots = 0, tc_p_bufs = 0;
   const int tc_smem =
-      p8 > 0 ? lse_tc_smem(a->dtype, p8, smem_optin, &tc_stages, &tc_q_slots, &tc_p_bufs) : -1;
+      p8 > 0 ? lse_tc_smem(a->dtype, p8, pl->scaled, smem_optin, &tc_stages, &tc_q_slots,
+                           &tc_p_bufs)
+             : -1;
   if (allow_tc && a->dtype != LSE_KV_F32 && a->head_dim == 128 &&
       t_ok && p8 > 0 && tc_smem > 0) {
     const int tile = lse_tc_key_tile();
@@ -349,6 +374,7 @@ int lse_attn_plan_query(const lse_attn_plan_t *pl, lse_attn_plan_info *info) {
   info->q_slots = tc ? pl->q_slots : 0;
   info->p_bufs = tc ? pl->p_bufs : 0;
   info->rows_per_chunk = tc ? pl->rows_per_chunk : 0;
+  info->scaled = pl->scaled;
   return LSE_OK;
 }
 
@@ -367,7 +393,15 @@ static int fill_params(const lse_attn_plan_t *pl, void *ws, LseKernelParams &p, 
   const lse_kv_arena *a = pl->arena;
   if (reinterpret_cast<uintptr_t>(ws) & 255u)
     return fail(err, LSE_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+  if (pl->scaled != (a->scales != nullptr))
+    return fail(err, LSE_ERR_INVALID_ARG, pl->scaled ? "plan made with per-vector scales, "
+                "arena has none now" : "arena has per-vector scales; the plan was made "
+                "without them");
+  if (a->scales &&
+      a->n_scales < int64_t(a->used.size()) * a->n_kv_heads * a->tokens_per_fragment)
+    return fail(err, LSE_ERR_INVALID_ARG, "the arena grew past its scale array");
   memset(&p, 0, sizeof p);
+  p.scales = a->scales;
   for (size_t c = 0; c < a->chunk_base.size(); ++c) p.chunk_base[c] = a->chunk_base[c];
   p.fragment_bytes = (long long)a->fragment_bytes;
   p.frags_per_chunk = a->frags_per_chunk;
@@ -468,7 +502,7 @@ int lse_attn_run(const lse_attn_plan_t *pl, const float *q, const int32_t *k_pag
       pl->maps_chunks = nch;
     }
     ce = lse_launch_partial_tcgen05(p, pl->maps.data(), nch, pl->dtype, pl->pairs_bucket,
-                                    pl->ctas, pl->n_splits, pl->stages, pl->q_slots,
+                                    pl->scaled, pl->ctas, pl->n_splits, pl->stages, pl->q_slots,
                                     pl->p_bufs, pl->box_tokens,
                                     pl->smem_bytes, stream);
   } else {

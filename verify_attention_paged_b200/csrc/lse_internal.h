@@ -23,6 +23,8 @@ struct lse_kv_arena {
   std::vector<int32_t> chunk_live;  // live fragments per chunk
   int32_t n_free = 0;
   int32_t scan_from = 0;            // lowest id that may be free
+  const float *scales = nullptr;    // per-vector scales by fragment (device), or null
+  int64_t n_scales = 0;             // floats in scales
 };
 
 struct lse_attn_plan_s {
@@ -51,6 +53,7 @@ struct lse_attn_plan_s {
   int pairs_bucket = 0;  // its compile-time pair count (P8)
   int rows_per_chunk = 0;  // tensor-core kernel: query rows per segment
   int box_tokens = 0;    // its TMA box height
+  int scaled = 0;        // made for an arena with per-vector scales
   // tensor maps of the arena chunks (built on first run, rebuilt on growth)
   mutable std::vector<uint8_t> maps;
   mutable int maps_chunks = 0;
@@ -94,6 +97,9 @@ struct LseKernelParams {
   int rows_per_chunk;  // tcgen05: query rows per segment (row chunk)
   int balanced;    // merge: 1 = slots are persistent-CTA pieces (tcgen05)
   int n_ctas;      // persistent grid size when balanced
+  // per-vector scales: a [kv_head][token] FP32 block per fragment id, or
+  // null for unit scales
+  const float *scales;
 };
 
 // Arguments of the K/V append kernel (lse_append.cu).
@@ -127,12 +133,13 @@ const char *lse_cuda_error_string(int code);
 
 // tensor-core partial pass (lse_tcgen05.cu)
 int lse_tc_pairs_bucket(int pairs);
-int lse_tc_smem(int dtype, int p8, int smem_optin, int *stages, int *q_slots, int *p_bufs);
+int lse_tc_smem(int dtype, int p8, int scaled, int smem_optin, int *stages, int *q_slots,
+                int *p_bufs);
 int lse_tc_key_tile();
 size_t lse_tc_map_bytes();
 int lse_tc_build_maps(const uint64_t *chunk_base, int n_chunks, size_t chunk_bytes,
                       int n_kv_heads, int dtype, int box_tokens, void *maps_out);
 int lse_launch_partial_tcgen05(const LseKernelParams &p, const void *maps, int n_maps,
-                               int dtype, int p8, int n_ctas, int n_slots, int stages,
-                               int q_slots, int p_bufs, int box_tokens, int smem,
+                               int dtype, int p8, int scaled, int n_ctas, int n_slots,
+                               int stages, int q_slots, int p_bufs, int box_tokens, int smem,
                                void *stream);

@@ -139,6 +139,17 @@ __device__ __forceinline__ const uint8_t *kv_addr(const LseKernelParams &p, cons
   return reinterpret_cast<const uint8_t *>(p.chunk_base[chunk]) + byte;
 }
 
+// Per-vector scale of key `key`, kv head g: entry (g, key % T) of the
+// [kv_head][token] scale block of its fragment (the caller has checked the
+// page-table entry).
+__device__ __forceinline__ float kv_scale(const LseKernelParams &p, const int32_t *table, int s,
+                                          int key, int g) {
+  const int T = p.tokens_per_fragment;
+  const int page = key / T;
+  const int frag = table[(long long)s * p.max_pages + page];
+  return __ldg(p.scales + ((long long)frag * p.n_kv_heads + g) * T + (key - page * T));
+}
+
 // ---- partial pass on CUDA cores ------------------------------------------
 
 template <int D>
@@ -240,6 +251,16 @@ __global__ void __launch_bounds__(kThreads)
           const uint4 vr = __ldg(reinterpret_cast<const uint4 *>(va) + c);
           Fmt::to_float(kr, kf);
           Fmt::to_float(vr, vf);
+          if (p.scales) {
+            // the stored vectors times their per-vector scales
+            const float ks = kv_scale(p, p.k_pages, s, key, g);
+            const float vs = kv_scale(p, p.v_pages, s, key, g);
+#pragma unroll
+            for (int e = 0; e < kElemPerVec; ++e) {
+              kf[e] *= ks;
+              vf[e] *= vs;
+            }
+          }
         } else {
 #pragma unroll
           for (int e = 0; e < kElemPerVec; ++e) kf[e] = vf[e] = 0.f;

@@ -196,6 +196,17 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map
       : "memory");
 }
 
+// Plain bulk copy global -> shared (no tensor map, no multicast), counted
+// on an mbarrier's transaction bytes.  Both addresses 16-byte aligned, bytes
+// a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 // UMMA shared-memory matrix descriptor.
 __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
                                               uint32_t layout) {
@@ -449,12 +460,32 @@ __device__ __forceinline__ void load_boxes(const TcParams &tp, int nbox, int box
   }
 }
 
-// Producer work for tile n: K slot, tile record, K boxes, V slot, V boxes.
-// Returns 0 when a wait gave up.
+// Per-vector scales of one tile's boxes (kv head g) into a row of 128 FP32
+// in shared memory: one bulk copy per box from entry (g, key % T) of the
+// [kv_head][token] scale block of its fragment (fragment ids ids[0..nbox)).
+__device__ __forceinline__ void load_scales(const LseKernelParams &p, int nbox, int box_t, int g,
+                                            int key0, const int *ids, uint32_t dst,
+                                            uint32_t full_bar) {
+  const int T = p.tokens_per_fragment;
+#pragma unroll 1
+  for (int b = 0; b < nbox; ++b) {
+    const int f = ids[b];
+    if (f < 0) continue;
+    const int kb = key0 + b * box_t;
+    bulk_load(dst + (uint32_t)(b * box_t * 4),
+              p.scales + ((long long)f * p.n_kv_heads + g) * T + kb % T, (uint32_t)box_t * 4u,
+              full_bar);
+  }
+}
+
+// Producer work for tile n: K slot, tile record, K boxes, V slot, V boxes
+// (and, with sdst != 0, the tile's K and V scales into sdst[0..128) and
+// sdst[128..256), counted on the V slot's barrier).  Returns 0 when a wait
+// gave up.
 __device__ __forceinline__ int produce_tile(const TcParams &tp, int n, int NS, int nbox,
                                             int box_t, int regions, int g, int tile, int L,
                                             const int *pk, const int *pv, uint32_t kdst,
-                                            uint32_t vdst, const uint32_t *bars_k,
+                                            uint32_t vdst, uint32_t sdst, const uint32_t *bars_k,
                                             const uint32_t *bars_v, uint32_t info_bar,
                                             uint4 *info, volatile int *abort_flag) {
   const LseKernelParams &p = tp.p;
@@ -478,8 +509,14 @@ __device__ __forceinline__ int produce_tile(const TcParams &tp, int n, int NS, i
   mbar_expect_tx(bars_k[1], (uint32_t)__popc(kmask) * box_bytes);
   load_boxes(tp, nbox, box_t, regions, g, key0, pk, kdst, bars_k[1]);
   if (!mbar_wait(bars_v[0], ph, abort_flag, p.err)) return 0;
-  mbar_expect_tx(bars_v[1], (uint32_t)__popc(vmask) * box_bytes);
+  const uint32_t scale_bytes =
+      sdst ? (uint32_t)(__popc(kmask) + __popc(vmask)) * (uint32_t)box_t * 4u : 0u;
+  mbar_expect_tx(bars_v[1], (uint32_t)__popc(vmask) * box_bytes + scale_bytes);
   load_boxes(tp, nbox, box_t, regions, g, key0, pv, vdst, bars_v[1]);
+  if (sdst) {
+    load_scales(p, nbox, box_t, g, key0, pk, sdst, bars_v[1]);
+    load_scales(p, nbox, box_t, g, key0, pv, sdst + kTK * 4, bars_v[1]);
+  }
   return 1;
 }
 
@@ -572,11 +609,13 @@ struct TcLayout {
                                     kSeqTab * (int)sizeof(SeqRec);
   // one K or V tile: 128 keys of 128 dims (two 64-dim regions when 16-bit)
   static constexpr int kHalfStage = kF8 ? kRegionBytes : 2 * kRegionBytes;
+  // per-vector scales of one tile, K then V (128 FP32 each), per ring stage
+  static constexpr int kScStage = 2 * kTK * 4;
   // stages: K/V ring depth; q_slots: Q ring depth (1 or 2); p_bufs: P tiles
-  // per softmax group (1 or 2)
-  static int smem_bytes(int stages, int q_slots, int p_bufs) {
+  // per softmax group (1 or 2); scaled: per-vector scale rows per stage
+  static int smem_bytes(int stages, int q_slots, int p_bufs, bool scaled) {
     return 1024 + stages * 2 * kHalfStage + q_slots * kQBytes + 2 * p_bufs * kPBytes +
-           kMiscBytes;
+           (scaled ? stages * kScStage : 0) + kMiscBytes;
   }
 };
 
@@ -859,11 +898,12 @@ __device__ __forceinline__ bool stage_q(const LseKernelParams &p, int t, int g, 
   return true;
 }
 
-template <int DT, int P8>
+template <int DT, int P8, bool kSc>
 __global__ void __launch_bounds__(kThreads, 1)
     partial_tcgen05_kernel(const __grid_constant__ TcParams tp) {
   using Lay = TcLayout<DT, P8>;
   constexpr bool kF8 = Lay::kF8;
+  static_assert(!kSc || kF8, "per-vector scales go with the 8-bit formats");
   constexpr bool kE5 = DT == LSE_KV_FP8_E5M2;
   constexpr int kNQ = Lay::kNQ;
   constexpr int kN = Lay::kN;
@@ -882,7 +922,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t v_base = k_base + NS * Lay::kHalfStage;        // V ring
   const uint32_t q_base = v_base + NS * Lay::kHalfStage;        // Q slots
   const uint32_t p_base = q_base + QS * Lay::kQBytes;          // P tiles [group][buffer]
-  uint8_t *misc = smem + (p_base - sbase) + 2 * PB * Lay::kPBytes;
+  const uint32_t sc_base = p_base + 2 * PB * Lay::kPBytes;     // scale rows [stage]
+  uint8_t *misc = smem + (sc_base - sbase) + (kSc ? NS * Lay::kScStage : 0);
   // the P tile of group grp used with its tile of index n (n & 1 == grp)
   auto p_tile = [&](int grp, int n) {
     return p_base + (uint32_t)((grp * PB + ((n >> 1) % PB)) * Lay::kPBytes);
@@ -1042,7 +1083,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           go = produce_tile(tp, n, NS, nbox, box_t, kF8 ? 1 : 2, tg, tt, tl, pk + i * 16,
                             pv + i * 16,
                             k_base + (n % NS) * Lay::kHalfStage,
-                            v_base + (n % NS) * Lay::kHalfStage, bars_k, bars_v,
+                            v_base + (n % NS) * Lay::kHalfStage,
+                            kSc ? sc_base + (n % NS) * Lay::kScStage : 0u, bars_k, bars_v,
                             bar(kBarInfo + (n & 7)), tile_info + (n & 7), abort_flag);
         }
         go = __shfl_sync(0xffffffffu, go, 0);
@@ -1330,6 +1372,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int pbuf_n = (n >> 1) % PB, use = (n >> 1) / PB;
         if (w && use >= 1)
           w = mbar_wait(bar(kBarPEmpty + 2 * grp + pbuf_n), (use - 1) & 1, abort_flag, p.err);
+        // per-vector scales land with the tile's V (the V slot outlives
+        // this pass: its output product waits for this tile's P)
+        if (kSc && w)
+          w = mbar_wait(bar(kBarFullV + n % NS), (n / NS) & 1, abort_flag, p.err);
         if (named_or(bar_id, 128, !w)) {
           ok = false;
           break;
@@ -1339,6 +1385,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int key = key0 + j;
         const uint32_t both = inf.x & inf.y;
         const bool kvalid = j < (int)inf.z && (both >> (j / box_t) & 1u);
+        // Per-vector scales.  The key's score is multiplied by its K scale;
+        // its V scale sV enters through the probability: with u = x + log2 sV
+        // in place of the score x, the running max and P follow u, P.V sums
+        // 2^(u - m) V = 2^(x - m) sV V, and the row sums add 2^(u - m) / sV =
+        // 2^(x - m), so the output and log-sum-exp come out unchanged while P
+        // stays within the range the unscaled path gives it.  (A V scale
+        // below 2^-64 is read as 2^-64; a dead key keeps unit scales.)
+        float ks = 1.f, lv = 0.f, ivs = 1.f;
+        if constexpr (kSc) {
+          if (kvalid) {
+            const float *scs = reinterpret_cast<const float *>(
+                smem + (sc_base - sbase) + (n % NS) * Lay::kScStage);
+            ks = scs[j];
+            float vs = scs[kTK + j];
+            vs = vs < 0x1p-64f ? 0x1p-64f : vs;  // (NaN stays NaN)
+            lv = log2f(vs);
+            ivs = 1.f / vs;
+          }
+        }
         // visibility of this key to each pair, as a bit mask
         unsigned long long vis;
         if (key0 + kTK <= Cctx && inf.z == (uint32_t)kTK && both == full_boxes) {
@@ -1364,6 +1429,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 8; ++i) sv[c + i] *= isg[c + i];
           }
+        }
+        if constexpr (kSc) {
+#pragma unroll
+          for (int q = 0; q < P8; ++q) sv[q] = fmaf(sv[q], ks, lv);
         }
         if (vis != ~0ull) {
 #pragma unroll
@@ -1474,8 +1543,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if constexpr (kLAcc) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) lacc[c + i] += e[i];
+            for (int i = 0; i < 8; ++i) lacc[c + i] = kSc ? fmaf(e[i], ivs, lacc[c + i])
+                                                          : lacc[c + i] + e[i];
           } else {
+            if constexpr (kSc) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) e[i] *= ivs;  // (P was stored above)
+            }
             const float ws = warp_sum8(e, lane);
             if ((lane & 3) == 0) lp[c + (lane >> 2)] = ws;
           }
@@ -1587,9 +1661,9 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-template <int DT, int P8>
+template <int DT, int P8, bool kSc>
 int launch_tc(const TcParams &tp, int smem, cudaStream_t st) {
-  auto k = partial_tcgen05_kernel<DT, P8>;
+  auto k = partial_tcgen05_kernel<DT, P8, kSc>;
   static int set_for = -1;  // largest dynamic smem already allowed (per device run)
   if (smem > set_for) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -1600,34 +1674,34 @@ int launch_tc(const TcParams &tp, int smem, cudaStream_t st) {
   return (int)cudaGetLastError();
 }
 
-template <int DT>
+template <int DT, bool kSc>
 int launch_tc_p(const TcParams &tp, int p8, int smem, cudaStream_t st) {
   switch (p8) {
-    case 8: return launch_tc<DT, 8>(tp, smem, st);
-    case 16: return launch_tc<DT, 16>(tp, smem, st);
-    case 24: return launch_tc<DT, 24>(tp, smem, st);
-    case 32: return launch_tc<DT, 32>(tp, smem, st);
-    case 48: return launch_tc<DT, 48>(tp, smem, st);
+    case 8: return launch_tc<DT, 8, kSc>(tp, smem, st);
+    case 16: return launch_tc<DT, 16, kSc>(tp, smem, st);
+    case 24: return launch_tc<DT, 24, kSc>(tp, smem, st);
+    case 32: return launch_tc<DT, 32, kSc>(tp, smem, st);
+    case 48: return launch_tc<DT, 48, kSc>(tp, smem, st);
   }
   return (int)cudaErrorInvalidValue;
 }
 
 template <int DT>
-int smem_for_p(int p8, int stages, int q_slots, int p_bufs) {
+int smem_for_p(int p8, int stages, int q_slots, int p_bufs, bool scaled) {
   switch (p8) {
-    case 8: return TcLayout<DT, 8>::smem_bytes(stages, q_slots, p_bufs);
-    case 16: return TcLayout<DT, 16>::smem_bytes(stages, q_slots, p_bufs);
-    case 24: return TcLayout<DT, 24>::smem_bytes(stages, q_slots, p_bufs);
-    case 32: return TcLayout<DT, 32>::smem_bytes(stages, q_slots, p_bufs);
-    case 48: return TcLayout<DT, 48>::smem_bytes(stages, q_slots, p_bufs);
+    case 8: return TcLayout<DT, 8>::smem_bytes(stages, q_slots, p_bufs, scaled);
+    case 16: return TcLayout<DT, 16>::smem_bytes(stages, q_slots, p_bufs, scaled);
+    case 24: return TcLayout<DT, 24>::smem_bytes(stages, q_slots, p_bufs, scaled);
+    case 32: return TcLayout<DT, 32>::smem_bytes(stages, q_slots, p_bufs, scaled);
+    case 48: return TcLayout<DT, 48>::smem_bytes(stages, q_slots, p_bufs, scaled);
   }
   return -1;
 }
 
-int smem_for(int dtype, int p8, int stages, int q_slots, int p_bufs) {
+int smem_for(int dtype, int p8, int stages, int q_slots, int p_bufs, bool scaled) {
   // the two 16-bit formats share a layout, and so do the two 8-bit ones
-  return is_f8(dtype) ? smem_for_p<LSE_KV_FP8_E4M3>(p8, stages, q_slots, p_bufs)
-                      : smem_for_p<LSE_KV_BF16>(p8, stages, q_slots, p_bufs);
+  return is_f8(dtype) ? smem_for_p<LSE_KV_FP8_E4M3>(p8, stages, q_slots, p_bufs, scaled)
+                      : smem_for_p<LSE_KV_BF16>(p8, stages, q_slots, p_bufs, scaled);
 }
 
 }  // namespace
@@ -1647,11 +1721,13 @@ int lse_tc_pairs_bucket(int pairs) {
 // staging with the end of the previous segment) when it fits as well.  The
 // kernel also runs with two P tiles per group (p_bufs = 2), which the planner
 // does not pick.
-int lse_tc_smem(int dtype, int p8, int smem_optin, int *stages, int *q_slots, int *p_bufs) {
+int lse_tc_smem(int dtype, int p8, int scaled, int smem_optin, int *stages, int *q_slots,
+                int *p_bufs) {
+  if (scaled && !is_f8(dtype)) return -1;
   for (int pb = 1; pb >= 1; --pb)
     for (int ns = kMaxStages; ns >= 2; --ns)
       for (int qs = 2; qs >= 1; --qs) {
-        const int b = smem_for(dtype, p8, ns, qs, pb);
+        const int b = smem_for(dtype, p8, ns, qs, pb, scaled != 0);
         if (b > 0 && b <= smem_optin) {
           *stages = ns;
           *q_slots = qs;
@@ -1701,8 +1777,8 @@ int lse_tc_build_maps(const uint64_t *chunk_base, int n_chunks, size_t chunk_byt
 size_t lse_tc_map_bytes() { return sizeof(CUtensorMap); }
 
 int lse_launch_partial_tcgen05(const LseKernelParams &p, const void *maps, int n_maps,
-                               int dtype, int p8, int n_ctas, int n_slots, int stages,
-                               int q_slots, int p_bufs, int box_tokens, int smem,
+                               int dtype, int p8, int scaled, int n_ctas, int n_slots,
+                               int stages, int q_slots, int p_bufs, int box_tokens, int smem,
                                void *stream) {
   static_assert(sizeof(TcParams) < 30000, "kernel parameter block too large");
   TcParams tp;
@@ -1717,10 +1793,16 @@ int lse_launch_partial_tcgen05(const LseKernelParams &p, const void *maps, int n
   tp.box_tokens = box_tokens;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   switch (dtype) {
-    case LSE_KV_BF16: return launch_tc_p<LSE_KV_BF16>(tp, p8, smem, st);
-    case LSE_KV_F16: return launch_tc_p<LSE_KV_F16>(tp, p8, smem, st);
-    case LSE_KV_FP8_E4M3: return launch_tc_p<LSE_KV_FP8_E4M3>(tp, p8, smem, st);
-    case LSE_KV_FP8_E5M2: return launch_tc_p<LSE_KV_FP8_E5M2>(tp, p8, smem, st);
+    case LSE_KV_BF16:
+      return scaled ? (int)cudaErrorInvalidValue : launch_tc_p<LSE_KV_BF16, false>(tp, p8, smem, st);
+    case LSE_KV_F16:
+      return scaled ? (int)cudaErrorInvalidValue : launch_tc_p<LSE_KV_F16, false>(tp, p8, smem, st);
+    case LSE_KV_FP8_E4M3:
+      return scaled ? launch_tc_p<LSE_KV_FP8_E4M3, true>(tp, p8, smem, st)
+                    : launch_tc_p<LSE_KV_FP8_E4M3, false>(tp, p8, smem, st);
+    case LSE_KV_FP8_E5M2:
+      return scaled ? launch_tc_p<LSE_KV_FP8_E5M2, true>(tp, p8, smem, st)
+                    : launch_tc_p<LSE_KV_FP8_E5M2, false>(tp, p8, smem, st);
   }
   return (int)cudaErrorInvalidValue;
 }

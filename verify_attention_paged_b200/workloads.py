@@ -135,6 +135,7 @@ def build(
     gen: torch.Generator | None = None,
     scaled: bool = False,
     scale_spread: float = 0.0,
+    magnitude_spread: float = 0.0,
 ) -> Workload:
     """Lay out one seeded problem.
 
@@ -144,9 +145,13 @@ def build(
 
     ``scaled`` (8-bit formats) stores every K and V vector with a per-vector
     FP32 scale, amax / (largest finite value of the format), the stored
-    elements being the vector divided by it and cast; ``scale_spread``
-    first multiplies each vector by 2^u, u uniform in [-spread, spread], so
-    the scales span a range of magnitudes.
+    elements being the vector divided by it and cast.  ``magnitude_spread``
+    first multiplies each vector by 2^u, u uniform in [-spread, spread] (the
+    vectors' sizes vary, and their scales with them); ``scale_spread``
+    multiplies each scale by 2^u, u uniform in [0, spread] (the scales vary
+    over that many binades while the vectors they give back do not: the
+    stored elements shrink by the same factor, never past the format's
+    largest value).
     """
     g = gen if gen is not None else torch.Generator().manual_seed(seed)
     es = ELEM_SIZE[dtype]
@@ -200,10 +205,12 @@ def build(
             x = torch.randn((L, n_kv_heads, head_dim), generator=g, dtype=torch.float32)
             x = x * kv_std
             if scaled:
-                if scale_spread > 0:
-                    u = (torch.rand((L, n_kv_heads, 1), generator=g) * 2 - 1) * scale_spread
+                if magnitude_spread > 0:
+                    u = (torch.rand((L, n_kv_heads, 1), generator=g) * 2 - 1) * magnitude_spread
                     x = x * torch.exp2(u)
                 sc = x.abs().amax(dim=2) / torch.finfo(tdt).max      # [L, Hkv]
+                if scale_spread > 0:
+                    sc = sc * torch.exp2(torch.rand((L, n_kv_heads), generator=g) * scale_spread)
                 sc = torch.where(sc > 0, sc, torch.ones_like(sc))
                 x = x / sc[:, :, None]
                 sc = sc.numpy()
@@ -304,6 +311,16 @@ def long_e5m2(keep_logical=False) -> Workload:
                  keep_logical=keep_logical)
 
 
+def long_fp8_scaled(keep_logical=False) -> Workload:
+    """The long-context FP8 (E4M3) workload stored with per-vector FP32
+    scales (the README's fp8 "with scales" format): each K and V vector of
+    N(0, 0.5^2) values is divided by amax / 448 and cast, its scale kept in
+    the fragment's scale block."""
+    return build("long_fp8_scaled", "e4m3", [68173], [4], 24, 4, 128,
+                 fragment_bytes=512 * 4 * 128, chunk_bytes=256 * MIB, max_pages=256, seed=1243,
+                 kv_std=0.5, n_chunks=1, keep_logical=keep_logical, scaled=True)
+
+
 BUILDERS = {
     "tiny_decode": tiny_decode,
     "batched_decode": batched_decode,
@@ -311,9 +328,10 @@ BUILDERS = {
     "long_fp8": long_fp8,
     "tree_verify": tree_verify,
     "long_e5m2": long_e5m2,
+    "long_fp8_scaled": long_fp8_scaled,
 }
 # workloads beyond the five benchmark configurations
-EXTRA_NAMES = ["long_e5m2"]
+EXTRA_NAMES = ["long_e5m2", "long_fp8_scaled"]
 
 
 # ---------------------------------------------------------------------------
@@ -370,7 +388,8 @@ def fragment_ab_cases() -> list[Workload]:
 
 def small_case(dtype: str, seq_lens, rows, n_q_heads=8, n_kv_heads=2, head_dim=64,
                tokens_per_fragment=16, max_pages=None, seed=7, tree=False, kv_std=1.0,
-               keep_logical=True, n_chunks=None, scaled=False, scale_spread=0.0) -> Workload:
+               keep_logical=True, n_chunks=None, scaled=False, scale_spread=0.0,
+               magnitude_spread=0.0) -> Workload:
     """A small seeded problem of any shape, for parity and pin tests."""
     g = torch.Generator().manual_seed(seed)
     es = ELEM_SIZE[dtype]
@@ -385,4 +404,5 @@ def small_case(dtype: str, seq_lens, rows, n_q_heads=8, n_kv_heads=2, head_dim=6
     return build(f"small_{dtype}", dtype, list(seq_lens), list(rows), n_q_heads, n_kv_heads,
                  head_dim, fragment_bytes=fb, chunk_bytes=fb * fpc, max_pages=max_pages,
                  seed=seed, parents=parents, kv_std=kv_std, keep_logical=keep_logical,
-                 n_chunks=n_chunks, gen=g, scaled=scaled, scale_spread=scale_spread)
+                 n_chunks=n_chunks, gen=g, scaled=scaled, scale_spread=scale_spread,
+                 magnitude_spread=magnitude_spread)
