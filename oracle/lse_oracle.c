@@ -59,6 +59,13 @@
  * FP16/BF16 overflow to infinity as IEEE formats do; the FP8 formats
  * saturate to their largest finite value (E4M3 has no infinity; the pages
  * fix no overflow rule for E5M2, and saturating keeps a cache finite).
+ * With per-vector scales (8-bit formats) the append also picks each new
+ * vector's scale: the pages say only that scales exist, so the reading is
+ * the usual per-vector one, scale = (largest magnitude in the vector) /
+ * (largest finite value of the format), 1 for an all-zero vector, every
+ * element stored as the FP32 quotient element / scale rounded to the
+ * format.  Both divisions are FP32 operations (correctly rounded), so the
+ * stored code is fixed to the bit.
  */
 #include <math.h>
 #include <stddef.h>
@@ -461,13 +468,16 @@ int orc_kv_append(uint8_t *const *chunks, int n_chunks, int64_t chunk_bytes,
                   int64_t fragment_bytes, int dtype, int n_kv_heads, int head_dim, int n_seqs,
                   int max_pages, const int32_t *k_pages, const int32_t *v_pages,
                   const int32_t *seq_lens_before, const int32_t *new_offsets,
-                  const float *k_new, const float *v_new) {
+                  const float *k_new, const float *v_new, float *scales, int64_t n_scales) {
   const int es = elem_size(dtype);
   if (es == 0) return ORC_BAD_DTYPE;
   if (n_kv_heads < 1 || head_dim < 1 || fragment_bytes < (int64_t)n_kv_heads * head_dim * es)
     return ORC_BAD_SHAPE;
   const int64_t T = fragment_bytes / ((int64_t)n_kv_heads * head_dim * es);
   const int64_t per_chunk = chunk_bytes / fragment_bytes;
+  if (scales && (es != 1 || n_scales < per_chunk * n_chunks * n_kv_heads * T))
+    return ORC_BAD_SHAPE;  /* 8-bit formats, a block for every fragment */
+  const float fmt_max = dtype == ORC_E4M3 ? 448.0f : 57344.0f;
   int status = ORC_OK;
   for (int s = 0; s < n_seqs; ++s) {
     for (int32_t i = new_offsets[s]; i < new_offsets[s + 1]; ++i) {
@@ -487,13 +497,23 @@ int orc_kv_append(uint8_t *const *chunks, int n_chunks, int64_t chunk_bytes,
         }
         uint8_t *dst = chunks[frag / per_chunk] + (frag % per_chunk) * fragment_bytes +
                        off * (int64_t)n_kv_heads * head_dim * es;
-        for (int g = 0; g < n_kv_heads; ++g)
+        for (int g = 0; g < n_kv_heads; ++g) {
+          const float *x = src + ((int64_t)i * n_kv_heads + g) * head_dim;
+          float sc = 1.0f;
+          if (scales) {
+            float amax = 0.0f;
+            for (int d = 0; d < head_dim; ++d)
+              if (fabsf(x[d]) > amax) amax = fabsf(x[d]);
+            if (amax > 0.0f) sc = amax / fmt_max;
+            scales[((int64_t)frag * n_kv_heads + g) * T + off] = sc;
+          }
           for (int d = 0; d < head_dim; ++d) {
-            const int64_t e = ((int64_t)i * n_kv_heads + g) * head_dim + d;
-            const uint32_t bits = orc_encode(dtype, (double)src[e]);
+            const float q = scales ? x[d] / sc : x[d];
+            const uint32_t bits = orc_encode(dtype, (double)q);
             uint8_t *o = dst + ((int64_t)g * head_dim + d) * es;
             for (int b = 0; b < es; ++b) o[b] = (uint8_t)((bits >> (8 * b)) & 0xffu);
           }
+        }
       }
     }
   }

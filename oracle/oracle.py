@@ -90,7 +90,7 @@ def _load():
         lib.orc_kv_append.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int,
                                       ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
                                       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                      vp, vp, vp, vp, vp, vp]
+                                      vp, vp, vp, vp, vp, vp, vp, ctypes.c_int64]
         lib.orc_kv_append.restype = ctypes.c_int
         for f in (lib.orc_attention, lib.orc_attention_one, lib.orc_attention_split):
             f.restype = ctypes.c_int
@@ -211,12 +211,16 @@ def encode(dtype: str, x: float) -> int:
 
 
 def kv_append(chunks, chunk_bytes, fragment_bytes, dtype, n_kv_heads, head_dim, k_pages,
-              v_pages, seq_lens_before, new_offsets, k_new, v_new):
+              v_pages, seq_lens_before, new_offsets, k_new, v_new, scales=None):
     """Write new tokens' K/V into host copies of the arena chunks (modified in
     place): token i of sequence s (new_offsets[s] <= i < new_offsets[s+1])
-    goes to key position seq_lens_before[s] + i - new_offsets[s].  Returns
-    the oracle status (0, or 2 when some position has no fragment; the
-    others are written)."""
+    goes to key position seq_lens_before[s] + i - new_offsets[s].  With
+    ``scales`` (a float32 per-vector scale array, 8-bit formats; modified in
+    place) each vector is stored divided by its new scale.  Returns the
+    oracle status (0, or 2 when some position has no fragment; the others
+    are written)."""
+    if scales is not None:
+        assert scales.dtype == np.float32 and scales.flags["C_CONTIGUOUS"]
     for c in chunks:
         assert c.dtype == np.uint8 and c.flags["C_CONTIGUOUS"]
     kp, vp_ = _as(k_pages, np.int32), _as(v_pages, np.int32)
@@ -227,4 +231,5 @@ def kv_append(chunks, chunk_bytes, fragment_bytes, dtype, n_kv_heads, head_dim, 
         ctypes.cast(ptrs, ctypes.POINTER(ctypes.c_void_p)), len(chunks), int(chunk_bytes),
         int(fragment_bytes), DTYPE_CODES[dtype], int(n_kv_heads), int(head_dim), len(sl),
         kp.shape[1], kp.ctypes.data, vp_.ctypes.data, sl.ctypes.data, no.ctypes.data,
-        kn.ctypes.data, vn.ctypes.data))
+        kn.ctypes.data, vn.ctypes.data, None if scales is None else scales.ctypes.data,
+        0 if scales is None else scales.size))

@@ -165,3 +165,57 @@ def test_append_past_the_page_table_is_reported_and_skipped():
     b = off * w.fragment_bytes + 7 * 16
     assert np.array_equal(chunks[c][b:b + 16].view(np.uint16),
                           np.full(8, 0x3F80, np.uint16))  # bf16 1.0
+
+
+@pytest.mark.parametrize("dtype", ["e4m3", "e5m2"])
+def test_scaled_append_restores_the_generator_bytes_and_scales(dtype):
+    # the generator drew per-vector scales amax / (largest finite value) and
+    # stored each vector divided by its scale (FP32 division, torch's cast);
+    # re-appending the last keys of each sequence from the same FP32 vectors
+    # gives back the same bytes and the same scales, bit for bit
+    w = wl.small_case(dtype, [40, 9, 1, 33], [1, 2, 1, 3], n_q_heads=4, n_kv_heads=2,
+                      head_dim=16, tokens_per_fragment=8, seed=44, scaled=True,
+                      magnitude_spread=4.0)
+    chunks = [c.copy() for c in w.chunks]
+    scales = w.scales.copy()
+    T, Hkv = w.tokens_per_fragment, w.n_kv_heads
+    fpc = w.chunk_bytes // w.fragment_bytes
+    row = Hkv * w.head_dim
+    n_new = 11
+    before, offs, ks, vs = [], [0], [], []
+    for s in range(w.n_seqs):
+        L = int(w.seq_lens[s])
+        m = min(n_new, L)
+        before.append(L - m)
+        offs.append(offs[-1] + m)
+        for j in range(L - m, L):
+            for table in (w.k_pages, w.v_pages):
+                f = int(table[s, j // T])
+                c, off = divmod(f, fpc)
+                b = off * w.fragment_bytes + (j % T) * row
+                chunks[c][b:b + row] = 0xFF
+                scales[f * Hkv * T + np.arange(Hkv) * T + j % T] = np.nan
+        ks.append(w.logical_k_src[s][L - m:L].numpy())
+        vs.append(w.logical_v_src[s][L - m:L].numpy())
+    st = orc.kv_append(chunks, w.chunk_bytes, w.fragment_bytes, dtype, Hkv, w.head_dim,
+                       w.k_pages, w.v_pages, np.array(before, np.int32),
+                       np.array(offs, np.int32), np.concatenate(ks), np.concatenate(vs),
+                       scales=scales)
+    assert st == 0
+    for a, b in zip(chunks, w.chunks):
+        assert np.array_equal(a, b)
+    assert np.array_equal(scales.view(np.uint32), w.scales.view(np.uint32))
+
+
+def test_scaled_append_of_a_zero_vector_uses_unit_scale():
+    w = wl.small_case("e4m3", [8], [1], n_q_heads=2, n_kv_heads=1, head_dim=8,
+                      tokens_per_fragment=8, seed=45, scaled=True)
+    chunks = [c.copy() for c in w.chunks]
+    scales = w.scales.copy()
+    z = np.zeros((1, 1, 8), np.float32)
+    st = orc.kv_append(chunks, w.chunk_bytes, w.fragment_bytes, "e4m3", 1, 8, w.k_pages,
+                       w.v_pages, np.array([7], np.int32), np.array([0, 1], np.int32), z, z,
+                       scales=scales)
+    assert st == 0
+    for table in (w.k_pages, w.v_pages):
+        assert scales[int(table[0, 0]) * 8 + 7] == 1.0

@@ -58,6 +58,10 @@ MUTANTS = {
                                 "int64_t at = ((int64_t)frag * T + j % T) * pb->n_kv_heads + g;"),
     "v_scale_through_k_table": ("vec_scale(pb, pb->v_pages", "vec_scale(pb, pb->k_pages"),
     "v_scale_in_denominator": ("    l += p;\n", "    l += p * sv;\n"),
+    "append_not_divided_by_scale": ("const float q = scales ? x[d] / sc : x[d];",
+                                    "const float q = x[d];"),
+    "append_scale_formats_swapped": ("dtype == ORC_E4M3 ? 448.0f : 57344.0f",
+                                     "dtype == ORC_E4M3 ? 57344.0f : 448.0f"),
 }
 
 
@@ -143,6 +147,8 @@ def _pins_fail(lib) -> list:
         check("encoder_ties_e5m2", lambda: pins_append.test_encoder_rounds_ties_to_even("e5m2"))
         check("append_bf16", lambda: append("bf16"))
         check("scaled_sdpa_e4m3", lambda: pins_scale.test_scaled_matches_library_sdpa("e4m3", True))
+        check("scaled_append_e4m3",
+              lambda: pins_append.test_scaled_append_restores_the_generator_bytes_and_scales("e4m3"))
         check("sdpa_bf16_tree", lambda: sdpa("bf16", True))
         check("sdpa_e4m3_chain", lambda: sdpa("e4m3", False))
         check("split", split)

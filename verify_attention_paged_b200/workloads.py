@@ -67,6 +67,9 @@ class Workload:
     scales: np.ndarray | None = None
     logical_k_scale: list = field(default_factory=list)  # per seq float32 [L, Hkv]
     logical_v_scale: list = field(default_factory=list)
+    # scaled: the FP32 vectors before they were divided by their scales
+    logical_k_src: list = field(default_factory=list)    # per seq float32 [L, Hkv, D]
+    logical_v_src: list = field(default_factory=list)
 
     @property
     def n_seqs(self) -> int:
@@ -199,6 +202,7 @@ def build(
     scales = np.full(n_chunks * fpc * n_kv_heads * T, np.nan, np.float32) if scaled else None
     logical_k, logical_v = [], []
     logical_ks, logical_vs = [], []
+    src_k, src_v = [], []
     for s in range(S):
         L = seq_lens[s]
         for which, table in (("k", k_pages), ("v", v_pages)):
@@ -208,6 +212,8 @@ def build(
                 if magnitude_spread > 0:
                     u = (torch.rand((L, n_kv_heads, 1), generator=g) * 2 - 1) * magnitude_spread
                     x = x * torch.exp2(u)
+                if keep_logical:
+                    (src_k if which == "k" else src_v).append(x.clone())
                 sc = x.abs().amax(dim=2) / torch.finfo(tdt).max      # [L, Hkv]
                 if scale_spread > 0:
                     sc = sc * torch.exp2(torch.rand((L, n_kv_heads), generator=g) * scale_spread)
@@ -237,7 +243,8 @@ def build(
         row_offsets=row_offsets, row_masks=row_masks, q=q, scale=1.0 / math.sqrt(head_dim),
         seed=seed, logical_k=logical_k, logical_v=logical_v,
         parents=parents if parents is not None else [], scales=scales,
-        logical_k_scale=logical_ks, logical_v_scale=logical_vs)
+        logical_k_scale=logical_ks, logical_v_scale=logical_vs, logical_k_src=src_k,
+        logical_v_src=src_v)
 
 
 # ---------------------------------------------------------------------------
