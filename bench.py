@@ -63,8 +63,7 @@ def measured_peaks():
 
 # the sources each measured kernel (and its launch plan) is built from
 KERNEL_SOURCES = {
-    "partial": ("lse_host.cpp", "lse_internal.h", "lse_kernels.cu", "lse_static.cu",
-                "lse_tcgen05.cu"),
+    "partial": ("lse_host.cpp", "lse_internal.h", "lse_tcgen05.cu"),
     "append": ("lse_append.cu", "lse_host.cpp", "lse_internal.h"),
 }
 

@@ -160,11 +160,13 @@ LSE_API int lse_kv_arena_query(const lse_kv_arena *arena, lse_kv_arena_info *inf
  *           non-negative; a V scale below 2^-64 may be read as 2^-64 (the
  *           value it weights changes by less than 2^-64 of the output).
  *   scales = NULL removes them (unit scales).
- * Plans record whether the arena had scales when they were made; running a
- * plan after the arena's scales were added or removed is LSE_ERR_INVALID_ARG.
+ * Attention reads the scales; lse_kv_append writes the scales of the
+ * vectors it stores.  Plans record whether the arena had scales when they
+ * were made; running a plan after the arena's scales were added or removed
+ * is LSE_ERR_INVALID_ARG.
  * Errors: LSE_ERR_UNSUPPORTED for 16-bit or FP32 arenas, LSE_ERR_INVALID_ARG
  * for a misaligned or short array. */
-LSE_API int lse_kv_arena_set_scales(lse_kv_arena *arena, const float *scales, int64_t n_floats,
+LSE_API int lse_kv_arena_set_scales(lse_kv_arena *arena, float *scales, int64_t n_floats,
                                     char **err);
 
 LSE_API void lse_kv_arena_destroy(lse_kv_arena *arena);
@@ -307,6 +309,11 @@ LSE_API int lse_attn_read_error(const lse_attn_plan_t *plan, void *workspace, vo
  * their fragments, cast from FP32 to the arena's storage format: the nearest
  * value of the format, ties to even; F16 and BF16 overflow to infinity,
  * E4M3 and E5M2 saturate at their largest finite value (448, 57344).
+ * When the arena has per-vector scales (lse_kv_arena_set_scales), each
+ * vector's scale is its largest magnitude over the format's largest finite
+ * value (1 for an all-zero vector), written to its entry of the scale
+ * array, and each element is stored as the FP32 quotient element / scale,
+ * rounded as above.
  *
  * Token i of sequence s, new_offsets[s] <= i < new_offsets[s+1], goes to key
  * position seq_lens_before[s] + i - new_offsets[s] of s (page = position / T,

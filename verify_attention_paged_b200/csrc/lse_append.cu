@@ -9,7 +9,12 @@
 // table, and each lane stores its converted slices (coalesced across the
 // warp).  Casts: nearest value, ties to
 // even (cvt.rn); FP8 through cvt.rn.satfinite (saturating at the largest
-// finite value); F16 and BF16 overflow to infinity.
+// finite value); F16 and BF16 overflow to infinity.  With per-vector scales
+// (8-bit arenas) the warp also takes each vector's largest magnitude (a
+// butterfly max), its scale = that / the format's largest finite value (1
+// for a zero vector), stores the elements divided by it (FP32 division,
+// correctly rounded) and lane 0 writes the scale to the [kv_head][token]
+// block of the fragment.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -91,6 +96,30 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) kv_append_kernel(const Ap
     xv[k] = fv.x;
     xv[k + 1] = fv.y;
   }
+  float sk = 1.f, sv = 1.f;
+  if constexpr (DT == LSE_KV_FP8_E4M3 || DT == LSE_KV_FP8_E5M2) {
+    if (a.scales) {
+      float mk = 0.f, mv = 0.f;
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        mk = fmaxf(mk, fabsf(xk[k]));
+        mv = fmaxf(mv, fabsf(xv[k]));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        mk = fmaxf(mk, __shfl_xor_sync(0xffffffffu, mk, o));
+        mv = fmaxf(mv, __shfl_xor_sync(0xffffffffu, mv, o));
+      }
+      constexpr float kFmtMax = DT == LSE_KV_FP8_E4M3 ? 448.f : 57344.f;
+      if (mk > 0.f) sk = __fdiv_rn(mk, kFmtMax);
+      if (mv > 0.f) sv = __fdiv_rn(mv, kFmtMax);
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        xk[k] = __fdiv_rn(xk[k], sk);
+        xv[k] = __fdiv_rn(xv[k], sv);
+      }
+    }
+  }
   // the token's sequence, the last s with new_offsets[s] <= i: each round the
   // 32 lanes test 32 evenly spaced offsets of the remaining range
   int lo = 0, span = a.n_seqs;  // s in [lo, lo + span)
@@ -126,6 +155,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) kv_append_kernel(const Ap
                    (long long)(frag - c * a.frags_per_chunk) * a.fragment_bytes +
                    ((slot * a.n_kv_heads + g) * D + lane * kPer) * kEs;
     store_slice<DT, kPer>(kv ? xv : xk, dst);
+    if (a.scales && lane == 0)
+      a.scales[((long long)frag * a.n_kv_heads + g) * a.tokens_per_fragment + slot] = kv ? sv : sk;
   }
 }
 

@@ -134,8 +134,7 @@ int lse_kv_arena_add_chunk(lse_kv_arena *a, void *chunk_base, int32_t *first_id,
   return LSE_OK;
 }
 
-int lse_kv_arena_set_scales(lse_kv_arena *a, const float *scales, int64_t n_floats,
-                            char **err) {
+int lse_kv_arena_set_scales(lse_kv_arena *a, float *scales, int64_t n_floats, char **err) {
   if (!a) return fail(err, LSE_ERR_INVALID_ARG, "arena is NULL");
   if (!scales) {
     a->scales = nullptr;
@@ -460,6 +459,11 @@ int lse_kv_append(const lse_kv_arena *a, int n_seqs, int max_pages, const float 
   p.seq_lens_before = seq_lens_before;
   p.new_offsets = new_offsets;
   p.err = err_word;
+  if (a->scales) {
+    if (a->n_scales < int64_t(a->used.size()) * a->n_kv_heads * a->tokens_per_fragment)
+      return fail(err, LSE_ERR_INVALID_ARG, "the arena grew past its scale array");
+    p.scales = a->scales;
+  }
   const int ce = lse_launch_kv_append(p, a->dtype, a->head_dim, stream);
   if (ce) return cuda_fail(err, ce, "append kernel launch");
   return LSE_OK;

@@ -23,7 +23,7 @@ struct lse_kv_arena {
   std::vector<int32_t> chunk_live;  // live fragments per chunk
   int32_t n_free = 0;
   int32_t scan_from = 0;            // lowest id that may be free
-  const float *scales = nullptr;    // per-vector scales by fragment (device), or null
+  float *scales = nullptr;          // per-vector scales by fragment (device), or null
   int64_t n_scales = 0;             // floats in scales
 };
 
@@ -120,6 +120,7 @@ struct AppendParams {
   const int32_t *seq_lens_before;
   const int32_t *new_offsets;
   unsigned int *err;
+  float *scales;  // 8-bit arenas with per-vector scales: written with the vectors
 };
 int lse_launch_kv_append(const AppendParams &a, int dtype, int head_dim, void *stream);
 

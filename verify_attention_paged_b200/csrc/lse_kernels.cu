@@ -393,15 +393,14 @@ constexpr int kMergeThreads = kMergeWarps * 32;
 // row's sequence and which partials of its segment are live (the scan over
 // the sequences reads only call inputs, all threads at once, so it overlaps
 // the partial pass's tail).  Each warp then loads its share of the partials
-// (warp w: partials w, w + 8, ..., eight in flight per lane, each lane a D/32
-// slice of the head dim) and keeps a running maximum of their lse; the
+// (warp w: partials w, w + 8, ..., kUnroll in flight per lane, each lane a
+// D/32 slice of the head dim) and keeps a running maximum of their lse; the
 // warps' sums are rescaled to the common maximum and added in warp order in
 // shared memory.
-template <int D>
+template <int D, int kUnroll>
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
     const __grid_constant__ LseKernelParams p) {
   constexpr int kPerLane = D / 32;
-  constexpr int kUnroll = 8;
   __shared__ float s_m[kMergeWarps], s_w[kMergeWarps];
   __shared__ float s_acc[kMergeWarps][D];
   __shared__ long long s_cnt[kMergeWarps][2];
@@ -609,7 +608,8 @@ int lse_launch_partial_cuda_core(const LseKernelParams &p, int dtype, int head_d
 template <int D>
 int launch_merge_d(const LseKernelParams &p, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)p.max_total_rows * (unsigned)p.n_q_heads, 1, 1);
+  const long long grid = (long long)p.max_total_rows * p.n_q_heads;
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
   cfg.blockDim = dim3(kMergeThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
@@ -618,7 +618,13 @@ int launch_merge_d(const LseKernelParams &p, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return (int)cudaLaunchKernelEx(&cfg, merge_kernel<D>, p);
+  // With no more (row, head) CTAs than the partial pass had SMs, each CTA has
+  // an SM to itself and merges up to 2 x SMs partials: it keeps 16 loads in
+  // flight per lane (the round trips set its time).  Otherwise 8, which
+  // leaves room for more resident CTAs.
+  if (D <= 128 && p.balanced && grid <= p.n_ctas)
+    return (int)cudaLaunchKernelEx(&cfg, merge_kernel<D, 16>, p);
+  return (int)cudaLaunchKernelEx(&cfg, merge_kernel<D, 8>, p);
 }
 
 int lse_launch_merge(const LseKernelParams &p, int head_dim, void *stream) {
