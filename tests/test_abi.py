@@ -183,3 +183,48 @@ def test_per_vector_scales_only_for_8_bit_arenas():
     with pytest.raises(b.LseError, match="8-bit"):
         b.lse_kv_arena_set_scales(a, FAKE, 1 << 20)
     b.lse_kv_arena_destroy(a)
+
+
+def test_scaled_arena_bytes_per_token_match_the_readme_table():
+    # the README's table: fp8/bf8 "with scales" take 33,280 bytes per token
+    # for 16 KV layers of four kv heads of 256 dims (K and V).  The library's
+    # layout: T tokens of elements per fragment plus the smallest scale array
+    # it accepts (one FP32 per token and kv head of each fragment)
+    import os
+    rows = [ln.split() for ln in open(os.path.join(os.path.dirname(__file__), "golden",
+                                                   "kv_bytes_per_token.txt"))
+            if ln.strip() and not ln.startswith("#")]
+    want = {r[1]: int(r[2]) for r in rows}
+    for dtype in ("e4m3", "e5m2"):
+        frag = 256 << 10
+        a = b.lse_kv_arena_create([FAKE], 4 * frag, frag, dtype, 4, 256)
+        info = b.lse_kv_arena_query(a)
+        T, n_frag = info["tokens_per_fragment"], info["n_fragments"]
+        need = None
+        for n in range(n_frag * 4 * T - 2, n_frag * 4 * T + 2):
+            try:
+                b.lse_kv_arena_set_scales(a, FAKE, n)
+                need = n
+                break
+            except b.LseError:
+                pass
+        assert need is not None
+        per_token_one_tensor = (frag + need * 4 // n_frag) / T
+        assert 16 * 2 * per_token_one_tensor == want[dtype]
+        b.lse_kv_arena_destroy(a)
+
+
+def test_append_argument_checks_without_launching():
+    a = b.lse_kv_arena_create([FAKE], 1 << 20, 256 << 10, "e4m3", 4, 128)
+    F = FAKE
+    with pytest.raises(b.LseError, match="NULL"):
+        b.lse_kv_append(a, 1, 4, F, F, 0, F, F, F, 3)
+    with pytest.raises(b.LseError, match="n_seqs"):
+        b.lse_kv_append(a, 0, 4, F, F, F, F, F, F, 3)
+    b.lse_kv_append(a, 1, 4, 0, 0, F, F, F, F, 0)   # nothing to write: no launch, ok
+    # a scaled arena that grew past its scale array is refused before launch
+    b.lse_kv_arena_set_scales(a, F, 4 * 4 * 512)
+    b.lse_kv_arena_add_chunk(a, F * 2)
+    with pytest.raises(b.LseError, match="grew"):
+        b.lse_kv_append(a, 1, 4, F, F, F, F, F, F, 3)
+    b.lse_kv_arena_destroy(a)
