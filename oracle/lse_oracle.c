@@ -25,7 +25,11 @@
  *    "Long-context split attention".  The R query rows are the last R
  *    positions of the sequence; every row sees the whole cached context and,
  *    among the draft positions, the ones set in its ancestor mask (the chain
- *    default is "itself and all earlier drafts").
+ *    default is "itself and all earlier drafts").  Without masks the rows
+ *    may be any number (a prefill block: row r sees positions up to its
+ *    own, the causal rule of the long-query paged attention of LSE
+ *    releases, v0.4.14 "Improvements", whose kernel skips 256-key windows
+ *    that no row of a block sees); masks (tree rows) are 64 bits, so R <= 64.
  *  - Split attention with one partial family and one merge family, the
  *    partition count taken from page-table capacity, empty partitions
  *    skipped: LSE releases, v0.4.19 and v0.4.20.  The merge is the
@@ -280,8 +284,12 @@ static uint64_t row_mask(const orc_problem *pb, int s, int r) {
   return (r >= 63) ? ~(uint64_t)0 : (((uint64_t)1 << (r + 1)) - 1);
 }
 
-static int visible(int64_t j, int64_t C, uint64_t mask) {
+/* Key j visible to row r (C context keys): the context always; among the
+ * drafts, the bits of the row's mask, or without masks the chain (drafts up
+ * to the row itself, for any number of rows). */
+static int visible(const orc_problem *pb, int64_t j, int64_t C, int r, uint64_t mask) {
   if (j < C) return 1;
+  if (!pb->row_masks) return j - C <= r;
   return (int)((mask >> (j - C)) & 1u);
 }
 
@@ -302,9 +310,10 @@ static int check_problem(const orc_problem *pb) {
   for (int s = 0; s < pb->n_seqs; ++s) {
     int64_t L = pb->seq_lens[s];
     int R = pb->row_offsets[s + 1] - pb->row_offsets[s];
-    if (R < 0 || R > 64 || L < R || L > (int64_t)pb->max_pages * T) return ORC_BAD_SHAPE;
+    if (R < 0 || (pb->row_masks && R > 64) || L < R || L > (int64_t)pb->max_pages * T)
+      return ORC_BAD_SHAPE;
     if (R > 0 && L < 1) return ORC_BAD_SHAPE;
-    for (int r = 0; r < R; ++r) {
+    for (int r = 0; pb->row_masks && r < R; ++r) {
       uint64_t m = row_mask(pb, s, r);
       if (!((m >> r) & 1u)) return ORC_BAD_MASK;                 /* sees itself */
       if (r < 63 && (m >> (r + 1)) != 0) return ORC_BAD_MASK;    /* no later draft */
@@ -327,14 +336,14 @@ static int attend_range(const orc_problem *pb, int s, int r, int h, int64_t key_
   const int64_t L = pb->seq_lens[s];
   const int R = pb->row_offsets[s + 1] - pb->row_offsets[s];
   const int64_t C = L - R;
-  const uint64_t mask = row_mask(pb, s, r);
+  const uint64_t mask = pb->row_masks ? row_mask(pb, s, r) : 0;
   const float *q = pb->q + ((int64_t)(pb->row_offsets[s] + r) * pb->n_q_heads + h) * D;
   const int es = elem_size(pb->dtype);
 
   /* pass 1: the maximum score */
   double m = -INFINITY;
   for (int64_t j = key_begin; j < key_end; ++j) {
-    if (!visible(j, C, mask)) continue;
+    if (!visible(pb, j, C, r, mask)) continue;
     const uint8_t *k = kv_row(pb, pb->k_pages, s, j, g, &status);
     const double sk = vec_scale(pb, pb->k_pages, s, j, g, &status);
     if (status) return status;
@@ -351,7 +360,7 @@ static int attend_range(const orc_problem *pb, int s, int r, int h, int64_t key_
   /* pass 2: weights, their sum and the weighted sum of V */
   double l = 0.0;
   for (int64_t j = key_begin; j < key_end; ++j) {
-    if (!visible(j, C, mask)) continue;
+    if (!visible(pb, j, C, r, mask)) continue;
     const uint8_t *k = kv_row(pb, pb->k_pages, s, j, g, &status);
     const uint8_t *v = kv_row(pb, pb->v_pages, s, j, g, &status);
     const double sk = vec_scale(pb, pb->k_pages, s, j, g, &status);

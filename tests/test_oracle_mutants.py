@@ -58,6 +58,8 @@ MUTANTS = {
                                 "int64_t at = ((int64_t)frag * T + j % T) * pb->n_kv_heads + g;"),
     "v_scale_through_k_table": ("vec_scale(pb, pb->v_pages", "vec_scale(pb, pb->k_pages"),
     "v_scale_in_denominator": ("    l += p;\n", "    l += p * sv;\n"),
+    "long_chain_excludes_itself": ("if (!pb->row_masks) return j - C <= r;",
+                                   "if (!pb->row_masks) return j - C < r;"),
     "append_not_divided_by_scale": ("const float q = scales ? x[d] / sc : x[d];",
                                     "const float q = x[d];"),
     "append_scale_formats_swapped": ("dtype == ORC_E4M3 ? 448.0f : 57344.0f",

@@ -311,3 +311,35 @@ def test_rejects_bad_input():
         orc.attention(to_problem(w, row_masks=np.array([2, 3], np.uint64)))
     with pytest.raises(orc.OracleError, match="bad mask"):   # row 0 may not see row 1
         orc.attention(to_problem(w, row_masks=np.array([3, 3], np.uint64)))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "e4m3"])
+def test_long_query_block_matches_library_sdpa(dtype):
+    # a prefill-style block of more than 64 chained rows (no masks): row r
+    # sees the context and positions up to its own
+    w = wl.small_case(dtype, [300, 90], [150, 70], n_q_heads=4, n_kv_heads=2, head_dim=16,
+                      tokens_per_fragment=16, seed=21)
+    assert w.row_masks is None and w.max_rows > 64
+    out, lse = orc.attention(to_problem(w))
+    assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
+    np.testing.assert_allclose(out, sdpa_reference(w), rtol=1e-12, atol=1e-13)
+
+
+def test_long_query_block_in_256_key_windows_equals_unsplit():
+    # cutting the keys into 256-key windows (the windows past a row's own
+    # position are empty for it and drop out of the merge) changes nothing
+    w = wl.small_case("bf16", [700, 300], [200, 100], n_q_heads=4, n_kv_heads=2, head_dim=16,
+                      tokens_per_fragment=16, seed=22)
+    a = orc.attention(to_problem(w))
+    for kp in (256, 64):
+        b_ = orc.attention_split(to_problem(w), kp)
+        np.testing.assert_allclose(b_[0], a[0], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(b_[1], a[1], rtol=1e-12, atol=1e-13)
+
+
+def test_masked_rows_stay_limited_to_64():
+    w = wl.small_case("bf16", [100], [70], n_q_heads=2, n_kv_heads=1, head_dim=8,
+                      tokens_per_fragment=16, seed=23)
+    masks = np.array([(1 << min(r + 1, 64)) - 1 for r in range(70)], dtype=np.uint64)
+    with pytest.raises(orc.OracleError):
+        orc.attention(to_problem(w, row_masks=masks))
