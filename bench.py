@@ -467,8 +467,9 @@ def run_append(args, world, rank, local):
         at += 2 * pages[s_]
     dev = lambda a: torch.from_numpy(a).cuda()  # noqa: E731
     total = n_seqs * new
-    k_new = torch.randn((total, hkv, d), device="cuda")
-    v_new = torch.randn((total, hkv, d), device="cuda")
+    gen = torch.Generator().manual_seed(1240)   # seeded on the host, then uploaded
+    k_new = torch.randn((total, hkv, d), generator=gen).cuda()
+    v_new = torch.randn((total, hkv, d), generator=gen).cuda()
     offs = dev(np.arange(0, total + 1, new, dtype=np.int32))
     kp_d, vp_d, before_d = dev(kp), dev(vp), dev(before)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
