@@ -18,6 +18,7 @@
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cfloat>
 #include <climits>
 #include <cstdint>
@@ -532,15 +533,37 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
         wt > 0.f ? (M + log2f(wt)) * 0.69314718055994530942f : -INFINITY;
 }
 
+// Largest dynamic shared memory already allowed for one kernel, per device
+// ordinal (the attribute is per device).  Zero-initialised static storage;
+// threads may race to raise it, which is harmless.
+constexpr int kMaxDevices = 64;
+struct SmemAllowed {
+  std::atomic<int> bytes[kMaxDevices];
+};
+
+template <class K>
+int allow_dynamic_smem(K kernel, int smem, SmemAllowed &allowed) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return (int)e;
+  const bool cached = dev >= 0 && dev < kMaxDevices;
+  if (cached && allowed.bytes[dev].load(std::memory_order_relaxed) >= smem) return 0;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return (int)e;
+  if (cached) {
+    int cur = allowed.bytes[dev].load(std::memory_order_relaxed);
+    while (cur < smem && !allowed.bytes[dev].compare_exchange_weak(cur, smem)) {
+    }
+  }
+  return 0;
+}
+
 template <int DT, int D>
 int launch_cc(const LseKernelParams &p, int gx, int gy, int gz, int smem, cudaStream_t st) {
   auto k = partial_cuda_core_kernel<DT, D>;
-  static int set_for = -1;
-  if (smem > set_for) {
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return (int)e;
-    set_for = smem;
-  }
+  static SmemAllowed allowed;
+  const int e = allow_dynamic_smem(k, smem, allowed);
+  if (e) return e;
   k<<<dim3(gx, gy, gz), kThreads, smem, st>>>(p);
   return (int)cudaGetLastError();
 }
