@@ -138,3 +138,14 @@ def test_scale_array_must_cover_the_arena():
     w = scaled_case("e5m2", seed=66)
     with pytest.raises(orc.OracleError):
         orc.attention(to_problem(with_scales(w, w.scales[:-1])))
+
+
+def test_scaled_contiguous_cache_is_bitwise_equal():
+    # relaying the fragments (and their scale blocks) into identity tables
+    # leaves the scaled problem unchanged, bit for bit
+    w = scaled_case("e5m2", seed=67)
+    c = wl.contiguous_copy(w)
+    a = orc.attention(to_problem(w))
+    b = orc.attention(to_problem(c))
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    assert np.isnan(c.scales).sum() == np.isnan(w.scales).sum()
