@@ -228,3 +228,34 @@ def test_append_argument_checks_without_launching():
     with pytest.raises(b.LseError, match="grew"):
         b.lse_kv_append(a, 1, 4, F, F, F, F, F, F, 3)
     b.lse_kv_arena_destroy(a)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "e4m3", "e5m2"])
+@pytest.mark.parametrize("scaled", [False, True])
+def test_planner_sweep_stays_within_device_limits(dtype, scaled):
+    # every (group size, rows) the tensor-core kernel takes: a plan that fits
+    # the B200's shared memory, a ring of 2-6 stages, row chunks of at most
+    # 48 pairs; scaled plans only for the 8-bit formats
+    if scaled and dtype in ("f16", "bf16"):
+        pytest.skip("scales go with the 8-bit formats")
+    esize = 1 if dtype.startswith("e") else 2
+    for T in (8, 16, 64, 128, 512):
+        frag = T * 4 * 128 * esize
+        a = b.lse_kv_arena_create([FAKE], frag * 8, frag, dtype, 4, 128)
+        if scaled:
+            b.lse_kv_arena_set_scales(a, FAKE, 8 * 4 * T)
+        for hq in (4, 8, 24, 48):
+            G = hq // 4
+            for rows in (1, 2, 3, 4, 5, 8, 9, 16, 33, 64):
+                p, _ = b.lse_attn_plan_ex(a, 2, rows, 2 * rows, hq, 16, **B200)
+                info = b.lse_attn_plan_query(p)
+                assert info["kernel_name"] == "tcgen05", (dtype, T, hq, rows)
+                assert info["smem_bytes"] <= B200["smem_optin"]
+                assert 2 <= info["stages"] <= 6 and info["q_slots"] in (1, 2)
+                assert info["scaled"] == int(scaled)
+                rc = info["rows_per_chunk"]
+                assert 1 <= rc <= rows and G * rc <= max(48, G)
+                if G * rows <= 48:
+                    assert rc == rows
+                b.lse_attn_plan_destroy(p)
+        b.lse_kv_arena_destroy(a)
