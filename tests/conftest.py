@@ -11,6 +11,10 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+    # temporary files (the oracle variants the tests compile) stay inside
+    # the repository, in a git-ignored folder
+    if not config.option.basetemp:
+        config.option.basetemp = os.path.join(ROOT, ".pytest_tmp")
 
 
 def to_problem(w, q=None, row_masks="keep", chunks=None, k_pages=None, v_pages=None):
