@@ -191,9 +191,8 @@ def test_scaled_arena_bytes_per_token_match_the_readme_table():
     # layout: T tokens of elements per fragment plus the smallest scale array
     # it accepts (one FP32 per token and kv head of each fragment)
     import os
-    rows = [ln.split() for ln in open(os.path.join(os.path.dirname(__file__), "golden",
-                                                   "kv_bytes_per_token.txt"))
-            if ln.strip() and not ln.startswith("#")]
+    with open(os.path.join(os.path.dirname(__file__), "golden", "kv_bytes_per_token.txt")) as f:
+        rows = [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
     want = {r[1]: int(r[2]) for r in rows}
     for dtype in ("e4m3", "e5m2"):
         frag = 256 << 10

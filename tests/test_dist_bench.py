@@ -30,7 +30,7 @@ def _rank(rank, world, port, times, out):
 @pytest.mark.parametrize("times", [(3.0, 5.0), (7.5, 2.5)])
 def test_replica_timing_takes_the_slowest_rank(times):
     world = 2
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.start_processes(_rank, args=(world, _free_port(), times, out), nprocs=world,
                            start_method="spawn")

@@ -68,7 +68,8 @@ MUTANTS = {
 
 
 def _build_mutant(tmp_path, name, old, new):
-    src = open(SRC).read()
+    with open(SRC) as f:
+        src = f.read()
     assert src.count(old) >= 1, name
     mutated = src.replace(old, new)
     c = tmp_path / f"{name}.c"

@@ -291,8 +291,8 @@ def test_codec_fp32_roundtrip():
 
 
 def test_kv_bytes_per_token_matches_readme_table():
-    rows = [l.split() for l in open(os.path.join(GOLDEN, "kv_bytes_per_token.txt"))
-            if l.strip() and not l.startswith("#")]
+    with open(os.path.join(GOLDEN, "kv_bytes_per_token.txt")) as f:
+        rows = [l.split() for l in f if l.strip() and not l.startswith("#")]
     assert len(rows) == 5
     for fmt, dt, want, scales in rows:
         assert orc.kv_bytes_per_token(dt, 16, 4, 256, bool(int(scales))) == int(want), fmt

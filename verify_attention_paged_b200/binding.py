@@ -106,7 +106,8 @@ class LseError(RuntimeError):
 
 def declared_symbols() -> list[str]:
     """Entry points declared in include/lse_attn.h."""
-    text = open(HEADER_PATH).read()
+    with open(HEADER_PATH) as f:
+        text = f.read()
     return sorted(set(re.findall(r"^LSE_API\s+[\w\s\*]*?\b(lse_\w+)\(", text, flags=re.M)))
 
 
