@@ -3,15 +3,19 @@
 
 One step = one pass of the whole hot path over one batch: the partial pass
 (lse_attn_run) and the merge pass (lse_attn_merge) through the C ABI, on
-resident inputs.  The default workload is the batched BF16 decode
-(8 sequences, lengths uniform in [1024, 16384], 24 query / 4 kv heads,
-head_dim 128, 256 KiB fragments).  L2 is flushed (a 256 MiB write) before
-every timed step, outside the step's CUDA-event interval.
+resident inputs.  By default every one of the five workloads is timed in
+turn (tiny FP32 decode, batched BF16 decode, BF16 chain verify, long-context
+FP8, mixed FP16 tree-verify batch); the line's headline ``value``, roofline,
+end-to-end and CPU-baseline figures are those of the largest, the
+tree-verify batch, and ``per_workload`` holds each workload's own figures.
+L2 is flushed (a 256 MiB write) before every timed step, outside the step's
+CUDA-event interval.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload all|NAME]
                   [--impl ours|reference]
 
---workload append times the K/V append kernel instead (see run_append).
+--workload append times the K/V append kernel instead (see run_append);
+--workload fragment_ab the fragment-addressing comparison.
 
 Prints one JSON line.  ``value`` is effective GB/s: (K + V + Q + out bytes of
 every call on every rank) / (max over ranks of the summed step times).
@@ -42,9 +46,10 @@ FLUSH_BYTES = 256 << 20
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--workload", default="batched_decode")
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="all",
+                    help="all (the five configurations) or one workload name")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -110,8 +115,16 @@ class ClockSampler:
             pass
         self._stop = threading.Event()
 
+    def active(self, on):
+        """Sample only while a timed loop runs (between workloads the box
+        is building inputs on the host)."""
+        self._on = on
+
     def _loop(self):
         while not self._stop.is_set():
+            if not getattr(self, "_on", True):
+                time.sleep(0.002)
+                continue
             try:
                 self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
                 r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
@@ -271,32 +284,23 @@ def workload_config(w):
             "timing": "CUDA events around a CUDA-graph replay of each step"}
 
 
-def run_ours(args, w, world, rank, local):
+HEADLINE = "tree_verify"   # the largest single-GPU workload carries the headline
+
+
+def time_workload(w, args, flush, dist, clk):
+    """Device times of one workload: `args.steps` graph replays of the whole
+    step (partial pass, then the merge as its programmatic dependent) and
+    as many of the partial pass alone, L2 flushed before each outside the
+    CUDA-event interval.  Returns the DeviceCall (kept for the end-to-end
+    leg) and the per-step millisecond lists."""
     import torch
-    torch.cuda.set_device(local)
-    dist = None
-    if world > 1:
-        import torch.distributed as dist
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
     from verify_attention_paged_b200 import binding as b
-
     call = b.DeviceCall(w)
-    stream = call.stream
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
-    bytes_call = w.call_bytes()
-    bytes_partial = w.kv_bytes() + w.total_rows * w.n_q_heads * w.head_dim * 4
-
     for _ in range(args.warmup):
         flush.fill_(1)
         call.run()
     torch.cuda.synchronize()
-    assert call.device_error() == 0, "device error during warm-up"
-
-    # the step (partial pass, then the merge as its programmatic dependent) is
-    # captured once into a CUDA graph, so the timed region holds device time
-    # only; the partial pass alone is captured too, for its roofline
+    assert call.device_error() == 0, f"{w.name}: device error during warm-up"
     g_step, g_part = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
     saved = call.stream
     with torch.cuda.graph(g_step):
@@ -313,72 +317,126 @@ def run_ours(args, w, world, rank, local):
         flush.fill_(3)
         g_part.replay()
     torch.cuda.synchronize()
-
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     evp = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        for i in range(args.steps):
-            flush.fill_(i & 0xff)                  # L2 flush, outside the interval
-            ev[i][0].record()
-            g_step.replay()
-            ev[i][1].record()
-        torch.cuda.synchronize()
+    clk.active(True)
+    for i in range(args.steps):
+        flush.fill_(i & 0xff)                  # L2 flush, outside the interval
+        ev[i][0].record()
+        g_step.replay()
+        ev[i][1].record()
+    torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    for i in range(args.steps):                    # the partial pass alone
+    for i in range(args.steps):                # the partial pass alone
         flush.fill_(i & 0xff)
         evp[i][0].record()
         g_part.replay()
         evp[i][1].record()
     torch.cuda.synchronize()
-    assert call.device_error() == 0, "device error during the timed steps"
+    clk.active(False)
+    assert call.device_error() == 0, f"{w.name}: device error during the timed steps"
     steps_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    part = [e[0].elapsed_time(e[1]) for e in evp]
+    part_ms = [e[0].elapsed_time(e[1]) for e in evp]
+    del g_step, g_part
+    return call, steps_ms, part_ms
+
+
+def workload_result(w, call, steps_ms, part_ms, world, dist, args, peak, peak_kind):
+    """One workload's figures: us per call, whole-job GB/s, and the roofline
+    of the partial pass (its algorithmic K + V + Q bytes over its
+    CUDA-event time, against the measured copy bandwidth)."""
     total_ms = reduce_max(sum(steps_ms), dist, "cuda")
+    part_mean = reduce_max(statistics.mean(part_ms), dist, "cuda")
+    bytes_call = w.call_bytes()
+    bytes_partial = w.kv_bytes() + w.total_rows * w.n_q_heads * w.head_dim * 4
+    achieved = bytes_partial / (part_mean * 1e-3) / 1e9
+    value = job_gbs(world, bytes_call, args.steps, total_ms)
+    info = call.info
+    bound = "hbm"
+    if bytes_call < 4 << 20:
+        # a quarter of a megabyte moves in well under a microsecond at HBM
+        # speed: launch and dependent-load latency set the time
+        bound = "launch"
+    return {
+        "value": value, "unit": "GB/s", "us_per_call": total_ms / args.steps * 1e3,
+        "us_per_call_median": statistics.median(steps_ms) * 1e3,
+        "partial_us_mean": part_mean * 1e3,
+        "merge_us_est": (total_ms / args.steps - part_mean) * 1e3,
+        "pct_of_8tbs": value / world / 8000.0 * 100.0,
+        "pct_of_measured_hbm": value / world / peak * 100.0,
+        "bytes_per_call": bytes_call,
+        "kernel": info["kernel_name"], "n_splits": info["n_splits"],
+        "dtype": compute_dtype(w.dtype, info["kernel"]),
+        "roofline": {"bound": bound, "kernel": "partial", "achieved": achieved, "peak": peak,
+                     "peak_kind": f"{peak_kind} (copy, burst)", "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": ncu_traffic(w.name),
+                     "algorithmic_bytes_per_launch": bytes_partial},
+    }
+
+
+def run_ours(args, names, world, rank, local):
+    import torch
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    from verify_attention_paged_b200 import workloads as wl
+
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    peak, peak_kind = measured_peaks()
+    head = HEADLINE if HEADLINE in names else names[0]
+    results, head_w, head_call = {}, None, None
+    clk = ClockSampler(local)
+    with clk:
+        for name in names:
+            w = wl.BUILDERS[name]()
+            call, steps_ms, part_ms = time_workload(w, args, flush, dist, clk)
+            results[name] = workload_result(w, call, steps_ms, part_ms, world, dist, args,
+                                            peak, peak_kind)
+            if name == head:
+                head_w, head_call = w, call
+            else:
+                call.close()
+                del call, w
+                torch.cuda.empty_cache()
 
     # end to end: pinned host inputs -> device -> run -> result back to host
     e2e = None
     if not args.no_e2e:
-        e2e = measure_e2e(call, w, args, stream, flush, dist)
+        e2e = measure_e2e(head_call, head_w, args, head_call.stream, flush, dist)
 
     if rank != 0:
         if dist:
             dist.destroy_process_group()
         return
-    peak, peak_kind = measured_peaks()
-    part_ms = statistics.mean(part)
-    achieved = bytes_partial / (part_ms * 1e-3) / 1e9
-    value = job_gbs(world, bytes_call, args.steps, total_ms)
-    info = call.info
+    r = results[head]
     line = {
-        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
-        "us_per_call": total_ms / args.steps * 1e3,
-        "us_per_call_median": statistics.median(steps_ms) * 1e3,
-        "partial_us_mean": part_ms * 1e3,
-        "merge_us_est": (total_ms / args.steps - part_ms) * 1e3,
-        "pct_of_8tbs": value / world / 8000.0 * 100.0,
-        "pct_of_measured_hbm": value / world / peak * 100.0,
+        "metric": METRIC, "value": r["value"], "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": r["us_per_call"] / 1e3,
+        "us_per_call": r["us_per_call"], "us_per_call_median": r["us_per_call_median"],
+        "partial_us_mean": r["partial_us_mean"], "merge_us_est": r["merge_us_est"],
+        "pct_of_8tbs": r["pct_of_8tbs"], "pct_of_measured_hbm": r["pct_of_measured_hbm"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": compute_dtype(w.dtype, info["kernel"]),
-        "data": "synthetic", "config": {**workload_config(w), "parallelism": f"replicas{world}",
-                                        "kernel": info["kernel_name"],
-                                        "n_splits": info["n_splits"],
-                                        "keys_per_split": info["keys_per_split"]},
-        "roofline": {"bound": "hbm", "kernel": "partial", "achieved": achieved, "peak": peak,
-                     "peak_kind": f"{peak_kind} (copy, burst)", "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": ncu_traffic(w.name),
-                     "algorithmic_bytes_per_launch": bytes_partial},
-        "gpu_launches": 2 * args.steps,
+        "dtype": r["dtype"], "data": "synthetic",
+        "config": {**workload_config(head_w), "parallelism": f"replicas{world}",
+                   "kernel": r["kernel"], "n_splits": r["n_splits"]},
+        "roofline": r["roofline"],
+        "per_workload": {n: {k: v for k, v in res.items()} for n, res in results.items()},
+        "gpu_launches": 4 * args.steps * len(names),
         "clocks": clk.summary(),
     }
     if e2e:
         line["e2e"] = e2e
     if world == 1:
-        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(head_w, args.cpu_seconds)
     print(json.dumps(line), flush=True)
     if dist:
         dist.destroy_process_group()
@@ -635,11 +693,12 @@ def main():
         run_append(args, world, rank, local)
         return
     from verify_attention_paged_b200 import workloads as wl
-    w = wl.BUILDERS[args.workload]()
+    names = list(wl.NAMES) if args.workload == "all" else [args.workload]
     if args.impl == "reference":
-        run_reference(args, w, world, rank)
+        head = HEADLINE if HEADLINE in names else names[0]
+        run_reference(args, wl.BUILDERS[head](), world, rank)
     else:
-        run_ours(args, w, world, rank, local)
+        run_ours(args, names, world, rank, local)
 
 
 if __name__ == "__main__":

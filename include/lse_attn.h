@@ -48,7 +48,10 @@
  *   library and released by their destroy calls.  Device pointers are passed
  *   as plain pointers; every launch goes to the caller's cudaStream_t (passed
  *   as void*; NULL = legacy default stream).  No call synchronises except
- *   lse_attn_read_error.  A plan may be used from one thread at a time.
+ *   the read-error calls.  Several host threads may run and merge with one
+ *   plan at the same time (each with its own workspace); a call that
+ *   changes an arena (alloc, free, add_chunk, set_scales) must not overlap a
+ *   call that reads it (planning, run, merge, append).
  *
  * Errors
  *   Every call returns LSE_OK (0) or an lse_status code.  When err is not
@@ -101,7 +104,8 @@ typedef enum {
 #define LSE_DEVERR_BAD_LENGTH 0x2u   /* L_s > capacity, R_s > L_s, R_s > max rows or rows past max_total_rows */
 
 #define LSE_MAX_CHUNKS 64     /* arena chunks a kernel can address          */
-#define LSE_MAX_TMA_CHUNKS 16 /* chunks the tensor-core kernel can address; more -> CUDA cores */
+#define LSE_MAX_TMA_CHUNKS 64 /* chunks the tensor-core kernel can address (every chunk
+                                 an arena can have: one TMA descriptor per chunk) */
 #define LSE_MAX_ROWS_PER_SEQ 64
 
 typedef struct lse_kv_arena lse_kv_arena;
@@ -345,8 +349,8 @@ LSE_API int lse_kv_append(const lse_kv_arena *arena, int n_seqs, int max_pages,
  * No-allocation variant (the pages have no counterpart: it exists for
  * callers that cannot allocate device memory when attention runs, such as
  * plugin or custom-op hosts that hand a kernel only its inputs and outputs,
- * serving loops that forbid allocation after warm-up, and code running under
- * CUDA-graph stream capture, where a synchronising allocation is illegal).
+ * and serving loops whose device memory is fixed at start-up, so that no
+ * allocation may happen after warm-up).
  * Runs lse_attn_run then lse_attn_merge on `stream` with the workspace taken
  * from a static device array of LSE_STATIC_SCRATCH_BYTES that the library
  * holds on every GPU that loads it until the process exits.  Arguments as
@@ -362,6 +366,8 @@ LSE_API int lse_kv_append(const lse_kv_arena *arena, int n_seqs, int max_pages,
  *     device error word is cleared at the start of each call.  Calls whose
  *     GPU work overlaps (other streams, other threads) race on the array:
  *     serialise them.
+ *   - The device error word of the latest call (bad fragment id, bad
+ *     length, pipeline timeout) is read with lse_attn_static_read_error.
  * ------------------------------------------------------------------------- */
 #define LSE_STATIC_SCRATCH_BYTES (32u << 20)
 
@@ -370,6 +376,13 @@ LSE_API int lse_attn_forward_static(const lse_attn_plan_t *plan, const float *q,
                                     const int32_t *seq_lens, const int32_t *row_offsets,
                                     const uint64_t *row_masks, float softmax_scale, float *out,
                                     float *lse_out, void *stream, char **err);
+
+/* Read (and clear) the device error word of the static scratch on the
+ * current device: the LSE_DEVERR_* bits the latest lse_attn_forward_static
+ * call on this device left (0 when clean).  Synchronises the stream.  Like
+ * the static call itself it allocates nothing; the first use on a device
+ * looks the scratch address up.  No counterpart on the pages. */
+LSE_API int lse_attn_static_read_error(void *stream, uint32_t *device_error, char **err);
 
 /* Release a string returned through an err argument. */
 LSE_API void lse_free(void *p);

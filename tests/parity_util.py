@@ -1,4 +1,8 @@
-"""Shared parity helpers: tolerances and comparison against the oracle."""
+"""Shared parity helpers: tolerances, comparison against the oracle, and
+the oracle over every output of a large problem on all host cores."""
+import os
+import threading
+
 import numpy as np
 
 # Per-element tolerance, written out: FP32 K/V -> max |gpu - oracle| <= 1e-5;
@@ -27,3 +31,49 @@ def assert_close(got, want, dtype, what="out"):
 
 def lse_tol(dtype):
     return FP32_ABS if dtype == "f32" else LOWP_TOL
+
+
+def oracle_all_outputs(pb, threads=None):
+    """Every (row, head) output of a problem from the float64 oracle, one
+    output per call on one thread per host core (the ctypes calls release
+    the GIL).  Same result as oracle.attention(pb), computed in parallel."""
+    from oracle import oracle as orc
+    m = orc.marshal(pb)
+    ro = np.asarray(pb.row_offsets)
+    rows = int(ro[-1])
+    hq, d = pb.n_q_heads, pb.head_dim
+    out = np.zeros((rows, hq, d), np.float64)
+    lse = np.zeros((rows, hq), np.float64)
+    items = [(s, r, h) for s in range(len(ro) - 1) for r in range(int(ro[s + 1] - ro[s]))
+             for h in range(hq)]
+    # the longest sequences first, so the threads finish together
+    lens = np.asarray(pb.seq_lens)
+    items.sort(key=lambda t: -int(lens[t[0]]))
+    lock = threading.Lock()
+    state = {"next": 0, "error": None}
+
+    def worker():
+        while True:
+            with lock:
+                if state["next"] >= len(items) or state["error"] is not None:
+                    return
+                s, r, h = items[state["next"]]
+                state["next"] += 1
+            try:
+                o, l = orc.attention_one(pb, s, r, h, marshalled=m)
+            except Exception as e:  # surfaced below, on the caller's thread
+                with lock:
+                    state["error"] = e
+                return
+            out[ro[s] + r, h] = o
+            lse[ro[s] + r, h] = l
+
+    n = threads or os.cpu_count() or 1
+    pool = [threading.Thread(target=worker) for _ in range(n)]
+    for t in pool:
+        t.start()
+    for t in pool:
+        t.join()
+    if state["error"] is not None:
+        raise state["error"]
+    return out, lse

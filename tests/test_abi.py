@@ -229,14 +229,12 @@ def test_append_argument_checks_without_launching():
     b.lse_kv_arena_destroy(a)
 
 
-@pytest.mark.parametrize("dtype", ["f16", "bf16", "e4m3", "e5m2"])
-@pytest.mark.parametrize("scaled", [False, True])
+@pytest.mark.parametrize("dtype,scaled", [("f16", False), ("bf16", False), ("e4m3", False),
+                                          ("e5m2", False), ("e4m3", True), ("e5m2", True)])
 def test_planner_sweep_stays_within_device_limits(dtype, scaled):
     # every (group size, rows) the tensor-core kernel takes: a plan that fits
     # the B200's shared memory, a ring of 2-6 stages, row chunks of at most
     # 48 pairs; scaled plans only for the 8-bit formats
-    if scaled and dtype in ("f16", "bf16"):
-        pytest.skip("scales go with the 8-bit formats")
     esize = 1 if dtype.startswith("e") else 2
     for T in (8, 16, 64, 128, 512):
         frag = T * 4 * 128 * esize
@@ -258,3 +256,28 @@ def test_planner_sweep_stays_within_device_limits(dtype, scaled):
                     assert rc == rows
                 b.lse_attn_plan_destroy(p)
         b.lse_kv_arena_destroy(a)
+
+
+@pytest.mark.parametrize("n_chunks", [1, 16, 17, 64])
+def test_tensor_core_plan_for_arenas_of_any_chunk_count(n_chunks):
+    # every chunk an arena can have gets its TMA descriptor: the planner
+    # keeps the tensor-core kernel however many chunks there are, and an
+    # arena grown after planning stays within the kernel's reach
+    frag = 256 << 10
+    a = b.lse_kv_arena_create([FAKE * (i + 1) for i in range(n_chunks)], frag * 4, frag,
+                              "bf16", 4, 128)
+    p, _ = b.lse_attn_plan_ex(a, 8, 1, 8, 24, 64, **B200, allow_tcgen05=1)
+    assert b.lse_attn_plan_query(p)["kernel_name"] == "tcgen05"
+    while b.lse_kv_arena_query(a)["n_chunks"] < 64:
+        b.lse_kv_arena_add_chunk(a, FAKE * 100)
+    with pytest.raises(b.LseError, match="64 chunks"):
+        b.lse_kv_arena_add_chunk(a, FAKE * 100)
+    b.lse_attn_plan_destroy(p)
+    b.lse_kv_arena_destroy(a)
+
+
+def test_tma_chunk_limit_is_every_chunk_an_arena_can_have():
+    text = open(b.HEADER_PATH).read()
+    import re
+    lim = {k: int(v) for k, v in re.findall(r"#define (LSE_MAX_\w*CHUNKS) (\d+)", text)}
+    assert lim["LSE_MAX_TMA_CHUNKS"] == lim["LSE_MAX_CHUNKS"]

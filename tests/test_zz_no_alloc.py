@@ -53,6 +53,8 @@ def test_static_matches_regular_entry_points_twice(binding, case):
         lse = torch.full_like(call.lse, float("nan"))
         _static_call(binding, call, out, lse)
         torch.cuda.synchronize()
+        # the static call's device error word (bad page, bad length, timeout)
+        assert binding.lse_attn_static_read_error(call.stream) == 0
         got = out[:w.total_rows].cpu().numpy()
         assert_close(got, ref_out, w.dtype, what=f"static {case}")
         np.testing.assert_allclose(lse[:w.total_rows].cpu().numpy(), ref_lse, rtol=0,
@@ -73,3 +75,21 @@ def test_static_refuses_plans_beyond_its_scratch(binding):
                                         call.out, None, call.stream)
     binding.lse_attn_plan_destroy(plan)
     call.close()
+
+
+def test_static_error_word_reports_a_bad_page(binding):
+    # a page-table entry naming no fragment: the static call flags it in the
+    # scratch's error word, which the static read-error call returns and
+    # clears; the next clean call reads 0
+    w = wl.small_case("bf16", [600], [2], n_q_heads=8, n_kv_heads=2, head_dim=128,
+                      tokens_per_fragment=128, seed=305)
+    kp = w.k_pages.copy()
+    kp[0, 1] = 10 ** 6
+    bad = wl.Workload(**{**w.__dict__, "k_pages": kp})
+    for case, want in ((bad, binding.DEVERR_BAD_FRAGMENT), (w, 0)):
+        call = binding.DeviceCall(case)
+        _static_call(binding, call, call.out, call.lse)
+        got = binding.lse_attn_static_read_error(call.stream)
+        assert got == want, f"error word {got:#x}, expected {want:#x}"
+        assert binding.lse_attn_static_read_error(call.stream) == 0  # cleared
+        call.close()

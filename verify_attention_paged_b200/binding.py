@@ -95,6 +95,7 @@ _sig("lse_attn_read_error", _i, _vp, _vp, _vp, ctypes.POINTER(ctypes.c_uint32), 
 _sig("lse_attn_forward_static", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _vp,
      _vp, _errp)
 _sig("lse_kv_append", _i, _vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _errp)
+_sig("lse_attn_static_read_error", _i, _vp, ctypes.POINTER(ctypes.c_uint32), _errp)
 STATIC_SCRATCH_BYTES = 32 << 20
 
 
@@ -284,6 +285,14 @@ def lse_attn_forward_static(plan, q, k_pages, v_pages, seq_lens, row_offsets, ro
     _call(_lib.lse_attn_forward_static, plan, _ptr(q), _ptr(k_pages), _ptr(v_pages),
           _ptr(seq_lens), _ptr(row_offsets), _ptr(row_masks), float(softmax_scale), _ptr(out),
           _ptr(lse_out), _ptr(stream))
+
+
+def lse_attn_static_read_error(stream=0) -> int:
+    """Read and clear the device error word of the static scratch (the
+    latest lse_attn_forward_static call on the current device)."""
+    v = ctypes.c_uint32()
+    _call(_lib.lse_attn_static_read_error, _ptr(stream), ctypes.byref(v))
+    return v.value
 
 
 def lse_attn_read_error(plan, workspace, stream=0) -> int:

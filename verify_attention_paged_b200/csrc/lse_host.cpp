@@ -492,9 +492,10 @@ int lse_attn_run(const lse_attn_plan_t *pl, const float *q, const int32_t *k_pag
   if (pl->kernel == LSE_KERNEL_TCGEN05) {
     const lse_kv_arena *a = pl->arena;
     const int nch = int(a->chunk_base.size());
-    if (nch > LSE_MAX_TMA_CHUNKS)
+    if (nch > LSE_MAX_TMA_CHUNKS)  // (the arena itself holds at most this many)
       return fail(err, LSE_ERR_UNSUPPORTED, "arena has %d chunks; the tensor-core kernel "
                   "addresses at most %d", nch, LSE_MAX_TMA_CHUNKS);
+    std::lock_guard<std::mutex> lock(pl->maps_mutex);
     if (pl->maps_chunks != nch) {
       pl->maps.assign(lse_tc_map_bytes() * nch, 0);
       ce = lse_tc_build_maps(a->chunk_base.data(), nch, a->chunk_bytes, a->n_kv_heads,

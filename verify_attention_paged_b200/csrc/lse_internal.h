@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -54,9 +55,11 @@ struct lse_attn_plan_s {
   int rows_per_chunk = 0;  // tensor-core kernel: query rows per segment
   int box_tokens = 0;    // its TMA box height
   int scaled = 0;        // made for an arena with per-vector scales
-  // tensor maps of the arena chunks (built on first run, rebuilt on growth)
+  // tensor maps of the arena chunks (built on first run, rebuilt on growth);
+  // maps_mutex guards them, so threads may run one plan at the same time
   mutable std::vector<uint8_t> maps;
   mutable int maps_chunks = 0;
+  mutable std::mutex maps_mutex;
   size_t ws_bytes = 0;
   size_t ws_o_off = 0;   // partial outputs  FP32 [rows][Hq][n_splits][D]
   size_t ws_lse_off = 0; // partial lse (log2 units) FP32 [rows][Hq][n_splits]

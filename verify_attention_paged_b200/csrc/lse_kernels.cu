@@ -24,6 +24,7 @@
 #include <cstdint>
 
 #include "lse_internal.h"
+#include "lse_smem_attr.h"
 
 namespace {
 
@@ -533,30 +534,8 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
         wt > 0.f ? (M + log2f(wt)) * 0.69314718055994530942f : -INFINITY;
 }
 
-// Largest dynamic shared memory already allowed for one kernel, per device
-// ordinal (the attribute is per device).  Zero-initialised static storage;
-// threads may race to raise it, which is harmless.
-constexpr int kMaxDevices = 64;
-struct SmemAllowed {
-  std::atomic<int> bytes[kMaxDevices];
-};
-
-template <class K>
-int allow_dynamic_smem(K kernel, int smem, SmemAllowed &allowed) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return (int)e;
-  const bool cached = dev >= 0 && dev < kMaxDevices;
-  if (cached && allowed.bytes[dev].load(std::memory_order_relaxed) >= smem) return 0;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return (int)e;
-  if (cached) {
-    int cur = allowed.bytes[dev].load(std::memory_order_relaxed);
-    while (cur < smem && !allowed.bytes[dev].compare_exchange_weak(cur, smem)) {
-    }
-  }
-  return 0;
-}
+using lse_detail::SmemAllowed;
+using lse_detail::allow_dynamic_smem;
 
 template <int DT, int D>
 int launch_cc(const LseKernelParams &p, int gx, int gy, int gz, int smem, cudaStream_t st) {

@@ -4,9 +4,9 @@
 // Some callers cannot call cudaMalloc at the point where they run
 // attention: engines whose device memory is carved up once at start-up by
 // a host framework (plugin and custom-op hosts that hand a kernel only its
-// inputs and outputs), real-time serving loops that forbid allocation
-// after warm-up, and code that runs while a CUDA graph is being captured,
-// where a synchronising allocation is not allowed.  This entry point gives
+// inputs and outputs) and real-time serving loops whose device memory is
+// fixed at start-up, so that nothing may be allocated after warm-up.  This
+// entry point gives
 // them the whole call (lse_attn_run, then lse_attn_merge) with the
 // workspace taken from a file-scope __device__ array instead of caller
 // memory.  It allocates nothing.
@@ -91,4 +91,23 @@ extern "C" LSE_API int lse_attn_forward_static(
                     ws, stream, err);
   if (st) return st;
   return lse_attn_merge(plan, seq_lens, row_offsets, ws, out, lse_out, stream, err);
+}
+
+// The first 32-bit word of the scratch is the device error word of the
+// latest static call on this device (the passes OR their LSE_DEVERR_* bits
+// into it).  Read it, then clear it, in stream order.
+extern "C" LSE_API int lse_attn_static_read_error(void *stream, uint32_t *device_error,
+                                                  char **err) {
+  if (!device_error) return fail_msg(err, LSE_ERR_INVALID_ARG, "device_error is NULL");
+  void *ws = nullptr;
+  int st = scratch_address(&ws, err);
+  if (st) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof v, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, sizeof v, s);
+  if (e != cudaSuccess) return fail_msg(err, LSE_ERR_CUDA, cudaGetErrorString(e));
+  *device_error = v;
+  return LSE_OK;
 }

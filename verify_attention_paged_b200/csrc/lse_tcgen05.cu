@@ -64,6 +64,7 @@
 #include <mutex>
 
 #include "lse_internal.h"
+#include "lse_smem_attr.h"
 
 namespace {
 
@@ -1664,12 +1665,9 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 template <int DT, int P8, bool kSc>
 int launch_tc(const TcParams &tp, int smem, cudaStream_t st) {
   auto k = partial_tcgen05_kernel<DT, P8, kSc>;
-  static int set_for = -1;  // largest dynamic smem already allowed (per device run)
-  if (smem > set_for) {
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return (int)e;
-    set_for = smem;
-  }
+  static lse_detail::SmemAllowed allowed;  // per device ordinal
+  const int e = lse_detail::allow_dynamic_smem(k, smem, allowed);
+  if (e) return e;
   k<<<tp.n_ctas, kThreads, smem, st>>>(tp);
   return (int)cudaGetLastError();
 }

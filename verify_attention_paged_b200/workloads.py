@@ -396,15 +396,19 @@ def fragment_ab_cases() -> list[Workload]:
 def small_case(dtype: str, seq_lens, rows, n_q_heads=8, n_kv_heads=2, head_dim=64,
                tokens_per_fragment=16, max_pages=None, seed=7, tree=False, kv_std=1.0,
                keep_logical=True, n_chunks=None, scaled=False, scale_spread=0.0,
-               magnitude_spread=0.0) -> Workload:
-    """A small seeded problem of any shape, for parity and pin tests."""
+               magnitude_spread=0.0, frags_per_chunk=None) -> Workload:
+    """A small seeded problem of any shape, for parity and pin tests.
+    ``frags_per_chunk`` cuts the arena into chunks of that many fragments
+    (enough chunks for every live fragment), so a problem spans many chunks."""
     g = torch.Generator().manual_seed(seed)
     es = ELEM_SIZE[dtype]
     fb = tokens_per_fragment * n_kv_heads * head_dim * es
     need = 2 * sum(math.ceil(L / tokens_per_fragment) for L in seq_lens)
     if max_pages is None:
         max_pages = max(1, max(math.ceil(L / tokens_per_fragment) for L in seq_lens))
-    fpc = max(4, need)
+    fpc = max(4, need) if frags_per_chunk is None else int(frags_per_chunk)
+    if frags_per_chunk is not None and n_chunks is None:
+        n_chunks = math.ceil(need / fpc)
     parents = None
     if tree:
         parents = [[int(torch.randint(-1, i, (1,), generator=g)) for i in range(R)] for R in rows]
