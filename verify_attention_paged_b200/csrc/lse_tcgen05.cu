@@ -637,6 +637,7 @@ enum {
   kBarInfo = 49,    // [8] one per tile record
   kBarPEmpty = 57,  // [4] = group * 2 + P buffer: the P tile has been read
   kBarDoneV = 61,   // the output issuer's MMAs have completed
+  kBarSEmpty = 62,  // [2] per softmax group: its score buffer has been read out
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -713,13 +714,13 @@ __device__ __forceinline__ void f8_terms(float *x, uint2 *out) {
 }
 
 // Eight FP32 values -> F16 (round to nearest), then kTerms E5M2 terms of
-// the F16 values.  E5M2 is the upper byte of F16 (same sign and exponent
-// fields), so the nearest E5M2 of each half of a packed F16 pair is its bit
-// pattern with the low byte rounded away (ties to even; a carry out of the
-// mantissa raises the exponent), done for both halves in integer arithmetic
-// (a half stays far below 0xFF80 here, so no carry crosses halves).  Each
-// remainder is an exact F16 subtraction, and four terms of 3 significant
-// bits hold all 11 bits of an F16.
+// the F16 values.  E5M2 has F16's sign and exponent fields, so every E5M2
+// value is an F16 value and the nearest E5M2 of an F16 (round to nearest,
+// ties to even) leaves a remainder that F16 holds exactly: each term is the
+// hardware conversion of the remainder so far, converted back and
+// subtracted (an exact F16 subtraction).  Four terms of 3 significant bits
+// hold all 11 bits of an F16.  (The inputs stay far below E5M2's largest
+// finite value, so the saturating conversion never clips.)
 template <int kTerms>
 __device__ __forceinline__ void e5_terms_f16(const float *x, uint2 *out) {
   uint32_t h[4];
@@ -731,10 +732,14 @@ __device__ __forceinline__ void e5_terms_f16(const float *x, uint2 *out) {
     uint32_t w[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t r = (h[i] + 0x007F007Fu + ((h[i] >> 8) & 0x00010001u)) & 0xFF00FF00u;
-      // bytes 1 and 3 of r: the lower value's E5M2 in the low byte
-      asm("prmt.b32 %0, %1, 0, 0x0031;" : "=r"(w[i]) : "r"(r));
-      if (t + 1 < kTerms) asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(h[i]) : "r"(h[i]), "r"(r));
+      uint16_t e;
+      asm("cvt.rn.satfinite.e5m2x2.f16x2 %0, %1;" : "=h"(e) : "r"(h[i]));
+      w[i] = e;
+      if (t + 1 < kTerms) {
+        uint32_t back;
+        asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(back) : "h"(e));
+        asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(h[i]) : "r"(h[i]), "r"(back));
+      }
     }
     out[t] = make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
   }
@@ -812,6 +817,28 @@ __device__ __forceinline__ float warp_sum8(const float *e, int lane) {
   float x = (b2 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? w2[0] : w2[1], 4);
   x += __shfl_xor_sync(0xffffffffu, x, 2);
   x += __shfl_xor_sync(0xffffffffu, x, 1);
+  return x;
+}
+
+// Maximum of eight per-lane values over the 32 lanes of a warp, by the same
+// fixed butterfly as warp_sum8: every lane returns the warp maximum of value
+// (lane >> 2).
+__device__ __forceinline__ float warp_max8(const float *e, int lane) {
+  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+  float w4[4], w2[2];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float keep = b4 ? e[4 + i] : e[i], give = b4 ? e[i] : e[4 + i];
+    w4[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, give, 16));
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float keep = b3 ? w4[2 + i] : w4[i], give = b3 ? w4[i] : w4[2 + i];
+    w2[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, give, 8));
+  }
+  float x = fmaxf(b2 ? w2[1] : w2[0], __shfl_xor_sync(0xffffffffu, b2 ? w2[0] : w2[1], 4));
+  x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 2));
+  x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 1));
   return x;
 }
 
@@ -958,7 +985,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // the merge pass may be scheduled now; it waits for this grid to finish
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  // ---- prologue: total live tiles, barriers, TMEM -------------------------------
+  // ---- prologue: TMEM, total live tiles, barriers --------------------------------
+  if (warp == 1) {
+    // allocated first, while warp 0 reads the sequences' lengths
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(Lay::kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
   const bool use_tab = p.n_seqs <= kSeqTab;
   if (warp == 0) {
     // every sequence's tiles, lanes taking contiguous blocks; then a warp
@@ -1011,6 +1046,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarSFull + i), 1);
+      mbar_init(bar(kBarSEmpty + i), 128);
       mbar_init(bar(kBarPFull + i), 128);
       mbar_init(bar(kBarQFull + i), 1);
       // FP8: the softmax groups also hold the slot until they have copied
@@ -1024,25 +1060,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (tid < 64) pair_row[tid] = tid / p.group;
-  __syncthreads();
-  const long long U = *shared_u;
-  // working CTAs: never more than tiles, so no working range is empty and a
-  // segment's pieces never outnumber its tiles
-  const int C = (int)(U < tp.n_ctas ? U : tp.n_ctas);
-  if (cta >= C) return;  // nothing for this CTA (uniform)
-  const long long t_begin = U * cta / C, t_stop = U * (cta + 1) / C;
-
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"(Lay::kTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const long long U = *shared_u;
+  // working CTAs: never more than tiles, so no working range is empty and a
+  // segment's pieces never outnumber its tiles
+  const int C = (int)(U < tp.n_ctas ? U : tp.n_ctas);
+  if (cta >= C) {  // nothing for this CTA (uniform): give the TMEM back
+    if (warp == 1)
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                   "r"(Lay::kTmemCols)
+                   : "memory");
+    return;
+  }
+  const long long t_begin = U * cta / C, t_stop = U * (cta + 1) / C;
   constexpr int kSW = Lay::kSW;
   auto tmem_s = [&](int grp) { return tmem + (uint32_t)(grp * kSW); };
   constexpr int kOS = Lay::kOSlots;
@@ -1130,12 +1163,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (first) ++seg_q;
         const int st = nq % NS;
         // the segment's Q, the K tile, and the group's score buffer, which
-        // its softmax finished reading with tile nq - 2
+        // its softmax read out (into registers) at the start of tile nq - 2
         bool go = !first || mbar_wait(bar(kBarQFull + seg_q % QS), (seg_q / QS) & 1, abort_flag,
                                       p.err);
         go = go && mbar_wait(bar(kBarFullK + st), (nq / NS) & 1, abort_flag, p.err);
         go = go && (nq < 2 ||
-                    mbar_wait(bar(kBarPFull + (nq & 1)), ((nq - 2) >> 1) & 1, abort_flag, p.err));
+                    mbar_wait(bar(kBarSEmpty + (nq & 1)), ((nq - 2) >> 1) & 1, abort_flag, p.err));
         if (!__all_sync(0xffffffffu, go)) break;
         tc_fence_after();
         const uint32_t kaddr = k_base + st * Lay::kHalfStage;
@@ -1368,11 +1401,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // tile record, published by the producer on its own barrier (the
         // K ring may already hold a later tile)
         if (w) w = mbar_wait(bar(kBarInfo + (n & 7)), (n >> 3) & 1, abort_flag, p.err);
-        // this tile's P buffer is free once the output product that last
-        // read it (the group's tile n - 2 PB) has completed
+        // (this tile's P buffer is waited for just before pass 2 writes it)
         const int pbuf_n = (n >> 1) % PB, use = (n >> 1) / PB;
-        if (w && use >= 1)
-          w = mbar_wait(bar(kBarPEmpty + 2 * grp + pbuf_n), (use - 1) & 1, abort_flag, p.err);
         // per-vector scales land with the tile's V (the V slot outlives
         // this pass: its output product waits for this tile's P)
         if (kSc && w)
@@ -1424,12 +1454,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the running max by 2^tau?
         float sv[P8], mr[P8];
 #pragma unroll
-        for (int c = 0; c < P8; c += 8) {
-          tmem_load_sum8<kSW / kNQ>(s_addr + c, kNQ, sv + c);
-          if constexpr (kF8) {
+        for (int c = 0; c < P8; c += 8) tmem_load_sum8<kSW / kNQ>(s_addr + c, kNQ, sv + c);
+        // the scores are in registers: the group's next score product may
+        // overwrite the buffer while this tile's probabilities are built
+        tc_fence_before();
+        mbar_arrive(bar(kBarSEmpty + grp));
+        if constexpr (kF8) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) sv[c + i] *= isg[c + i];
-          }
+          for (int q = 0; q < P8; ++q) sv[q] *= isg[q];
         }
         if constexpr (kSc) {
 #pragma unroll
@@ -1451,20 +1483,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         float gap = -INFINITY;
 #pragma unroll
         for (int q = 0; q < P8; ++q) gap = fmaxf(gap, sv[q] - mr[q]);
-        float *scr = scratch(n);
         if (named_or(bar_id, 128, gap > kTau)) {
-          // per-pair maximum over the tile's keys, through this tile's P
-          // buffer as FP32 scratch [key][pair] (free: waited for above)
+          // per-pair maximum over the tile's keys: each warp folds its 32
+          // keys by a butterfly, and the four warps' maxima meet in red
+          // [warp quarter][pair]
 #pragma unroll
-          for (int c = 0; c < P8; c += 4)
-            *reinterpret_cast<float4 *>(scr + j * P8 + c) =
-                make_float4(sv[c], sv[c + 1], sv[c + 2], sv[c + 3]);
-          named_sync(bar_id, 128);
-          column_reduce<P8, false>(scr, j, red, bar_id);  // red[q] = max over keys
+          for (int c = 0; c < P8; c += 8) {
+            const float wm = warp_max8(sv + c, lane);
+            if ((lane & 3) == 0) red[quarter * 64 + c + (lane >> 2)] = wm;
+          }
           named_sync(bar_id, 128);
           if (j < P8) {
             const float mo = m_run[j];
-            const float mn = fmaxf(mo, red[j]);
+            const float mn = fmaxf(mo, fmaxf(fmaxf(red[j], red[64 + j]),
+                                             fmaxf(red[128 + j], red[192 + j])));
             const float al = ex2(mo - mn);
             alpha[j] = al;
             m_run[j] = mn;
@@ -1485,11 +1517,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (had_tile) {
             // rescale this group's output once every earlier P.V of the group
-            // has completed (with two P buffers, tile n - 2's used the other)
-            bool wo = true;
-            if (PB == 2 && n >= 2)
-              wo = mbar_wait(bar(kBarPEmpty + 2 * grp + (pbuf_n ^ 1)), (((n >> 1) - 1) >> 1) & 1,
-                             abort_flag, p.err);
+            // has completed: the output products complete in issue order, so
+            // the one of the group's previous tile (n - 2) covers them all
+            const int pn = (n - 2) >> 1;
+            const bool wo = mbar_wait(bar(kBarPEmpty + 2 * grp + pn % PB), (pn / PB) & 1,
+                                      abort_flag, p.err);
             if (named_or(bar_id, 128, !wo)) {
               ok = false;
               break;
@@ -1508,6 +1540,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               tmem_st8(ob + c, v);
             }
             tmem_st_wait();
+          }
+        }
+        // this tile's P buffer is free once the output product that last
+        // read it (the group's tile n - 2 PB) has completed
+        if (use >= 1) {
+          const bool wp =
+              mbar_wait(bar(kBarPEmpty + 2 * grp + pbuf_n), (use - 1) & 1, abort_flag, p.err);
+          if (named_or(bar_id, 128, !wp)) {
+            ok = false;
+            break;
           }
         }
         // pass 2: probabilities -> this group's P tile, row j (16-bit: hi block
