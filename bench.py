@@ -66,6 +66,29 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def measured_bf16_tflops():
+    """Dense BF16 tensor peak (burst) measured on this machine's B200s."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
+def attention_flops(w):
+    """Algorithmic FLOPs of one call: 4 D per (row, query head, visible key)
+    (the score and output products, 2 each); a block row at position C + r
+    sees C + r + 1 keys (chain rows, no masks)."""
+    lens = np.asarray(w.seq_lens, np.int64)
+    offs = np.asarray(w.row_offsets, np.int64)
+    vis = 0
+    for s in range(len(lens)):
+        R = int(offs[s + 1] - offs[s])
+        C = int(lens[s]) - R
+        vis += R * C + R * (R + 1) // 2
+    return 4 * w.head_dim * w.n_q_heads * vis
+
+
 # the sources each measured kernel (and its launch plan) is built from
 KERNEL_SOURCES = {
     "partial": ("lse_host.cpp", "lse_internal.h", "lse_tcgen05.cu"),
@@ -272,7 +295,7 @@ def compute_dtype(kv_dtype, kernel):
     """The arithmetic the partial pass runs in: the tensor-core kernel takes
     16-bit K/V times 16-bit hi + lo terms of Q and P, or 8-bit K/V times 8-bit
     terms, accumulating in FP32; the CUDA-core kernel is FP32 throughout."""
-    return f"{kv_dtype}-mma/f32" if kernel == 1 else "f32"
+    return f"{kv_dtype}-mma/f32" if kernel in (1, 2) else "f32"
 
 
 def workload_config(w):
@@ -289,10 +312,13 @@ HEADLINE = "tree_verify"   # the largest single-GPU workload carries the headlin
 
 def time_workload(w, args, flush, dist, clk):
     """Device times of one workload: `args.steps` graph replays of the whole
-    step (partial pass, then the merge as its programmatic dependent) and
-    as many of the partial pass alone, L2 flushed before each outside the
-    CUDA-event interval.  Returns the DeviceCall (kept for the end-to-end
-    leg) and the per-step millisecond lists."""
+    step (lse_attn_forward: on tensor-core plans one launch, the merge fused
+    into the partial pass; on CUDA-core plans the partial pass and the merge
+    as its programmatic dependent) and as many of the dominant kernel alone
+    (the partial pass of a two-kernel step; the step itself when it is one
+    kernel), L2 flushed before each outside the CUDA-event interval.
+    Returns the DeviceCall (kept for the end-to-end leg) and the per-step
+    millisecond lists."""
     import torch
     from verify_attention_paged_b200 import binding as b
     call = b.DeviceCall(w)
@@ -301,15 +327,18 @@ def time_workload(w, args, flush, dist, clk):
         call.run()
     torch.cuda.synchronize()
     assert call.device_error() == 0, f"{w.name}: device error during warm-up"
+    one_kernel = call.info["kernel_name"] in ("tcgen05", "prefill")
     g_step, g_part = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
     saved = call.stream
     with torch.cuda.graph(g_step):
         call.stream = torch.cuda.current_stream()
-        call.run_partial()
-        call.run_merge()
+        call.run()
     with torch.cuda.graph(g_part):
         call.stream = torch.cuda.current_stream()
-        call.run_partial()
+        if one_kernel:
+            call.run()
+        else:
+            call.run_partial()
     call.stream = saved
     for _ in range(3):
         flush.fill_(2)
@@ -347,21 +376,45 @@ def time_workload(w, args, flush, dist, clk):
 
 def workload_result(w, call, steps_ms, part_ms, world, dist, args, peak, peak_kind):
     """One workload's figures: us per call, whole-job GB/s, and the roofline
-    of the partial pass (its algorithmic K + V + Q bytes over its
-    CUDA-event time, against the measured copy bandwidth)."""
+    of the dominant kernel (the algorithmic K + V + Q bytes of the partial
+    pass over that kernel's CUDA-event time, against the measured copy
+    bandwidth)."""
     total_ms = reduce_max(sum(steps_ms), dist, "cuda")
     part_mean = reduce_max(statistics.mean(part_ms), dist, "cuda")
+    info = call.info
+    fused = info["kernel_name"] in ("tcgen05", "prefill")
     bytes_call = w.call_bytes()
-    bytes_partial = w.kv_bytes() + w.total_rows * w.n_q_heads * w.head_dim * 4
+    # the dominant kernel's algorithmic bytes: K + V + Q (+ out when the
+    # merge is fused into it)
+    bytes_partial = w.call_bytes() if fused else (
+        w.kv_bytes() + w.total_rows * w.n_q_heads * w.head_dim * 4)
     achieved = bytes_partial / (part_mean * 1e-3) / 1e9
     value = job_gbs(world, bytes_call, args.steps, total_ms)
-    info = call.info
     bound = "hbm"
     if bytes_call < 4 << 20:
         # a quarter of a megabyte moves in well under a microsecond at HBM
         # speed: launch and dependent-load latency set the time
         bound = "launch"
+    roof = {"bound": bound,
+            "kernel": "partial pass with the merge fused" if fused else "partial",
+            "achieved": achieved, "peak": peak,
+            "peak_kind": f"{peak_kind} (copy, burst)", "unit": "GB/s",
+            "frac": achieved / peak, "traffic": ncu_traffic(w.name),
+            "algorithmic_bytes_per_launch": bytes_partial}
+    extra = {}
+    if info["kernel_name"] == "prefill":
+        # a long query block is a dense contraction: its roofline is the
+        # tensor peak (the products carry hi + lo operand terms, so at most
+        # half of it counts as algorithmic FLOPs)
+        tf_peak, tf_kind = measured_bf16_tflops()
+        tflops = attention_flops(w) / (part_mean * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": "long-query-block pass", "achieved": tflops,
+                "peak": tf_peak, "peak_kind": f"{tf_kind} (cuBLAS bf16, burst)",
+                "unit": "TFLOP/s", "frac": tflops / tf_peak, "traffic": ncu_traffic(w.name),
+                "algorithmic_flops_per_launch": attention_flops(w)}
+        extra = {"tflops": tflops}
     return {
+        **extra,
         "value": value, "unit": "GB/s", "us_per_call": total_ms / args.steps * 1e3,
         "us_per_call_median": statistics.median(steps_ms) * 1e3,
         "partial_us_mean": part_mean * 1e3,
@@ -370,11 +423,9 @@ def workload_result(w, call, steps_ms, part_ms, world, dist, args, peak, peak_ki
         "pct_of_measured_hbm": value / world / peak * 100.0,
         "bytes_per_call": bytes_call,
         "kernel": info["kernel_name"], "n_splits": info["n_splits"],
+        "launches_per_call": 1 if fused else 2,
         "dtype": compute_dtype(w.dtype, info["kernel"]),
-        "roofline": {"bound": bound, "kernel": "partial", "achieved": achieved, "peak": peak,
-                     "peak_kind": f"{peak_kind} (copy, burst)", "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": ncu_traffic(w.name),
-                     "algorithmic_bytes_per_launch": bytes_partial},
+        "roofline": roof,
     }
 
 
@@ -430,7 +481,7 @@ def run_ours(args, names, world, rank, local):
                    "kernel": r["kernel"], "n_splits": r["n_splits"]},
         "roofline": r["roofline"],
         "per_workload": {n: {k: v for k, v in res.items()} for n, res in results.items()},
-        "gpu_launches": 4 * args.steps * len(names),
+        "gpu_launches": 2 * args.steps * sum(res["launches_per_call"] for res in results.values()),
         "clocks": clk.summary(),
     }
     if e2e:
@@ -444,33 +495,20 @@ def run_ours(args, names, world, rank, local):
 
 def measure_e2e(call, w, args, stream, flush, dist):
     """Same metric through the public API with this step's inputs (Q, page
-    tables, lengths, row offsets, masks) copied from pinned host memory and
-    the result (out and lse) read back, inside the timed interval."""
+    tables, lengths, row offsets, masks, packed in one pinned host buffer)
+    copied to the device in one copy and the result (out and lse, packed)
+    read back in one copy, inside the timed interval."""
     import torch
-    host_in = [torch.from_numpy(np.ascontiguousarray(w.q)).pin_memory(),
-               torch.from_numpy(np.ascontiguousarray(w.k_pages)).pin_memory(),
-               torch.from_numpy(np.ascontiguousarray(w.v_pages)).pin_memory(),
-               torch.from_numpy(np.ascontiguousarray(w.seq_lens)).pin_memory(),
-               torch.from_numpy(np.ascontiguousarray(w.row_offsets)).pin_memory()]
-    dev_in = [call.q, call.k_pages, call.v_pages, call.seq_lens, call.row_offsets]
-    if w.row_masks is not None:
-        host_in.append(torch.from_numpy(np.ascontiguousarray(w.row_masks).view(np.int64))
-                       .pin_memory())
-        dev_in.append(call.row_masks)
-    rows = w.total_rows
-    host_out = torch.empty((rows, w.n_q_heads, w.head_dim), dtype=torch.float32).pin_memory()
-    host_lse = torch.empty((rows, w.n_q_heads), dtype=torch.float32).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host_in)
-    d2h = host_out.numel() * 4 + host_lse.numel() * 4
+    host_in = call.host_inputs
+    host_out = torch.empty(call.outputs.numel(), dtype=torch.float32).pin_memory()
+    h2d = host_in.numel()
+    d2h = host_out.numel() * 4
     steps = max(10, args.steps // 5)
 
     def step():
-        with torch.cuda.stream(stream):
-            for h, d in zip(host_in, dev_in):
-                d.copy_(h, non_blocking=True)
-            call.run()
-            host_out.copy_(call.out[:rows], non_blocking=True)
-            host_lse.copy_(call.lse[:rows], non_blocking=True)
+        call.upload(host_in)
+        call.run()
+        call.download(host_out)
 
     for _ in range(3):
         step()
@@ -479,17 +517,18 @@ def measure_e2e(call, w, args, stream, flush, dist):
            for _ in range(steps)]
     if dist:
         dist.barrier()
-    for i in range(steps):
-        flush.fill_(i & 0xff)
-        evs[i][0].record(stream)
-        step()
-        evs[i][1].record(stream)
+    with torch.cuda.stream(stream):
+        for i in range(steps):
+            flush.fill_(i & 0xff)
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
     torch.cuda.synchronize()
     ms = reduce_max(sum(a.elapsed_time(b) for a, b in evs), dist, "cuda")
     world = dist.get_world_size() if dist else 1
     return {"value": job_gbs(world, w.call_bytes(), steps, ms), "unit": "GB/s",
             "us_per_call": ms / steps * 1e3, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h}
+            "d2h_bytes_per_step": d2h, "copies_per_step": {"h2d": 1, "d2h": 1}}
 
 
 APPEND_METRIC = "K/V append us/call and GB/s (FP32 read + stored bytes)"
@@ -591,8 +630,7 @@ def _step_times(call, steps, flush):
     saved = call.stream
     with torch.cuda.graph(g):
         call.stream = torch.cuda.current_stream()
-        call.run_partial()
-        call.run_merge()
+        call.run()
     call.stream = saved
     for i in range(3):
         flush.fill_(i)
@@ -693,7 +731,8 @@ def main():
         run_append(args, world, rank, local)
         return
     from verify_attention_paged_b200 import workloads as wl
-    names = list(wl.NAMES) if args.workload == "all" else [args.workload]
+    # the five configurations, then the long query block (its own roofline)
+    names = list(wl.NAMES) + ["prefill_block"] if args.workload == "all" else [args.workload]
     if args.impl == "reference":
         head = HEADLINE if HEADLINE in names else names[0]
         run_reference(args, wl.BUILDERS[head](), world, rank)

@@ -106,7 +106,8 @@ typedef enum {
 #define LSE_MAX_CHUNKS 64     /* arena chunks a kernel can address          */
 #define LSE_MAX_TMA_CHUNKS 64 /* chunks the tensor-core kernel can address (every chunk
                                  an arena can have: one TMA descriptor per chunk) */
-#define LSE_MAX_ROWS_PER_SEQ 64
+#define LSE_MAX_ROWS_PER_SEQ 64    /* rows per sequence of the verify kernels (64-bit masks) */
+#define LSE_MAX_BLOCK_ROWS 32768   /* rows per sequence of a long query block (chain only) */
 
 typedef struct lse_kv_arena lse_kv_arena;
 typedef struct lse_attn_plan_s lse_attn_plan_t;
@@ -210,16 +211,18 @@ LSE_API int lse_attn_plan_ex(const lse_kv_arena *arena, int n_seqs, int max_rows
 /* Kernel families a plan can select. */
 #define LSE_KERNEL_CUDA_CORE 0 /* FP32 math on CUDA cores (any dtype, any P) */
 #define LSE_KERNEL_TCGEN05 1   /* tensor-core (tcgen05) partial pass           */
+#define LSE_KERNEL_PREFILL 2   /* tensor-core pass for long query blocks (rows as M) */
 
 /* For LSE_KERNEL_CUDA_CORE the partitions are fixed ranges of K_p keys,
  * n_splits = ceil(capacity / K_p), and partitions past a sequence's live
  * keys are skipped.  For LSE_KERNEL_TCGEN05 the partial pass is persistent
  * (one CTA per SM): the live 128-key tiles of all (sequence, kv head) pairs
  * are laid end to end and cut into equal contiguous ranges, one per CTA;
- * each piece yields one partial per softmax warpgroup, so n_splits =
- * 2 * min(CTAs, capacity tiles) bounds the partials of one (sequence, kv
- * head); keys_per_split reports the tile (128); capacity without live keys
- * is never visited. */
+ * a CTA's share of one (sequence, kv head) is a piece, which yields one
+ * partial (the CTA combines its two softmax warpgroups), so n_splits =
+ * min(CTAs, capacity tiles) bounds the partials of one (sequence, kv head);
+ * keys_per_split reports the tile (128); capacity without live keys is
+ * never visited. */
 typedef struct {
   int32_t n_splits;        /* partial slots per (row, head)                  */
   int32_t keys_per_split;  /* K_p (CUDA-core) or the key tile (tcgen05)      */
@@ -250,7 +253,8 @@ LSE_API int lse_attn_plan_query(const lse_attn_plan_t *plan, lse_attn_plan_info 
 LSE_API int lse_attn_split_rule(int64_t capacity_keys, int units, int n_sms, int ctas_per_sm,
                         int key_tile, int32_t *keys_per_split);
 
-/* Zero the workspace's error word (once after allocation; any time to clear). */
+/* Zero the workspace's error word and the fused pass's segment counters
+ * (once after allocation; any time to clear). */
 LSE_API int lse_attn_workspace_init(const lse_attn_plan_t *plan, void *workspace, void *stream,
                             char **err);
 
@@ -289,6 +293,29 @@ LSE_API int lse_attn_merge(const lse_attn_plan_t *plan, const int32_t *seq_lens,
                    float *lse_out, void *stream, char **err);
 
 /* ---------------------------------------------------------------------------
+ * Partial and merge passes in one call (LSE releases, v0.4.19: one partial
+ * and one merge family; v0.4.20: empty partitions skipped).  Arguments as
+ * lse_attn_run plus lse_attn_merge's out / lse_out; the result equals
+ * lse_attn_run followed by lse_attn_merge up to FP32 rounding.
+ * For tensor-core plans the merge runs inside the partial pass's launch: a
+ * CTA whose share of a (sequence, kv head) is the whole of it writes the
+ * final output directly; the partials of a shared one are merged at the end
+ * of the launch by the CTAs that computed them, after a bounded wait for
+ * the other pieces.  That launch is cooperative (every CTA resident at
+ * once; the call fails with LSE_ERR_CUDA where the device cannot hold the
+ * grid) and uses the workspace's segment counters, which each call leaves
+ * at zero.  After a call that set a device error bit, read it with
+ * lse_attn_read_error (which then also clears the counters) or call
+ * lse_attn_workspace_init before the next call.  For CUDA-core plans this
+ * is lse_attn_run then lse_attn_merge.
+ * ------------------------------------------------------------------------- */
+LSE_API int lse_attn_forward(const lse_attn_plan_t *plan, const float *q, const int32_t *k_pages,
+                             const int32_t *v_pages, const int32_t *seq_lens,
+                             const int32_t *row_offsets, const uint64_t *row_masks,
+                             float softmax_scale, void *workspace, float *out, float *lse_out,
+                             void *stream, char **err);
+
+/* ---------------------------------------------------------------------------
  * Host-side validation of HOST copies of the device inputs: every live page
  * names a fragment of the arena (sequences may share read-only fragments),
  * L_s <= capacity,
@@ -301,7 +328,8 @@ LSE_API int lse_attn_validate(const lse_attn_plan_t *plan, const int32_t *k_page
                       const int32_t *row_offsets, const uint64_t *row_masks, char **err);
 
 /* Read (and clear) the workspace's device error word.  Synchronises the
- * stream.  *device_error receives LSE_DEVERR_* bits, 0 when clean. */
+ * stream.  *device_error receives LSE_DEVERR_* bits, 0 when clean; when it
+ * is not, the fused pass's segment counters are cleared as well. */
 LSE_API int lse_attn_read_error(const lse_attn_plan_t *plan, void *workspace, void *stream,
                         uint32_t *device_error, char **err);
 
@@ -383,6 +411,16 @@ LSE_API int lse_attn_forward_static(const lse_attn_plan_t *plan, const float *q,
  * the static call itself it allocates nothing; the first use on a device
  * looks the scratch address up.  No counterpart on the pages. */
 LSE_API int lse_attn_static_read_error(void *stream, uint32_t *device_error, char **err);
+
+/* Testing the bounded waits (no counterpart on the pages).  Every wait of
+ * the tensor-core pass gives up after about 2 s, sets LSE_DEVERR_TIMEOUT,
+ * drains the copies and products in flight, releases TMEM and returns, so
+ * a fault upstream never leaves the GPU blocked.  After this call every
+ * later launch of `plan` skips loading each CTA's tile of local index
+ * `tile` (nothing arrives on that tile's barriers), so those waits run out;
+ * tile = -1 restores normal loading.  For tests only.  Returns
+ * LSE_ERR_UNSUPPORTED for plans of other kernels. */
+LSE_API int lse_attn_test_withhold_tile(lse_attn_plan_t *plan, int tile);
 
 /* Release a string returned through an err argument. */
 LSE_API void lse_free(void *p);

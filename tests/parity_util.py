@@ -33,19 +33,22 @@ def lse_tol(dtype):
     return FP32_ABS if dtype == "f32" else LOWP_TOL
 
 
-def oracle_all_outputs(pb, threads=None):
+def oracle_all_outputs(pb, threads=None, rows=None):
     """Every (row, head) output of a problem from the float64 oracle, one
     output per call on one thread per host core (the ctypes calls release
-    the GIL).  Same result as oracle.attention(pb), computed in parallel."""
+    the GIL).  Same result as oracle.attention(pb), computed in parallel.
+    ``rows`` (call row indices) restricts it to those rows; the other
+    entries stay 0."""
     from oracle import oracle as orc
     m = orc.marshal(pb)
     ro = np.asarray(pb.row_offsets)
-    rows = int(ro[-1])
+    n_rows = int(ro[-1])
     hq, d = pb.n_q_heads, pb.head_dim
-    out = np.zeros((rows, hq, d), np.float64)
-    lse = np.zeros((rows, hq), np.float64)
+    out = np.zeros((n_rows, hq, d), np.float64)
+    lse = np.zeros((n_rows, hq), np.float64)
+    keep = None if rows is None else set(int(x) for x in rows)
     items = [(s, r, h) for s in range(len(ro) - 1) for r in range(int(ro[s + 1] - ro[s]))
-             for h in range(hq)]
+             for h in range(hq) if keep is None or int(ro[s]) + r in keep]
     # the longest sequences first, so the threads finish together
     lens = np.asarray(pb.seq_lens)
     items.sort(key=lambda t: -int(lens[t[0]]))

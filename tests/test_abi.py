@@ -105,8 +105,8 @@ def test_plan_workspace_size():
 
 def test_plan_rejects_bad_shapes():
     a = b.lse_kv_arena_create([FAKE], 1 << 20, 256 << 10, "bf16", 4, 128)
-    for args in [(1, 65, 65, 24, 10), (1, 0, 1, 24, 10), (1, 1, 1, 22, 10), (0, 1, 1, 24, 10),
-                 (2, 4, 9, 24, 10)]:
+    for args in [(1, 40000, 40000, 24, 10), (1, 0, 1, 24, 10), (1, 1, 1, 22, 10),
+                 (0, 1, 1, 24, 10), (2, 4, 9, 24, 10)]:
         with pytest.raises(b.LseError):
             b.lse_attn_plan_ex(a, *args, **B200)
 
@@ -281,3 +281,37 @@ def test_tma_chunk_limit_is_every_chunk_an_arena_can_have():
     import re
     lim = {k: int(v) for k, v in re.findall(r"#define (LSE_MAX_\w*CHUNKS) (\d+)", text)}
     assert lim["LSE_MAX_TMA_CHUNKS"] == lim["LSE_MAX_CHUNKS"]
+
+
+def test_long_query_block_plans():
+    # more than 64 rows per sequence: the rows-as-M tensor-core pass, for
+    # 16-bit and FP8 arenas at head_dim 128; refused (with the reason)
+    # elsewhere; it runs through lse_attn_forward only, without masks
+    a = b.lse_kv_arena_create([FAKE], 1 << 28, 256 << 10, "bf16", 4, 128)
+    p, ws = b.lse_attn_plan_ex(a, 2, 1024, 2048, 24, 64, **B200)
+    info = b.lse_attn_plan_query(p)
+    assert info["kernel_name"] == "prefill" and info["rows_per_chunk"] == 128
+    assert info["smem_bytes"] <= B200["smem_optin"] and 2 <= info["stages"] <= 6
+    assert ws >= 148 * 2 * 128 * 129 * 4
+    F = FAKE
+    with pytest.raises(b.LseError, match="lse_attn_forward"):
+        b.lse_attn_run(p, F, F, F, F, F, None, 0.1, F)       # refused before any launch
+    with pytest.raises(b.LseError, match="lse_attn_forward"):
+        b.lse_attn_merge(p, F, F, F, F)
+    with pytest.raises(b.LseError, match="row masks"):
+        b.lse_attn_forward(p, F, F, F, F, F, F, 0.1, F, F)
+    lens = np.array([1000, 70], np.int32)
+    offs = np.array([0, 900, 970], np.int32)
+    pages = np.zeros((2, 64), np.int32)
+    b.lse_attn_validate(p, pages, pages, lens, offs)
+    masks = np.full(970, 1, np.uint64)
+    with pytest.raises(b.LseError, match="masks take at most 64"):
+        b.lse_attn_validate(p, pages, pages, lens, offs, masks)
+    b.lse_attn_plan_destroy(p)
+    with pytest.raises(b.LseError, match="tcgen05"):
+        b.lse_attn_plan_ex(a, 1, 100, 100, 24, 64, **{**B200, "allow_tcgen05": 0})
+    b.lse_kv_arena_destroy(a)
+    f = b.lse_kv_arena_create([FAKE], 1 << 20, 64 << 10, "f32", 1, 128)
+    with pytest.raises(b.LseError, match="16-bit or FP8"):
+        b.lse_attn_plan_ex(f, 1, 100, 100, 8, 64, **B200)
+    b.lse_kv_arena_destroy(f)

@@ -30,7 +30,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 LSE_OK = 0
 KV_DTYPES = {"f32": 0, "f16": 1, "bf16": 2, "e4m3": 3, "e5m2": 4}
-KERNELS = {0: "cuda_core", 1: "tcgen05"}
+KERNELS = {0: "cuda_core", 1: "tcgen05", 2: "prefill"}
 DEVERR_BAD_FRAGMENT = 0x1
 DEVERR_BAD_LENGTH = 0x2
 DEVERR_TIMEOUT = 0x4
@@ -89,6 +89,8 @@ _sig("lse_attn_workspace_init", _i, _vp, _vp, _vp, _errp)
 _sig("lse_attn_plan_destroy", None, _vp)
 _sig("lse_attn_run", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _vp, _errp)
 _sig("lse_attn_merge", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _errp)
+_sig("lse_attn_forward", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _vp, _vp, _vp,
+     _vp, _errp)
 _sig("lse_attn_validate", _i, _vp, _i32p, _i32p, _i32p, _i32p,
      ctypes.POINTER(ctypes.c_uint64), _errp)
 _sig("lse_attn_read_error", _i, _vp, _vp, _vp, ctypes.POINTER(ctypes.c_uint32), _errp)
@@ -96,6 +98,7 @@ _sig("lse_attn_forward_static", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_
      _vp, _errp)
 _sig("lse_kv_append", _i, _vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _errp)
 _sig("lse_attn_static_read_error", _i, _vp, ctypes.POINTER(ctypes.c_uint32), _errp)
+_sig("lse_attn_test_withhold_tile", _i, _vp, _i)
 STATIC_SCRATCH_BYTES = 32 << 20
 
 
@@ -265,6 +268,14 @@ def lse_attn_merge(plan, seq_lens, row_offsets, workspace, out, lse_out=None, st
           _ptr(out), _ptr(lse_out), _ptr(stream))
 
 
+def lse_attn_forward(plan, q, k_pages, v_pages, seq_lens, row_offsets, row_masks, softmax_scale,
+                     workspace, out, lse_out=None, stream=0) -> None:
+    """Partial and merge passes in one call (one launch on tensor-core plans)."""
+    _call(_lib.lse_attn_forward, plan, _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(seq_lens),
+          _ptr(row_offsets), _ptr(row_masks), float(softmax_scale), _ptr(workspace), _ptr(out),
+          _ptr(lse_out), _ptr(stream))
+
+
 def lse_attn_validate(plan, k_pages, v_pages, seq_lens, row_offsets, row_masks=None) -> None:
     kp, kpp = _i32(k_pages)
     vp, vpp = _i32(v_pages)
@@ -285,6 +296,14 @@ def lse_attn_forward_static(plan, q, k_pages, v_pages, seq_lens, row_offsets, ro
     _call(_lib.lse_attn_forward_static, plan, _ptr(q), _ptr(k_pages), _ptr(v_pages),
           _ptr(seq_lens), _ptr(row_offsets), _ptr(row_masks), float(softmax_scale), _ptr(out),
           _ptr(lse_out), _ptr(stream))
+
+
+def lse_attn_test_withhold_tile(plan, tile: int) -> None:
+    """Tests of the bounded waits: later launches skip loading each CTA's
+    tile ``tile`` (-1 restores normal loading)."""
+    st = _lib.lse_attn_test_withhold_tile(plan, int(tile))
+    if st != LSE_OK:
+        raise LseError(st, "lse_attn_test_withhold_tile")
 
 
 def lse_attn_static_read_error(stream=0) -> int:
@@ -326,15 +345,31 @@ class DeviceCall:
                                ctas_per_sm=0, allow_tcgen05=int(kernel == "tcgen05"))
         self.w = problem
         self.chunks = [torch.from_numpy(c).to(dev) for c in problem.chunks]
-        self.k_pages = torch.from_numpy(np.ascontiguousarray(problem.k_pages)).to(dev)
-        self.v_pages = torch.from_numpy(np.ascontiguousarray(problem.v_pages)).to(dev)
-        self.seq_lens = torch.from_numpy(np.ascontiguousarray(problem.seq_lens)).to(dev)
-        self.row_offsets = torch.from_numpy(np.ascontiguousarray(problem.row_offsets)).to(dev)
-        self.row_masks = None
+        # a step's inputs (Q, page tables, lengths, row offsets, masks) live in
+        # one device buffer, mirrored by one pinned host buffer, so a step's
+        # inputs go up in one copy (upload)
+        host = [np.ascontiguousarray(problem.q, dtype=np.float32),
+                np.ascontiguousarray(problem.k_pages, dtype=np.int32),
+                np.ascontiguousarray(problem.v_pages, dtype=np.int32),
+                np.ascontiguousarray(problem.seq_lens, dtype=np.int32),
+                np.ascontiguousarray(problem.row_offsets, dtype=np.int32)]
         if problem.row_masks is not None:
-            self.row_masks = torch.from_numpy(
-                np.ascontiguousarray(problem.row_masks).view(np.int64)).to(dev)
-        self.q = torch.from_numpy(np.ascontiguousarray(problem.q)).to(dev)
+            host.append(np.ascontiguousarray(problem.row_masks).view(np.int64))
+        offs, total = [], 0
+        for a in host:
+            offs.append(total)
+            total += (a.nbytes + 255) // 256 * 256
+        packed = np.zeros(max(total, 256), np.uint8)
+        for a, o in zip(host, offs):
+            packed[o:o + a.nbytes] = a.reshape(-1).view(np.uint8)
+        self.host_inputs = torch.from_numpy(packed).pin_memory()
+        self.inputs = self.host_inputs.to(dev)
+        views = [self.inputs[o:o + a.nbytes].view(torch.float32 if a.dtype == np.float32 else
+                                                  torch.int64 if a.dtype == np.int64 else
+                                                  torch.int32).view(a.shape)
+                 for a, o in zip(host, offs)]
+        self.q, self.k_pages, self.v_pages, self.seq_lens, self.row_offsets = views[:5]
+        self.row_masks = views[5] if len(views) > 5 else None
         rows = int(problem.row_offsets[-1])
         self.total_rows = rows
         max_rows = max(1, int(np.max(np.diff(problem.row_offsets))))
@@ -360,11 +395,33 @@ class DeviceCall:
         self.workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
         self.stream = stream if stream is not None else torch.cuda.current_stream()
         lse_attn_workspace_init(self.plan, self.workspace, self.stream)
-        self.out = torch.empty((max(rows, 1), problem.n_q_heads, problem.head_dim),
-                               dtype=torch.float32, device=dev)
-        self.lse = torch.empty((max(rows, 1), problem.n_q_heads), dtype=torch.float32,
-                               device=dev)
+        # out and lse in one device buffer (one copy back: download)
+        n_out = max(rows, 1) * problem.n_q_heads * problem.head_dim
+        n_lse = max(rows, 1) * problem.n_q_heads
+        self.outputs = torch.empty(n_out + (n_lse + 63) // 64 * 64, dtype=torch.float32,
+                                   device=dev)
+        self.out = self.outputs[:n_out].view(max(rows, 1), problem.n_q_heads, problem.head_dim)
+        self.lse = self.outputs[n_out:n_out + n_lse].view(max(rows, 1), problem.n_q_heads)
         self.scale = float(problem.scale)
+
+    def upload(self, host_inputs=None):
+        """Copy a step's packed inputs (the layout of ``host_inputs``, a
+        pinned uint8 tensor) to the device in one copy on ``stream``."""
+        src = self.host_inputs if host_inputs is None else host_inputs
+        with self.torch.cuda.stream(self._torch_stream()):
+            self.inputs.copy_(src, non_blocking=True)
+
+    def download(self, host_outputs):
+        """Copy out and lse (packed, FP32) into a pinned host tensor of
+        ``outputs.numel()`` floats in one copy on ``stream``."""
+        with self.torch.cuda.stream(self._torch_stream()):
+            host_outputs.copy_(self.outputs, non_blocking=True)
+
+    def _torch_stream(self):
+        s = self.stream
+        if isinstance(s, self.torch.cuda.Stream):
+            return s
+        return self.torch.cuda.current_stream()
 
     def run_partial(self):
         lse_attn_run(self.plan, self.q, self.k_pages, self.v_pages, self.seq_lens,
@@ -375,6 +432,15 @@ class DeviceCall:
                        self.lse, self.stream)
 
     def run(self):
+        """Both passes through lse_attn_forward (on tensor-core plans, one
+        launch with the merge fused)."""
+        lse_attn_forward(self.plan, self.q, self.k_pages, self.v_pages, self.seq_lens,
+                         self.row_offsets, self.row_masks, self.scale, self.workspace, self.out,
+                         self.lse, self.stream)
+        return self.out, self.lse
+
+    def run_two_pass(self):
+        """lse_attn_run then lse_attn_merge (partials through the workspace)."""
         self.run_partial()
         self.run_merge()
         return self.out, self.lse

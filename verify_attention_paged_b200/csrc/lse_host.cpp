@@ -235,9 +235,9 @@ int lse_attn_plan_ex(const lse_kv_arena *a, int n_seqs, int max_rows, int max_to
   *out = nullptr;
   if (!a) return fail(err, LSE_ERR_INVALID_ARG, "arena is NULL");
   if (n_seqs < 1) return fail(err, LSE_ERR_INVALID_ARG, "n_seqs %d", n_seqs);
-  if (max_rows < 1 || max_rows > LSE_MAX_ROWS_PER_SEQ)
+  if (max_rows < 1 || max_rows > LSE_MAX_BLOCK_ROWS)
     return fail(err, LSE_ERR_INVALID_ARG, "max_rows_per_seq %d not in [1, %d]", max_rows,
-                LSE_MAX_ROWS_PER_SEQ);
+                LSE_MAX_BLOCK_ROWS);
   if (max_total_rows < 1 || max_total_rows > n_seqs * max_rows)
     return fail(err, LSE_ERR_INVALID_ARG, "max_total_rows %d not in [1, %d]", max_total_rows,
                 n_seqs * max_rows);
@@ -307,7 +307,38 @@ int lse_attn_plan_ex(const lse_kv_arena *a, int n_seqs, int max_rows, int max_to
       p8 > 0 ? lse_tc_smem(a->dtype, p8, pl->scaled, smem_optin, &tc_stages, &tc_q_slots,
                            &tc_p_bufs)
              : -1;
-  if (allow_tc && a->dtype != LSE_KV_F32 && a->head_dim == 128 &&
+  if (max_rows > LSE_MAX_ROWS_PER_SEQ) {
+    // a long query block (chain rows only): the rows-as-M tensor-core pass
+    const int rt = lse_pf_row_tile();
+    const int64_t row_tiles = int64_t(n_seqs) * ceil_div(max_rows, rt);
+    const char *why = !allow_tc ? "a device with tcgen05"
+                      : a->dtype == LSE_KV_F32 ? "16-bit or FP8 K/V"
+                      : a->head_dim != 128 ? "head_dim 128"
+                      : !t_ok ? "fragments of a multiple or divisor of 128 tokens (>= 8)"
+                      : pl->scaled ? "an arena without per-vector scales"
+                      : row_tiles > lse_pf_max_row_tiles() ? "at most 256 row tiles of 128 rows"
+                      : nullptr;
+    int pf_stages = 0;
+    const int pf_smem = why ? -1 : lse_pf_smem(a->dtype, smem_optin, &pf_stages);
+    if (!why && pf_smem < 0) why = "more shared memory";
+    if (why) {
+      delete pl;
+      return fail(err, LSE_ERR_UNSUPPORTED, "more than %d rows per sequence (a long query "
+                  "block) needs %s", LSE_MAX_ROWS_PER_SEQ, why);
+    }
+    pl->kernel = LSE_KERNEL_PREFILL;
+    pl->key_tile = lse_tc_key_tile();
+    pl->smem_bytes = pf_smem;
+    pl->stages = pf_stages;
+    pl->box_tokens = T < pl->key_tile ? T : pl->key_tile;
+    pl->ctas = n_sms;
+    pl->rows_per_chunk = rt;
+    // two partial slots of a 128-row tile per CTA: its first and last
+    // segments, the only ones it may share with other CTAs
+    pl->n_splits = 2;
+    pl->keys_per_split = pl->key_tile;
+    pl->n_seg_max = int(row_tiles) * n_q_heads;
+  } else if (allow_tc && a->dtype != LSE_KV_F32 && a->head_dim == 128 &&
       t_ok && p8 > 0 && tc_smem > 0) {
     const int tile = lse_tc_key_tile();
     pl->kernel = LSE_KERNEL_TCGEN05;
@@ -321,10 +352,11 @@ int lse_attn_plan_ex(const lse_kv_arena *a, int n_seqs, int max_rows, int max_to
     pl->box_tokens = T < tile ? T : tile;
     pl->ctas = n_sms;
     const int64_t cap_tiles = ceil_div(cap_keys, tile);
-    // a (sequence, kv head) has at most min(CTAs, tiles) pieces, and each
-    // piece holds one partial per softmax group
-    pl->n_splits = 2 * int(std::min<int64_t>(n_sms, cap_tiles));
+    // a segment (sequence, row chunk, kv head) has at most min(CTAs, tiles)
+    // pieces, one partial each (the CTA combines its two softmax groups)
+    pl->n_splits = int(std::min<int64_t>(n_sms, cap_tiles));
     pl->keys_per_split = tile;
+    pl->n_seg_max = n_seqs * int(ceil_div(max_rows, rows_per_chunk)) * a->n_kv_heads;
   } else {
     pl->kernel = LSE_KERNEL_CUDA_CORE;
     pl->key_tile = 32;
@@ -349,8 +381,11 @@ int lse_attn_plan_ex(const lse_kv_arena *a, int n_seqs, int max_rows, int max_to
     pl->keys_per_split = kp;
   }
 
-  const size_t n_part = size_t(max_total_rows) * n_q_heads * pl->n_splits;
-  pl->ws_o_off = kWsHeader;
+  const size_t n_part = pl->kernel == LSE_KERNEL_PREFILL
+                            ? size_t(n_sms) * 2 * lse_pf_row_tile()
+                            : size_t(max_total_rows) * n_q_heads * pl->n_splits;
+  pl->ws_cnt_off = kWsHeader;
+  pl->ws_o_off = align256(pl->ws_cnt_off + size_t(pl->n_seg_max) * 2 * sizeof(uint32_t));
   pl->ws_lse_off = align256(pl->ws_o_off + n_part * a->head_dim * sizeof(float));
   pl->ws_bytes = align256(pl->ws_lse_off + n_part * sizeof(float));
   if (ws_bytes) *ws_bytes = pl->ws_bytes;
@@ -366,22 +401,30 @@ int lse_attn_plan_query(const lse_attn_plan_t *pl, lse_attn_plan_info *info) {
   info->key_tile = pl->key_tile;
   info->pairs = pl->pairs;
   info->smem_bytes = pl->smem_bytes;
-  info->ctas = pl->kernel == LSE_KERNEL_TCGEN05 ? pl->ctas : 0;
+  info->ctas = pl->kernel != LSE_KERNEL_CUDA_CORE ? pl->ctas : 0;
   info->workspace_bytes = int64_t(pl->ws_bytes);
-  const bool tc = pl->kernel == LSE_KERNEL_TCGEN05;
-  info->stages = tc ? pl->stages : 0;
+  const bool tc = pl->kernel == LSE_KERNEL_TCGEN05, pf = pl->kernel == LSE_KERNEL_PREFILL;
+  info->stages = tc || pf ? pl->stages : 0;
   info->q_slots = tc ? pl->q_slots : 0;
   info->p_bufs = tc ? pl->p_bufs : 0;
-  info->rows_per_chunk = tc ? pl->rows_per_chunk : 0;
+  info->rows_per_chunk = tc || pf ? pl->rows_per_chunk : 0;
   info->scaled = pl->scaled;
   return LSE_OK;
 }
 
 void lse_attn_plan_destroy(lse_attn_plan_t *pl) { delete pl; }
 
+int lse_attn_test_withhold_tile(lse_attn_plan_t *pl, int tile) {
+  if (!pl || tile < -1) return LSE_ERR_INVALID_ARG;
+  if (pl->kernel != LSE_KERNEL_TCGEN05) return LSE_ERR_UNSUPPORTED;
+  pl->withhold_tile = tile;
+  return LSE_OK;
+}
+
 int lse_attn_workspace_init(const lse_attn_plan_t *pl, void *ws, void *stream, char **err) {
   if (!pl || !ws) return fail(err, LSE_ERR_INVALID_ARG, "plan or workspace is NULL");
-  int ce = (int)cudaMemsetAsync(ws, 0, kWsHeader, reinterpret_cast<cudaStream_t>(stream));
+  // the error word and the fused merge's segment counters
+  int ce = (int)cudaMemsetAsync(ws, 0, pl->ws_o_off, reinterpret_cast<cudaStream_t>(stream));
   if (ce) return cuda_fail(err, ce, "cudaMemsetAsync");
   return LSE_OK;
 }
@@ -419,6 +462,7 @@ static int fill_params(const lse_attn_plan_t *pl, void *ws, LseKernelParams &p, 
   p.rows_per_chunk = pl->rows_per_chunk > 0 ? pl->rows_per_chunk : 1;
   char *base = static_cast<char *>(ws);
   p.err = reinterpret_cast<unsigned int *>(base);
+  p.seg_count = reinterpret_cast<unsigned int *>(base + pl->ws_cnt_off);
   p.o_part = reinterpret_cast<float *>(base + pl->ws_o_off);
   p.lse_part = reinterpret_cast<float *>(base + pl->ws_lse_off);
   return LSE_OK;
@@ -469,10 +513,13 @@ int lse_kv_append(const lse_kv_arena *a, int n_seqs, int max_pages, const float 
   return LSE_OK;
 }
 
-int lse_attn_run(const lse_attn_plan_t *pl, const float *q, const int32_t *k_pages,
-                 const int32_t *v_pages, const int32_t *seq_lens, const int32_t *row_offsets,
-                 const uint64_t *row_masks, float softmax_scale, void *ws, void *stream,
-                 char **err) {
+// The partial pass; with `fused` (tensor-core plans only) the same launch
+// also merges and writes out / lse_out.
+static int launch_partial(const lse_attn_plan_t *pl, const float *q, const int32_t *k_pages,
+                          const int32_t *v_pages, const int32_t *seq_lens,
+                          const int32_t *row_offsets, const uint64_t *row_masks,
+                          float softmax_scale, void *ws, float *out, float *lse_out, int fused,
+                          void *stream, char **err) {
   if (!pl) return fail(err, LSE_ERR_INVALID_ARG, "plan is NULL");
   if (!q || !k_pages || !v_pages || !seq_lens || !row_offsets || !ws)
     return fail(err, LSE_ERR_INVALID_ARG, "a required device pointer is NULL");
@@ -488,8 +535,16 @@ int lse_attn_run(const lse_attn_plan_t *pl, const float *q, const int32_t *k_pag
   p.seq_lens = seq_lens;
   p.row_offsets = row_offsets;
   p.row_masks = reinterpret_cast<const unsigned long long *>(row_masks);
+  p.out = out;
+  p.lse_out = lse_out;
   int ce = 0;
-  if (pl->kernel == LSE_KERNEL_TCGEN05) {
+  if (pl->kernel == LSE_KERNEL_PREFILL && !fused)
+    return fail(err, LSE_ERR_UNSUPPORTED, "a long-query-block plan (more than %d rows per "
+                "sequence) runs through lse_attn_forward", LSE_MAX_ROWS_PER_SEQ);
+  if (pl->kernel == LSE_KERNEL_PREFILL && row_masks)
+    return fail(err, LSE_ERR_INVALID_ARG, "row masks take at most %d rows per sequence; a "
+                "long query block is a chain (row_masks = NULL)", LSE_MAX_ROWS_PER_SEQ);
+  if (pl->kernel != LSE_KERNEL_CUDA_CORE) {
     const lse_kv_arena *a = pl->arena;
     const int nch = int(a->chunk_base.size());
     if (nch > LSE_MAX_TMA_CHUNKS)  // (the arena itself holds at most this many)
@@ -506,10 +561,14 @@ int lse_attn_run(const lse_attn_plan_t *pl, const float *q, const int32_t *k_pag
       }
       pl->maps_chunks = nch;
     }
-    ce = lse_launch_partial_tcgen05(p, pl->maps.data(), nch, pl->dtype, pl->pairs_bucket,
-                                    pl->scaled, pl->ctas, pl->n_splits, pl->stages, pl->q_slots,
-                                    pl->p_bufs, pl->box_tokens,
-                                    pl->smem_bytes, stream);
+    if (pl->kernel == LSE_KERNEL_PREFILL)
+      ce = lse_launch_prefill_tcgen05(p, pl->maps.data(), nch, pl->dtype, pl->ctas, pl->stages,
+                                      pl->box_tokens, pl->smem_bytes, stream);
+    else
+      ce = lse_launch_partial_tcgen05(p, pl->maps.data(), nch, pl->dtype, pl->pairs_bucket,
+                                      pl->scaled, pl->ctas, pl->n_splits, pl->stages,
+                                      pl->q_slots, pl->p_bufs, pl->box_tokens, pl->smem_bytes,
+                                      fused, pl->withhold_tile, stream);
   } else {
     ce = lse_launch_partial_cuda_core(p, pl->dtype, pl->head_dim, pl->n_splits, pl->n_kv_heads,
                                       pl->n_seqs, pl->smem_bytes, stream);
@@ -518,9 +577,35 @@ int lse_attn_run(const lse_attn_plan_t *pl, const float *q, const int32_t *k_pag
   return LSE_OK;
 }
 
+int lse_attn_run(const lse_attn_plan_t *pl, const float *q, const int32_t *k_pages,
+                 const int32_t *v_pages, const int32_t *seq_lens, const int32_t *row_offsets,
+                 const uint64_t *row_masks, float softmax_scale, void *ws, void *stream,
+                 char **err) {
+  return launch_partial(pl, q, k_pages, v_pages, seq_lens, row_offsets, row_masks,
+                        softmax_scale, ws, nullptr, nullptr, 0, stream, err);
+}
+
+int lse_attn_forward(const lse_attn_plan_t *pl, const float *q, const int32_t *k_pages,
+                     const int32_t *v_pages, const int32_t *seq_lens, const int32_t *row_offsets,
+                     const uint64_t *row_masks, float softmax_scale, void *ws, float *out,
+                     float *lse_out, void *stream, char **err) {
+  if (!pl) return fail(err, LSE_ERR_INVALID_ARG, "plan is NULL");
+  if (!out) return fail(err, LSE_ERR_INVALID_ARG, "out is NULL");
+  if (pl->kernel != LSE_KERNEL_CUDA_CORE)
+    return launch_partial(pl, q, k_pages, v_pages, seq_lens, row_offsets, row_masks,
+                          softmax_scale, ws, out, lse_out, 1, stream, err);
+  const int st = launch_partial(pl, q, k_pages, v_pages, seq_lens, row_offsets, row_masks,
+                                softmax_scale, ws, nullptr, nullptr, 0, stream, err);
+  if (st) return st;
+  return lse_attn_merge(pl, seq_lens, row_offsets, ws, out, lse_out, stream, err);
+}
+
 int lse_attn_merge(const lse_attn_plan_t *pl, const int32_t *seq_lens, const int32_t *row_offsets,
                    const void *ws, float *out, float *lse_out, void *stream, char **err) {
   if (!pl) return fail(err, LSE_ERR_INVALID_ARG, "plan is NULL");
+  if (pl->kernel == LSE_KERNEL_PREFILL)
+    return fail(err, LSE_ERR_UNSUPPORTED, "a long-query-block plan runs through "
+                "lse_attn_forward");
   if (!seq_lens || !row_offsets || !ws || !out)
     return fail(err, LSE_ERR_INVALID_ARG, "a required device pointer is NULL");
   LseKernelParams p;
@@ -545,7 +630,9 @@ int lse_attn_read_error(const lse_attn_plan_t *pl, void *ws, void *stream, uint3
   uint32_t v = 0;
   int ce = (int)cudaMemcpyAsync(&v, ws, sizeof v, cudaMemcpyDeviceToHost, st);
   if (!ce) ce = (int)cudaStreamSynchronize(st);
-  if (!ce) ce = (int)cudaMemsetAsync(ws, 0, sizeof v, st);
+  // after a fault the fused merge's segment counters may be left part-way:
+  // clear them with the error word
+  if (!ce) ce = (int)cudaMemsetAsync(ws, 0, v ? pl->ws_o_off : sizeof v, st);
   if (ce) return cuda_fail(err, ce, "reading the device error word");
   *device_error = v;
   return LSE_OK;
@@ -583,6 +670,9 @@ int lse_attn_validate(const lse_attn_plan_t *pl, const int32_t *k_pages, const i
                       s, which ? "V" : "K", (long long)pg, f);
       }
     }
+    if (row_masks && R > LSE_MAX_ROWS_PER_SEQ)
+      return fail(err, LSE_ERR_BAD_INPUT, "sequence %d: %d rows with masks (masks take at "
+                  "most %d rows)", s, R, LSE_MAX_ROWS_PER_SEQ);
     for (int r = 0; r < R && row_masks; ++r) {
       const uint64_t m = row_masks[row_offsets[s] + r];
       if (!((m >> r) & 1u))

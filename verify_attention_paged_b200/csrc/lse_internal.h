@@ -55,12 +55,15 @@ struct lse_attn_plan_s {
   int rows_per_chunk = 0;  // tensor-core kernel: query rows per segment
   int box_tokens = 0;    // its TMA box height
   int scaled = 0;        // made for an arena with per-vector scales
+  int withhold_tile = -1;  // tests of the bounded waits (lse_attn_test_withhold_tile)
   // tensor maps of the arena chunks (built on first run, rebuilt on growth);
   // maps_mutex guards them, so threads may run one plan at the same time
   mutable std::vector<uint8_t> maps;
   mutable int maps_chunks = 0;
   mutable std::mutex maps_mutex;
   size_t ws_bytes = 0;
+  size_t ws_cnt_off = 0; // tensor-core kernel: per-segment counters of the fused merge
+  int n_seg_max = 0;     //   (two uint32 per segment), zeroed by lse_attn_workspace_init
   size_t ws_o_off = 0;   // partial outputs  FP32 [rows][Hq][n_splits][D]
   size_t ws_lse_off = 0; // partial lse (log2 units) FP32 [rows][Hq][n_splits]
 };
@@ -103,6 +106,8 @@ struct LseKernelParams {
   // per-vector scales: a [kv_head][token] FP32 block per fragment id, or
   // null for unit scales
   const float *scales;
+  // tensor-core kernel with the merge fused: two counters per segment
+  unsigned int *seg_count;
 };
 
 // Arguments of the K/V append kernel (lse_append.cu).
@@ -146,4 +151,10 @@ int lse_tc_build_maps(const uint64_t *chunk_base, int n_chunks, size_t chunk_byt
 int lse_launch_partial_tcgen05(const LseKernelParams &p, const void *maps, int n_maps,
                                int dtype, int p8, int scaled, int n_ctas, int n_slots,
                                int stages, int q_slots, int p_bufs, int box_tokens, int smem,
-                               void *stream);
+                               int fused, int withhold_tile, void *stream);
+// long query blocks (lse_prefill.cu)
+int lse_pf_row_tile();
+int lse_pf_max_row_tiles();
+int lse_pf_smem(int dtype, int smem_optin, int *stages);
+int lse_launch_prefill_tcgen05(const LseKernelParams &p, const void *maps, int n_maps, int dtype,
+                               int n_ctas, int stages, int box_tokens, int smem, void *stream);

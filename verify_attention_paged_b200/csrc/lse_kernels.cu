@@ -458,8 +458,8 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
     const long long first = before + ((long long)(r / Rc) * p.n_kv_heads + g) * n_s;
     const long long last = first + n_s - 1;
     const long long C = U < p.n_ctas ? U : p.n_ctas;  // working CTAs of the partial pass
-    // two partials (one per softmax group) per piece
-    n_live = n_s > 0 ? 2 * (int(((last + 1) * C - 1) / U - ((first + 1) * C - 1) / U) + 1) : 0;
+    // one partial per piece (the CTA combines its two softmax groups)
+    n_live = n_s > 0 ? int(((last + 1) * C - 1) / U - ((first + 1) * C - 1) / U) + 1 : 0;
   } else if (live_row) {
     n_live = min((L + p.keys_per_split - 1) / p.keys_per_split, p.n_splits);
   }

@@ -65,14 +65,16 @@
 
 #include "lse_internal.h"
 #include "lse_smem_attr.h"
+#include "lse_tc_ptx.h"
 
 namespace {
+
+using namespace lse_ptx;
 
 constexpr int kTK = 128;           // keys per tile = M of the score product
 constexpr int kD = 128;            // head dim = M of the output product
 constexpr int kThreads = 384;
 constexpr float kTau = 8.f;        // lazy-rescale threshold (log2 units)
-constexpr long long kWaitCycles = 4000000000ll;  // ~2 s at 2 GHz
 constexpr int kRegionBytes = kTK * 128;          // 128 rows x 128 B (64 dims)
 
 struct __align__(64) TcParams {
@@ -84,203 +86,9 @@ struct __align__(64) TcParams {
   int q_slots;
   int p_bufs;
   int box_tokens;
+  int fused;  // 1: the merge runs in this pass and writes p.out / p.lse_out
+  int withhold_tile;  // tests of the bounded waits: each CTA's tile of this index is not loaded
 };
-
-// ---- PTX helpers --------------------------------------------------------------
-
-__device__ __forceinline__ uint32_t smem_u32(const void *ptr) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(ptr));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// As mbar_try_wait, but a thread whose phase is not complete is suspended
-// (until the phase completes, or for at most about a microsecond) instead of
-// returning at once, so waiting warps leave their issue slots to the warps
-// doing work.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity), "n"(1000)
-      : "memory");
-  return ok != 0;
-}
-
-// Slow path of mbar_wait (out of line: it runs only when the phase is not
-// complete at the first test).
-__device__ __noinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity,
-                                            volatile int *abort_flag, unsigned int *err) {
-  const long long t0 = clock64();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait_sleep(bar, parity)) return true;
-    if ((i & 3u) == 0) {
-      if (*abort_flag) return false;
-      if (clock64() - t0 > kWaitCycles) {
-        *abort_flag = 1;
-        atomicOr(err, LSE_DEVERR_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
-
-// Wait for the phase of `bar` with the given parity; false when the wait ran
-// out (then the CTA-wide abort flag is set) or another role aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                          unsigned int *err) {
-  return mbar_try_wait(bar, parity) || mbar_wait_spin(bar, parity, abort_flag, err);
-}
-
-// Time-bounded wait that ignores the abort flag: used to drain copies and
-// MMAs already in flight before the CTA releases TMEM and exits.
-__device__ __noinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
-  const long long t0 = clock64();
-  while (!mbar_try_wait_sleep(bar, parity))
-    if (clock64() - t0 > kWaitCycles) return;
-}
-
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void named_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-__device__ __forceinline__ bool named_or(int id, int n, bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred a, b;\n\t"
-      "setp.ne.u32 a, %1, 0;\n\t"
-      "bar.red.or.pred b, %2, %3, a;\n\t"
-      "selp.u32 %0, 1, 0, b;\n\t}\n"
-      : "=r"(r)
-      : "r"((uint32_t)v), "r"(id), "r"(n)
-      : "memory");
-  return r != 0;
-}
-
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
-                                            int x, int y, int z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
-      : "memory");
-}
-
-// Plain bulk copy global -> shared (no tensor map, no multicast), counted
-// on an mbarrier's transaction bytes.  Both addresses 16-byte aligned, bytes
-// a multiple of 16.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
-                                          uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-      : "memory");
-}
-
-// UMMA shared-memory matrix descriptor.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
-                                              uint32_t layout) {
-  return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
-}
-constexpr uint32_t kLayoutNone = 0;
-constexpr uint32_t kLayoutSw128 = 2;
-
-// Instruction descriptor, FP32 accumulation.  Formats: kind::f16 takes
-// 0 = F16, 1 = BF16 (A and B alike); kind::f8f6f4 takes 0 = E4M3, 1 = E5M2
-// for A and B independently.  a_mn / b_mn: 1 = MN-major operand.
-__host__ __device__ constexpr uint32_t instr_desc(uint32_t a_fmt, uint32_t b_fmt, uint32_t a_mn,
-                                                  uint32_t b_mn, uint32_t M, uint32_t N) {
-  return (1u << 4) | (a_fmt << 7) | (b_fmt << 10) | (a_mn << 15) | (b_mn << 16) |
-         ((N >> 3) << 17) | ((M >> 4) << 24);
-}
-
-// One lane of the warp (elect.sync): 1 in that lane, 0 in the others.
-__device__ __forceinline__ uint32_t elect_one() {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred e;\n\t.reg .b32 x;\n\t"
-      "elect.sync x|e, 0xffffffff;\n\t"
-      "selp.u32 %0, 1, 0, e;\n\t}\n"
-      : "=r"(r));
-  return r;
-}
-
-// The MMA issue helpers run in all lanes of a converged warp with the same
-// operands; only the lane with `leader` set issues.
-__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                        uint32_t accumulate, uint32_t leader) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "setp.ne.b32 e, %5, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(leader)
-      : "memory");
-}
-// 8-bit operands, K = 32 per instruction.
-__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                       uint32_t accumulate, uint32_t leader) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "setp.ne.b32 e, %5, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(leader)
-      : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint32_t bar, uint32_t leader) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\t"
-      "setp.ne.b32 e, %1, 0;\n\t"
-      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(bar),
-      "r"(leader)
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float *v) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
-          taddr),
-      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
-      : "memory");
-}
-__device__ __forceinline__ void tmem_st_wait() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
 
 // ---- work decomposition ---------------------------------------------------------
 
@@ -306,10 +114,10 @@ __device__ __forceinline__ int seq_chunks(const LseKernelParams &p, int R) {
 
 // Per-sequence record built once per CTA in shared memory (sequences up to
 // kSeqTab): tiles of all segments before the sequence, its 128-key tiles,
-// L, first row, R.
+// L, first row, R, and the number of segments before the sequence.
 constexpr int kSeqTab = 256;
 struct SeqRec {
-  int prefix, n_tiles, L, row0, R;
+  int prefix, n_tiles, L, row0, R, seg_prefix;
 };
 
 // Walks the CTA's contiguous range of global tiles, segment by segment.  The
@@ -321,6 +129,7 @@ struct TileIter {
   int s, c, g, tile, n_tiles;  // segment (sequence, row chunk, kv head), tile within it
   int n_chunks;
   int L, row0, R;              // the sequence
+  int seg_id;                  // index of the segment among all segments of the call
   long long seg_first;         // global index of the segment's first tile
   long long t, t_end;          // current / end global tile
   const SeqRec *tab;           // shared-memory sequence table or null
@@ -354,7 +163,9 @@ struct TileIter {
     tab = table;
     s = 0;
     long long base = 0;
+    int seg_base = 0;
     n_tiles = 0;
+    seg_id = 0;
     if (t >= t_end) return;
     if (tab) {
       // last sequence whose first tile is at or before t (idle sequences share
@@ -367,11 +178,13 @@ struct TileIter {
       }
       s = lo;
       base = tab[s].prefix;
+      seg_base = tab[s].seg_prefix;
       next_seq(p);
     } else {
       next_seq(p);
       while (base + (long long)n_chunks * p.n_kv_heads * n_tiles <= t) {
         base += (long long)n_chunks * p.n_kv_heads * n_tiles;
+        seg_base += n_chunks * p.n_kv_heads;
         ++s;
         next_seq(p);
       }
@@ -381,6 +194,7 @@ struct TileIter {
     g = sg - c * p.n_kv_heads;
     tile = int((t - base) - (long long)sg * n_tiles);
     seg_first = base + (long long)sg * n_tiles;
+    seg_id = seg_base + sg;
   }
   __device__ bool valid() const { return t < t_end; }
   __device__ bool seg_start(long long t_begin) const { return t == t_begin || tile == 0; }
@@ -397,6 +211,7 @@ struct TileIter {
     if (++tile == n_tiles) {
       tile = 0;
       seg_first += n_tiles;
+      ++seg_id;
       if (++g == p.n_kv_heads) {
         g = 0;
         if (++c == n_chunks) {
@@ -556,6 +371,20 @@ __device__ __forceinline__ void column_reduce(const float *tile, int t, float *o
   }
 }
 
+// A segment this CTA shares with other CTAs, merged after the CTA's own
+// tiles when the merge is fused into the pass (at most two per CTA: the
+// first and the last segment of its range; every segment in between lies
+// in this CTA alone).
+struct EndRec {
+  int seg_id, n_pieces, piece, row0, rows, g;
+};
+// shared memory of the epilogue and end phase: each group's published
+// per-pair maximum and row sum and its "had a tile" flag, double-buffered
+// by segment parity [2][2][64] x 2 + [2][2], then up to two end records and
+// their count
+constexpr int kPubBytes = 2 * 2 * 64 * 4 * 2 + 2 * 2 * 4;
+constexpr int kEndBytes = kPubBytes + 2 * 4 + 2 * (int)sizeof(EndRec) + 8;
+
 // ---- shared-memory and TMEM layout ------------------------------------------------
 
 constexpr bool is_f8(int dt) { return dt == LSE_KV_FP8_E4M3 || dt == LSE_KV_FP8_E5M2; }
@@ -600,14 +429,14 @@ struct TcLayout {
                                  : kTmemNeed <= 256 ? 256 : 512;
   static_assert(kTmemNeed <= 512, "TMEM holds at most 512 columns");
   static_assert(kSW <= 256 && kN <= 256, "MMA N is at most 256");
-  static constexpr int kBars = 64;
+  static constexpr int kBars = 72;
   // row sums of P per group [2][64] and their per-warp partials
   // [2 groups][2 buffers][4 warps][P8]
   static constexpr int kLBytes = 2 * 64 * 4 + 2 * 2 * 4 * P8 * 4;
   static constexpr int kMiscBytes = kBars * 8 + 16 + 2 * 64 * 4 * 2 + 2 * 4 * 64 * 4 +
                                     2 * 64 * 8 * 2 + 64 * 4 + 8 * 16 + 2 * 32 * 16 * 4 +
                                     (kF8 ? 4 * 64 * 4 : 0) + kLBytes +
-                                    kSeqTab * (int)sizeof(SeqRec);
+                                    kSeqTab * (int)sizeof(SeqRec) + kEndBytes;
   // one K or V tile: 128 keys of 128 dims (two 64-dim regions when 16-bit)
   static constexpr int kHalfStage = kF8 ? kRegionBytes : 2 * kRegionBytes;
   // per-vector scales of one tile, K then V (128 FP32 each), per ring stage
@@ -638,165 +467,8 @@ enum {
   kBarPEmpty = 57,  // [4] = group * 2 + P buffer: the P tile has been read
   kBarDoneV = 61,   // the output issuer's MMAs have completed
   kBarSEmpty = 62,  // [2] per softmax group: its score buffer has been read out
+  kBarEpiMeet = 64, // [2] per output slot: both groups' sums and maxima of a piece are in
 };
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ float lg2(float x) {
-  float y;
-  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ float rcp(float x) {
-  float y;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// Two FP32 values -> packed hi (nearest 16-bit) and lo (its rounding error).
-template <int DT>
-__device__ __forceinline__ void split2(float x0, float x1, uint32_t &hi, uint32_t &lo);
-template <>
-__device__ __forceinline__ void split2<LSE_KV_BF16>(float x0, float x1, uint32_t &hi,
-                                                    uint32_t &lo) {
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(hi) : "f"(x1), "f"(x0));
-  const float h0 = __uint_as_float(hi << 16), h1 = __uint_as_float(hi & 0xffff0000u);
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(lo) : "f"(x1 - h1), "f"(x0 - h0));
-}
-template <>
-__device__ __forceinline__ void split2<LSE_KV_F16>(float x0, float x1, uint32_t &hi,
-                                                   uint32_t &lo) {
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(hi) : "f"(x1), "f"(x0));
-  const float2 h = __half22float2(*reinterpret_cast<const __half2 *>(&hi));
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(lo) : "f"(x1 - h.y), "f"(x0 - h.x));
-}
-
-// Two FP32 values -> the nearest 8-bit pair (x1 in the high byte, saturating
-// at the format's largest finite value), and the values that pair decodes
-// to (exactly, through F16, which holds every E4M3 and E5M2 value).
-template <bool kE5>
-__device__ __forceinline__ uint32_t f8x2(float x0, float x1, float &d0, float &d1) {
-  uint16_t r;
-  uint32_t h;
-  if (kE5) {
-    asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(x1), "f"(x0));
-    asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h) : "h"(r));
-  } else {
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(x1), "f"(x0));
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(r));
-  }
-  const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h));
-  d0 = f.x;
-  d1 = f.y;
-  return r;
-}
-
-// Eight FP32 values -> kTerms 8-byte words of 8-bit values whose sum is the
-// input up to the last term's rounding (each term takes the remainder left
-// by the ones before it; the subtractions are exact).
-template <bool kE5, int kTerms>
-__device__ __forceinline__ void f8_terms(float *x, uint2 *out) {
-#pragma unroll
-  for (int t = 0; t < kTerms; ++t) {
-    uint32_t w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float d0, d1;
-      w[i] = f8x2<kE5>(x[2 * i], x[2 * i + 1], d0, d1);
-      x[2 * i] -= d0;
-      x[2 * i + 1] -= d1;
-    }
-    out[t] = make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
-  }
-}
-
-// Eight FP32 values -> F16 (round to nearest), then kTerms E5M2 terms of
-// the F16 values.  E5M2 has F16's sign and exponent fields, so every E5M2
-// value is an F16 value and the nearest E5M2 of an F16 (round to nearest,
-// ties to even) leaves a remainder that F16 holds exactly: each term is the
-// hardware conversion of the remainder so far, converted back and
-// subtracted (an exact F16 subtraction).  Four terms of 3 significant bits
-// hold all 11 bits of an F16.  (The inputs stay far below E5M2's largest
-// finite value, so the saturating conversion never clips.)
-template <int kTerms>
-__device__ __forceinline__ void e5_terms_f16(const float *x, uint2 *out) {
-  uint32_t h[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h[i]) : "f"(x[2 * i + 1]), "f"(x[2 * i]));
-#pragma unroll
-  for (int t = 0; t < kTerms; ++t) {
-    uint32_t w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint16_t e;
-      asm("cvt.rn.satfinite.e5m2x2.f16x2 %0, %1;" : "=h"(e) : "r"(h[i]));
-      w[i] = e;
-      if (t + 1 < kTerms) {
-        uint32_t back;
-        asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(back) : "h"(e));
-        asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(h[i]) : "r"(h[i]), "r"(back));
-      }
-    }
-    out[t] = make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
-  }
-}
-
-// 2^e as a float, e in [-126, 127].
-__device__ __forceinline__ float exp2i(int e) { return __int_as_float((e + 127) << 23); }
-
-// TMEM: this thread's lane, N consecutive 32-bit columns (N a multiple of 8),
-// one wait for all of them.  The TMEM loads carry no memory clobber (TMEM is
-// not memory the compiler tracks): volatile keeps them in order with the
-// barrier waits and fences, and shared-memory traffic may overlap them.
-template <int N>
-__device__ __forceinline__ void tmem_load(uint32_t taddr, float *v) {
-  static_assert(N % 8 == 0, "columns in groups of 8");
-  uint32_t r[N];
-#pragma unroll
-  for (int c = 0; c < N; c += 8)
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-        : "=r"(r[c]), "=r"(r[c + 1]), "=r"(r[c + 2]), "=r"(r[c + 3]), "=r"(r[c + 4]),
-          "=r"(r[c + 5]), "=r"(r[c + 6]), "=r"(r[c + 7])
-        : "r"(taddr + c));
-  asm volatile("tcgen05.wait::ld.sync.aligned;");
-  // tie every register to the wait so no use is scheduled above it
-#pragma unroll
-  for (int c = 0; c < N; ++c) {
-    asm volatile("" : "+r"(r[c]));
-    v[c] = __uint_as_float(r[c]);
-  }
-}
-
-// TMEM: this thread's lane, 8 columns from each of T blocks `stride`
-// columns apart, summed in block order; one wait for all loads.
-template <int T>
-__device__ __forceinline__ void tmem_load_sum8(uint32_t taddr, int stride, float *v) {
-  uint32_t r[T][8];
-#pragma unroll
-  for (int t = 0; t < T; ++t)
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-        : "=r"(r[t][0]), "=r"(r[t][1]), "=r"(r[t][2]), "=r"(r[t][3]), "=r"(r[t][4]),
-          "=r"(r[t][5]), "=r"(r[t][6]), "=r"(r[t][7])
-        : "r"(taddr + (uint32_t)(t * stride)));
-  asm volatile("tcgen05.wait::ld.sync.aligned;");
-#pragma unroll
-  for (int t = 0; t < T; ++t)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) asm volatile("" : "+r"(r[t][c]));
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    float a = __uint_as_float(r[0][c]);
-#pragma unroll
-    for (int t = 1; t < T; ++t) a += __uint_as_float(r[t][c]);
-    v[c] = a;
-  }
-}
 
 // Sum of eight per-lane values over the 32 lanes of a warp, by a fixed
 // butterfly (halving the values each lane keeps, then full sums): every
@@ -926,6 +598,83 @@ __device__ __forceinline__ bool stage_q(const LseKernelParams &p, int t, int g, 
   return true;
 }
 
+// End phase of the fused pass: for each segment this CTA shares with other
+// CTAs, wait until every piece's partial is written (the segment's arrival
+// count reaches two per piece), then merge this CTA's share of the
+// segment's (pair, dim) outputs: share k of n covers elements
+// [k E / n, (k+1) E / n) of the E = pairs x D outputs, each the
+// log-sum-exp-weighted mean of the pieces' partials (the same merge as the
+// separate merge pass).  The last CTA to finish a segment clears its two
+// counters for the next call.  The wait is bounded like every other wait;
+// the launch is cooperative, so every CTA of the grid is resident and each
+// arrives for its own pieces without waiting on any other CTA.
+__device__ __noinline__ void fused_end_merge(const TcParams &tp, const EndRec *rec, int n_rec,
+                                             volatile int *abort_flag, int *go_flag) {
+  const LseKernelParams &p = tp.p;
+  const int tid = threadIdx.x;
+#pragma unroll 1
+  for (int k = 0; k < n_rec; ++k) {
+    const EndRec r = rec[k];
+    unsigned int *cnt = p.seg_count + 2 * r.seg_id;
+    if (tid == 0) {
+      int go = *abort_flag == 0;
+      const long long t0 = clock64();
+      while (go) {
+        unsigned int v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
+        if (v >= 2u * (unsigned)r.n_pieces) break;
+        if (clock64() - t0 > kWaitCycles) {
+          *abort_flag = 1;
+          atomicOr(p.err, LSE_DEVERR_TIMEOUT);
+          go = 0;
+        }
+        __nanosleep(256);
+      }
+      *go_flag = go;
+    }
+    __syncthreads();
+    const bool go = *go_flag != 0;
+    if (go) {
+      const int G = p.group;
+      const long long E = (long long)G * r.rows * kD;
+      const long long e0 = E * r.piece / r.n_pieces, e1 = E * (r.piece + 1) / r.n_pieces;
+#pragma unroll 1
+      for (long long e = e0 + tid; e < e1; e += kThreads) {
+        const int q = (int)(e / kD), d = (int)(e - (long long)q * kD);
+        const int rr = q / G, h = r.g * G + (q - rr * G);
+        const long long oi = (long long)(r.row0 + rr) * p.n_q_heads + h;
+        const long long base = oi * tp.n_slots;
+        // partials written by other CTAs: read through L2
+        float M = -INFINITY;
+#pragma unroll 4
+        for (int i = 0; i < r.n_pieces; ++i) M = fmaxf(M, __ldcg(p.lse_part + base + i));
+        float W = 0.f, acc = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll 4
+          for (int i = 0; i < r.n_pieces; ++i) {
+            const float l = __ldcg(p.lse_part + base + i);
+            const float w = l == -INFINITY ? 0.f : ex2(l - M);
+            W += w;
+            acc = fmaf(w, __ldcg(p.o_part + (base + i) * kD + d), acc);
+          }
+        }
+        p.out[oi * kD + d] = W > 0.f ? acc * rcp(W) : 0.f;
+        if (d == 0 && p.lse_out)
+          p.lse_out[oi] = W > 0.f ? (M + lg2(W)) * 0.69314718055994530942f : -INFINITY;
+      }
+    }
+    __syncthreads();
+    if (tid == 0 && go) {
+      // leaving the segment: the last CTA out clears its counters
+      const unsigned int left = atomicAdd(cnt + 1, 1u);
+      if (left + 1u == (unsigned)r.n_pieces) {
+        atomicExch(cnt, 0u);
+        atomicExch(cnt + 1, 0u);
+      }
+    }
+  }
+}
+
 template <int DT, int P8, bool kSc>
 __global__ void __launch_bounds__(kThreads, 1)
     partial_tcgen05_kernel(const __grid_constant__ TcParams tp) {
@@ -981,6 +730,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   float *lsum_all = isig_all + (kF8 ? 4 * 64 : 0);                           // [2][64]
   float *lpart_all = lsum_all + 2 * 64;                                      // [2][2][4][P8]
   SeqRec *seq_tab = reinterpret_cast<SeqRec *>(lpart_all + 2 * 2 * 4 * P8);  // [kSeqTab]
+  // per-pair statistics a group publishes for the other one at a piece's
+  // end: [segment parity][group][pair]; a group resets its own running
+  // state at the next segment while the other may still be reading these
+  float *pub_m = reinterpret_cast<float *>(seq_tab + kSeqTab);              // [2][2][64]
+  float *pub_l = pub_m + 2 * 2 * 64;                                         // [2][2][64]
+  int *pub_had = reinterpret_cast<int *>(pub_l + 2 * 2 * 64);                // [2][2]
+  int *had_all = pub_had + 4;                                                // [2] (end phase)
+  EndRec *end_rec = reinterpret_cast<EndRec *>(had_all + 2);                 // [2]
+  int *n_end = reinterpret_cast<int *>(end_rec + 2);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
   // the merge pass may be scheduled now; it waits for this grid to finish
@@ -1009,7 +767,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bad = true;
         n = 0;
       }
-      if (use_tab) seq_tab[q] = SeqRec{0, n, L, r0, R};
+      if (use_tab) seq_tab[q] = SeqRec{0, n, L, r0, R, 0};
       // all segments of the sequence: row chunks x kv heads
       mine += (long long)n * (n > 0 ? seq_chunks(p, R) : 0) * p.n_kv_heads;
     }
@@ -1020,11 +778,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane >= o) incl += v;
     }
     if (use_tab) {
+      // segments of the lanes before this one (a second warp scan)
+      int segs = 0;
+      for (int q = s0; q < s1; ++q) {
+        const int n = seq_tab[q].n_tiles;
+        segs += n > 0 ? seq_chunks(p, seq_tab[q].R) * p.n_kv_heads : 0;
+      }
+      int seg_incl = segs;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, seg_incl, o);
+        if (lane >= o) seg_incl += v;
+      }
       long long run = incl - mine;
+      int seg_run = seg_incl - segs;
       for (int q = s0; q < s1; ++q) {
         seq_tab[q].prefix = (int)run;
+        seq_tab[q].seg_prefix = seg_run;
         const int n = seq_tab[q].n_tiles;
         run += (long long)n * (n > 0 ? seq_chunks(p, seq_tab[q].R) : 0) * p.n_kv_heads;
+        seg_run += n > 0 ? seq_chunks(p, seq_tab[q].R) * p.n_kv_heads : 0;
       }
     }
     bad = __any_sync(0xffffffffu, bad);
@@ -1042,8 +815,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(bar(kBarOFull + i), 1);
-      mbar_init(bar(kBarOEmpty + i), 128);
+      // both softmax groups read both groups' output blocks of a piece
+      mbar_init(bar(kBarOEmpty + i), 256);
     }
+    for (int i = 0; i < 2; ++i) mbar_init(bar(kBarEpiMeet + i), 256);
+    *n_end = 0;
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarSFull + i), 1);
       mbar_init(bar(kBarSEmpty + i), 128);
@@ -1111,7 +887,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int tt = __shfl_sync(0xffffffffu, mine.tile, i);
         const int tl = __shfl_sync(0xffffffffu, mine.L, i);
         int go = 1;
-        if (lane == 0) {
+        if (lane == 0 && n != tp.withhold_tile) {
           const uint32_t bars_k[2] = {bar(kBarEmptyK + n % NS), bar(kBarFullK + n % NS)};
           const uint32_t bars_v[2] = {bar(kBarEmptyV + n % NS), bar(kBarFullV + n % NS)};
           go = produce_tile(tp, n, NS, nbox, box_t, kF8 ? 1 : 2, tg, tt, tl, pk + i * 16,
@@ -1616,14 +1392,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 
       if (last) {
-        // ---- epilogue of this group's piece: normalised output and log2-sum-exp ----
+        // ---- epilogue of the piece: the two groups' results combined ----
         const bool w = mbar_wait(bar(kBarOFull + 2 * grp + oslot), (seg / kOS) & 1, abort_flag,
                                  p.err);
         if (named_or(bar_id, 128, !w)) {
           ok = false;
           break;
         }
-        const float *lt_of = lsum;  // the group's row sums of P, per pair
         if constexpr (kLAcc) {
           // column sums of the threads' sums, through one of the group's P
           // tiles as FP32 scratch [key][pair] (free: the piece's last P.V has
@@ -1635,44 +1410,99 @@ __global__ void __launch_bounds__(kThreads, 1)
                 make_float4(lacc[c], lacc[c + 1], lacc[c + 2], lacc[c + 3]);
           named_sync(bar_id, 128);
           column_reduce<P8, true>(scr, j, red, bar_id);  // red[q] = sum over keys
-          lt_of = red;
         } else {
           fold();  // the group's last tile's partials
         }
-        named_sync(bar_id, 128);
+        // publish this group's per-pair maximum and row sum (its running
+        // copies are reset at its next segment, maybe before the other group
+        // has read them)
+        const int pb = seg & 1;
+        if (j < P8) {
+          pub_m[(pb * 2 + grp) * 64 + j] = m_run[j];
+          pub_l[(pb * 2 + grp) * 64 + j] = kLAcc ? red[j] : lsum[j];
+        }
+        if (j == 0) pub_had[pb * 2 + grp] = had_tile ? 1 : 0;
+        // this group's row sums, maxima and output block are complete; meet
+        // the other group (an mbarrier wait, so a group that gave up never
+        // leaves the other one waiting)
+        tc_fence_before();
+        mbar_arrive(bar(kBarEpiMeet + oslot));
+        const bool wm = mbar_wait(bar(kBarEpiMeet + oslot), (seg / kOS) & 1, abort_flag, p.err);
+        if (named_or(bar_id, 128, !wm)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         __syncwarp();
+        // the piece: its place among the segment's pieces
         const int c_first = cta_of_tile(it.seg_first, U, C);
-        const int slot = 2 * (cta - c_first) + grp;
+        const int c_last = cta_of_tile(it.seg_first + it.n_tiles - 1, U, C);
+        const int n_pieces = c_last - c_first + 1, piece = cta - c_first;
+        const bool direct = tp.fused && n_pieces == 1;  // the final output, no partial
+        const bool had0 = pub_had[pb * 2] != 0, had1 = pub_had[pb * 2 + 1] != 0;
+        const float *lt0 = pub_l + pb * 2 * 64, *lt1 = lt0 + 64;    // the groups' row sums
+        const float *mx0 = pub_m + pb * 2 * 64, *mx1 = mx0 + 64;    // and maxima
         const int d = j;  // output lane = head dim
-        const uint32_t ob = tmem_o(grp, oslot) + lane_off;
         const long long row_stride = (long long)p.n_q_heads * tp.n_slots * kD;
         const long long base =
-            ((long long)it.crow0(p) * p.n_q_heads + it.g * G) * tp.n_slots + slot;
+            ((long long)it.crow0(p) * p.n_q_heads + it.g * G) * tp.n_slots + piece;
+        // the groups take alternate blocks of 8 pairs
 #pragma unroll 1
-        for (int c = 0; c < P8; c += 8) {
-          float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int c = 8 * grp; c < P8; c += 16) {
+          float o0[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          float o1[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
           // the output blocks (hi and lo, or the P terms) summed
-          if (had_tile) tmem_load_sum8<kN / Lay::kOBlk>(ob + c, Lay::kOBlk, o);
+          if (had0) tmem_load_sum8<kN / Lay::kOBlk>(tmem_o(0, oslot) + lane_off + c, Lay::kOBlk, o0);
+          if (had1) tmem_load_sum8<kN / Lay::kOBlk>(tmem_o(1, oslot) + lane_off + c, Lay::kOBlk, o1);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int q = c + i;
             if (q < P) {
+              const float l0 = lt0[q], l1 = lt1[q];
+              const float m0 = mx0[q], m1 = mx1[q];
+              const float M = l0 > 0.f ? (l1 > 0.f ? fmaxf(m0, m1) : m0) : m1;
+              const float a0 = l0 > 0.f ? ex2(m0 - M) : 0.f;
+              const float a1 = l1 > 0.f ? ex2(m1 - M) : 0.f;
+              const float lt = a0 * l0 + a1 * l1;
+              const float v = lt > 0.f ? (a0 * o0[i] + a1 * o1[i]) * rcp(lt) : 0.f;
+              // log2-sum-exp (FP8 sums carry P's factor 2^7)
+              const float lse2 = lt > 0.f ? M + lg2(lt) - (kF8 ? kPScaleLog2 : 0) : -INFINITY;
               const int r = pair_row[q];
-              const long long idx =
-                  base + r * row_stride / kD + (long long)(q - r * G) * tp.n_slots;
-              const float lt = lt_of[q];
-              p.o_part[idx * kD + d] = lt > 0.f ? o[i] * rcp(lt) : 0.f;
-              // (FP8 sums carry P's factor 2^7)
-              if (d == q)
-                p.lse_part[idx] = lt > 0.f ? m_run[q] + lg2(lt) - (kF8 ? kPScaleLog2 : 0)
-                                           : -INFINITY;
+              const int h = it.g * G + (q - r * G);
+              if (direct) {
+                const long long oi = (long long)(it.crow0(p) + r) * p.n_q_heads + h;
+                p.out[oi * kD + d] = v;
+                if (d == q && p.lse_out) p.lse_out[oi] = lse2 * 0.69314718055994530942f;
+              } else {
+                const long long idx =
+                    base + r * row_stride / kD + (long long)(q - r * G) * tp.n_slots;
+                p.o_part[idx * kD + d] = v;
+                if (d == q) p.lse_part[idx] = lse2;
+              }
             }
           }
         }
+        // both groups have read both output blocks when both have arrived
         tc_fence_before();
-        named_sync(bar_id, 128);
-        mbar_arrive(bar(kBarOEmpty + 2 * grp + oslot));
+        mbar_arrive(bar(kBarOEmpty + oslot));
+        mbar_arrive(bar(kBarOEmpty + 2 + oslot));
+        if (tp.fused && n_pieces > 1) {
+          // this group's share of the piece's partial is written: count it on
+          // the segment (two arrivals per piece); the CTA merges its share of
+          // the segment once every piece is in (end phase)
+          __threadfence();
+          named_sync(bar_id, 128);
+          if (j == 0) {
+            atomicAdd(p.seg_count + 2 * it.seg_id, 1u);
+            if (grp == 0) {
+              const int k = *n_end;
+              if (k < 2) {
+                end_rec[k] = EndRec{it.seg_id, n_pieces, piece, it.crow0(p), it.crows(p), it.g};
+                *n_end = k + 1;
+              }
+            }
+          }
+        }
       }
     }
   }
@@ -1686,6 +1516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(Lay::kTmemCols)
                  : "memory");
+  if (tp.fused) fused_end_merge(tp, end_rec, *n_end, abort_flag, had_all);
 }
 
 // ---- host side ------------------------------------------------------------------------
@@ -1710,8 +1541,23 @@ int launch_tc(const TcParams &tp, int smem, cudaStream_t st) {
   static lse_detail::SmemAllowed allowed;  // per device ordinal
   const int e = lse_detail::allow_dynamic_smem(k, smem, allowed);
   if (e) return e;
-  k<<<tp.n_ctas, kThreads, smem, st>>>(tp);
-  return (int)cudaGetLastError();
+  if (!tp.fused) {
+    k<<<tp.n_ctas, kThreads, smem, st>>>(tp);
+    return (int)cudaGetLastError();
+  }
+  // the fused merge waits (bounded) for other CTAs' pieces: a cooperative
+  // launch, so every CTA of the grid is resident at once (or the launch fails)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(tp.n_ctas);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return (int)cudaLaunchKernelEx(&cfg, k, tp);
 }
 
 template <int DT, bool kSc>
@@ -1819,7 +1665,7 @@ size_t lse_tc_map_bytes() { return sizeof(CUtensorMap); }
 int lse_launch_partial_tcgen05(const LseKernelParams &p, const void *maps, int n_maps,
                                int dtype, int p8, int scaled, int n_ctas, int n_slots,
                                int stages, int q_slots, int p_bufs, int box_tokens, int smem,
-                               void *stream) {
+                               int fused, int withhold_tile, void *stream) {
   static_assert(sizeof(TcParams) < 30000, "kernel parameter block too large");
   TcParams tp;
   memset(&tp, 0, sizeof tp);
@@ -1831,6 +1677,8 @@ int lse_launch_partial_tcgen05(const LseKernelParams &p, const void *maps, int n
   tp.q_slots = q_slots;
   tp.p_bufs = p_bufs;
   tp.box_tokens = box_tokens;
+  tp.fused = fused;
+  tp.withhold_tile = withhold_tile;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   switch (dtype) {
     case LSE_KV_BF16:

@@ -328,6 +328,16 @@ def long_fp8_scaled(keep_logical=False) -> Workload:
                  kv_std=0.5, n_chunks=1, keep_logical=keep_logical, scaled=True)
 
 
+def prefill_block(keep_logical=False) -> Workload:
+    """A long query block (the releases page's prefill chunks of 1024 rows,
+    v0.4.14): 1 sequence of 16384 keys whose last 1024 positions are a chain
+    of query rows over 15360 cached keys, 24/4 heads, head_dim 128, BF16 in
+    256 KiB fragments in shuffled order."""
+    return build("prefill_block", "bf16", [16384], [1024], 24, 4, 128,
+                 fragment_bytes=256 * KIB, chunk_bytes=256 * MIB, max_pages=64, seed=1244,
+                 n_chunks=1, keep_logical=keep_logical)
+
+
 BUILDERS = {
     "tiny_decode": tiny_decode,
     "batched_decode": batched_decode,
@@ -336,9 +346,10 @@ BUILDERS = {
     "tree_verify": tree_verify,
     "long_e5m2": long_e5m2,
     "long_fp8_scaled": long_fp8_scaled,
+    "prefill_block": prefill_block,
 }
 # workloads beyond the five benchmark configurations
-EXTRA_NAMES = ["long_e5m2", "long_fp8_scaled"]
+EXTRA_NAMES = ["long_e5m2", "long_fp8_scaled", "prefill_block"]
 
 
 # ---------------------------------------------------------------------------
