@@ -91,7 +91,8 @@ def attention_flops(w):
 
 # the sources each measured kernel (and its launch plan) is built from
 KERNEL_SOURCES = {
-    "partial": ("lse_host.cpp", "lse_internal.h", "lse_tcgen05.cu"),
+    "partial": ("lse_host.cpp", "lse_internal.h", "lse_tcgen05.cu", "lse_tc_ptx.h"),
+    "prefill": ("lse_host.cpp", "lse_internal.h", "lse_prefill.cu", "lse_tc_ptx.h"),
     "append": ("lse_append.cu", "lse_host.cpp", "lse_internal.h"),
 }
 
@@ -410,7 +411,8 @@ def workload_result(w, call, steps_ms, part_ms, world, dist, args, peak, peak_ki
         tflops = attention_flops(w) / (part_mean * 1e-3) / 1e12
         roof = {"bound": "tensor", "kernel": "long-query-block pass", "achieved": tflops,
                 "peak": tf_peak, "peak_kind": f"{tf_kind} (cuBLAS bf16, burst)",
-                "unit": "TFLOP/s", "frac": tflops / tf_peak, "traffic": ncu_traffic(w.name),
+                "unit": "TFLOP/s", "frac": tflops / tf_peak,
+                "traffic": ncu_traffic(w.name, "prefill"),
                 "algorithmic_flops_per_launch": attention_flops(w)}
         extra = {"tflops": tflops}
     return {

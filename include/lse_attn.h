@@ -232,13 +232,15 @@ typedef struct {
   int32_t smem_bytes;      /* dynamic shared memory of the partial kernel  */
   int32_t ctas;            /* partial-pass CTAs when persistent, else 0     */
   int64_t workspace_bytes;
-  int32_t stages;          /* tensor-core kernel: K/V ring depth, else 0      */
+  int32_t stages;          /* tensor-core kernels: K ring depth (long query
+                              blocks: K/V ring depth), else 0              */
   int32_t q_slots;         /* tensor-core kernel: Q ring depth, else 0        */
   int32_t p_bufs;          /* tensor-core kernel: P tiles per softmax group   */
   int32_t rows_per_chunk;  /* tensor-core kernel: query rows per segment (a
                               sequence with more rows is split into row
                               chunks, each reading its keys), else 0       */
   int32_t scaled;          /* 1: made for an arena with per-vector scales  */
+  int32_t v_stages;        /* verify tensor-core kernel: V ring depth, else 0 */
 } lse_attn_plan_info;
 
 LSE_API int lse_attn_plan_query(const lse_attn_plan_t *plan, lse_attn_plan_info *info);

@@ -161,7 +161,8 @@ def test_per_vector_scales_attach_and_plan():
     info0 = b.lse_attn_plan_query(p0)
     assert info0["scaled"] == 0
     # the scale rows take shared memory from the same ring
-    assert info["smem_bytes"] > info0["smem_bytes"] or info["stages"] < info0["stages"]
+    slots = lambda i: i["stages"] + i["v_stages"]  # noqa: E731  (K and V ring slots)
+    assert info["smem_bytes"] > info0["smem_bytes"] or slots(info) < slots(info0)
     # a plan runs only on an arena in the state it was made for (checked
     # before any launch)
     with pytest.raises(b.LseError, match="scales"):
@@ -315,3 +316,20 @@ def test_long_query_block_plans():
     with pytest.raises(b.LseError, match="16-bit or FP8"):
         b.lse_attn_plan_ex(f, 1, 100, 100, 8, 64, **B200)
     b.lse_kv_arena_destroy(f)
+
+
+def test_benchmark_plans_keep_their_ring_depth():
+    # the shared-memory budget of the tensor-core pass: the benchmark
+    # workloads keep the K/V ring depth that their throughput depends on
+    # (K and V tile slots together)
+    want = {"batched_decode": 6, "chain_verify": 4, "long_fp8": 10, "tree_verify": 4,
+            "long_e5m2": 10}
+    for name, slots in want.items():
+        w = wl.BUILDERS[name]()
+        a, p, _ = _plan_for(w, n_sms=148, smem_optin=232448, ctas_per_sm=0, allow_tcgen05=1)
+        info = b.lse_attn_plan_query(p)
+        assert info["kernel_name"] == "tcgen05", name
+        assert info["stages"] + info["v_stages"] >= slots, (name, info)
+        assert 2 <= info["stages"] <= info["v_stages"] <= 8
+        b.lse_attn_plan_destroy(p)
+        b.lse_kv_arena_destroy(a)

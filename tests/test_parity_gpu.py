@@ -277,6 +277,18 @@ def test_tcgen05_many_segments_per_cta(binding, dtype):
     assert_close(out_tc, out_cc, dtype, what="tcgen05 vs cuda_core")
 
 
+@pytest.mark.parametrize("dtype", ["f16", "e4m3"])
+def test_tcgen05_more_sequences_than_the_cta_table(binding, dtype):
+    # 130 sequences: more than the per-CTA sequence table holds, so the tile
+    # iterator reads lengths from global memory (and numbers segments itself)
+    rng = np.random.default_rng(6)
+    lens = [int(x) for x in rng.integers(1, 900, 130)]
+    rows = [int(min(L, r)) for L, r in zip(lens, rng.integers(0, 5, 130))]
+    w = wl.small_case(dtype, lens, rows, n_q_heads=24, n_kv_heads=4, head_dim=128,
+                      tokens_per_fragment=128, tree=True, seed=227)
+    check_kernel(binding, w, "tcgen05", two_pass=True)
+
+
 @pytest.mark.parametrize("dtype", ["f16", "e5m2"])
 def test_tcgen05_fewer_tiles_than_ctas(binding, dtype):
     w = wl.small_case(dtype, [200], [2], n_q_heads=8, n_kv_heads=2, head_dim=128,

@@ -302,10 +302,10 @@ int lse_attn_plan_ex(const lse_kv_arena *a, int n_seqs, int max_rows, int max_to
   const int rows_per_chunk =
       pl->pairs <= max_tile_pairs ? max_rows : max_tile_pairs / pl->group;
   const int p8 = rows_per_chunk > 0 ? lse_tc_pairs_bucket(pl->group * rows_per_chunk) : -1;
-  int tc_stages = 0, tc_q_slots = 0, tc_p_bufs = 0;
+  int tc_stages = 0, tc_v_stages = 0, tc_q_slots = 0, tc_p_bufs = 0;
   const int tc_smem =
-      p8 > 0 ? lse_tc_smem(a->dtype, p8, pl->scaled, smem_optin, &tc_stages, &tc_q_slots,
-                           &tc_p_bufs)
+      p8 > 0 ? lse_tc_smem(a->dtype, p8, pl->scaled, smem_optin, &tc_stages, &tc_v_stages,
+                           &tc_q_slots, &tc_p_bufs)
              : -1;
   if (max_rows > LSE_MAX_ROWS_PER_SEQ) {
     // a long query block (chain rows only): the rows-as-M tensor-core pass
@@ -345,6 +345,7 @@ int lse_attn_plan_ex(const lse_kv_arena *a, int n_seqs, int max_rows, int max_to
     pl->key_tile = tile;
     pl->smem_bytes = tc_smem;
     pl->stages = tc_stages;
+    pl->v_stages = tc_v_stages;
     pl->q_slots = tc_q_slots;
     pl->p_bufs = tc_p_bufs;
     pl->pairs_bucket = p8;
@@ -409,6 +410,7 @@ int lse_attn_plan_query(const lse_attn_plan_t *pl, lse_attn_plan_info *info) {
   info->p_bufs = tc ? pl->p_bufs : 0;
   info->rows_per_chunk = tc || pf ? pl->rows_per_chunk : 0;
   info->scaled = pl->scaled;
+  info->v_stages = tc ? pl->v_stages : 0;
   return LSE_OK;
 }
 
@@ -567,8 +569,8 @@ static int launch_partial(const lse_attn_plan_t *pl, const float *q, const int32
     else
       ce = lse_launch_partial_tcgen05(p, pl->maps.data(), nch, pl->dtype, pl->pairs_bucket,
                                       pl->scaled, pl->ctas, pl->n_splits, pl->stages,
-                                      pl->q_slots, pl->p_bufs, pl->box_tokens, pl->smem_bytes,
-                                      fused, pl->withhold_tile, stream);
+                                      pl->v_stages, pl->q_slots, pl->p_bufs, pl->box_tokens,
+                                      pl->smem_bytes, fused, pl->withhold_tile, stream);
   } else {
     ce = lse_launch_partial_cuda_core(p, pl->dtype, pl->head_dim, pl->n_splits, pl->n_kv_heads,
                                       pl->n_seqs, pl->smem_bytes, stream);

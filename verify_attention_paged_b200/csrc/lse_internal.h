@@ -48,7 +48,8 @@ struct lse_attn_plan_s {
   int smem_bytes = 0;
   int n_sms = 0;
   int ctas = 0;          // persistent grid of the tensor-core kernel
-  int stages = 0;        // its pipeline depth
+  int stages = 0;        // its K ring depth (prefill: the K/V ring depth)
+  int v_stages = 0;      // its V ring depth
   int q_slots = 0;       // and its Q ring depth
   int p_bufs = 0;        // and its P tiles per softmax group
   int pairs_bucket = 0;  // its compile-time pair count (P8)
@@ -142,16 +143,17 @@ const char *lse_cuda_error_string(int code);
 
 // tensor-core partial pass (lse_tcgen05.cu)
 int lse_tc_pairs_bucket(int pairs);
-int lse_tc_smem(int dtype, int p8, int scaled, int smem_optin, int *stages, int *q_slots,
-                int *p_bufs);
+int lse_tc_smem(int dtype, int p8, int scaled, int smem_optin, int *k_stages, int *v_stages,
+                int *q_slots, int *p_bufs);
 int lse_tc_key_tile();
 size_t lse_tc_map_bytes();
 int lse_tc_build_maps(const uint64_t *chunk_base, int n_chunks, size_t chunk_bytes,
                       int n_kv_heads, int dtype, int box_tokens, void *maps_out);
 int lse_launch_partial_tcgen05(const LseKernelParams &p, const void *maps, int n_maps,
                                int dtype, int p8, int scaled, int n_ctas, int n_slots,
-                               int stages, int q_slots, int p_bufs, int box_tokens, int smem,
-                               int fused, int withhold_tile, void *stream);
+                               int k_stages, int v_stages, int q_slots, int p_bufs,
+                               int box_tokens, int smem, int fused, int withhold_tile,
+                               void *stream);
 // long query blocks (lse_prefill.cu)
 int lse_pf_row_tile();
 int lse_pf_max_row_tiles();

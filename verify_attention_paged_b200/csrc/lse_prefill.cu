@@ -33,9 +33,13 @@
 //    several CTAs share are merged at the end of the launch (log-sum-exp
 //    weights) by those CTAs, after a bounded wait for the others' partials
 //    (a cooperative launch, so all CTAs are resident).
-//  * Roles (192 threads): warp 0 streams K and V tiles through the page
-//    table by TMA, warp 1 issues the MMAs (and owns TMEM), warps 2-5 stage
-//    each segment's Q, run the softmax (thread = row) and write the results.
+//  * Roles (320 threads): warp 0 streams K and V tiles through the page
+//    table by TMA, warp 1 issues the MMAs (and owns TMEM), and two groups of
+//    four warps (2-5 and 6-9) stage each segment's Q, run the softmax and
+//    write the results: thread r of each group holds row r, the first group
+//    the tile's keys 0-63 (and head dims 0-63 of the output), the second
+//    keys 64-127 (dims 64-127); the groups meet at named barriers to share
+//    each row's maximum and sum.
 //    Every wait is bounded and reports LSE_DEVERR_TIMEOUT when it runs out.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -55,7 +59,7 @@ using namespace lse_ptx;
 constexpr int kTK = 128;        // keys per tile = N of the score product
 constexpr int kRT = 128;        // query rows per tile = M of both products
 constexpr int kD = 128;         // head dim = N of the output product
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr float kTau = 8.f;     // lazy-rescale threshold (log2 units)
 constexpr int kRegion = 128 * 128;  // 128 rows x 128 bytes
 constexpr int kQBytes = 4 * kRegion;  // Q terms: 16-bit hi | lo (two regions each), or 4 FP8
@@ -99,19 +103,22 @@ enum {
   kFullV = 16,   // [8]
   kEmptyV = 24,  // [8]
   kSFull = 32,   // [2] score buffer complete
-  kPFull = 34,   // [2] probabilities written over the score buffer (128 arrivals)
+  kPFull = 34,   // [2] probabilities written over the score buffer (256 arrivals)
   kPvDone = 36,  // [2] output product of a tile of this parity complete
-  kQFull = 38,   // Q of a segment staged (128 arrivals)
+  kQFull = 38,   // Q of a segment staged (256 arrivals)
   kQEmpty = 39,  // the segment's score products complete (Q may be replaced)
   kOFull = 40,   // the piece's last output product complete
-  kOEmpty = 41,  // the piece's output read out (128 arrivals)
+  kOEmpty = 41,  // the piece's output read out (256 arrivals)
   kDoneMma = 42, // every MMA issued has completed
   kInfo = 43,    // [8] tile records
   kBarsPf = 56,
 };
 
+// exchange of the two softmax groups: per row, partial maxima [2 tiles][2
+// groups][128], partial sums [2 groups][128], Q maxima [2 groups][128]
+constexpr int kXchBytes = (2 * 2 * 128 + 2 * 128 + 2 * 128) * 4;
 constexpr int kMiscPf = kBarsPf * 8 + 16 + 8 * 16 + 2 * 32 * 16 * 4 + kRowTab * (int)sizeof(RowTile) +
-                        2 * (int)sizeof(EndRecP) + 64;
+                        2 * (int)sizeof(EndRecP) + 64 + kXchBytes;
 
 int prefill_smem_bytes(int dt, int stages) {
   return 1024 + kQBytes + stages * 2 * half_stage(dt) + kMiscPf;
@@ -253,26 +260,29 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *v) {
       : "memory");
 }
 
-// Stage row r of a segment's Q (128 FP32 dims times the softmax scale in
-// log2 units) into the score product's operand layout: 16-bit, hi and lo
-// terms of two 64-dim regions each; FP8, four E4M3 terms under the row's
-// power-of-2 scale 2^e (max |x| 2^e in [128, 256)), whose inverse is
-// returned.  Rows past the sequence's rows are zero.
+// Stage dims 64 kh .. 64 kh + 63 of row r of a segment's Q (FP32 times the
+// softmax scale in log2 units) into the score product's operand layout:
+// 16-bit, hi and lo terms of the 64-dim region kh; FP8, four E4M3 terms under
+// the row's power-of-2 scale 2^e (max |x| 2^e in [128, 256) over all 128
+// dims: the two groups' maxima meet in qmax), whose inverse is returned.
+// Rows past the sequence's rows are zero.
 template <int DT>
 __device__ __forceinline__ float pf_stage_q(const LseKernelParams &p, const float *src, bool live,
-                                            int r, uint8_t *qs) {
+                                            int r, int kh, uint8_t *qs, float *qmax, int bar_id) {
   const float sc = p.scale_log2;
   float isig = 1.f;
   if constexpr (is_f8(DT)) {
     float mx = 0.f;
     if (live) {
 #pragma unroll 4
-      for (int c = 0; c < 32; ++c) {
-        const float4 v = __ldg(reinterpret_cast<const float4 *>(src) + c);
+      for (int c = 0; c < 16; ++c) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(src) + 16 * kh + c);
         mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
       }
-      mx *= fabsf(sc);
     }
+    qmax[kh * 128 + r] = mx;
+    named_sync(bar_id, 256);
+    mx = fmaxf(qmax[r], qmax[128 + r]) * fabsf(sc);
     int e = 0;
     if (mx > 0.f && mx <= FLT_MAX) {
       const int E = ((__float_as_int(mx) >> 23) & 0xff) - 127;
@@ -281,7 +291,7 @@ __device__ __forceinline__ float pf_stage_q(const LseKernelParams &p, const floa
     const float sg = sc * exp2i(e);
     isig = exp2i(-e);
 #pragma unroll 1
-    for (int c = 0; c < 16; ++c) {  // 16-byte chunk c = dims 8c .. 8c + 7
+    for (int c = 8 * kh; c < 8 * kh + 8; ++c) {  // 8-dim chunk c = dims 8c .. 8c + 7
       float x[8];
       if (live) {
         const float4 a = __ldg(reinterpret_cast<const float4 *>(src) + 2 * c);
@@ -300,7 +310,7 @@ __device__ __forceinline__ float pf_stage_q(const LseKernelParams &p, const floa
     }
   } else {
 #pragma unroll 1
-    for (int c = 0; c < 16; ++c) {
+    for (int c = 8 * kh; c < 8 * kh + 8; ++c) {
       uint4 vh = make_uint4(0, 0, 0, 0), vl = make_uint4(0, 0, 0, 0);
       if (live) {
         const float4 a = __ldg(reinterpret_cast<const float4 *>(src) + 2 * c);
@@ -424,6 +434,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tcgen05_kernel(const __gr
   int *n_end = reinterpret_cast<int *>(end_rec + 2);
   int *go_flag = n_end + 1;
   int *n_rt_sh = n_end + 2;
+  float *xch_m = reinterpret_cast<float *>(n_end + 16);  // [2 tiles][2 groups][128]
+  float *xch_l = xch_m + 2 * 2 * 128;                   // [2 groups][128]
+  float *xch_q = xch_l + 2 * 128;                       // [2 groups][128]
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
   if (warp == 1) {
@@ -505,13 +518,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tcgen05_kernel(const __gr
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kSFull + i), 1);
-      mbar_init(bar(kPFull + i), 128);
+      mbar_init(bar(kPFull + i), 256);
       mbar_init(bar(kPvDone + i), 1);
     }
-    mbar_init(bar(kQFull), 128);
+    mbar_init(bar(kQFull), 256);
     mbar_init(bar(kQEmpty), 1);
     mbar_init(bar(kOFull), 1);
-    mbar_init(bar(kOEmpty), 128);
+    mbar_init(bar(kOEmpty), 256);
     mbar_init(bar(kDoneMma), 1);
     *n_end = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -704,15 +717,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tcgen05_kernel(const __gr
     mma_commit(bar(kDoneMma), leader);
     mbar_drain(bar(kDoneMma), 0);
   } else {
-    // ============== Q staging, softmax and epilogue: warps 2-5 ==============
+    // ====== Q staging, softmax and epilogue: warps 2-5 (keys 0-63) and 6-9 (64-127) ======
+    const int kh = (warp - 2) >> 2;               // key half of the tile, head-dim half of O
     const int quarter = warp & 3;                 // TMEM lane quarter
     const int r = quarter * 32 + lane;            // the row of the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    constexpr int kBar = 1;                       // named barrier of these 128 threads
+    constexpr int kBar = 1;                       // named barrier of these 256 threads
+    constexpr int kHK = kTK / 2;                  // keys of a half
     PfIter it;
     it.init(tab, n_rt, Hq, t_begin, t_stop);
     int seg = -1;
-    float m_run = -FLT_MAX, l_run = 0.f, isig = 1.f;
+    float m_run = -FLT_MAX, l_run = 0.f, isig = 1.f;  // l_run: this half's keys only
     bool had = false, ok = true;
 #pragma unroll 1
     for (int n = 0; it.valid() && ok; it.advance(), ++n) {
@@ -724,9 +739,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tcgen05_kernel(const __gr
         ++seg;
         // the previous segment's score products are done: replace Q
         bool w = seg == 0 || mbar_wait(bar(kQEmpty), (seg - 1) & 1, abort_flag, p.err);
-        if (named_or(kBar, 128, !w)) { ok = false; break; }
+        if (named_or(kBar, 256, !w)) { ok = false; break; }
         const float *src = p.q + ((long long)(rt.row0 + rt.r0 + r) * Hq + it.h) * kD;
-        isig = pf_stage_q<DT>(p, src, row_live, r, smem);
+        isig = pf_stage_q<DT>(p, src, row_live, r, kh, smem, xch_q, kBar);
         fence_proxy_async();
         mbar_arrive(bar(kQFull));
         m_run = -FLT_MAX;
@@ -736,51 +751,58 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tcgen05_kernel(const __gr
       // ---- tile n: scores -> probabilities ----
       bool w = mbar_wait(bar(kSFull + (n & 1)), (n >> 1) & 1, abort_flag, p.err);
       w = w && mbar_wait(bar(kInfo + (n & 7)), (n >> 3) & 1, abort_flag, p.err);
-      if (named_or(kBar, 128, !w)) { ok = false; break; }
+      if (named_or(kBar, 256, !w)) { ok = false; break; }
       tc_fence_after();
       const uint4 inf = tile_info[n & 7];
       const int key0 = it.kt * kTK;
       const uint32_t both = inf.x & inf.y;
       const bool tile_full = inf.z == (uint32_t)kTK && both == full_boxes;
-      float sv[kTK];
+      const int kc = kh * kHK;                    // this half's first key in the tile
+      float sv[kHK];
 #pragma unroll
-      for (int c = 0; c < kTK; c += 32) tmem_load<32>(tmem_s(n & 1) + lane_off + c, sv + c);
+      for (int c = 0; c < kHK; c += 32) tmem_load<32>(tmem_s(n & 1) + lane_off + kc + c, sv + c);
       if constexpr (kF8) {
 #pragma unroll
-        for (int j = 0; j < kTK; ++j) sv[j] *= isig;
+        for (int j = 0; j < kHK; ++j) sv[j] *= isig;
       }
       // every row of the tile sees every key of this tile?
       const bool all_vis = tile_full && key0 + kTK - 1 <= rt.C + rt.r0;
       if (!all_vis || !row_live) {
 #pragma unroll
-        for (int j = 0; j < kTK; ++j) {
-          const bool vis = row_live && key0 + j <= pos && j < (int)inf.z &&
-                           ((both >> (j / box_t)) & 1u);
+        for (int j = 0; j < kHK; ++j) {
+          const int jj = kc + j;
+          const bool vis = row_live && key0 + jj <= pos && jj < (int)inf.z &&
+                           ((both >> (jj / box_t)) & 1u);
           if (!vis) sv[j] = -INFINITY;
         }
       }
-      float mx = -INFINITY;
+      float mh = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < kTK; ++j) mx = fmaxf(mx, sv[j]);
-      const bool need = mx > m_run + kTau;
+      for (int j = 0; j < kHK; ++j) mh = fmaxf(mh, sv[j]);
+      // the row's maximum over both halves (double-buffered by tile parity)
+      float *xm = xch_m + (n & 1) * 256;
+      xm[kh * 128 + r] = mh;
+      named_sync(kBar, 256);
+      const float mx = fmaxf(xm[r], xm[128 + r]);
+      const bool need = mx > m_run + kTau;        // the same in both groups
       if (__any_sync(0xffffffffu, need)) {
         const float m_new = need ? mx : m_run;
         const float alpha = ex2(m_run - m_new);
         if (had) {
-          // rescale this row's output once the previous output product of
-          // the piece has completed (products complete in issue order)
+          // rescale this row's half of the output once the previous output
+          // product of the piece has completed (products complete in order)
           const int pn = n - 1;
           const bool wo = mbar_wait(bar(kPvDone + (pn & 1)), (pn >> 1) & 1, abort_flag, p.err);
           if (!__all_sync(0xffffffffu, wo)) { ok = false; }
           if (ok) {
             tc_fence_after();
 #pragma unroll 1
-            for (int c = 0; c < kD; c += 8) {
+            for (int c = 0; c < kD / 2; c += 8) {
               float v[8];
-              tmem_load<8>(tmem_o + lane_off + c, v);
+              tmem_load<8>(tmem_o + lane_off + kh * (kD / 2) + c, v);
 #pragma unroll
               for (int i = 0; i < 8; ++i) v[i] *= alpha;
-              tmem_st8(tmem_o + lane_off + c, v);
+              tmem_st8(tmem_o + lane_off + kh * (kD / 2) + c, v);
             }
             tmem_st_wait();
           }
@@ -788,14 +810,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tcgen05_kernel(const __gr
         l_run *= alpha;
         m_run = m_new;
       }
-      if (named_or(kBar, 128, !ok)) { ok = false; break; }
-      // probabilities over the score columns (A operand of the output product)
+      if (named_or(kBar, 256, !ok)) { ok = false; break; }
+      // probabilities over this half's score columns (A operand of the
+      // output product)
       float lsum = 0.f;
       if constexpr (kF8) {
         // P 2^7 as four E5M2 terms of its F16 rounding: term t of keys
         // 4c .. 4c + 3 in column 32 t + c
 #pragma unroll
-        for (int c0 = 0; c0 < kTK; c0 += 32) {
+        for (int c0 = 0; c0 < kHK; c0 += 32) {
           uint32_t words[4][8];
 #pragma unroll
           for (int c = 0; c < 32; c += 8) {
@@ -815,75 +838,79 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tcgen05_kernel(const __gr
           }
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
-            // 8 columns of term t: keys c0 .. c0 + 31
+            // 8 columns of term t: keys kc + c0 .. kc + c0 + 31
             asm volatile(
                 "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
-                    tmem_s(n & 1) + lane_off + (uint32_t)(32 * t + c0 / 4)),
+                    tmem_s(n & 1) + lane_off + (uint32_t)(32 * t + (kc + c0) / 4)),
                 "r"(words[t][0]), "r"(words[t][1]), "r"(words[t][2]), "r"(words[t][3]),
                 "r"(words[t][4]), "r"(words[t][5]), "r"(words[t][6]), "r"(words[t][7])
                 : "memory");
           }
         }
       } else {
-        // hi terms in columns 0 .. 63, lo terms in 64 .. 127 (two keys a column)
+        // hi terms in columns 0 .. 63, lo terms in 64 .. 127 (two keys a
+        // column): this half's 32 columns of each
+        uint32_t hi[32], lo[32];
 #pragma unroll
-        for (int c0 = 0; c0 < kTK; c0 += 64) {
-          uint32_t hi[32], lo[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float e0 = ex2(sv[c0 + 2 * c] - m_run), e1 = ex2(sv[c0 + 2 * c + 1] - m_run);
-            lsum += e0 + e1;
-            split2<DT>(e0, e1, hi[c], lo[c]);
-          }
-          tmem_st32(tmem_s(n & 1) + lane_off + (uint32_t)(c0 / 2), hi);
-          tmem_st32(tmem_s(n & 1) + lane_off + (uint32_t)(64 + c0 / 2), lo);
+        for (int c = 0; c < 32; ++c) {
+          const float e0 = ex2(sv[2 * c] - m_run), e1 = ex2(sv[2 * c + 1] - m_run);
+          lsum += e0 + e1;
+          split2<DT>(e0, e1, hi[c], lo[c]);
         }
+        tmem_st32(tmem_s(n & 1) + lane_off + (uint32_t)(kc / 2), hi);
+        tmem_st32(tmem_s(n & 1) + lane_off + (uint32_t)(64 + kc / 2), lo);
       }
       tmem_st_wait();
       l_run += lsum;
       had = true;
       if (!tile_full) {
         // a V row that holds no live key may hold any bits: zero it (its
-        // probability is 0, and 0 x NaN would not be)
-        const bool wv = mbar_wait(bar(kFullV + n % NS), (n / NS) & 1, abort_flag, p.err);
-        const bool dead = !(r < (int)inf.z && ((both >> (r / box_t)) & 1u));
-        if (wv && dead) {
-          uint8_t *v0 = smem + kQBytes + NS * kHalf + (n % NS) * kHalf + r * 128;
+        // probability is 0, and 0 x NaN would not be); the first group's
+        // thread r takes V row r
+        bool wv = true;
+        if (kh == 0) {
+          wv = mbar_wait(bar(kFullV + n % NS), (n / NS) & 1, abort_flag, p.err);
+          const bool dead = !(r < (int)inf.z && ((both >> (r / box_t)) & 1u));
+          if (wv && dead) {
+            uint8_t *v0 = smem + kQBytes + NS * kHalf + (n % NS) * kHalf + r * 128;
 #pragma unroll 1
-          for (int c = 0; c < (kF8 ? 8 : 16); ++c)
-            *reinterpret_cast<uint4 *>(v0 + (c >> 3) * kRegion + (c & 7) * 16) =
-                make_uint4(0, 0, 0, 0);
+            for (int c = 0; c < (kF8 ? 8 : 16); ++c)
+              *reinterpret_cast<uint4 *>(v0 + (c >> 3) * kRegion + (c & 7) * 16) =
+                  make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async();
         }
-        if (named_or(kBar, 128, !wv)) { ok = false; break; }
-        fence_proxy_async();
+        if (named_or(kBar, 256, !wv)) { ok = false; break; }
       }
       tc_fence_before();
       mbar_arrive(bar(kPFull + (n & 1)));
 
       if (last) {
-        // ---- epilogue of the piece ----
+        // ---- epilogue of the piece: this group writes head dims 64 kh .. ----
         bool we = mbar_wait(bar(kOFull), seg & 1, abort_flag, p.err);
-        if (named_or(kBar, 128, !we)) { ok = false; break; }
+        xch_l[kh * 128 + r] = l_run;
+        if (named_or(kBar, 256, !we)) { ok = false; break; }
         tc_fence_after();
+        const float lt = xch_l[r] + xch_l[128 + r];
         const int c_first = cta_of(it.seg_first, U, C);
         const int c_last = cta_of(it.seg_first + it.n_kt - 1, U, C);
         const int n_pieces = c_last - c_first + 1, piece = cta - c_first;
-        const float inv = l_run > 0.f ? rcp(l_run) : 0.f;
+        const float inv = lt > 0.f ? rcp(lt) : 0.f;
         const float lse2 =
-            l_run > 0.f ? m_run + lg2(l_run) - (kF8 ? (float)kPScaleLog2 : 0.f) : -INFINITY;
+            lt > 0.f ? m_run + lg2(lt) - (kF8 ? (float)kPScaleLog2 : 0.f) : -INFINITY;
         float *dst;
         if (n_pieces == 1) {
           dst = p.out + ((long long)(rt.row0 + rt.r0 + r) * Hq + it.h) * kD;
-          if (row_live && p.lse_out)
+          if (kh == 0 && row_live && p.lse_out)
             p.lse_out[(long long)(rt.row0 + rt.r0 + r) * Hq + it.h] = lse2 * 0.69314718055994530942f;
         } else {
           const int slot = t_begin >= it.seg_first ? 0 : 1;
           const long long pi = (long long)cta * 2 + slot;
           dst = p.o_part + pi * kRT * kD + (long long)r * kD;
-          p.lse_part[pi * kRT + r] = row_live ? lse2 : -INFINITY;
+          if (kh == 0) p.lse_part[pi * kRT + r] = row_live ? lse2 : -INFINITY;
         }
 #pragma unroll 1
-        for (int c = 0; c < kD; c += 8) {
+        for (int c = kh * (kD / 2); c < (kh + 1) * (kD / 2); c += 8) {
           float v[8];
           tmem_load<8>(tmem_o + lane_off + c, v);
           if (row_live || n_pieces > 1) {
@@ -898,8 +925,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tcgen05_kernel(const __gr
         mbar_arrive(bar(kOEmpty));
         if (n_pieces > 1) {
           __threadfence();
-          named_sync(kBar, 128);
-          if (r == 0) {
+          named_sync(kBar, 256);
+          if (kh == 0 && r == 0) {
             atomicAdd(p.seg_count + 2 * it.seg_id, 1u);
             const int k = *n_end;
             if (k < 2) {

@@ -82,7 +82,8 @@ struct __align__(64) TcParams {
   LseKernelParams p;
   int n_ctas;
   int n_slots;
-  int stages;
+  int k_stages;  // K ring depth
+  int v_stages;  // V ring depth (V tiles are held longer: through the softmax and P.V)
   int q_slots;
   int p_bufs;
   int box_tokens;
@@ -115,7 +116,7 @@ __device__ __forceinline__ int seq_chunks(const LseKernelParams &p, int R) {
 // Per-sequence record built once per CTA in shared memory (sequences up to
 // kSeqTab): tiles of all segments before the sequence, its 128-key tiles,
 // L, first row, R, and the number of segments before the sequence.
-constexpr int kSeqTab = 256;
+constexpr int kSeqTab = 96;
 struct SeqRec {
   int prefix, n_tiles, L, row0, R, seg_prefix;
 };
@@ -298,14 +299,14 @@ __device__ __forceinline__ void load_scales(const LseKernelParams &p, int nbox, 
 // (and, with sdst != 0, the tile's K and V scales into sdst[0..128) and
 // sdst[128..256), counted on the V slot's barrier).  Returns 0 when a wait
 // gave up.
-__device__ __forceinline__ int produce_tile(const TcParams &tp, int n, int NS, int nbox,
+__device__ __forceinline__ int produce_tile(const TcParams &tp, int n, int NK, int NV, int nbox,
                                             int box_t, int regions, int g, int tile, int L,
                                             const int *pk, const int *pv, uint32_t kdst,
                                             uint32_t vdst, uint32_t sdst, const uint32_t *bars_k,
                                             const uint32_t *bars_v, uint32_t info_bar,
                                             uint4 *info, volatile int *abort_flag) {
   const LseKernelParams &p = tp.p;
-  const uint32_t ph = ((n / NS) & 1) ^ 1;
+  const uint32_t ph_k = ((n / NK) & 1) ^ 1, ph_v = ((n / NV) & 1) ^ 1;
   const int key0 = tile * kTK;
   uint32_t kmask = 0, vmask = 0;
 #pragma unroll 1
@@ -315,16 +316,16 @@ __device__ __forceinline__ int produce_tile(const TcParams &tp, int n, int NS, i
   }
   const int live = L - key0 < kTK ? L - key0 : kTK;
   const uint32_t box_bytes = (uint32_t)regions * (uint32_t)box_t * 128u;
-  if (!mbar_wait(bars_k[0], ph, abort_flag, p.err)) return 0;
+  if (!mbar_wait(bars_k[0], ph_k, abort_flag, p.err)) return 0;
   // the record slot was last read by the softmax of tile n - 8, which has
   // finished: the K slot of tile n was freed by the score product of tile
-  // n - NS, issued in order after the softmax of tiles up to n - NS - 2
-  // (>= n - 8 for NS <= 6) released their score buffers
+  // n - NK, issued in order after the softmax of tiles up to n - NK - 2
+  // (>= n - 8 for NK <= 6) read their scores
   *info = make_uint4(kmask, vmask, (uint32_t)live, 0u);
   mbar_arrive(info_bar);  // publishes the record
   mbar_expect_tx(bars_k[1], (uint32_t)__popc(kmask) * box_bytes);
   load_boxes(tp, nbox, box_t, regions, g, key0, pk, kdst, bars_k[1]);
-  if (!mbar_wait(bars_v[0], ph, abort_flag, p.err)) return 0;
+  if (!mbar_wait(bars_v[0], ph_v, abort_flag, p.err)) return 0;
   const uint32_t scale_bytes =
       sdst ? (uint32_t)(__popc(kmask) + __popc(vmask)) * (uint32_t)box_t * 4u : 0u;
   mbar_expect_tx(bars_v[1], (uint32_t)__popc(vmask) * box_bytes + scale_bytes);
@@ -441,11 +442,12 @@ struct TcLayout {
   static constexpr int kHalfStage = kF8 ? kRegionBytes : 2 * kRegionBytes;
   // per-vector scales of one tile, K then V (128 FP32 each), per ring stage
   static constexpr int kScStage = 2 * kTK * 4;
-  // stages: K/V ring depth; q_slots: Q ring depth (1 or 2); p_bufs: P tiles
-  // per softmax group (1 or 2); scaled: per-vector scale rows per stage
-  static int smem_bytes(int stages, int q_slots, int p_bufs, bool scaled) {
-    return 1024 + stages * 2 * kHalfStage + q_slots * kQBytes + 2 * p_bufs * kPBytes +
-           (scaled ? stages * kScStage : 0) + kMiscBytes;
+  // k_stages / v_stages: K and V ring depths; q_slots: Q ring depth (1 or
+  // 2); p_bufs: P tiles per softmax group (1 or 2); scaled: per-vector scale
+  // rows per V stage
+  static int smem_bytes(int k_stages, int v_stages, int q_slots, int p_bufs, bool scaled) {
+    return 1024 + (k_stages + v_stages) * kHalfStage + q_slots * kQBytes + 2 * p_bufs * kPBytes +
+           (scaled ? v_stages * kScStage : 0) + kMiscBytes;
   }
 };
 
@@ -467,7 +469,7 @@ enum {
   kBarPEmpty = 57,  // [4] = group * 2 + P buffer: the P tile has been read
   kBarDoneV = 61,   // the output issuer's MMAs have completed
   kBarSEmpty = 62,  // [2] per softmax group: its score buffer has been read out
-  kBarEpiMeet = 64, // [2] per output slot: both groups' sums and maxima of a piece are in
+  kBarPub = 64,     // [2] per output slot: the non-closing group's sums and maxima are published
 };
 
 // Sum of eight per-lane values over the 32 lanes of a warp, by a fixed
@@ -600,18 +602,26 @@ __device__ __forceinline__ bool stage_q(const LseKernelParams &p, int t, int g, 
 
 // End phase of the fused pass: for each segment this CTA shares with other
 // CTAs, wait until every piece's partial is written (the segment's arrival
-// count reaches two per piece), then merge this CTA's share of the
-// segment's (pair, dim) outputs: share k of n covers elements
-// [k E / n, (k+1) E / n) of the E = pairs x D outputs, each the
-// log-sum-exp-weighted mean of the pieces' partials (the same merge as the
-// separate merge pass).  The last CTA to finish a segment clears its two
-// counters for the next call.  The wait is bounded like every other wait;
-// the launch is cooperative, so every CTA of the grid is resident and each
-// arrives for its own pieces without waiting on any other CTA.
+// count reaches its number of pieces), then merge this CTA's share of the
+// segment's (row, head) pairs: pair q goes to the segment's piece q mod n,
+// so the n CTAs of the segment split its pairs.  A pair is merged by one or
+// more warps, each taking every k-th piece with its loads issued together
+// (lanes over the head dim, four dims a lane) and a running maximum; the
+// warps' sums meet in shared memory (the K/V ring, idle by now).  Same
+// arithmetic as the separate merge pass: M = max lse, weights 2^(lse - M).
+// The last CTA to finish a segment clears its two counters for the next
+// call.  The wait is bounded like every other wait; the launch is
+// cooperative, so every CTA of the grid is resident and each arrives for its
+// own pieces without waiting on any other CTA.
 __device__ __noinline__ void fused_end_merge(const TcParams &tp, const EndRec *rec, int n_rec,
-                                             volatile int *abort_flag, int *go_flag) {
+                                             volatile int *abort_flag, int *go_flag,
+                                             float *scratch) {
   const LseKernelParams &p = tp.p;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  constexpr int kWarps = kThreads / 32;
+  float *w_m = scratch;                 // [warp] running maximum
+  float *w_l = scratch + kWarps;        // [warp] sum of weights
+  float *w_acc = scratch + 2 * kWarps;  // [warp][kD] weighted sums
 #pragma unroll 1
   for (int k = 0; k < n_rec; ++k) {
     const EndRec r = rec[k];
@@ -622,46 +632,96 @@ __device__ __noinline__ void fused_end_merge(const TcParams &tp, const EndRec *r
       while (go) {
         unsigned int v;
         asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
-        if (v >= 2u * (unsigned)r.n_pieces) break;
+        if (v >= (unsigned)r.n_pieces) break;
         if (clock64() - t0 > kWaitCycles) {
           *abort_flag = 1;
           atomicOr(p.err, LSE_DEVERR_TIMEOUT);
           go = 0;
         }
-        __nanosleep(256);
+        __nanosleep(64);
       }
       *go_flag = go;
     }
     __syncthreads();
     const bool go = *go_flag != 0;
-    if (go) {
-      const int G = p.group;
-      const long long E = (long long)G * r.rows * kD;
-      const long long e0 = E * r.piece / r.n_pieces, e1 = E * (r.piece + 1) / r.n_pieces;
+    const int G = p.group, P = G * r.rows, n = r.n_pieces;
+    // this CTA's pairs: r.piece, r.piece + n, ...
+    const int mine = r.piece < P ? (P - 1 - r.piece) / n + 1 : 0;
 #pragma unroll 1
-      for (long long e = e0 + tid; e < e1; e += kThreads) {
-        const int q = (int)(e / kD), d = (int)(e - (long long)q * kD);
+    for (int b = 0; go && b < mine; b += kWarps) {
+      const int np = min(kWarps, mine - b);           // pairs in this round
+      const int kw = kWarps / np;                      // warps per pair
+      const int slot = warp / kw, sub = warp - slot * kw;
+      const bool active = slot < np;
+      float m = -INFINITY, l = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      long long base = 0;
+      if (active) {
+        const int q = r.piece + (b + slot) * n;
         const int rr = q / G, h = r.g * G + (q - rr * G);
         const long long oi = (long long)(r.row0 + rr) * p.n_q_heads + h;
-        const long long base = oi * tp.n_slots;
-        // partials written by other CTAs: read through L2
-        float M = -INFINITY;
-#pragma unroll 4
-        for (int i = 0; i < r.n_pieces; ++i) M = fmaxf(M, __ldcg(p.lse_part + base + i));
-        float W = 0.f, acc = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll 4
-          for (int i = 0; i < r.n_pieces; ++i) {
-            const float l = __ldcg(p.lse_part + base + i);
-            const float w = l == -INFINITY ? 0.f : ex2(l - M);
-            W += w;
-            acc = fmaf(w, __ldcg(p.o_part + (base + i) * kD + d), acc);
+        base = oi * tp.n_slots;
+        // pieces sub, sub + kw, ...: loads first, then the running maximum
+#pragma unroll 1
+        for (int i0 = sub; i0 < n; i0 += 8 * kw) {
+          float li[8];
+          float4 vi[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * kw;
+            li[u] = i < n ? __ldcg(p.lse_part + base + i) : -INFINITY;
+            vi[u] = i < n ? __ldcg(reinterpret_cast<const float4 *>(p.o_part + (base + i) * kD) +
+                                   lane)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
           }
+          float mc = m;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) mc = fmaxf(mc, li[u]);
+          if (mc == -INFINITY) continue;
+          const float sc = ex2(m - mc);  // 0 while m = -inf
+          l *= sc;
+          acc.x *= sc; acc.y *= sc; acc.z *= sc; acc.w *= sc;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const float w = li[u] == -INFINITY ? 0.f : ex2(li[u] - mc);
+            l += w;
+            acc.x = fmaf(w, vi[u].x, acc.x);
+            acc.y = fmaf(w, vi[u].y, acc.y);
+            acc.z = fmaf(w, vi[u].z, acc.z);
+            acc.w = fmaf(w, vi[u].w, acc.w);
+          }
+          m = mc;
         }
-        p.out[oi * kD + d] = W > 0.f ? acc * rcp(W) : 0.f;
-        if (d == 0 && p.lse_out)
+      }
+      if (lane == 0) {
+        w_m[warp] = m;
+        w_l[warp] = l;
+      }
+      reinterpret_cast<float4 *>(w_acc + warp * kD)[lane] = acc;
+      __syncthreads();
+      // the pair's warps combined in a fixed order (warp `slot * kw` writes)
+      if (active && sub == 0) {
+        float M = -INFINITY;
+        for (int s2 = 0; s2 < kw; ++s2) M = fmaxf(M, w_m[warp + s2]);
+        float W = 0.f;
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s2 = 0; s2 < kw; ++s2) {
+          const float sc = w_m[warp + s2] == -INFINITY ? 0.f : ex2(w_m[warp + s2] - M);
+          W += w_l[warp + s2] * sc;
+          const float4 v = reinterpret_cast<const float4 *>(w_acc + (warp + s2) * kD)[lane];
+          a.x = fmaf(sc, v.x, a.x);
+          a.y = fmaf(sc, v.y, a.y);
+          a.z = fmaf(sc, v.z, a.z);
+          a.w = fmaf(sc, v.w, a.w);
+        }
+        const float inv = W > 0.f ? rcp(W) : 0.f;
+        const long long oi = base / tp.n_slots;
+        reinterpret_cast<float4 *>(p.out + oi * kD)[lane] =
+            make_float4(a.x * inv, a.y * inv, a.z * inv, a.w * inv);
+        if (lane == 0 && p.lse_out)
           p.lse_out[oi] = W > 0.f ? (M + lg2(W)) * 0.69314718055994530942f : -INFINITY;
       }
+      __syncthreads();
     }
     __syncthreads();
     if (tid == 0 && go) {
@@ -687,7 +747,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int QS = tp.q_slots;
   const int PB = tp.p_bufs;
   const LseKernelParams &p = tp.p;
-  const int NS = tp.stages;
+  const int NK = tp.k_stages, NV = tp.v_stages;
   const int cta = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -696,11 +756,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
   const uint32_t sbase = smem_u32(smem);
   const uint32_t k_base = sbase;                                // K ring
-  const uint32_t v_base = k_base + NS * Lay::kHalfStage;        // V ring
-  const uint32_t q_base = v_base + NS * Lay::kHalfStage;        // Q slots
+  const uint32_t v_base = k_base + NK * Lay::kHalfStage;        // V ring
+  const uint32_t q_base = v_base + NV * Lay::kHalfStage;        // Q slots
   const uint32_t p_base = q_base + QS * Lay::kQBytes;          // P tiles [group][buffer]
   const uint32_t sc_base = p_base + 2 * PB * Lay::kPBytes;     // scale rows [stage]
-  uint8_t *misc = smem + (sc_base - sbase) + (kSc ? NS * Lay::kScStage : 0);
+  uint8_t *misc = smem + (sc_base - sbase) + (kSc ? NV * Lay::kScStage : 0);
   // the P tile of group grp used with its tile of index n (n & 1 == grp)
   auto p_tile = [&](int grp, int n) {
     return p_base + (uint32_t)((grp * PB + ((n >> 1) % PB)) * Lay::kPBytes);
@@ -815,10 +875,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 4; ++i) {
       mbar_init(bar(kBarOFull + i), 1);
-      // both softmax groups read both groups' output blocks of a piece
-      mbar_init(bar(kBarOEmpty + i), 256);
+      // released by the group that combines the piece (it read both blocks)
+      mbar_init(bar(kBarOEmpty + i), 128);
     }
-    for (int i = 0; i < 2; ++i) mbar_init(bar(kBarEpiMeet + i), 256);
+    for (int i = 0; i < 2; ++i) mbar_init(bar(kBarPub + i), 128);
     *n_end = 0;
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarSFull + i), 1);
@@ -888,13 +948,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int tl = __shfl_sync(0xffffffffu, mine.L, i);
         int go = 1;
         if (lane == 0 && n != tp.withhold_tile) {
-          const uint32_t bars_k[2] = {bar(kBarEmptyK + n % NS), bar(kBarFullK + n % NS)};
-          const uint32_t bars_v[2] = {bar(kBarEmptyV + n % NS), bar(kBarFullV + n % NS)};
-          go = produce_tile(tp, n, NS, nbox, box_t, kF8 ? 1 : 2, tg, tt, tl, pk + i * 16,
+          const uint32_t bars_k[2] = {bar(kBarEmptyK + n % NK), bar(kBarFullK + n % NK)};
+          const uint32_t bars_v[2] = {bar(kBarEmptyV + n % NV), bar(kBarFullV + n % NV)};
+          go = produce_tile(tp, n, NK, NV, nbox, box_t, kF8 ? 1 : 2, tg, tt, tl, pk + i * 16,
                             pv + i * 16,
-                            k_base + (n % NS) * Lay::kHalfStage,
-                            v_base + (n % NS) * Lay::kHalfStage,
-                            kSc ? sc_base + (n % NS) * Lay::kScStage : 0u, bars_k, bars_v,
+                            k_base + (n % NK) * Lay::kHalfStage,
+                            v_base + (n % NV) * Lay::kHalfStage,
+                            kSc ? sc_base + (n % NV) * Lay::kScStage : 0u, bars_k, bars_v,
                             bar(kBarInfo + (n & 7)), tile_info + (n & 7), abort_flag);
         }
         go = __shfl_sync(0xffffffffu, go, 0);
@@ -908,9 +968,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // drain: every copy issued must have landed before the CTA exits
     if (lane == 0)
 #pragma unroll 1
-      for (int k = (n > NS ? n - NS : 0); k < n; ++k) {
-        mbar_drain(bar(kBarFullK + k % NS), (k / NS) & 1);
-        mbar_drain(bar(kBarFullV + k % NS), (k / NS) & 1);
+      for (int k = (n > NV ? n - NV : 0); k < n; ++k) {
+        if (k >= n - NK) mbar_drain(bar(kBarFullK + k % NK), (k / NK) & 1);
+        mbar_drain(bar(kBarFullV + k % NV), (k / NV) & 1);
       }
   } else if (warp == 1 || warp == 2) {
     // ====================== MMA issuers (one thread each) ======================
@@ -937,12 +997,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int nq = 0; nq < n_total; ++nq, iq.advance(p)) {
         const bool first = iq.seg_start(t_begin), last = iq.seg_end();
         if (first) ++seg_q;
-        const int st = nq % NS;
+        const int st = nq % NK;
         // the segment's Q, the K tile, and the group's score buffer, which
         // its softmax read out (into registers) at the start of tile nq - 2
         bool go = !first || mbar_wait(bar(kBarQFull + seg_q % QS), (seg_q / QS) & 1, abort_flag,
                                       p.err);
-        go = go && mbar_wait(bar(kBarFullK + st), (nq / NS) & 1, abort_flag, p.err);
+        go = go && mbar_wait(bar(kBarFullK + st), (nq / NK) & 1, abort_flag, p.err);
         go = go && (nq < 2 ||
                     mbar_wait(bar(kBarSEmpty + (nq & 1)), ((nq - 2) >> 1) & 1, abort_flag, p.err));
         if (!__all_sync(0xffffffffu, go)) break;
@@ -992,9 +1052,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int grp = nv & 1, slot = seg_v % kOS;
         const uint32_t oe_par = ((seg_v / kOS) & 1) ^ 1;
-        const int st = nv % NS;
+        const int st = nv % NV;
         bool go = mbar_wait(bar(kBarPFull + grp), (nv >> 1) & 1, abort_flag, p.err);
-        go = go && mbar_wait(bar(kBarFullV + st), (nv / NS) & 1, abort_flag, p.err);
+        go = go && mbar_wait(bar(kBarFullV + st), (nv / NV) & 1, abort_flag, p.err);
         // a group's output slot must have been read out kOS segments ago
         const bool mine = (started >> grp) & 1u, other = (started >> (grp ^ 1)) & 1u;
         if (!mine)
@@ -1182,7 +1242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // per-vector scales land with the tile's V (the V slot outlives
         // this pass: its output product waits for this tile's P)
         if (kSc && w)
-          w = mbar_wait(bar(kBarFullV + n % NS), (n / NS) & 1, abort_flag, p.err);
+          w = mbar_wait(bar(kBarFullV + n % NV), (n / NV) & 1, abort_flag, p.err);
         if (named_or(bar_id, 128, !w)) {
           ok = false;
           break;
@@ -1203,7 +1263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (kSc) {
           if (kvalid) {
             const float *scs = reinterpret_cast<const float *>(
-                smem + (sc_base - sbase) + (n % NS) * Lay::kScStage);
+                smem + (sc_base - sbase) + (n % NV) * Lay::kScStage);
             ks = scs[j];
             float vs = scs[kTK + j];
             vs = vs < 0x1p-64f ? 0x1p-64f : vs;  // (NaN stays NaN)
@@ -1377,8 +1437,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         pbuf = buf;
         if (!kvalid) {
           // a dead slot may hold any bits: give it a zero V row (P is 0 there)
-          mbar_wait(bar(kBarFullV + n % NS), (n / NS) & 1, abort_flag, p.err);
-          uint8_t *v0 = smem + (v_base - sbase) + (n % NS) * Lay::kHalfStage + j * 128;
+          mbar_wait(bar(kBarFullV + n % NV), (n / NV) & 1, abort_flag, p.err);
+          uint8_t *v0 = smem + (v_base - sbase) + (n % NV) * Lay::kHalfStage + j * 128;
           constexpr int kChunks = kF8 ? 8 : 16;  // 16-byte chunks of the row
 #pragma unroll 1
           for (int c = 0; c < kChunks; ++c)
@@ -1422,12 +1482,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           pub_l[(pb * 2 + grp) * 64 + j] = kLAcc ? red[j] : lsum[j];
         }
         if (j == 0) pub_had[pb * 2 + grp] = had_tile ? 1 : 0;
-        // this group's row sums, maxima and output block are complete; meet
-        // the other group (an mbarrier wait, so a group that gave up never
-        // leaves the other one waiting)
-        tc_fence_before();
-        mbar_arrive(bar(kBarEpiMeet + oslot));
-        const bool wm = mbar_wait(bar(kBarEpiMeet + oslot), (seg / kOS) & 1, abort_flag, p.err);
+        // The group that ran the piece's last tile closes the piece: it
+        // combines both groups' results.  The other group has finished its
+        // part earlier; it publishes its sums and maxima and goes on to its
+        // next segment (on its other output slot, or after the closer frees
+        // this one), never waiting for the closer.
+        const bool closer = (n & 1) == grp;
+        if (!closer) {
+          tc_fence_before();
+          mbar_arrive(bar(kBarPub + oslot));
+          continue;
+        }
+        const int other = grp ^ 1;
+        bool wm = mbar_wait(bar(kBarPub + oslot), (seg / kOS) & 1, abort_flag, p.err);
+        wm = wm && mbar_wait(bar(kBarOFull + 2 * other + oslot), (seg / kOS) & 1, abort_flag,
+                             p.err);
         if (named_or(bar_id, 128, !wm)) {
           ok = false;
           break;
@@ -1446,9 +1515,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const long long row_stride = (long long)p.n_q_heads * tp.n_slots * kD;
         const long long base =
             ((long long)it.crow0(p) * p.n_q_heads + it.g * G) * tp.n_slots + piece;
-        // the groups take alternate blocks of 8 pairs
+        // every pair, 8 at a time
 #pragma unroll 1
-        for (int c = 8 * grp; c < P8; c += 16) {
+        for (int c = 0; c < P8; c += 8) {
           float o0[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
           float o1[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
           // the output blocks (hi and lo, or the P terms) summed
@@ -1482,24 +1551,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        // both groups have read both output blocks when both have arrived
+        // both output blocks are read: free both groups' slots
         tc_fence_before();
         mbar_arrive(bar(kBarOEmpty + oslot));
         mbar_arrive(bar(kBarOEmpty + 2 + oslot));
         if (tp.fused && n_pieces > 1) {
-          // this group's share of the piece's partial is written: count it on
-          // the segment (two arrivals per piece); the CTA merges its share of
-          // the segment once every piece is in (end phase)
+          // the piece's partial is written: count it on the segment; the CTA
+          // merges its share of the segment once every piece is in (end phase)
           __threadfence();
           named_sync(bar_id, 128);
           if (j == 0) {
             atomicAdd(p.seg_count + 2 * it.seg_id, 1u);
-            if (grp == 0) {
-              const int k = *n_end;
-              if (k < 2) {
-                end_rec[k] = EndRec{it.seg_id, n_pieces, piece, it.crow0(p), it.crows(p), it.g};
-                *n_end = k + 1;
-              }
+            const int k = *n_end;
+            if (k < 2) {
+              end_rec[k] = EndRec{it.seg_id, n_pieces, piece, it.crow0(p), it.crows(p), it.g};
+              *n_end = k + 1;
             }
           }
         }
@@ -1516,7 +1582,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(Lay::kTmemCols)
                  : "memory");
-  if (tp.fused) fused_end_merge(tp, end_rec, *n_end, abort_flag, had_all);
+  // (the K/V ring is idle: the end phase's scratch)
+  if (tp.fused)
+    fused_end_merge(tp, end_rec, *n_end, abort_flag, had_all,
+                    reinterpret_cast<float *>(smem + (k_base - sbase)));
 }
 
 // ---- host side ------------------------------------------------------------------------
@@ -1573,21 +1642,23 @@ int launch_tc_p(const TcParams &tp, int p8, int smem, cudaStream_t st) {
 }
 
 template <int DT>
-int smem_for_p(int p8, int stages, int q_slots, int p_bufs, bool scaled) {
+int smem_for_p(int p8, int k_stages, int v_stages, int q_slots, int p_bufs, bool scaled) {
   switch (p8) {
-    case 8: return TcLayout<DT, 8>::smem_bytes(stages, q_slots, p_bufs, scaled);
-    case 16: return TcLayout<DT, 16>::smem_bytes(stages, q_slots, p_bufs, scaled);
-    case 24: return TcLayout<DT, 24>::smem_bytes(stages, q_slots, p_bufs, scaled);
-    case 32: return TcLayout<DT, 32>::smem_bytes(stages, q_slots, p_bufs, scaled);
-    case 48: return TcLayout<DT, 48>::smem_bytes(stages, q_slots, p_bufs, scaled);
+    case 8: return TcLayout<DT, 8>::smem_bytes(k_stages, v_stages, q_slots, p_bufs, scaled);
+    case 16: return TcLayout<DT, 16>::smem_bytes(k_stages, v_stages, q_slots, p_bufs, scaled);
+    case 24: return TcLayout<DT, 24>::smem_bytes(k_stages, v_stages, q_slots, p_bufs, scaled);
+    case 32: return TcLayout<DT, 32>::smem_bytes(k_stages, v_stages, q_slots, p_bufs, scaled);
+    case 48: return TcLayout<DT, 48>::smem_bytes(k_stages, v_stages, q_slots, p_bufs, scaled);
   }
   return -1;
 }
 
-int smem_for(int dtype, int p8, int stages, int q_slots, int p_bufs, bool scaled) {
+int smem_for(int dtype, int p8, int k_stages, int v_stages, int q_slots, int p_bufs,
+             bool scaled) {
   // the two 16-bit formats share a layout, and so do the two 8-bit ones
-  return is_f8(dtype) ? smem_for_p<LSE_KV_FP8_E4M3>(p8, stages, q_slots, p_bufs, scaled)
-                      : smem_for_p<LSE_KV_BF16>(p8, stages, q_slots, p_bufs, scaled);
+  return is_f8(dtype)
+             ? smem_for_p<LSE_KV_FP8_E4M3>(p8, k_stages, v_stages, q_slots, p_bufs, scaled)
+             : smem_for_p<LSE_KV_BF16>(p8, k_stages, v_stages, q_slots, p_bufs, scaled);
 }
 
 }  // namespace
@@ -1601,26 +1672,34 @@ int lse_tc_pairs_bucket(int pairs) {
   return -1;
 }
 
-// Shared-memory configuration: the deepest K/V ring with one P tile per
-// softmax group (the groups then alternate on the SM's pipes, which their
-// exponentials and conversions keep busy), a second Q slot (overlapping Q
-// staging with the end of the previous segment) when it fits as well.  The
-// kernel also runs with two P tiles per group (p_bufs = 2), which the planner
-// does not pick.
-int lse_tc_smem(int dtype, int p8, int scaled, int smem_optin, int *stages, int *q_slots,
-                int *p_bufs) {
+// Shared-memory configuration: the most K and V tile slots with one P tile
+// per softmax group (the groups then alternate on the SM's pipes, which
+// their exponentials and conversions keep busy), a second Q slot
+// (overlapping Q staging with the end of the previous segment) when it fits
+// as well.  The slots are split about 1 : 2 between the K and the V ring (at
+// least two each, K at most kMaxStages, V at most 8): a K slot is free again
+// once its score product is done, a V slot only after the softmax of its
+// tile and its output product.  The kernel also runs with two P tiles per
+// group (p_bufs = 2), which the planner does not pick.
+int lse_tc_smem(int dtype, int p8, int scaled, int smem_optin, int *k_stages, int *v_stages,
+                int *q_slots, int *p_bufs) {
   if (scaled && !is_f8(dtype)) return -1;
   for (int pb = 1; pb >= 1; --pb)
-    for (int ns = kMaxStages; ns >= 2; --ns)
+    for (int slots = kMaxStages + 8; slots >= 4; --slots) {
+      const int nk = slots / 3 < 2 ? 2 : (slots / 3 > kMaxStages ? kMaxStages : slots / 3);
+      const int nv = slots - nk;
+      if (nv < 2 || nv > 8) continue;
       for (int qs = 2; qs >= 1; --qs) {
-        const int b = smem_for(dtype, p8, ns, qs, pb, scaled != 0);
+        const int b = smem_for(dtype, p8, nk, nv, qs, pb, scaled != 0);
         if (b > 0 && b <= smem_optin) {
-          *stages = ns;
+          *k_stages = nk;
+          *v_stages = nv;
           *q_slots = qs;
           *p_bufs = pb;
           return b;
         }
       }
+    }
   return -1;
 }
 
@@ -1664,8 +1743,9 @@ size_t lse_tc_map_bytes() { return sizeof(CUtensorMap); }
 
 int lse_launch_partial_tcgen05(const LseKernelParams &p, const void *maps, int n_maps,
                                int dtype, int p8, int scaled, int n_ctas, int n_slots,
-                               int stages, int q_slots, int p_bufs, int box_tokens, int smem,
-                               int fused, int withhold_tile, void *stream) {
+                               int k_stages, int v_stages, int q_slots, int p_bufs,
+                               int box_tokens, int smem, int fused, int withhold_tile,
+                               void *stream) {
   static_assert(sizeof(TcParams) < 30000, "kernel parameter block too large");
   TcParams tp;
   memset(&tp, 0, sizeof tp);
@@ -1673,7 +1753,8 @@ int lse_launch_partial_tcgen05(const LseKernelParams &p, const void *maps, int n
   tp.p = p;
   tp.n_ctas = n_ctas;
   tp.n_slots = n_slots;
-  tp.stages = stages;
+  tp.k_stages = k_stages;
+  tp.v_stages = v_stages;
   tp.q_slots = q_slots;
   tp.p_bufs = p_bufs;
   tp.box_tokens = box_tokens;
