@@ -373,4 +373,81 @@ __device__ __forceinline__ void tmem_load_sum8(uint32_t taddr, int stride, float
   }
 }
 
+// TMEM: this thread's lane, 4 columns from each of T blocks `stride`
+// columns apart, summed in block order; one wait for all loads.
+template <int T>
+__device__ __forceinline__ void tmem_load_sum4(uint32_t taddr, int stride, float *v) {
+  uint32_t r[T][4];
+#pragma unroll
+  for (int t = 0; t < T; ++t)
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[t][0]), "=r"(r[t][1]), "=r"(r[t][2]), "=r"(r[t][3])
+                 : "r"(taddr + (uint32_t)(t * stride)));
+  asm volatile("tcgen05.wait::ld.sync.aligned;");
+#pragma unroll
+  for (int t = 0; t < T; ++t)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) asm volatile("" : "+r"(r[t][c]));
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    float a = __uint_as_float(r[0][c]);
+#pragma unroll
+    for (int t = 1; t < T; ++t) a += __uint_as_float(r[t][c]);
+    v[c] = a;
+  }
+}
+
+// TMEM: 4 columns of this thread's lane.
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, const float *v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr),
+               "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+               "r"(__float_as_uint(v[3]))
+               : "memory");
+}
+
+// Four FP32 values -> F16, then kTerms E5M2 terms of the F16 values (as
+// e5_terms_f16, four values): out[t] holds term t of value i in byte i.
+template <int kTerms>
+__device__ __forceinline__ void e5_terms4(const float *x, uint32_t *out) {
+  uint32_t h[2];
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h[0]) : "f"(x[1]), "f"(x[0]));
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h[1]) : "f"(x[3]), "f"(x[2]));
+#pragma unroll
+  for (int t = 0; t < kTerms; ++t) {
+    uint32_t w[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      uint16_t e;
+      asm("cvt.rn.satfinite.e5m2x2.f16x2 %0, %1;" : "=h"(e) : "r"(h[i]));
+      w[i] = e;
+      if (t + 1 < kTerms) {
+        uint32_t back;
+        asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(back) : "h"(e));
+        asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(h[i]) : "r"(h[i]), "r"(back));
+      }
+    }
+    out[t] = w[0] | (w[1] << 16);
+  }
+}
+
+// Sum (kMax: maximum) of four per-lane values over the 32 lanes of a warp,
+// by a fixed butterfly (halving the values each lane keeps, then full
+// reductions): every lane returns the warp result of value (lane >> 3) & 3.
+template <bool kMax>
+__device__ __forceinline__ float warp_reduce4(const float *e, int lane) {
+  auto op = [](float a, float b) { return kMax ? fmaxf(a, b) : a + b; };
+  const bool b4 = lane & 16, b3 = lane & 8;
+  float w2[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float keep = b4 ? e[2 + i] : e[i], give = b4 ? e[i] : e[2 + i];
+    w2[i] = op(keep, __shfl_xor_sync(0xffffffffu, give, 16));
+  }
+  float x = op(b3 ? w2[1] : w2[0], __shfl_xor_sync(0xffffffffu, b3 ? w2[0] : w2[1], 8));
+  x = op(x, __shfl_xor_sync(0xffffffffu, x, 4));
+  x = op(x, __shfl_xor_sync(0xffffffffu, x, 2));
+  x = op(x, __shfl_xor_sync(0xffffffffu, x, 1));
+  return x;
+}
+
 }  // namespace lse_ptx

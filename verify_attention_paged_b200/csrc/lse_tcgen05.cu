@@ -379,12 +379,9 @@ __device__ __forceinline__ void column_reduce(const float *tile, int t, float *o
 struct EndRec {
   int seg_id, n_pieces, piece, row0, rows, g;
 };
-// shared memory of the epilogue and end phase: each group's published
-// per-pair maximum and row sum and its "had a tile" flag, double-buffered
-// by segment parity [2][2][64] x 2 + [2][2], then up to two end records and
-// their count
-constexpr int kPubBytes = 2 * 2 * 64 * 4 * 2 + 2 * 2 * 4;
-constexpr int kEndBytes = kPubBytes + 2 * 4 + 2 * (int)sizeof(EndRec) + 8;
+// shared memory of the end phase: a flag word pair, up to two end records
+// and their count
+constexpr int kEndBytes = 2 * 4 + 2 * (int)sizeof(EndRec) + 8;
 
 // ---- shared-memory and TMEM layout ------------------------------------------------
 
@@ -400,15 +397,18 @@ template <int DT, int P8>
 struct TcLayout {
   static constexpr bool kF8 = is_f8(DT);
   static constexpr int kNQ = (P8 + 15) / 16 * 16;       // pairs rounded to 16 (MMA N step)
+  // each softmax group takes half of the (row, head) pairs of every tile
+  static constexpr int kH = P8 / 2;
+  static_assert(kH % 4 == 0, "a group's pairs come in blocks of 4");
   // Every product carries its operand terms side by side along N, so one
   // MMA per K step covers them all (the issue of an MMA costs the same
-  // whatever its N).  Score columns per group: 16-bit, Q hi | Q lo blocks of
+  // whatever its N).  Score columns of a tile: 16-bit, Q hi | Q lo blocks of
   // kNQ; FP8, four Q-term blocks of kNQ.
   static constexpr int kSW = kF8 ? kQTerms * kNQ : 2 * kNQ;
-  // Output columns per group and slot: 16-bit, P hi | P lo blocks of P8;
-  // FP8, four P-term blocks of kNQ when they fit in TMEM, else one block
-  // that the four terms accumulate into (four MMAs per K step)
-  static constexpr bool kPSide = !kF8 || 4 * kSW <= 256;
+  // Output columns of a slot: 16-bit, P hi | P lo blocks of P8; FP8, four
+  // P-term blocks of kNQ when they fit in TMEM, else one block that the
+  // four terms accumulate into (four MMAs per K step)
+  static constexpr bool kPSide = !kF8 || 2 * kSW + kPTerms * kNQ <= 512;
   static constexpr int kOBlk = kF8 ? kNQ : P8;            // width of one output block
   static constexpr int kN = kF8 ? (kPSide ? kPTerms * kNQ : kNQ) : 2 * P8;
   static constexpr int kQRegion = kNQ * 128;             // kNQ rows of 128 bytes
@@ -421,32 +421,28 @@ struct TcLayout {
   // hi block then lo block (16-bit) or term blocks of kNQ (FP8)
   static constexpr int kPCols = kF8 ? kPTerms * kNQ : 2 * P8;
   static constexpr int kPLbo = (kF8 ? kPCols / 16 : kPCols / 8) * 128;
-  static constexpr int kPBytes = kTK / 8 * kPLbo;        // one group's P tile
-  // TMEM: S per group, then per group and output slot O^T (kN columns);
-  // two output slots when they fit
-  static constexpr int kOSlots = (2 * kSW + 4 * kN <= 512) ? 2 : 1;
-  static constexpr int kTmemNeed = 2 * kSW + 2 * kOSlots * kN;
+  static constexpr int kPBytes = kTK / 8 * kPLbo;        // one tile's P
+  // TMEM: two score buffers (tiles alternate), then the output slots (two
+  // when they fit: a piece's output is read out while the next one builds)
+  static constexpr int kOSlots = (2 * kSW + 2 * kN <= 512) ? 2 : 1;
+  static constexpr int kTmemNeed = 2 * kSW + kOSlots * kN;
   static constexpr int kTmemCols = kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                  : kTmemNeed <= 256 ? 256 : 512;
   static_assert(kTmemNeed <= 512, "TMEM holds at most 512 columns");
   static_assert(kSW <= 256 && kN <= 256, "MMA N is at most 256");
-  static constexpr int kBars = 72;
-  // row sums of P per group [2][64] and their per-warp partials
-  // [2 groups][2 buffers][4 warps][P8]
-  static constexpr int kLBytes = 2 * 64 * 4 + 2 * 2 * 4 * P8 * 4;
+  static constexpr int kBars = 64;
   static constexpr int kMiscBytes = kBars * 8 + 16 + 2 * 64 * 4 * 2 + 2 * 4 * 64 * 4 +
                                     2 * 64 * 8 * 2 + 64 * 4 + 8 * 16 + 2 * 32 * 16 * 4 +
-                                    (kF8 ? 4 * 64 * 4 : 0) + kLBytes +
+                                    (kF8 ? 4 * 64 * 4 : 0) +
                                     kSeqTab * (int)sizeof(SeqRec) + kEndBytes;
   // one K or V tile: 128 keys of 128 dims (two 64-dim regions when 16-bit)
   static constexpr int kHalfStage = kF8 ? kRegionBytes : 2 * kRegionBytes;
   // per-vector scales of one tile, K then V (128 FP32 each), per ring stage
   static constexpr int kScStage = 2 * kTK * 4;
   // k_stages / v_stages: K and V ring depths; q_slots: Q ring depth (1 or
-  // 2); p_bufs: P tiles per softmax group (1 or 2); scaled: per-vector scale
-  // rows per V stage
+  // 2); p_bufs: P tiles (1 or 2); scaled: per-vector scale rows per V stage
   static int smem_bytes(int k_stages, int v_stages, int q_slots, int p_bufs, bool scaled) {
-    return 1024 + (k_stages + v_stages) * kHalfStage + q_slots * kQBytes + 2 * p_bufs * kPBytes +
+    return 1024 + (k_stages + v_stages) * kHalfStage + q_slots * kQBytes + p_bufs * kPBytes +
            (scaled ? v_stages * kScStage : 0) + kMiscBytes;
   }
 };
@@ -458,63 +454,18 @@ enum {
   kBarEmptyK = 8,   // [8]
   kBarFullV = 16,   // [8]
   kBarEmptyV = 24,  // [8]
-  kBarSFull = 32,   // [2] per softmax group
-  kBarPFull = 34,   // [2]
+  kBarSFull = 32,   // [2] per score buffer: its product is complete
+  kBarPFull = 34,   // [2] per P tile: both groups wrote their probabilities (256)
   kBarQFull = 36,   // [2]
   kBarQEmpty = 38,  // [2]
-  kBarOFull = 40,   // [4] = group * 2 + slot
-  kBarOEmpty = 44,  // [4]
-  kBarDone = 48,     // the score issuer's MMAs have completed
-  kBarInfo = 49,    // [8] one per tile record
-  kBarPEmpty = 57,  // [4] = group * 2 + P buffer: the P tile has been read
-  kBarDoneV = 61,   // the output issuer's MMAs have completed
-  kBarSEmpty = 62,  // [2] per softmax group: its score buffer has been read out
-  kBarPub = 64,     // [2] per output slot: the non-closing group's sums and maxima are published
+  kBarOFull = 40,   // [2] per output slot: the piece's last output product is complete
+  kBarOEmpty = 42,  // [2] per output slot: both groups read it out (256)
+  kBarDone = 44,    // the score issuer's MMAs have completed
+  kBarInfo = 45,    // [8] one per tile record
+  kBarPEmpty = 53,  // [2] per P tile: the output product that read it is complete
+  kBarDoneV = 55,   // the output issuer's MMAs have completed
+  kBarSEmpty = 56,  // [2] per score buffer: both groups read it out (256)
 };
-
-// Sum of eight per-lane values over the 32 lanes of a warp, by a fixed
-// butterfly (halving the values each lane keeps, then full sums): every
-// lane returns the warp sum of value (lane >> 2).
-__device__ __forceinline__ float warp_sum8(const float *e, int lane) {
-  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
-  float w4[4], w2[2];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float keep = b4 ? e[4 + i] : e[i], give = b4 ? e[i] : e[4 + i];
-    w4[i] = keep + __shfl_xor_sync(0xffffffffu, give, 16);
-  }
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const float keep = b3 ? w4[2 + i] : w4[i], give = b3 ? w4[i] : w4[2 + i];
-    w2[i] = keep + __shfl_xor_sync(0xffffffffu, give, 8);
-  }
-  float x = (b2 ? w2[1] : w2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? w2[0] : w2[1], 4);
-  x += __shfl_xor_sync(0xffffffffu, x, 2);
-  x += __shfl_xor_sync(0xffffffffu, x, 1);
-  return x;
-}
-
-// Maximum of eight per-lane values over the 32 lanes of a warp, by the same
-// fixed butterfly as warp_sum8: every lane returns the warp maximum of value
-// (lane >> 2).
-__device__ __forceinline__ float warp_max8(const float *e, int lane) {
-  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
-  float w4[4], w2[2];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float keep = b4 ? e[4 + i] : e[i], give = b4 ? e[i] : e[4 + i];
-    w4[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, give, 16));
-  }
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const float keep = b3 ? w4[2 + i] : w4[i], give = b3 ? w4[i] : w4[2 + i];
-    w2[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, give, 8));
-  }
-  float x = fmaxf(b2 ? w2[1] : w2[0], __shfl_xor_sync(0xffffffffu, b2 ? w2[0] : w2[1], 4));
-  x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 2));
-  x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 1));
-  return x;
-}
 
 // Stage one segment's Q into a Q slot, by T threads (t = 0 .. T-1): each
 // (pair row n, 8-dim chunk c) item is scaled by the softmax scale (log2
@@ -602,7 +553,8 @@ __device__ __forceinline__ bool stage_q(const LseKernelParams &p, int t, int g, 
 
 // End phase of the fused pass: for each segment this CTA shares with other
 // CTAs, wait until every piece's partial is written (the segment's arrival
-// count reaches its number of pieces), then merge this CTA's share of the
+// count reaches two per piece: one per softmax group), then merge this CTA's
+// share of the
 // segment's (row, head) pairs: pair q goes to the segment's piece q mod n,
 // so the n CTAs of the segment split its pairs.  A pair is merged by one or
 // more warps, each taking every k-th piece with its loads issued together
@@ -632,7 +584,7 @@ __device__ __noinline__ void fused_end_merge(const TcParams &tp, const EndRec *r
       while (go) {
         unsigned int v;
         asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
-        if (v >= (unsigned)r.n_pieces) break;
+        if (v >= 2u * (unsigned)r.n_pieces) break;
         if (clock64() - t0 > kWaitCycles) {
           *abort_flag = 1;
           atomicOr(p.err, LSE_DEVERR_TIMEOUT);
@@ -758,13 +710,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t k_base = sbase;                                // K ring
   const uint32_t v_base = k_base + NK * Lay::kHalfStage;        // V ring
   const uint32_t q_base = v_base + NV * Lay::kHalfStage;        // Q slots
-  const uint32_t p_base = q_base + QS * Lay::kQBytes;          // P tiles [group][buffer]
-  const uint32_t sc_base = p_base + 2 * PB * Lay::kPBytes;     // scale rows [stage]
+  const uint32_t p_base = q_base + QS * Lay::kQBytes;          // P tiles [buffer]
+  const uint32_t sc_base = p_base + PB * Lay::kPBytes;         // scale rows [stage]
   uint8_t *misc = smem + (sc_base - sbase) + (kSc ? NV * Lay::kScStage : 0);
-  // the P tile of group grp used with its tile of index n (n & 1 == grp)
-  auto p_tile = [&](int grp, int n) {
-    return p_base + (uint32_t)((grp * PB + ((n >> 1) % PB)) * Lay::kPBytes);
-  };
+  // the P tile of tile n
+  auto p_tile = [&](int n) { return p_base + (uint32_t)((n % PB) * Lay::kPBytes); };
   uint64_t *bars = reinterpret_cast<uint64_t *>(misc);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + Lay::kBars * 8);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + Lay::kBars * 8 + 4);
@@ -785,18 +735,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // FP8: the inverse of Q's per-pair scale, per Q slot [0, 2) and the
   // copy each softmax group keeps for its segment [2, 4)
   float *isig_all = reinterpret_cast<float *>(page_buf + 2 * 32 * 16);       // [4][64]
-  // row sums of P per softmax group, and each warp's partial sums of the
-  // group's latest tile (double buffered)
-  float *lsum_all = isig_all + (kF8 ? 4 * 64 : 0);                           // [2][64]
-  float *lpart_all = lsum_all + 2 * 64;                                      // [2][2][4][P8]
-  SeqRec *seq_tab = reinterpret_cast<SeqRec *>(lpart_all + 2 * 2 * 4 * P8);  // [kSeqTab]
-  // per-pair statistics a group publishes for the other one at a piece's
-  // end: [segment parity][group][pair]; a group resets its own running
-  // state at the next segment while the other may still be reading these
-  float *pub_m = reinterpret_cast<float *>(seq_tab + kSeqTab);              // [2][2][64]
-  float *pub_l = pub_m + 2 * 2 * 64;                                         // [2][2][64]
-  int *pub_had = reinterpret_cast<int *>(pub_l + 2 * 2 * 64);                // [2][2]
-  int *had_all = pub_had + 4;                                                // [2] (end phase)
+  SeqRec *seq_tab =
+      reinterpret_cast<SeqRec *>(isig_all + (kF8 ? 4 * 64 : 0));            // [kSeqTab]
+  int *had_all = reinterpret_cast<int *>(seq_tab + kSeqTab);                 // [2] (end phase)
   EndRec *end_rec = reinterpret_cast<EndRec *>(had_all + 2);                 // [2]
   int *n_end = reinterpret_cast<int *>(end_rec + 2);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
@@ -865,6 +806,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && bad && cta == 0) atomicOr(p.err, LSE_DEVERR_BAD_LENGTH);
   }
   const SeqRec *tab = use_tab ? seq_tab : nullptr;
+  if (tid < 64) pair_row[tid] = tid / p.group;
   if (tid == 32) {
     *abort_flag = 0;
     for (int i = 0; i < 8; ++i) {
@@ -873,17 +815,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(kBarFullV + i), 1);
       mbar_init(bar(kBarEmptyV + i), 1);
     }
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarOFull + i), 1);
-      // released by the group that combines the piece (it read both blocks)
-      mbar_init(bar(kBarOEmpty + i), 128);
+      mbar_init(bar(kBarOEmpty + i), 256);  // both groups read their pairs out
     }
-    for (int i = 0; i < 2; ++i) mbar_init(bar(kBarPub + i), 128);
     *n_end = 0;
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarSFull + i), 1);
-      mbar_init(bar(kBarSEmpty + i), 128);
-      mbar_init(bar(kBarPFull + i), 128);
+      mbar_init(bar(kBarSEmpty + i), 256);  // both groups read their columns
+      mbar_init(bar(kBarPFull + i), 256);   // both groups wrote their columns
       mbar_init(bar(kBarQFull + i), 1);
       // FP8: the softmax groups also hold the slot until they have copied
       // the segment's Q scales
@@ -892,10 +832,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(kBarDone), 1);
     mbar_init(bar(kBarDoneV), 1);
     for (int i = 0; i < 8; ++i) mbar_init(bar(kBarInfo + i), 1);
-    for (int i = 0; i < 4; ++i) mbar_init(bar(kBarPEmpty + i), 1);
+    for (int i = 0; i < 2; ++i) mbar_init(bar(kBarPEmpty + i), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (tid < 64) pair_row[tid] = tid / p.group;
+        }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -913,11 +852,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const long long t_begin = U * cta / C, t_stop = U * (cta + 1) / C;
   constexpr int kSW = Lay::kSW;
-  auto tmem_s = [&](int grp) { return tmem + (uint32_t)(grp * kSW); };
+  // score buffer of tile n: n & 1; output slot of the CTA's segment seg: seg % kOS
+  auto tmem_s = [&](int buf) { return tmem + (uint32_t)(buf * kSW); };
   constexpr int kOS = Lay::kOSlots;
-  auto tmem_o = [&](int grp, int slot) {
-    return tmem + (uint32_t)(2 * kSW + (grp * kOS + slot) * kN);
-  };
+  auto tmem_o = [&](int slot) { return tmem + (uint32_t)(2 * kSW + slot * kN); };
 
   const int box_t = tp.box_tokens;
   const int nbox = box_t >= kTK ? 1 : kTK / box_t;
@@ -1036,37 +974,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(bar(kBarDone), leader);
       mbar_drain(bar(kBarDone), 0);
     } else {
-      // ---- O^T += V^T P^T into the group's output slot ----
+      // ---- O^T += V^T P^T into the piece's output slot ----
       constexpr uint32_t idesc_pv =
           instr_desc(kvfmt, pfmt, 1, 1, kD, (kF8 && !Lay::kPSide) ? kNQ : kN);
       TileIter iv;
       iv.init(p, t_begin, t_stop, tab);
       int seg_v = -1;
-      uint32_t started = 0;  // bit g: group g has an output product in this piece
 #pragma unroll 1
       for (int nv = 0; nv < n_total; ++nv, iv.advance(p)) {
         const bool first = iv.seg_start(t_begin), last = iv.seg_end();
-        if (first) {
-          ++seg_v;
-          started = 0;
-        }
-        const int grp = nv & 1, slot = seg_v % kOS;
-        const uint32_t oe_par = ((seg_v / kOS) & 1) ^ 1;
+        if (first) ++seg_v;
+        const int slot = seg_v % kOS;
         const int st = nv % NV;
-        bool go = mbar_wait(bar(kBarPFull + grp), (nv >> 1) & 1, abort_flag, p.err);
+        // both groups' probabilities of tile nv, its V tile, and (for the
+        // piece's first product) the slot's previous piece read out
+        bool go = mbar_wait(bar(kBarPFull + nv % PB), (nv / PB) & 1, abort_flag, p.err);
         go = go && mbar_wait(bar(kBarFullV + st), (nv / NV) & 1, abort_flag, p.err);
-        // a group's output slot must have been read out kOS segments ago
-        const bool mine = (started >> grp) & 1u, other = (started >> (grp ^ 1)) & 1u;
-        if (!mine)
-          go = go && mbar_wait(bar(kBarOEmpty + 2 * grp + slot), oe_par, abort_flag, p.err);
-        if (last && !other)
-          go = go && mbar_wait(bar(kBarOEmpty + 2 * (grp ^ 1) + slot), oe_par, abort_flag, p.err);
+        if (first)
+          go = go && mbar_wait(bar(kBarOEmpty + slot), ((seg_v / kOS) & 1) ^ 1, abort_flag,
+                               p.err);
         if (!__all_sync(0xffffffffu, go)) break;
         tc_fence_after();
         const uint32_t vaddr = v_base + st * Lay::kHalfStage;
-        const uint32_t paddr = p_tile(grp, nv);
-        const uint32_t d = tmem_o(grp, slot);
-        const uint64_t b0 = smem_desc(paddr, Lay::kPLbo, 128, kLayoutNone);
+        const uint32_t d = tmem_o(slot);
+        const uint64_t b0 = smem_desc(p_tile(nv), Lay::kPLbo, 128, kLayoutNone);
         if constexpr (kF8) {
           // V^T is MN-major with one 128-byte swizzle atom across the dims
           // (LBO unused); K steps of 32 keys
@@ -1077,13 +1008,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t b = b0 + (uint64_t)(k * 4 * Lay::kPLbo / 16);
             if constexpr (Lay::kPSide) {
               // the P terms side by side along N
-              mma_f8(d, a, b, idesc_pv, (mine || k > 0) ? 1u : 0u, leader);
+              mma_f8(d, a, b, idesc_pv, (!first || k > 0) ? 1u : 0u, leader);
             } else {
               // the P terms accumulate into the same columns
 #pragma unroll
               for (int t = 0; t < kPTerms; ++t)
                 mma_f8(d, a, b + (uint64_t)(t * (kNQ / 16) * 128 / 16), idesc_pv,
-                       (mine || k > 0 || t > 0) ? 1u : 0u, leader);
+                       (!first || k > 0 || t > 0) ? 1u : 0u, leader);
             }
           }
         } else {
@@ -1092,19 +1023,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < kTK / 16; ++k)
             mma_f16(d, a0 + (uint64_t)(k * 2048 / 16), b0 + (uint64_t)(k * 2 * Lay::kPLbo / 16),
-                    idesc_pv, (mine || k > 0) ? 1u : 0u, leader);
+                    idesc_pv, (!first || k > 0) ? 1u : 0u, leader);
         }
-        started |= 1u << grp;
         mma_commit(bar(kBarEmptyV + st), leader);
-        mma_commit(bar(kBarPEmpty + 2 * grp + ((nv >> 1) % PB)), leader);
-        // this group's last tile of the piece: the tile is the piece's
-        // last, or the next one (the other group's) is
-        const bool next_is_last =
-            !last && (iv.t + 1 == iv.t_end - 1 || iv.tile + 1 == iv.n_tiles - 1);
-        if (last || next_is_last) mma_commit(bar(kBarOFull + 2 * grp + slot), leader);
-        // the other group had no tile in this piece: release its (empty)
-        // output slot all the same (its previous use was read out)
-        if (last && !other) mma_commit(bar(kBarOFull + 2 * (grp ^ 1) + slot), leader);
+        mma_commit(bar(kBarPEmpty + nv % PB), leader);
+        if (last) mma_commit(bar(kBarOFull + slot), leader);
       }
       mma_commit(bar(kBarDoneV), leader);
       mbar_drain(bar(kBarDoneV), 0);
@@ -1132,42 +1055,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ============== softmax and epilogue: two groups of 128 threads ==============
-    // Scores are read from TMEM eight pairs at a time in loops whose code does
-    // not grow with the pair count.  The row sums of P are summed here: each
-    // warp reduces its 32 keys per pair, and the four warps' partials are
-    // folded into the group's sums after the next group barrier, in a fixed
-    // order (so results repeat bit for bit).
-    const int grp = (warp - 4) >> 2;           // tiles of this parity
+    // Both groups work on every tile, each on half of the (row, head) pairs:
+    // group g takes pairs [g H, g H + H), H = P8 / 2, so a tile's softmax
+    // takes half as long and the groups never combine results.  Thread j of
+    // a group owns key j of the tile (its TMEM lane), reads its half of the
+    // key's scores four pairs at a time, keeps the key's sums of P per pair
+    // in registers over the segment, and the four warps' sums meet once per
+    // piece (a warp butterfly, then a fixed-order fold).
+    constexpr int kHq = Lay::kH;
+    const int grp = (warp - 4) >> 2;
+    const int q0 = grp * kHq;                  // this group's first pair
     const int j = tid - 128 - grp * 128;       // key of the tile = TMEM lane (scores)
     const int quarter = warp & 3;              // TMEM lane quarter of this warp
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const int bar_id = 1 + grp;
-    float *m_run = m_run_all + grp * 64;
-    float *alpha = alpha_all + grp * 64;
-    float *red = red_all + grp * 4 * 64;
+    float *m_run = m_run_all + grp * 64;       // indexed by pair
+    float *alpha = alpha_all + grp * 64;       // (at a piece's end: the pairs' row sums)
+    float *red = red_all + grp * 4 * 64;       // [warp quarter][pair]
     unsigned long long *masks = masks_all + grp * 64;
     unsigned long long *visk = visk_all + grp * 64;
-    // FP32 scratch [key][pair] in one of the group's P tiles
-    auto scratch = [&](int tile_n) {
-      return reinterpret_cast<float *>(smem + (p_tile(grp, tile_n) - sbase));
-    };
     float *isg = isig_all + (2 + grp) * 64;    // FP8: the segment's inverse Q scales
-    float *lsum = lsum_all + grp * 64;         // row sums of P of the segment so far
-    float *lpart = lpart_all + grp * 2 * 4 * P8;  // [buffer][warp][pair] partials
-    bool pend = false;                         // partials of buffer pbuf not yet folded
-    int pbuf = 0;
-    auto fold = [&]() {
-      if (pend && j < P8) {
-        const float *pp = lpart + pbuf * 4 * P8 + j;
-        lsum[j] += ((pp[0] + pp[P8]) + pp[2 * P8]) + pp[3 * P8];
-      }
-      pend = false;
-    };
-    // Up to 32 pairs each thread keeps its key's sums of P over the segment
-    // in registers (one column reduction per segment); beyond that, each
-    // tile's sums are reduced across the warp and folded into lsum.
-    constexpr bool kLAcc = P8 <= 32;
-    float lacc[kLAcc ? P8 : 1];
+    float lacc[kHq];
     TileIter it;
     it.init(p, t_begin, t_stop, tab);
     int n = 0, seg = -1;
@@ -1182,14 +1090,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++seg;
         // a finite floor keeps exp2(-inf - m) at 0 (never NaN) for pairs
         // with no visible key yet
-        if (j < P8) {
-          m_run[j] = -FLT_MAX;
-          lsum[j] = 0.f;
-        }
-        if constexpr (kLAcc) {
+        if (j < kHq) m_run[q0 + j] = -FLT_MAX;
 #pragma unroll
-          for (int q = 0; q < P8; ++q) lacc[q] = 0.f;
-        }
+        for (int q = 0; q < kHq; ++q) lacc[q] = 0.f;
         if (j < it.crows(p)) {
           // the chunk's rows; the default mask is the chain (row r sees drafts
           // 0 .. r of its sequence)
@@ -1231,276 +1134,225 @@ __global__ void __launch_bounds__(kThreads, 1)
           visk[j] = v;
         }
       }
-      if ((n & 1) == grp) {
-        bool w = mbar_wait(bar(kBarSFull + grp), (n >> 1) & 1, abort_flag, p.err);
-        tc_fence_after();
-        // tile record, published by the producer on its own barrier (the
-        // K ring may already hold a later tile)
-        if (w) w = mbar_wait(bar(kBarInfo + (n & 7)), (n >> 3) & 1, abort_flag, p.err);
-        // (this tile's P buffer is waited for just before pass 2 writes it)
-        const int pbuf_n = (n >> 1) % PB, use = (n >> 1) / PB;
-        // per-vector scales land with the tile's V (the V slot outlives
-        // this pass: its output product waits for this tile's P)
-        if (kSc && w)
-          w = mbar_wait(bar(kBarFullV + n % NV), (n / NV) & 1, abort_flag, p.err);
-        if (named_or(bar_id, 128, !w)) {
-          ok = false;
-          break;
+      // ---- tile n: this group's pairs ----
+      bool w = mbar_wait(bar(kBarSFull + (n & 1)), (n >> 1) & 1, abort_flag, p.err);
+      tc_fence_after();
+      // tile record, published by the producer on its own barrier (the K ring
+      // may already hold a later tile)
+      if (w) w = mbar_wait(bar(kBarInfo + (n & 7)), (n >> 3) & 1, abort_flag, p.err);
+      // per-vector scales land with the tile's V (the V slot outlives this
+      // pass: its output product waits for this tile's P)
+      if (kSc && w) w = mbar_wait(bar(kBarFullV + n % NV), (n / NV) & 1, abort_flag, p.err);
+      if (named_or(bar_id, 128, !w)) {
+        ok = false;
+        break;
+      }
+      const uint4 inf = tile_info[n & 7];
+      const int key0 = it.tile * kTK;
+      const int key = key0 + j;
+      const uint32_t both = inf.x & inf.y;
+      const bool kvalid = j < (int)inf.z && (both >> (j / box_t) & 1u);
+      // Per-vector scales.  The key's score is multiplied by its K scale;
+      // its V scale sV enters through the probability: with u = x + log2 sV
+      // in place of the score x, the running max and P follow u, P.V sums
+      // 2^(u - m) V = 2^(x - m) sV V, and the row sums add 2^(u - m) / sV =
+      // 2^(x - m), so the output and log-sum-exp come out unchanged while P
+      // stays within the range the unscaled path gives it.  (A V scale
+      // below 2^-64 is read as 2^-64; a dead key keeps unit scales.)
+      float ks = 1.f, lv = 0.f, ivs = 1.f;
+      if constexpr (kSc) {
+        if (kvalid) {
+          const float *scs = reinterpret_cast<const float *>(
+              smem + (sc_base - sbase) + (n % NV) * Lay::kScStage);
+          ks = scs[j];
+          float vs = scs[kTK + j];
+          vs = vs < 0x1p-64f ? 0x1p-64f : vs;  // (NaN stays NaN)
+          lv = log2f(vs);
+          ivs = 1.f / vs;
         }
-        const uint4 inf = tile_info[n & 7];
-        const int key0 = it.tile * kTK;
-        const int key = key0 + j;
-        const uint32_t both = inf.x & inf.y;
-        const bool kvalid = j < (int)inf.z && (both >> (j / box_t) & 1u);
-        // Per-vector scales.  The key's score is multiplied by its K scale;
-        // its V scale sV enters through the probability: with u = x + log2 sV
-        // in place of the score x, the running max and P follow u, P.V sums
-        // 2^(u - m) V = 2^(x - m) sV V, and the row sums add 2^(u - m) / sV =
-        // 2^(x - m), so the output and log-sum-exp come out unchanged while P
-        // stays within the range the unscaled path gives it.  (A V scale
-        // below 2^-64 is read as 2^-64; a dead key keeps unit scales.)
-        float ks = 1.f, lv = 0.f, ivs = 1.f;
-        if constexpr (kSc) {
-          if (kvalid) {
-            const float *scs = reinterpret_cast<const float *>(
-                smem + (sc_base - sbase) + (n % NV) * Lay::kScStage);
-            ks = scs[j];
-            float vs = scs[kTK + j];
-            vs = vs < 0x1p-64f ? 0x1p-64f : vs;  // (NaN stays NaN)
-            lv = log2f(vs);
-            ivs = 1.f / vs;
-          }
+      }
+      // visibility of this key to each pair, as a bit mask
+      unsigned long long vis;
+      if (key0 + kTK <= Cctx && inf.z == (uint32_t)kTK && both == full_boxes) {
+        vis = ~0ull;  // context tile (pairs past P have zero Q rows; never read)
+      } else {
+        vis = 0;
+        if (kvalid) {
+          vis = key < Cctx ? (P >= 64 ? ~0ull : ((1ull << P) - 1ull)) : visk[key - Cctx];
         }
-        // visibility of this key to each pair, as a bit mask
-        unsigned long long vis;
-        if (key0 + kTK <= Cctx && inf.z == (uint32_t)kTK && both == full_boxes) {
-          vis = ~0ull;  // context tile (pairs past P have zero Q rows; never read)
-        } else {
-          vis = 0;
-          if (kvalid) {
-            vis = key < Cctx ? (P >= 64 ? ~0ull : ((1ull << P) - 1ull)) : visk[key - Cctx];
-          }
+      }
+      const uint32_t s_addr = tmem_s(n & 1) + lane_off;
+      __syncwarp();
+      // pass 1: this group's scores into registers, the score terms summed
+      // (16-bit: Q hi and lo blocks; FP8: four Q-term blocks, times the
+      // pair's inverse Q scale), -inf where not visible; does any score pass
+      // the running max by 2^tau?
+      float sv[kHq], mr[kHq];
+#pragma unroll
+      for (int i = 0; i < kHq; i += 4) tmem_load_sum4<kSW / kNQ>(s_addr + q0 + i, kNQ, sv + i);
+      // the scores are in registers: the next score product into this
+      // buffer may overwrite it while the probabilities are built
+      tc_fence_before();
+      mbar_arrive(bar(kBarSEmpty + (n & 1)));
+      if constexpr (kF8) {
+#pragma unroll
+        for (int i = 0; i < kHq; ++i) sv[i] *= isg[q0 + i];
+      }
+      if constexpr (kSc) {
+#pragma unroll
+        for (int i = 0; i < kHq; ++i) sv[i] = fmaf(sv[i], ks, lv);
+      }
+      if (vis != ~0ull) {
+#pragma unroll
+        for (int i = 0; i < kHq; ++i)
+          if (!((vis >> (q0 + i)) & 1ull)) sv[i] = -INFINITY;
+      }
+#pragma unroll
+      for (int i = 0; i < kHq; i += 4) {
+        const float4 m4 = *reinterpret_cast<const float4 *>(m_run + q0 + i);
+        mr[i] = m4.x;
+        mr[i + 1] = m4.y;
+        mr[i + 2] = m4.z;
+        mr[i + 3] = m4.w;
+      }
+      float gap = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < kHq; ++i) gap = fmaxf(gap, sv[i] - mr[i]);
+      if (named_or(bar_id, 128, gap > kTau)) {
+        // per-pair maximum over the tile's keys: each warp folds its 32
+        // keys by a butterfly, and the four warps' maxima meet in red
+#pragma unroll
+        for (int i = 0; i < kHq; i += 4) {
+          const float wm = warp_reduce4<true>(sv + i, lane);
+          if ((lane & 7) == 0) red[quarter * 64 + q0 + i + ((lane >> 3) & 3)] = wm;
         }
-        const uint32_t s_addr = tmem_s(grp) + lane_off;
-        __syncwarp();
-        if constexpr (!kLAcc) fold();  // the previous tile's partials (written before the barrier above)
-        // pass 1: the key's scores into registers, the score terms summed
-        // (16-bit: Q hi and lo blocks; FP8: four Q-term blocks, times the
-        // pair's inverse Q scale), -inf where not visible; does any score pass
-        // the running max by 2^tau?
-        float sv[P8], mr[P8];
-#pragma unroll
-        for (int c = 0; c < P8; c += 8) tmem_load_sum8<kSW / kNQ>(s_addr + c, kNQ, sv + c);
-        // the scores are in registers: the group's next score product may
-        // overwrite the buffer while this tile's probabilities are built
-        tc_fence_before();
-        mbar_arrive(bar(kBarSEmpty + grp));
-        if constexpr (kF8) {
-#pragma unroll
-          for (int q = 0; q < P8; ++q) sv[q] *= isg[q];
+        named_sync(bar_id, 128);
+        if (j < kHq) {
+          const int q = q0 + j;
+          const float mo = m_run[q];
+          const float mn = fmaxf(mo, fmaxf(fmaxf(red[q], red[64 + q]),
+                                           fmaxf(red[128 + q], red[192 + q])));
+          alpha[q] = ex2(mo - mn);
+          m_run[q] = mn;
         }
-        if constexpr (kSc) {
+        named_sync(bar_id, 128);
 #pragma unroll
-          for (int q = 0; q < P8; ++q) sv[q] = fmaf(sv[q], ks, lv);
-        }
-        if (vis != ~0ull) {
-#pragma unroll
-          for (int q = 0; q < P8; ++q)
-            if (!((vis >> q) & 1ull)) sv[q] = -INFINITY;
+        for (int i = 0; i < kHq; i += 4) {
+          const float4 m4 = *reinterpret_cast<const float4 *>(m_run + q0 + i);
+          mr[i] = m4.x;
+          mr[i + 1] = m4.y;
+          mr[i + 2] = m4.z;
+          mr[i + 3] = m4.w;
         }
 #pragma unroll
-        for (int q = 0; q < P8; q += 4) {
-          const float4 m4 = *reinterpret_cast<const float4 *>(m_run + q);
-          mr[q] = m4.x;
-          mr[q + 1] = m4.y;
-          mr[q + 2] = m4.z;
-          mr[q + 3] = m4.w;
-        }
-        float gap = -INFINITY;
-#pragma unroll
-        for (int q = 0; q < P8; ++q) gap = fmaxf(gap, sv[q] - mr[q]);
-        if (named_or(bar_id, 128, gap > kTau)) {
-          // per-pair maximum over the tile's keys: each warp folds its 32
-          // keys by a butterfly, and the four warps' maxima meet in red
-          // [warp quarter][pair]
-#pragma unroll
-          for (int c = 0; c < P8; c += 8) {
-            const float wm = warp_max8(sv + c, lane);
-            if ((lane & 3) == 0) red[quarter * 64 + c + (lane >> 2)] = wm;
-          }
-          named_sync(bar_id, 128);
-          if (j < P8) {
-            const float mo = m_run[j];
-            const float mn = fmaxf(mo, fmaxf(fmaxf(red[j], red[64 + j]),
-                                             fmaxf(red[128 + j], red[192 + j])));
-            const float al = ex2(mo - mn);
-            alpha[j] = al;
-            m_run[j] = mn;
-            lsum[j] *= al;  // (this thread folded pair j's partials above)
-          }
-          named_sync(bar_id, 128);
-#pragma unroll
-          for (int q = 0; q < P8; q += 4) {
-            const float4 m4 = *reinterpret_cast<const float4 *>(m_run + q);
-            mr[q] = m4.x;
-            mr[q + 1] = m4.y;
-            mr[q + 2] = m4.z;
-            mr[q + 3] = m4.w;
-          }
-          if constexpr (kLAcc) {
-#pragma unroll
-            for (int q = 0; q < P8; ++q) lacc[q] *= alpha[q];
-          }
-          if (had_tile) {
-            // rescale this group's output once every earlier P.V of the group
-            // has completed: the output products complete in issue order, so
-            // the one of the group's previous tile (n - 2) covers them all
-            const int pn = (n - 2) >> 1;
-            const bool wo = mbar_wait(bar(kBarPEmpty + 2 * grp + pn % PB), (pn / PB) & 1,
-                                      abort_flag, p.err);
-            if (named_or(bar_id, 128, !wo)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            __syncwarp();
-            const uint32_t ob = tmem_o(grp, oslot) + lane_off;
-#pragma unroll 1
-            for (int c = 0; c < kN; c += 8) {
-              const int cc = c % Lay::kOBlk;
-              if (cc >= P8) continue;  // padding columns
-              float v[8];
-              tmem_load<8>(ob + c, v);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) v[i] *= alpha[cc + i];
-              tmem_st8(ob + c, v);
-            }
-            tmem_st_wait();
-          }
-        }
-        // this tile's P buffer is free once the output product that last
-        // read it (the group's tile n - 2 PB) has completed
-        if (use >= 1) {
-          const bool wp =
-              mbar_wait(bar(kBarPEmpty + 2 * grp + pbuf_n), (use - 1) & 1, abort_flag, p.err);
-          if (named_or(bar_id, 128, !wp)) {
+        for (int i = 0; i < kHq; ++i) lacc[i] *= alpha[q0 + i];
+        if (had_tile) {
+          // rescale this group's output columns once every earlier output
+          // product has completed (they complete in issue order: the one of
+          // tile n - 1 covers them all)
+          const bool wo = mbar_wait(bar(kBarPEmpty + (n - 1) % PB), ((n - 1) / PB) & 1,
+                                    abort_flag, p.err);
+          if (named_or(bar_id, 128, !wo)) {
             ok = false;
             break;
           }
-        }
-        // pass 2: probabilities -> this group's P tile, row j (16-bit: hi block
-        // then lo block; FP8: P 2^7 as kPTerms E5M2 terms, a block each), and
-        // this warp's sums of them per pair
-        uint8_t *prow = smem + (p_tile(grp, n) - sbase) + (j >> 3) * Lay::kPLbo + (j & 7) * 16;
-        const int buf = (n >> 1) & 1;
-        float *lp = lpart + buf * 4 * P8 + quarter * P8;
-#pragma unroll
-        for (int c = 0; c < P8; c += 8) {
-          float e[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) e[i] = ex2(sv[c + i] - mr[c + i]);  // 0 where not visible
-          if constexpr (kF8) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) e[i] *= (float)(1 << kPScaleLog2);
-            uint2 w[kPTerms];
-            e5_terms_f16<kPTerms>(e, w);
-            // 16 FP8 columns per core matrix: term t's pair c sits in column
-            // t kNQ + c
-#pragma unroll
-            for (int t = 0; t < kPTerms; ++t) {
-              const int col = t * kNQ + c;
-              *reinterpret_cast<uint2 *>(prow + (col >> 4) * 128 + ((col >> 3) & 1) * 8) = w[t];
-            }
-          } else {
-            uint4 vh, vl;
-            split2<DT>(e[0], e[1], vh.x, vl.x);
-            split2<DT>(e[2], e[3], vh.y, vl.y);
-            split2<DT>(e[4], e[5], vh.z, vl.z);
-            split2<DT>(e[6], e[7], vh.w, vl.w);
-            *reinterpret_cast<uint4 *>(prow + (c >> 3) * 128) = vh;
-            *reinterpret_cast<uint4 *>(prow + ((P8 + c) >> 3) * 128) = vl;
-          }
-          if constexpr (kLAcc) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) lacc[c + i] = kSc ? fmaf(e[i], ivs, lacc[c + i])
-                                                          : lacc[c + i] + e[i];
-          } else {
-            if constexpr (kSc) {
-#pragma unroll
-              for (int i = 0; i < 8; ++i) e[i] *= ivs;  // (P was stored above)
-            }
-            const float ws = warp_sum8(e, lane);
-            if ((lane & 3) == 0) lp[c + (lane >> 2)] = ws;
-          }
-        }
-        pend = !kLAcc;
-        pbuf = buf;
-        if (!kvalid) {
-          // a dead slot may hold any bits: give it a zero V row (P is 0 there)
-          mbar_wait(bar(kBarFullV + n % NV), (n / NV) & 1, abort_flag, p.err);
-          uint8_t *v0 = smem + (v_base - sbase) + (n % NV) * Lay::kHalfStage + j * 128;
-          constexpr int kChunks = kF8 ? 8 : 16;  // 16-byte chunks of the row
+          tc_fence_after();
+          __syncwarp();
+          const uint32_t ob = tmem_o(oslot) + lane_off;
 #pragma unroll 1
-          for (int c = 0; c < kChunks; ++c)
-            *reinterpret_cast<uint4 *>(v0 + (c >> 3) * kRegionBytes + (c & 7) * 16) =
-                make_uint4(0, 0, 0, 0);
+          for (int blk = 0; blk < kN / Lay::kOBlk; ++blk)
+#pragma unroll 1
+            for (int i = 0; i < kHq; i += 4) {
+              const uint32_t col = (uint32_t)(blk * Lay::kOBlk + q0 + i);
+              float v[4];
+              tmem_load_sum4<1>(ob + col, 0, v);
+#pragma unroll
+              for (int u = 0; u < 4; ++u) v[u] *= alpha[q0 + i + u];
+              tmem_st4(ob + col, v);
+            }
+          tmem_st_wait();
         }
-        fence_proxy_async();
-        tc_fence_before();
-        mbar_arrive(bar(kBarPFull + grp));
-        had_tile = true;
       }
+      // this tile's P buffer is free once the output product that last read
+      // it (tile n - PB) has completed
+      if (n >= PB) {
+        const bool wp =
+            mbar_wait(bar(kBarPEmpty + n % PB), ((n / PB) - 1) & 1, abort_flag, p.err);
+        if (named_or(bar_id, 128, !wp)) {
+          ok = false;
+          break;
+        }
+      }
+      // pass 2: probabilities of this group's pairs -> the tile's P tile, row
+      // j (16-bit: hi block then lo block; FP8: P 2^7 as kPTerms E5M2 terms,
+      // a block each), and this thread's sums of them per pair
+      uint8_t *prow = smem + (p_tile(n) - sbase) + (j >> 3) * Lay::kPLbo + (j & 7) * 16;
+#pragma unroll
+      for (int i = 0; i < kHq; i += 4) {
+        float e[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) e[u] = ex2(sv[i + u] - mr[i + u]);  // 0 where not visible
+        if constexpr (kF8) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) e[u] *= (float)(1 << kPScaleLog2);
+          uint32_t wt[kPTerms];
+          e5_terms4<kPTerms>(e, wt);
+          // 16 FP8 columns per core matrix: term t's pair q sits in column
+          // t kNQ + q
+#pragma unroll
+          for (int t = 0; t < kPTerms; ++t) {
+            const int col = t * kNQ + q0 + i;
+            *reinterpret_cast<uint32_t *>(prow + (col >> 4) * 128 + (col & 15)) = wt[t];
+          }
+        } else {
+          uint32_t h0, l0, h1, l1;
+          split2<DT>(e[0], e[1], h0, l0);
+          split2<DT>(e[2], e[3], h1, l1);
+          // 8 16-bit columns per core matrix: pair q's hi term in column q,
+          // its lo term in column P8 + q
+          const int ch = q0 + i, cl = P8 + q0 + i;
+          *reinterpret_cast<uint2 *>(prow + (ch >> 3) * 128 + (ch & 7) * 2) = make_uint2(h0, h1);
+          *reinterpret_cast<uint2 *>(prow + (cl >> 3) * 128 + (cl & 7) * 2) = make_uint2(l0, l1);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) lacc[i + u] = kSc ? fmaf(e[u], ivs, lacc[i + u])
+                                                      : lacc[i + u] + e[u];
+      }
+      if (!kvalid && grp == 0) {
+        // a dead slot may hold any bits: give it a zero V row (P is 0 there)
+        mbar_wait(bar(kBarFullV + n % NV), (n / NV) & 1, abort_flag, p.err);
+        uint8_t *v0 = smem + (v_base - sbase) + (n % NV) * Lay::kHalfStage + j * 128;
+        constexpr int kChunks = kF8 ? 8 : 16;  // 16-byte chunks of the row
+#pragma unroll 1
+        for (int c = 0; c < kChunks; ++c)
+          *reinterpret_cast<uint4 *>(v0 + (c >> 3) * kRegionBytes + (c & 7) * 16) =
+              make_uint4(0, 0, 0, 0);
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      mbar_arrive(bar(kBarPFull + n % PB));
+      had_tile = true;
 
       if (last) {
-        // ---- epilogue of the piece: the two groups' results combined ----
-        const bool w = mbar_wait(bar(kBarOFull + 2 * grp + oslot), (seg / kOS) & 1, abort_flag,
-                                 p.err);
-        if (named_or(bar_id, 128, !w)) {
+        // ---- epilogue of the piece: this group's pairs ----
+        const bool we = mbar_wait(bar(kBarOFull + oslot), (seg / kOS) & 1, abort_flag, p.err);
+        if (named_or(bar_id, 128, !we)) {
           ok = false;
           break;
         }
-        if constexpr (kLAcc) {
-          // column sums of the threads' sums, through one of the group's P
-          // tiles as FP32 scratch [key][pair] (free: the piece's last P.V has
-          // completed)
-          float *scr = scratch(grp);
+        // the row sums of P: each warp folds its 32 keys per pair, the four
+        // warps' sums are added in a fixed order (results repeat bit for bit)
 #pragma unroll
-          for (int c = 0; c < P8; c += 4)
-            *reinterpret_cast<float4 *>(scr + j * P8 + c) =
-                make_float4(lacc[c], lacc[c + 1], lacc[c + 2], lacc[c + 3]);
-          named_sync(bar_id, 128);
-          column_reduce<P8, true>(scr, j, red, bar_id);  // red[q] = sum over keys
-        } else {
-          fold();  // the group's last tile's partials
+        for (int i = 0; i < kHq; i += 4) {
+          const float ws = warp_reduce4<false>(lacc + i, lane);
+          if ((lane & 7) == 0) red[quarter * 64 + q0 + i + ((lane >> 3) & 3)] = ws;
         }
-        // publish this group's per-pair maximum and row sum (its running
-        // copies are reset at its next segment, maybe before the other group
-        // has read them)
-        const int pb = seg & 1;
-        if (j < P8) {
-          pub_m[(pb * 2 + grp) * 64 + j] = m_run[j];
-          pub_l[(pb * 2 + grp) * 64 + j] = kLAcc ? red[j] : lsum[j];
+        named_sync(bar_id, 128);
+        if (j < kHq) {
+          const int q = q0 + j;
+          alpha[q] = ((red[q] + red[64 + q]) + red[128 + q]) + red[192 + q];
         }
-        if (j == 0) pub_had[pb * 2 + grp] = had_tile ? 1 : 0;
-        // The group that ran the piece's last tile closes the piece: it
-        // combines both groups' results.  The other group has finished its
-        // part earlier; it publishes its sums and maxima and goes on to its
-        // next segment (on its other output slot, or after the closer frees
-        // this one), never waiting for the closer.
-        const bool closer = (n & 1) == grp;
-        if (!closer) {
-          tc_fence_before();
-          mbar_arrive(bar(kBarPub + oslot));
-          continue;
-        }
-        const int other = grp ^ 1;
-        bool wm = mbar_wait(bar(kBarPub + oslot), (seg / kOS) & 1, abort_flag, p.err);
-        wm = wm && mbar_wait(bar(kBarOFull + 2 * other + oslot), (seg / kOS) & 1, abort_flag,
-                             p.err);
-        if (named_or(bar_id, 128, !wm)) {
-          ok = false;
-          break;
-        }
+        named_sync(bar_id, 128);
         tc_fence_after();
         __syncwarp();
         // the piece: its place among the segment's pieces
@@ -1508,34 +1360,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int c_last = cta_of_tile(it.seg_first + it.n_tiles - 1, U, C);
         const int n_pieces = c_last - c_first + 1, piece = cta - c_first;
         const bool direct = tp.fused && n_pieces == 1;  // the final output, no partial
-        const bool had0 = pub_had[pb * 2] != 0, had1 = pub_had[pb * 2 + 1] != 0;
-        const float *lt0 = pub_l + pb * 2 * 64, *lt1 = lt0 + 64;    // the groups' row sums
-        const float *mx0 = pub_m + pb * 2 * 64, *mx1 = mx0 + 64;    // and maxima
         const int d = j;  // output lane = head dim
+        const uint32_t ob = tmem_o(oslot) + lane_off;
         const long long row_stride = (long long)p.n_q_heads * tp.n_slots * kD;
         const long long base =
             ((long long)it.crow0(p) * p.n_q_heads + it.g * G) * tp.n_slots + piece;
-        // every pair, 8 at a time
 #pragma unroll 1
-        for (int c = 0; c < P8; c += 8) {
-          float o0[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-          float o1[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int i = 0; i < kHq; i += 4) {
+          float o[4];
           // the output blocks (hi and lo, or the P terms) summed
-          if (had0) tmem_load_sum8<kN / Lay::kOBlk>(tmem_o(0, oslot) + lane_off + c, Lay::kOBlk, o0);
-          if (had1) tmem_load_sum8<kN / Lay::kOBlk>(tmem_o(1, oslot) + lane_off + c, Lay::kOBlk, o1);
+          tmem_load_sum4<kN / Lay::kOBlk>(ob + q0 + i, Lay::kOBlk, o);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int q = c + i;
+          for (int u = 0; u < 4; ++u) {
+            const int q = q0 + i + u;
             if (q < P) {
-              const float l0 = lt0[q], l1 = lt1[q];
-              const float m0 = mx0[q], m1 = mx1[q];
-              const float M = l0 > 0.f ? (l1 > 0.f ? fmaxf(m0, m1) : m0) : m1;
-              const float a0 = l0 > 0.f ? ex2(m0 - M) : 0.f;
-              const float a1 = l1 > 0.f ? ex2(m1 - M) : 0.f;
-              const float lt = a0 * l0 + a1 * l1;
-              const float v = lt > 0.f ? (a0 * o0[i] + a1 * o1[i]) * rcp(lt) : 0.f;
+              const float lt = alpha[q];
+              const float v = lt > 0.f ? o[u] * rcp(lt) : 0.f;
               // log2-sum-exp (FP8 sums carry P's factor 2^7)
-              const float lse2 = lt > 0.f ? M + lg2(lt) - (kF8 ? kPScaleLog2 : 0) : -INFINITY;
+              const float lse2 =
+                  lt > 0.f ? m_run[q] + lg2(lt) - (kF8 ? kPScaleLog2 : 0) : -INFINITY;
               const int r = pair_row[q];
               const int h = it.g * G + (q - r * G);
               if (direct) {
@@ -1551,21 +1394,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        // both output blocks are read: free both groups' slots
+        // every thread of the group has read the pairs' maxima and sums
+        // before any thread resets them at its next segment
         tc_fence_before();
+        if (tp.fused && n_pieces > 1) __threadfence();
+        named_sync(bar_id, 128);
         mbar_arrive(bar(kBarOEmpty + oslot));
-        mbar_arrive(bar(kBarOEmpty + 2 + oslot));
         if (tp.fused && n_pieces > 1) {
-          // the piece's partial is written: count it on the segment; the CTA
+          // this group's share of the piece's partial is written (and fenced
+          // above): count it on the segment (two arrivals per piece); the CTA
           // merges its share of the segment once every piece is in (end phase)
-          __threadfence();
-          named_sync(bar_id, 128);
           if (j == 0) {
             atomicAdd(p.seg_count + 2 * it.seg_id, 1u);
-            const int k = *n_end;
-            if (k < 2) {
-              end_rec[k] = EndRec{it.seg_id, n_pieces, piece, it.crow0(p), it.crows(p), it.g};
-              *n_end = k + 1;
+            if (grp == 0) {
+              const int k = *n_end;
+              if (k < 2) {
+                end_rec[k] = EndRec{it.seg_id, n_pieces, piece, it.crow0(p), it.crows(p), it.g};
+                *n_end = k + 1;
+              }
             }
           }
         }
@@ -1672,23 +1518,21 @@ int lse_tc_pairs_bucket(int pairs) {
   return -1;
 }
 
-// Shared-memory configuration: the most K and V tile slots with one P tile
-// per softmax group (the groups then alternate on the SM's pipes, which
-// their exponentials and conversions keep busy), a second Q slot
-// (overlapping Q staging with the end of the previous segment) when it fits
-// as well.  The slots are split about 1 : 2 between the K and the V ring (at
-// least two each, K at most kMaxStages, V at most 8): a K slot is free again
-// once its score product is done, a V slot only after the softmax of its
-// tile and its output product.  The kernel also runs with two P tiles per
-// group (p_bufs = 2), which the planner does not pick.
+// Shared-memory configuration: the most K and V tile slots, then a second P
+// tile (the next tile's probabilities are written while the output product
+// reads this one) and a second Q slot (overlapping Q staging with the end of
+// the previous segment) when they fit as well.  The slots are split about
+// 1 : 2 between the K and the V ring (at least two each, K at most
+// kMaxStages, V at most 8): a K slot is free again once its score product is
+// done, a V slot only after the softmax of its tile and its output product.
 int lse_tc_smem(int dtype, int p8, int scaled, int smem_optin, int *k_stages, int *v_stages,
                 int *q_slots, int *p_bufs) {
   if (scaled && !is_f8(dtype)) return -1;
-  for (int pb = 1; pb >= 1; --pb)
-    for (int slots = kMaxStages + 8; slots >= 4; --slots) {
-      const int nk = slots / 3 < 2 ? 2 : (slots / 3 > kMaxStages ? kMaxStages : slots / 3);
-      const int nv = slots - nk;
-      if (nv < 2 || nv > 8) continue;
+  for (int slots = kMaxStages + 8; slots >= 4; --slots) {
+    const int nk = slots / 3 < 2 ? 2 : (slots / 3 > kMaxStages ? kMaxStages : slots / 3);
+    const int nv = slots - nk;
+    if (nv < 2 || nv > 8) continue;
+    for (int pb = 2; pb >= 1; --pb)
       for (int qs = 2; qs >= 1; --qs) {
         const int b = smem_for(dtype, p8, nk, nv, qs, pb, scaled != 0);
         if (b > 0 && b <= smem_optin) {
@@ -1699,7 +1543,7 @@ int lse_tc_smem(int dtype, int p8, int scaled, int smem_optin, int *k_stages, in
           return b;
         }
       }
-    }
+  }
   return -1;
 }
 
