@@ -755,6 +755,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const bool use_tab = p.n_seqs <= kSeqTab;
   if (warp == 0) {
+    // the barriers first (the producer uses them as soon as its table is
+    // built, without waiting for the other warps)
+    if (lane == 0) {
+    *abort_flag = 0;
+    for (int i = 0; i < 8; ++i) {
+      mbar_init(bar(kBarFullK + i), 1);
+      mbar_init(bar(kBarEmptyK + i), 1);
+      mbar_init(bar(kBarFullV + i), 1);
+      mbar_init(bar(kBarEmptyV + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(kBarOFull + i), 1);
+      mbar_init(bar(kBarOEmpty + i), 256);  // both groups read their pairs out
+    }
+    *n_end = 0;
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(kBarSFull + i), 1);
+      mbar_init(bar(kBarSEmpty + i), 256);  // both groups read their columns
+      mbar_init(bar(kBarPFull + i), 256);   // both groups wrote their columns
+      mbar_init(bar(kBarQFull + i), 1);
+      // FP8: the softmax groups also hold the slot until they have copied
+      // the segment's Q scales
+      mbar_init(bar(kBarQEmpty + i), kF8 ? 3 : 1);
+    }
+    mbar_init(bar(kBarDone), 1);
+    mbar_init(bar(kBarDoneV), 1);
+    for (int i = 0; i < 8; ++i) mbar_init(bar(kBarInfo + i), 1);
+    for (int i = 0; i < 2; ++i) mbar_init(bar(kBarPEmpty + i), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+      }
+    __syncwarp();
     // every sequence's tiles, lanes taking contiguous blocks; then a warp
     // exclusive scan gives each sequence its first tile
     const int per = (p.n_seqs + 31) / 32;
@@ -807,38 +838,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const SeqRec *tab = use_tab ? seq_tab : nullptr;
   if (tid < 64) pair_row[tid] = tid / p.group;
-  if (tid == 32) {
-    *abort_flag = 0;
-    for (int i = 0; i < 8; ++i) {
-      mbar_init(bar(kBarFullK + i), 1);
-      mbar_init(bar(kBarEmptyK + i), 1);
-      mbar_init(bar(kBarFullV + i), 1);
-      mbar_init(bar(kBarEmptyV + i), 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(kBarOFull + i), 1);
-      mbar_init(bar(kBarOEmpty + i), 256);  // both groups read their pairs out
-    }
-    *n_end = 0;
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(kBarSFull + i), 1);
-      mbar_init(bar(kBarSEmpty + i), 256);  // both groups read their columns
-      mbar_init(bar(kBarPFull + i), 256);   // both groups wrote their columns
-      mbar_init(bar(kBarQFull + i), 1);
-      // FP8: the softmax groups also hold the slot until they have copied
-      // the segment's Q scales
-      mbar_init(bar(kBarQEmpty + i), kF8 ? 3 : 1);
-    }
-    mbar_init(bar(kBarDone), 1);
-    mbar_init(bar(kBarDoneV), 1);
-    for (int i = 0; i < 8; ++i) mbar_init(bar(kBarInfo + i), 1);
-    for (int i = 0; i < 2; ++i) mbar_init(bar(kBarPEmpty + i), 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  // The other warps wait for warp 0's table, barriers and TMEM address;
+  // warp 0 only announces its part (bar.arrive) and goes on to the loads.
+  if (warp == 0) {
+    asm volatile("bar.arrive 15, %0;" ::"n"(kThreads) : "memory");
+  } else {
+    tc_fence_before();
+    asm volatile("bar.sync 15, %0;" ::"n"(kThreads) : "memory");
+    tc_fence_after();
+  }
+  __syncwarp();
+  const uint32_t tmem = warp == 0 ? 0u : *tmem_slot;  // (warp 0 never touches TMEM)
   const long long U = *shared_u;
   // working CTAs: never more than tiles, so no working range is empty and a
   // segment's pieces never outnumber its tiles
