@@ -397,6 +397,34 @@ __device__ __forceinline__ void tmem_load_sum4(uint32_t taddr, int stride, float
   }
 }
 
+// TMEM: this thread's lane, C columns (a multiple of 4) from each of T
+// blocks `stride` columns apart, summed in block order; every load is
+// issued before the one wait.
+template <int T, int C>
+__device__ __forceinline__ void tmem_load_sum(uint32_t taddr, int stride, float *v) {
+  static_assert(C % 4 == 0, "columns in groups of 4");
+  uint32_t r[T][C];
+#pragma unroll
+  for (int t = 0; t < T; ++t)
+#pragma unroll
+    for (int c = 0; c < C; c += 4)
+      asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(r[t][c]), "=r"(r[t][c + 1]), "=r"(r[t][c + 2]), "=r"(r[t][c + 3])
+                   : "r"(taddr + (uint32_t)(t * stride + c)));
+  asm volatile("tcgen05.wait::ld.sync.aligned;");
+#pragma unroll
+  for (int t = 0; t < T; ++t)
+#pragma unroll
+    for (int c = 0; c < C; ++c) asm volatile("" : "+r"(r[t][c]));
+#pragma unroll
+  for (int c = 0; c < C; ++c) {
+    float a = __uint_as_float(r[0][c]);
+#pragma unroll
+    for (int t = 1; t < T; ++t) a += __uint_as_float(r[t][c]);
+    v[c] = a;
+  }
+}
+
 // TMEM: 4 columns of this thread's lane.
 __device__ __forceinline__ void tmem_st4(uint32_t taddr, const float *v) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr),

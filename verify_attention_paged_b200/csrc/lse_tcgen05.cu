@@ -1143,6 +1143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if ((masks[r] >> j) & 1ull) v |= row_pairs << (r * G);
           visk[j] = v;
         }
+        named_sync(bar_id, 128);  // visk and m_run ready for the group
       }
       // ---- tile n: this group's pairs ----
       bool w = mbar_wait(bar(kBarSFull + (n & 1)), (n >> 1) & 1, abort_flag, p.err);
@@ -1153,11 +1154,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // per-vector scales land with the tile's V (the V slot outlives this
       // pass: its output product waits for this tile's P)
       if (kSc && w) w = mbar_wait(bar(kBarFullV + n % NV), (n / NV) & 1, abort_flag, p.err);
-      if (named_or(bar_id, 128, !w)) {
-        ok = false;
-        break;
-      }
-      const uint4 inf = tile_info[n & 7];
+      // (a thread whose wait gave up goes on without side effects up to the
+      // group barrier after pass 1, where the whole group learns of it)
+      const uint4 inf = w ? tile_info[n & 7] : make_uint4(0u, 0u, 0u, 0u);
       const int key0 = it.tile * kTK;
       const int key = key0 + j;
       const uint32_t both = inf.x & inf.y;
@@ -1198,8 +1197,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // pair's inverse Q scale), -inf where not visible; does any score pass
       // the running max by 2^tau?
       float sv[kHq], mr[kHq];
+      // the loads of up to 16 pairs (16-bit) or of 12 or 8 pairs (FP8: four
+      // terms each) before one wait
+      constexpr int kLd = !kF8 ? (kHq <= 16 ? kHq : 12)
+                               : kHq % 12 == 0 ? 12 : kHq % 8 == 0 ? 8 : 4;
 #pragma unroll
-      for (int i = 0; i < kHq; i += 4) tmem_load_sum4<kSW / kNQ>(s_addr + q0 + i, kNQ, sv + i);
+      for (int i = 0; i < kHq; i += kLd)
+        tmem_load_sum<kSW / kNQ, kLd>(s_addr + q0 + i, kNQ, sv + i);
       // the scores are in registers: the next score product into this
       // buffer may overwrite it while the probabilities are built
       tc_fence_before();
@@ -1228,7 +1232,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       float gap = -INFINITY;
 #pragma unroll
       for (int i = 0; i < kHq; ++i) gap = fmaxf(gap, sv[i] - mr[i]);
-      if (named_or(bar_id, 128, gap > kTau)) {
+      // this tile's P buffer is free once the output product that last read
+      // it (tile n - PB) has completed
+      if (n >= PB && w)
+        w = mbar_wait(bar(kBarPEmpty + n % PB), ((n / PB) - 1) & 1, abort_flag, p.err);
+      // one group barrier per tile in the common case: does any thread need
+      // the rescale, or has any wait given up?
+      if (named_or(bar_id, 128, !w || gap > kTau)) {
+        if (named_or(bar_id, 128, !w)) {  // (uniform over the group)
+          ok = false;
+          break;
+        }
         // per-pair maximum over the tile's keys: each warp folds its 32
         // keys by a butterfly, and the four warps' maxima meet in red
 #pragma unroll
@@ -1281,16 +1295,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               tmem_st4(ob + col, v);
             }
           tmem_st_wait();
-        }
-      }
-      // this tile's P buffer is free once the output product that last read
-      // it (tile n - PB) has completed
-      if (n >= PB) {
-        const bool wp =
-            mbar_wait(bar(kBarPEmpty + n % PB), ((n / PB) - 1) & 1, abort_flag, p.err);
-        if (named_or(bar_id, 128, !wp)) {
-          ok = false;
-          break;
         }
       }
       // pass 2: probabilities of this group's pairs -> the tile's P tile, row
