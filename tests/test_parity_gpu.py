@@ -278,6 +278,34 @@ def test_tcgen05_many_segments_per_cta(binding, dtype):
 
 
 @pytest.mark.parametrize("dtype", ["f16", "e4m3"])
+@pytest.mark.parametrize("n_sms", [3, 7, 16])
+def test_tcgen05_segment_weighted_cut(binding, dtype, n_sms):
+    # few working CTAs, so each takes at least 24 tiles and the cut charges
+    # every segment 3 extra tiles: CTA ranges then start and end inside
+    # short segments' overhead positions, and a segment's pieces are counted
+    # by position in the pass (fused merge) and in the separate merge
+    rng = np.random.default_rng(40 + n_sms)
+    lens = [int(x) for x in rng.integers(1, 2500, 14)] + [130, 129, 1, 6000]
+    rows = [int(min(L, r)) for L, r in zip(lens, rng.integers(0, 13, len(lens)))]
+    w = wl.small_case(dtype, lens, rows, n_q_heads=24, n_kv_heads=4, head_dim=128,
+                      tokens_per_fragment=128, tree=True, seed=240 + n_sms)
+    props = torch.cuda.get_device_properties(0)
+    limits = dict(n_sms=n_sms, smem_optin=props.shared_memory_per_block_optin, ctas_per_sm=0,
+                  allow_tcgen05=1)
+    ref_out, ref_lse = orc.attention(to_problem(w))
+    call = binding.DeviceCall(w, plan_limits=limits)
+    assert call.info["kernel_name"] == "tcgen05" and call.info["ctas"] == n_sms
+    for label, fn in (("fused", call.run), ("two-pass", call.run_two_pass)):
+        out, lse = fn()
+        torch.cuda.synchronize()
+        assert call.device_error() == 0, label
+        assert_close(out[:w.total_rows].cpu().numpy(), ref_out, dtype, what=label)
+        np.testing.assert_allclose(lse[:w.total_rows].cpu().numpy(), ref_lse, rtol=0,
+                                   atol=lse_tol(dtype) * 4)
+    call.close()
+
+
+@pytest.mark.parametrize("dtype", ["f16", "e4m3"])
 def test_tcgen05_more_sequences_than_the_cta_table(binding, dtype):
     # 130 sequences: more than the per-CTA sequence table holds, so the tile
     # iterator reads lengths from global memory (and numbers segments itself)

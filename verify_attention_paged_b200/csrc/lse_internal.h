@@ -72,6 +72,15 @@ struct lse_attn_plan_s {
 // Bytes reserved at the head of the workspace (error word + padding).
 constexpr size_t kWsHeader = 256;
 
+// Cut of the tensor-core pass's live tiles into CTA ranges, shared by the
+// pass and the separate merge (which counts each segment's pieces): every
+// segment counts kLseSegWeight tiles more than it has, when the call has at
+// most kLseSeqTab sequences (the pass keeps them in a shared-memory table)
+// and each working CTA's share is at least kLseSegMinShare tiles.
+constexpr int kLseSeqTab = 96;
+constexpr int kLseSegWeight = 3;
+constexpr int kLseSegMinShare = 8 * kLseSegWeight;
+
 // Parameters passed by value to the partial and merge kernels.
 struct LseKernelParams {
   unsigned long long chunk_base[LSE_MAX_CHUNKS];

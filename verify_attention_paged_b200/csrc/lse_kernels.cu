@@ -405,7 +405,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
   constexpr int kPerLane = D / 32;
   __shared__ float s_m[kMergeWarps], s_w[kMergeWarps];
   __shared__ float s_acc[kMergeWarps][D];
-  __shared__ long long s_cnt[kMergeWarps][2];
+  __shared__ long long s_cnt[kMergeWarps][4];
   __shared__ int s_seq;
   const int h = blockIdx.x % p.n_q_heads;
   const int grow = blockIdx.x / p.n_q_heads;  // the row, over all sequences
@@ -424,42 +424,58 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(
   if (p.balanced && live_row) {
     // pieces of the row's segment (sequence, row chunk, kv head) written by
     // the persistent tensor-core pass: the tiles of all segments end to end
-    // (per sequence: row chunks x kv heads segments of its tiles), CTA c
-    // owning [c U / C, (c+1) U / C); the tiles before sequence s and in all,
-    // summed over the CTA
+    // (per sequence: row chunks x kv heads segments of its tiles), each
+    // segment weighted by W more tiles, CTA c owning positions
+    // [c UW / C, (c+1) UW / C); the tiles and segments before sequence s and
+    // in all, summed over the CTA
     const int Rc = p.rows_per_chunk;
-    long long mine_before = 0, mine_all = 0;
+    long long mine_before = 0, mine_all = 0, segs_before = 0, segs_all = 0;
     for (int q = tid; q < p.n_seqs; q += kMergeThreads) {
       int Lq, r0q, Rq;
       const int n = seq_tiles_merge(p, q, Lq, r0q, Rq);
-      const long long tq = (long long)n * ((Rq + Rc - 1) / Rc) * p.n_kv_heads;
+      const long long sq = n > 0 ? (long long)((Rq + Rc - 1) / Rc) * p.n_kv_heads : 0;
+      const long long tq = (long long)n * sq;
       mine_all += tq;
-      if (q < s) mine_before += tq;
+      segs_all += sq;
+      if (q < s) {
+        mine_before += tq;
+        segs_before += sq;
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       mine_before += __shfl_xor_sync(0xffffffffu, mine_before, o);
       mine_all += __shfl_xor_sync(0xffffffffu, mine_all, o);
+      segs_before += __shfl_xor_sync(0xffffffffu, segs_before, o);
+      segs_all += __shfl_xor_sync(0xffffffffu, segs_all, o);
     }
     if (lane == 0) {
       s_cnt[warp][0] = mine_before;
       s_cnt[warp][1] = mine_all;
+      s_cnt[warp][2] = segs_before;
+      s_cnt[warp][3] = segs_all;
     }
     __syncthreads();
-    long long before = 0, U = 0;
+    long long before = 0, U = 0, sb = 0, S = 0;
 #pragma unroll
     for (int w = 0; w < kMergeWarps; ++w) {
       before += s_cnt[w][0];
       U += s_cnt[w][1];
+      sb += s_cnt[w][2];
+      S += s_cnt[w][3];
     }
     int Ls, r0s, Rs;
     const int n_s = seq_tiles_merge(p, s, Ls, r0s, Rs);
     const int g = h / p.group;
+    const long long sid = sb + (long long)(r / Rc) * p.n_kv_heads + g;  // the segment
     const long long first = before + ((long long)(r / Rc) * p.n_kv_heads + g) * n_s;
-    const long long last = first + n_s - 1;
     const long long C = U < p.n_ctas ? U : p.n_ctas;  // working CTAs of the partial pass
-    // one partial per piece (the CTA combines its two softmax groups)
-    n_live = n_s > 0 ? int(((last + 1) * C - 1) / U - ((first + 1) * C - 1) / U) + 1 : 0;
+    const long long W =
+        p.n_seqs <= kLseSeqTab && C > 0 && U / C >= kLseSegMinShare ? kLseSegWeight : 0;
+    const long long UW = U + W * S;
+    const long long pos0 = first + W * (sid + 1), pos1 = pos0 + n_s - 1;
+    // one partial per piece
+    n_live = n_s > 0 ? int(((pos1 + 1) * C - 1) / UW - ((pos0 + 1) * C - 1) / UW) + 1 : 0;
   } else if (live_row) {
     n_live = min((L + p.keys_per_split - 1) / p.keys_per_split, p.n_splits);
   }

@@ -942,12 +942,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_tcgen05_kernel(const __gr
   // ---- teardown ----
   tc_fence_before();
   __syncthreads();
-  tc_fence_after();
-  __syncwarp();
-  if (warp == 1)
+  pf_end_merge(tp, tab, end_rec, *n_end, U, C, abort_flag, go_flag);
+  // TMEM is released last: only its owner fences after the barrier
+  if (warp == 1) {
+    tc_fence_after();
+    __syncwarp();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512)
                  : "memory");
-  pf_end_merge(tp, tab, end_rec, *n_end, U, C, abort_flag, go_flag);
+  }
 }
 
 template <int DT>

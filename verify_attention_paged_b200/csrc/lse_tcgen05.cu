@@ -46,9 +46,10 @@
 //    N), and the two products are issued by two threads; the row sums of P
 //    are summed by the softmax warps.
 //
-// Roles (384 threads): warp 0 TMA producer, warp 1 score-product issuer
-// (and TMEM owner), warp 2 output-product issuer, warp 3 stages Q, warps 4-7
-// and 8-11 the two softmax groups.
+// Roles: warp 0 TMA producer, warp 1 score-product issuer (and TMEM
+// owner), warp 2 output-product issuer, warp 3 stages Q, then two to four
+// softmax groups of four warps (128 threads, one per key of a tile), each
+// taking an equal share of the tile's (row, head) pairs.
 // Every wait is bounded: a wait that runs out sets LSE_DEVERR_TIMEOUT and
 // every role leaves its loop; TMEM is released and outstanding copies are
 // drained before the CTA exits.
@@ -73,7 +74,12 @@ using namespace lse_ptx;
 
 constexpr int kTK = 128;           // keys per tile = M of the score product
 constexpr int kD = 128;            // head dim = M of the output product
-constexpr int kThreads = 384;
+// Softmax groups per CTA for a pairs bucket: more groups give each thread
+// fewer pairs of a tile (each group's share is a multiple of 4 pairs).
+template <int P8>
+constexpr int tc_groups() { return P8 == 48 || P8 == 24 ? 3 : 2; }
+template <int P8>
+constexpr int tc_threads() { return 128 * (1 + tc_groups<P8>()); }
 constexpr float kTau = 8.f;        // lazy-rescale threshold (log2 units)
 constexpr int kRegionBytes = kTK * 128;          // 128 rows x 128 B (64 dims)
 
@@ -116,7 +122,7 @@ __device__ __forceinline__ int seq_chunks(const LseKernelParams &p, int R) {
 // Per-sequence record built once per CTA in shared memory (sequences up to
 // kSeqTab): tiles of all segments before the sequence, its 128-key tiles,
 // L, first row, R, and the number of segments before the sequence.
-constexpr int kSeqTab = 96;
+constexpr int kSeqTab = kLseSeqTab;
 struct SeqRec {
   int prefix, n_tiles, L, row0, R, seg_prefix;
 };
@@ -225,9 +231,41 @@ struct TileIter {
   }
 };
 
-// CTA whose range holds global tile t, for ranges [c U / C, (c+1) U / C).
-__device__ __forceinline__ int cta_of_tile(long long t, long long U, int C) {
-  return int(((t + 1) * (long long)C - 1) / U);
+// Cut of the live tiles into the working CTAs' ranges.  Every segment
+// counts W tiles more than it has (the fixed cost of starting and ending
+// one: its Q staged, its first tile's rescale, its epilogue), so a CTA whose
+// range crosses many short segments gets fewer tiles.  Tile t of segment
+// sid sits at position t + W (sid + 1) of UW = U + W S positions, and CTA c
+// takes the tiles at positions [c UW / C, (c+1) UW / C).  W is 0 when the
+// sequences are not in the shared-memory table, or when a CTA's share is
+// under kSegMinShare tiles (there W would be a coarse share of a CTA's work;
+// it also keeps every range non-empty).
+constexpr int kSegWeight = kLseSegWeight;
+constexpr int kSegMinShare = kLseSegMinShare;
+
+// CTA whose range holds position x.
+__device__ __forceinline__ int cta_of_pos(long long x, long long UW, int C) {
+  return int(((x + 1) * (long long)C - 1) / UW);
+}
+
+// First tile at or after position x (U when x is past the last tile).
+__device__ long long tile_at(const SeqRec *tab, int n_seqs, const LseKernelParams &p, int W,
+                             long long U, long long UW, long long x) {
+  if (x >= UW) return U;
+  // last sequence whose weighted start is at or before x (an idle sequence
+  // starts where the next one does, so the last such index has tiles)
+  int lo = 0, hi = n_seqs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((long long)tab[mid].prefix + (long long)W * tab[mid].seg_prefix <= x) lo = mid;
+    else hi = mid - 1;
+  }
+  const SeqRec r = tab[lo];
+  const long long o = x - ((long long)r.prefix + (long long)W * r.seg_prefix);
+  const int nseg = seq_chunks(p, r.R) * p.n_kv_heads;
+  const long long j = o / (r.n_tiles + W), k = o - j * (r.n_tiles + W);
+  if (j >= nseg) return (long long)r.prefix + (long long)nseg * r.n_tiles;
+  return (long long)r.prefix + j * r.n_tiles + (k > W ? k - W : 0);
 }
 
 
@@ -338,40 +376,6 @@ __device__ __forceinline__ int produce_tile(const TcParams &tp, int n, int NK, i
 }
 
 
-// Column reduction of a [128 keys][P8 pairs] FP32 tile in shared memory by
-// the 128 threads of a softmax group: out[q] = max (or sum) over keys of
-// tile[key][q].  Each pair gets kSplit = max(2, 128 / P8) threads, each
-// folding a contiguous share of the keys; the shares are combined through
-// out[64 ...] (out holds 4 x 64 floats).
-template <int P8, bool kSum>
-__device__ __forceinline__ void column_reduce(const float *tile, int t, float *out, int bar_id) {
-  constexpr int kSplit = 128 / P8 >= 2 ? 128 / P8 : 2;
-  constexpr int kRows = (128 + kSplit - 1) / kSplit;
-  static_assert(kSplit * P8 <= 192, "shares must fit out[64 .. 256)");
-  const int q = t % P8, part = t / P8;
-  float a = kSum ? 0.f : -INFINITY;
-  if (part < kSplit) {
-#pragma unroll 8
-    for (int k = 0; k < kRows; ++k) {
-      const int row = part * kRows + k;
-      if (row < 128) {
-        const float v = tile[row * P8 + q];
-        a = kSum ? a + v : fmaxf(a, v);
-      }
-    }
-  }
-  float *shares = out + 64;
-  if (part < kSplit) shares[part * P8 + q] = a;
-  named_sync(bar_id, 128);
-  if (t < P8) {
-    float r = kSum ? 0.f : -INFINITY;
-#pragma unroll 1
-    for (int k = 0; k < kSplit; ++k)
-      r = kSum ? r + shares[k * P8 + t] : fmaxf(r, shares[k * P8 + t]);
-    out[t] = r;
-  }
-}
-
 // A segment this CTA shares with other CTAs, merged after the CTA's own
 // tiles when the merge is fused into the pass (at most two per CTA: the
 // first and the last segment of its range; every segment in between lies
@@ -380,8 +384,8 @@ struct EndRec {
   int seg_id, n_pieces, piece, row0, rows, g;
 };
 // shared memory of the end phase: a flag word pair, up to two end records
-// and their count
-constexpr int kEndBytes = 2 * 4 + 2 * (int)sizeof(EndRec) + 8;
+// and their count; then the CTA's tile range {t_begin, t_stop, UW, W}
+constexpr int kEndBytes = 2 * 4 + 2 * (int)sizeof(EndRec) + 8 + 8 + 4 * 8;
 
 // ---- shared-memory and TMEM layout ------------------------------------------------
 
@@ -397,8 +401,10 @@ template <int DT, int P8>
 struct TcLayout {
   static constexpr bool kF8 = is_f8(DT);
   static constexpr int kNQ = (P8 + 15) / 16 * 16;       // pairs rounded to 16 (MMA N step)
-  // each softmax group takes half of the (row, head) pairs of every tile
-  static constexpr int kH = P8 / 2;
+  // each softmax group takes an equal share of the (row, head) pairs of
+  // every tile
+  static constexpr int kG = tc_groups<P8>();
+  static constexpr int kH = P8 / kG;
   static_assert(kH % 4 == 0, "a group's pairs come in blocks of 4");
   // Every product carries its operand terms side by side along N, so one
   // MMA per K step covers them all (the issue of an MMA costs the same
@@ -431,9 +437,9 @@ struct TcLayout {
   static_assert(kTmemNeed <= 512, "TMEM holds at most 512 columns");
   static_assert(kSW <= 256 && kN <= 256, "MMA N is at most 256");
   static constexpr int kBars = 64;
-  static constexpr int kMiscBytes = kBars * 8 + 16 + 2 * 64 * 4 * 2 + 2 * 4 * 64 * 4 +
-                                    2 * 64 * 8 * 2 + 64 * 4 + 8 * 16 + 2 * 32 * 16 * 4 +
-                                    (kF8 ? 4 * 64 * 4 : 0) +
+  static constexpr int kMiscBytes = kBars * 8 + 16 + kG * 64 * 4 * 2 + kG * 4 * 64 * 4 +
+                                    kG * 64 * 8 * 2 + 64 * 4 + 8 * 16 + 2 * 32 * 16 * 4 +
+                                    (kF8 ? (2 + kG) * 64 * 4 : 0) +
                                     kSeqTab * (int)sizeof(SeqRec) + kEndBytes;
   // one K or V tile: 128 keys of 128 dims (two 64-dim regions when 16-bit)
   static constexpr int kHalfStage = kF8 ? kRegionBytes : 2 * kRegionBytes;
@@ -455,24 +461,25 @@ enum {
   kBarFullV = 16,   // [8]
   kBarEmptyV = 24,  // [8]
   kBarSFull = 32,   // [2] per score buffer: its product is complete
-  kBarPFull = 34,   // [2] per P tile: both groups wrote their probabilities (256)
+  kBarPFull = 34,   // [2] per P tile: every group wrote its probabilities
   kBarQFull = 36,   // [2]
   kBarQEmpty = 38,  // [2]
   kBarOFull = 40,   // [2] per output slot: the piece's last output product is complete
-  kBarOEmpty = 42,  // [2] per output slot: both groups read it out (256)
+  kBarOEmpty = 42,  // [2] per output slot: every group read it out
   kBarDone = 44,    // the score issuer's MMAs have completed
   kBarInfo = 45,    // [8] one per tile record
   kBarPEmpty = 53,  // [2] per P tile: the output product that read it is complete
   kBarDoneV = 55,   // the output issuer's MMAs have completed
-  kBarSEmpty = 56,  // [2] per score buffer: both groups read it out (256)
+  kBarSEmpty = 56,  // [2] per score buffer: every group read it out
 };
 
 // Stage one segment's Q into a Q slot, by T threads (t = 0 .. T-1): each
 // (pair row n, 8-dim chunk c) item is scaled by the softmax scale (log2
 // units) and written in the operand layout of the score product.  Item
 // t + T k goes to thread t, so the 16 lanes of a half warp hold one row.
-// Items go in rounds of up to 8 per thread; the first round's loads are
-// issued before `before_store` (the wait for the slot) runs.  FP8: each row
+// Items go in rounds of up to 8 per thread; the first round's loads, and L2
+// prefetches of the later rounds' rows, are issued before `before_store` (the
+// wait for the slot) runs.  FP8: each row
 // is scaled by 2^e (max |x| 2^e in [128, 256)) and written as kQTerms E4M3
 // terms; 2^-e goes to isig[n].
 template <int DT, int P8, int T, class Wait>
@@ -485,6 +492,19 @@ __device__ __forceinline__ bool stage_q(const LseKernelParams &p, int t, int g, 
   static_assert(kItems * T == kNQ * 16, "items split evenly");
   const int G = p.group;
   const float sc = p.scale_log2;
+  auto src_of = [&](int n, int c) {
+    const int r = n / G, h = g * G + (n - r * G);
+    return reinterpret_cast<const float4 *>(p.q + ((long long)(row0 + r) * p.n_q_heads + h) * kD +
+                                            c * 8);
+  };
+  // the later rounds' rows into L2 (one prefetch per 128-byte line)
+#pragma unroll 1
+  for (int k = kRound; k < kItems; ++k) {
+    const int item = t + T * k;
+    const int n = item >> 4, c = item & 15;
+    if (n < P && (c & 3) == 0)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(src_of(n, c)) : "memory");
+  }
 #pragma unroll 1
   for (int r0 = 0; r0 < kItems; r0 += kRound) {
     float4 ld[kRound][2];
@@ -493,9 +513,7 @@ __device__ __forceinline__ bool stage_q(const LseKernelParams &p, int t, int g, 
       const int item = t + T * (r0 + k);
       const int n = item >> 4, c = item & 15;
       if (n < P) {
-        const int r = n / G, h = g * G + (n - r * G);
-        const float4 *src = reinterpret_cast<const float4 *>(
-            p.q + ((long long)(row0 + r) * p.n_q_heads + h) * kD + c * 8);
+        const float4 *src = src_of(n, c);
         ld[k][0] = __ldg(src);
         ld[k][1] = __ldg(src + 1);
       } else {
@@ -551,11 +569,24 @@ __device__ __forceinline__ bool stage_q(const LseKernelParams &p, int t, int g, 
   return true;
 }
 
+// L2 prefetch of one segment's Q: `rows` rows from row0, the G heads of kv
+// head g (G x 512 contiguous bytes per row), by the 32 lanes of a warp.
+__device__ __forceinline__ void prefetch_q(const LseKernelParams &p, int g, int row0, int rows,
+                                           int lane) {
+  const int G = p.group;
+  const int lines = G * 4;  // 128-byte lines per row
+  for (int i = lane; i < rows * lines; i += 32) {
+    const int r = i / lines, l = i - r * lines;
+    const float *a = p.q + ((long long)(row0 + r) * p.n_q_heads + g * G) * kD + l * 32;
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(a) : "memory");
+  }
+}
+
 // End phase of the fused pass: for each segment this CTA shares with other
 // CTAs, wait until every piece's partial is written (the segment's arrival
-// count reaches two per piece: one per softmax group), then merge this CTA's
-// share of the
-// segment's (row, head) pairs: pair q goes to the segment's piece q mod n,
+// count reaches kArrivals per piece: one per softmax group), then merge this
+// CTA's share of the segment's (row, head) pairs: pair q goes to the
+// segment's piece q mod n,
 // so the n CTAs of the segment split its pairs.  A pair is merged by one or
 // more warps, each taking every k-th piece with its loads issued together
 // (lanes over the head dim, four dims a lane) and a running maximum; the
@@ -565,12 +596,12 @@ __device__ __forceinline__ bool stage_q(const LseKernelParams &p, int t, int g, 
 // call.  The wait is bounded like every other wait; the launch is
 // cooperative, so every CTA of the grid is resident and each arrives for its
 // own pieces without waiting on any other CTA.
+template <int kWarps, int kArrivals>
 __device__ __noinline__ void fused_end_merge(const TcParams &tp, const EndRec *rec, int n_rec,
                                              volatile int *abort_flag, int *go_flag,
                                              float *scratch) {
   const LseKernelParams &p = tp.p;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  constexpr int kWarps = kThreads / 32;
   float *w_m = scratch;                 // [warp] running maximum
   float *w_l = scratch + kWarps;        // [warp] sum of weights
   float *w_acc = scratch + 2 * kWarps;  // [warp][kD] weighted sums
@@ -584,7 +615,7 @@ __device__ __noinline__ void fused_end_merge(const TcParams &tp, const EndRec *r
       while (go) {
         unsigned int v;
         asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
-        if (v >= 2u * (unsigned)r.n_pieces) break;
+        if (v >= (unsigned)kArrivals * (unsigned)r.n_pieces) break;
         if (clock64() - t0 > kWaitCycles) {
           *abort_flag = 1;
           atomicOr(p.err, LSE_DEVERR_TIMEOUT);
@@ -688,10 +719,12 @@ __device__ __noinline__ void fused_end_merge(const TcParams &tp, const EndRec *r
 }
 
 template <int DT, int P8, bool kSc>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(tc_threads<P8>(), 1)
     partial_tcgen05_kernel(const __grid_constant__ TcParams tp) {
   using Lay = TcLayout<DT, P8>;
   constexpr bool kF8 = Lay::kF8;
+  constexpr int kG = Lay::kG;                    // softmax groups
+  constexpr int kThreads = tc_threads<P8>();
   static_assert(!kSc || kF8, "per-vector scales go with the 8-bit formats");
   constexpr bool kE5 = DT == LSE_KV_FP8_E5M2;
   constexpr int kNQ = Lay::kNQ;
@@ -719,27 +752,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + Lay::kBars * 8);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + Lay::kBars * 8 + 4);
   long long *shared_u = reinterpret_cast<long long *>(misc + Lay::kBars * 8 + 8);
-  float *m_run_all = reinterpret_cast<float *>(misc + Lay::kBars * 8 + 16);  // [2][64]
-  float *alpha_all = m_run_all + 2 * 64;                                     // [2][64]
-  float *red_all = alpha_all + 2 * 64;                                       // [2][4][64]
+  float *m_run_all = reinterpret_cast<float *>(misc + Lay::kBars * 8 + 16);  // [kG][64]
+  float *alpha_all = m_run_all + kG * 64;                                    // [kG][64]
+  float *red_all = alpha_all + kG * 64;                                      // [kG][4][64]
   unsigned long long *masks_all =
-      reinterpret_cast<unsigned long long *>(red_all + 2 * 4 * 64);          // [2][64]
+      reinterpret_cast<unsigned long long *>(red_all + kG * 4 * 64);         // [kG][64]
   // per softmax group and draft key k of the sequence: the pairs that see it
-  unsigned long long *visk_all = masks_all + 2 * 64;                         // [2][64]
-  int *pair_row = reinterpret_cast<int *>(visk_all + 2 * 64);                // [64]
+  unsigned long long *visk_all = masks_all + kG * 64;                        // [kG][64]
+  int *pair_row = reinterpret_cast<int *>(visk_all + kG * 64);               // [64]
   // ring of 8 per-tile records written by the producer before its arrival on
   // the tile's K barrier: {K box mask, V box mask, keys of the tile below L}
   uint4 *tile_info = reinterpret_cast<uint4 *>(pair_row + 64);               // [8]
   // fragment ids of a batch of 32 tiles (up to 16 boxes each), K then V
   int *page_buf = reinterpret_cast<int *>(tile_info + 8);                    // [2][32][16]
   // FP8: the inverse of Q's per-pair scale, per Q slot [0, 2) and the
-  // copy each softmax group keeps for its segment [2, 4)
-  float *isig_all = reinterpret_cast<float *>(page_buf + 2 * 32 * 16);       // [4][64]
+  // copy each softmax group keeps for its segment [2, 2 + kG)
+  float *isig_all = reinterpret_cast<float *>(page_buf + 2 * 32 * 16);       // [2+kG][64]
   SeqRec *seq_tab =
-      reinterpret_cast<SeqRec *>(isig_all + (kF8 ? 4 * 64 : 0));            // [kSeqTab]
+      reinterpret_cast<SeqRec *>(isig_all + (kF8 ? (2 + kG) * 64 : 0));     // [kSeqTab]
   int *had_all = reinterpret_cast<int *>(seq_tab + kSeqTab);                 // [2] (end phase)
   EndRec *end_rec = reinterpret_cast<EndRec *>(had_all + 2);                 // [2]
   int *n_end = reinterpret_cast<int *>(end_rec + 2);
+  long long *range = reinterpret_cast<long long *>(
+      (reinterpret_cast<uintptr_t>(n_end + 1) + 7) & ~uintptr_t(7));  // [4]
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
   // the merge pass may be scheduled now; it waits for this grid to finish
@@ -767,17 +802,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarOFull + i), 1);
-      mbar_init(bar(kBarOEmpty + i), 256);  // both groups read their pairs out
+      mbar_init(bar(kBarOEmpty + i), 128 * kG);  // every group read its pairs out
     }
     *n_end = 0;
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarSFull + i), 1);
-      mbar_init(bar(kBarSEmpty + i), 256);  // both groups read their columns
-      mbar_init(bar(kBarPFull + i), 256);   // both groups wrote their columns
+      mbar_init(bar(kBarSEmpty + i), 128 * kG);  // every group read its columns
+      mbar_init(bar(kBarPFull + i), 128 * kG);   // every group wrote its columns
       mbar_init(bar(kBarQFull + i), 1);
       // FP8: the softmax groups also hold the slot until they have copied
       // the segment's Q scales
-      mbar_init(bar(kBarQEmpty + i), kF8 ? 3 : 1);
+      mbar_init(bar(kBarQEmpty + i), kF8 ? 1 + kG : 1);
     }
     mbar_init(bar(kBarDone), 1);
     mbar_init(bar(kBarDoneV), 1);
@@ -809,6 +844,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const long long v = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += v;
     }
+    int seg_total = 0;  // segments up to this lane's sequences (with the table)
     if (use_tab) {
       // segments of the lanes before this one (a second warp scan)
       int segs = 0;
@@ -822,6 +858,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int v = __shfl_up_sync(0xffffffffu, seg_incl, o);
         if (lane >= o) seg_incl += v;
       }
+      seg_total = seg_incl;
       long long run = incl - mine;
       int seg_run = seg_incl - segs;
       for (int q = s0; q < s1; ++q) {
@@ -835,6 +872,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     bad = __any_sync(0xffffffffu, bad);
     if (lane == 31) *shared_u = incl;
     if (lane == 0 && bad && cta == 0) atomicOr(p.err, LSE_DEVERR_BAD_LENGTH);
+    // this CTA's range of tiles
+    const long long U0 = __shfl_sync(0xffffffffu, incl, 31);
+    const int S0 = use_tab ? __shfl_sync(0xffffffffu, seg_total, 31) : 0;
+    if (lane == 0 && U0 > 0) {
+      const int C0 = (int)(U0 < tp.n_ctas ? U0 : tp.n_ctas);
+      const int W = use_tab && U0 / C0 >= kSegMinShare ? kSegWeight : 0;
+      const long long UW = U0 + (long long)W * S0;
+      long long b0 = UW * cta / C0, b1 = UW * (cta + 1) / C0;
+      if (W > 0) {
+        b0 = tile_at(seq_tab, p.n_seqs, p, W, U0, UW, b0);
+        b1 = tile_at(seq_tab, p.n_seqs, p, W, U0, UW, b1);
+      }
+      range[0] = b0;
+      range[1] = b1;
+      range[2] = UW;
+      range[3] = W;
+    }
   }
   const SeqRec *tab = use_tab ? seq_tab : nullptr;
   if (tid < 64) pair_row[tid] = tid / p.group;
@@ -860,7 +914,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                    : "memory");
     return;
   }
-  const long long t_begin = U * cta / C, t_stop = U * (cta + 1) / C;
+  const long long t_begin = range[0], t_stop = range[1], UW = range[2];
+  const int W = (int)range[3];
   constexpr int kSW = Lay::kSW;
   // score buffer of tile n: n & 1; output slot of the CTA's segment seg: seg % kOS
   auto tmem_s = [&](int buf) { return tmem + (uint32_t)(buf * kSW); };
@@ -996,7 +1051,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (first) ++seg_v;
         const int slot = seg_v % kOS;
         const int st = nv % NV;
-        // both groups' probabilities of tile nv, its V tile, and (for the
+        // every group's probabilities of tile nv, its V tile, and (for the
         // piece's first product) the slot's previous piece read out
         bool go = mbar_wait(bar(kBarPFull + nv % PB), (nv / PB) & 1, abort_flag, p.err);
         go = go && mbar_wait(bar(kBarFullV + st), (nv / NV) & 1, abort_flag, p.err);
@@ -1047,11 +1102,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Every segment after the first, ahead of the score products (softmax
     // group 0 stages the first: it is idle until the first scores arrive,
     // and 128 threads do it faster than one warp).
+    // At each segment's start the next segment's Q is prefetched into L2,
+    // so its staging (once the slot is free) reads L2, not HBM.
     TileIter it;
     it.init(p, t_begin, t_stop, tab);
     int seg = -1;
     for (; it.valid(); it.advance(p)) {
       if (!it.seg_start(t_begin)) continue;
+      const long long nxt = it.seg_first + it.n_tiles;
+      if (nxt < t_stop) {
+        TileIter nx;
+        nx.init(p, nxt, t_stop, tab);
+        prefetch_q(p, nx.g, nx.crow0(p), nx.crows(p), lane);
+      }
       if (++seg == 0) continue;
       const int slot = seg % QS;
       uint8_t *qs = smem + (q_base - sbase) + slot * Lay::kQBytes;
@@ -1064,12 +1127,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(bar(kBarQFull + slot));
     }
   } else {
-    // ============== softmax and epilogue: two groups of 128 threads ==============
-    // Both groups work on every tile, each on half of the (row, head) pairs:
-    // group g takes pairs [g H, g H + H), H = P8 / 2, so a tile's softmax
-    // takes half as long and the groups never combine results.  Thread j of
-    // a group owns key j of the tile (its TMEM lane), reads its half of the
-    // key's scores four pairs at a time, keeps the key's sums of P per pair
+    // ============== softmax and epilogue: kG groups of 128 threads ==============
+    // Every group works on every tile, each on its share of the (row, head)
+    // pairs: group g takes pairs [g H, g H + H), H = P8 / kG, so a tile's
+    // softmax is spread over kG groups that never combine results.  Thread j
+    // of a group owns key j of the tile (its TMEM lane), reads its share of
+    // the key's scores, keeps the key's sums of P per pair
     // in registers over the segment, and the four warps' sums meet once per
     // piece (a warp butterfly, then a fixed-order fold).
     constexpr int kHq = Lay::kH;
@@ -1370,8 +1433,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         __syncwarp();
         // the piece: its place among the segment's pieces
-        const int c_first = cta_of_tile(it.seg_first, U, C);
-        const int c_last = cta_of_tile(it.seg_first + it.n_tiles - 1, U, C);
+        const long long pos0 = it.seg_first + (long long)W * (it.seg_id + 1);
+        const int c_first = cta_of_pos(pos0, UW, C);
+        const int c_last = cta_of_pos(pos0 + it.n_tiles - 1, UW, C);
         const int n_pieces = c_last - c_first + 1, piece = cta - c_first;
         const bool direct = tp.fused && n_pieces == 1;  // the final output, no partial
         const int d = j;  // output lane = head dim
@@ -1416,7 +1480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar(kBarOEmpty + oslot));
         if (tp.fused && n_pieces > 1) {
           // this group's share of the piece's partial is written (and fenced
-          // above): count it on the segment (two arrivals per piece); the CTA
+          // above): count it on the segment (kG arrivals per piece); the CTA
           // merges its share of the segment once every piece is in (end phase)
           if (j == 0) {
             atomicAdd(p.seg_count + 2 * it.seg_id, 1u);
@@ -1436,16 +1500,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- teardown --------------------------------------------------------------
   tc_fence_before();
   __syncthreads();
-  tc_fence_after();
-  __syncwarp();
-  if (warp == 1)
+  // (the K/V ring is idle: the end phase's scratch)
+  if (tp.fused)
+    fused_end_merge<kThreads / 32, kG>(tp, end_rec, *n_end, abort_flag, had_all,
+                    reinterpret_cast<float *>(smem + (k_base - sbase)));
+  // TMEM is released last: only its owner fences after the barrier (the
+  // fence there held the merge back by several microseconds)
+  if (warp == 1) {
+    tc_fence_after();
+    __syncwarp();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(Lay::kTmemCols)
                  : "memory");
-  // (the K/V ring is idle: the end phase's scratch)
-  if (tp.fused)
-    fused_end_merge(tp, end_rec, *n_end, abort_flag, had_all,
-                    reinterpret_cast<float *>(smem + (k_base - sbase)));
+  }
 }
 
 // ---- host side ------------------------------------------------------------------------
@@ -1471,14 +1538,14 @@ int launch_tc(const TcParams &tp, int smem, cudaStream_t st) {
   const int e = lse_detail::allow_dynamic_smem(k, smem, allowed);
   if (e) return e;
   if (!tp.fused) {
-    k<<<tp.n_ctas, kThreads, smem, st>>>(tp);
+    k<<<tp.n_ctas, tc_threads<P8>(), smem, st>>>(tp);
     return (int)cudaGetLastError();
   }
   // the fused merge waits (bounded) for other CTAs' pieces: a cooperative
   // launch, so every CTA of the grid is resident at once (or the launch fails)
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(tp.n_ctas);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(tc_threads<P8>());
   cfg.dynamicSmemBytes = (size_t)smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
