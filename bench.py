@@ -313,11 +313,12 @@ HEADLINE = "tree_verify"   # the largest single-GPU workload carries the headlin
 
 def time_workload(w, args, flush, dist, clk):
     """Device times of one workload: `args.steps` graph replays of the whole
-    step (lse_attn_forward: on tensor-core plans one launch, the merge fused
-    into the partial pass; on CUDA-core plans the partial pass and the merge
-    as its programmatic dependent) and as many of the dominant kernel alone
-    (the partial pass of a two-kernel step; the step itself when it is one
-    kernel), L2 flushed before each outside the CUDA-event interval.
+    step (lse_attn_forward: one launch, the merge inside the partial pass,
+    on tensor-core plans and on CUDA-core plans with small merges; otherwise
+    the partial pass and the merge as its programmatic dependent) and as many
+    of the dominant kernel alone (the partial pass of a two-kernel step; the
+    step itself when it is one launch), L2 flushed before each outside the
+    CUDA-event interval.
     Returns the DeviceCall (kept for the end-to-end leg) and the per-step
     millisecond lists."""
     import torch
@@ -328,7 +329,7 @@ def time_workload(w, args, flush, dist, clk):
         call.run()
     torch.cuda.synchronize()
     assert call.device_error() == 0, f"{w.name}: device error during warm-up"
-    one_kernel = call.info["kernel_name"] in ("tcgen05", "prefill")
+    one_kernel = call.info["merge_in_pass"] == 1  # the step is one launch
     g_step, g_part = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
     saved = call.stream
     with torch.cuda.graph(g_step):
@@ -383,7 +384,7 @@ def workload_result(w, call, steps_ms, part_ms, world, dist, args, peak, peak_ki
     total_ms = reduce_max(sum(steps_ms), dist, "cuda")
     part_mean = reduce_max(statistics.mean(part_ms), dist, "cuda")
     info = call.info
-    fused = info["kernel_name"] in ("tcgen05", "prefill")
+    fused = info["merge_in_pass"] == 1  # the merge runs inside the partial launch
     bytes_call = w.call_bytes()
     # the dominant kernel's algorithmic bytes: K + V + Q (+ out when the
     # merge is fused into it)

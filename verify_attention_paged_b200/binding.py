@@ -54,7 +54,8 @@ class PlanInfo(ctypes.Structure):
                 ("ctas", ctypes.c_int32), ("workspace_bytes", ctypes.c_int64),
                 ("stages", ctypes.c_int32), ("q_slots", ctypes.c_int32),
                 ("p_bufs", ctypes.c_int32), ("rows_per_chunk", ctypes.c_int32),
-                ("scaled", ctypes.c_int32), ("v_stages", ctypes.c_int32)]
+                ("scaled", ctypes.c_int32), ("v_stages", ctypes.c_int32),
+                ("merge_in_pass", ctypes.c_int32)]
 
 
 class DeviceLimits(ctypes.Structure):
