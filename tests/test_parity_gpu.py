@@ -282,7 +282,8 @@ def test_cuda_core_merge_in_pass(binding, dtype):
     # a CUDA-core plan with small merges: lse_attn_forward is one launch whose
     # last CTA per (sequence, kv head) merges the splits; twice in a row
     # (the counters return to zero), against the oracle and the two passes
-    w = wl.small_case(dtype, [900, 33, 1, 2047, 400], [2, 1, 1, 4, 3], n_q_heads=8,
+    # (capacity 304 keys: at most ten 32-key splits whatever the occupancy)
+    w = wl.small_case(dtype, [300, 33, 1, 170], [2, 1, 1, 3], n_q_heads=8,
                       n_kv_heads=2, head_dim=64, tokens_per_fragment=16, tree=True, seed=250)
     call = binding.DeviceCall(w, kernel="cuda_core")
     assert call.info["merge_in_pass"] == 1 and call.info["n_splits"] > 1
