@@ -314,8 +314,8 @@ HEADLINE = "tree_verify"   # the largest single-GPU workload carries the headlin
 def time_workload(w, args, flush, dist, clk):
     """Device times of one workload: `args.steps` graph replays of the whole
     step (lse_attn_forward: one launch, the merge inside the partial pass,
-    on tensor-core plans and on CUDA-core plans with small merges; otherwise
-    the partial pass and the merge as its programmatic dependent) and as many
+    on tensor-core plans; on CUDA-core plans the partial pass and the merge
+    as its programmatic dependent) and as many
     of the dominant kernel alone (the partial pass of a two-kernel step; the
     step itself when it is one launch), L2 flushed before each outside the
     CUDA-event interval.

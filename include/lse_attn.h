@@ -242,7 +242,8 @@ typedef struct {
   int32_t scaled;          /* 1: made for an arena with per-vector scales  */
   int32_t v_stages;        /* verify tensor-core kernel: V ring depth, else 0 */
   int32_t merge_in_pass;   /* 1: lse_attn_forward merges inside the partial
-                              pass's launch (one launch per call)          */
+                              pass's launch (tensor-core plans); 0: a
+                              partial launch and a merge launch            */
 } lse_attn_plan_info;
 
 LSE_API int lse_attn_plan_query(const lse_attn_plan_t *plan, lse_attn_plan_info *info);
@@ -310,11 +311,8 @@ LSE_API int lse_attn_merge(const lse_attn_plan_t *plan, const int32_t *seq_lens,
  * grid) and uses the workspace's segment counters, which each call leaves
  * at zero.  After a call that set a device error bit, read it with
  * lse_attn_read_error (which then also clears the counters) or call
- * lse_attn_workspace_init before the next call.  For CUDA-core plans whose
- * merges are small (one (sequence, kv head)'s partials at most 256 KB, at
- * most 64 splits) it is one launch too: the last CTA of each (sequence, kv
- * head) to finish merges its splits (same counters, same rule); for the
- * other CUDA-core plans it is lse_attn_run then lse_attn_merge.
+ * lse_attn_workspace_init before the next call.  For CUDA-core plans this
+ * is lse_attn_run then lse_attn_merge.
  * ------------------------------------------------------------------------- */
 LSE_API int lse_attn_forward(const lse_attn_plan_t *plan, const float *q, const int32_t *k_pages,
                              const int32_t *v_pages, const int32_t *seq_lens,

@@ -277,28 +277,6 @@ def test_tcgen05_many_segments_per_cta(binding, dtype):
     assert_close(out_tc, out_cc, dtype, what="tcgen05 vs cuda_core")
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_cuda_core_merge_in_pass(binding, dtype):
-    # a CUDA-core plan with small merges: lse_attn_forward is one launch whose
-    # last CTA per (sequence, kv head) merges the splits; twice in a row
-    # (the counters return to zero), against the oracle and the two passes
-    # (capacity 304 keys: at most ten 32-key splits whatever the occupancy)
-    w = wl.small_case(dtype, [300, 33, 1, 170], [2, 1, 1, 3], n_q_heads=8,
-                      n_kv_heads=2, head_dim=64, tokens_per_fragment=16, tree=True, seed=250)
-    call = binding.DeviceCall(w, kernel="cuda_core")
-    assert call.info["merge_in_pass"] == 1 and call.info["n_splits"] > 1
-    ref_out, ref_lse = orc.attention(to_problem(w))
-    for label, fn in (("one launch", call.run), ("again", call.run),
-                      ("two passes", call.run_two_pass)):
-        out, lse = fn()
-        torch.cuda.synchronize()
-        assert call.device_error() == 0, label
-        assert_close(out[:w.total_rows].cpu().numpy(), ref_out, dtype, what=label)
-        np.testing.assert_allclose(lse[:w.total_rows].cpu().numpy(), ref_lse, rtol=0,
-                                   atol=lse_tol(dtype) * 4)
-    call.close()
-
-
 @pytest.mark.parametrize("dtype", ["f16", "e4m3"])
 @pytest.mark.parametrize("n_sms", [3, 7, 16])
 def test_tcgen05_segment_weighted_cut(binding, dtype, n_sms):

@@ -380,11 +380,6 @@ int lse_attn_plan_ex(const lse_kv_arena *a, int n_seqs, int max_rows, int max_to
     pl->n_splits = lse_attn_split_rule(cap_keys, n_seqs * a->n_kv_heads, n_sms, ctas_per_sm,
                                        pl->key_tile, &kp);
     pl->keys_per_split = kp;
-    // small merges (one (sequence, kv head)'s partials at most 256 KB) run in
-    // the partial pass through lse_attn_forward: one launch instead of two
-    const int64_t merge_bytes = int64_t(pl->pairs) * pl->n_splits * (a->head_dim + 1) * 4;
-    pl->cc_fused = pl->n_splits <= 64 && merge_bytes <= (int64_t(256) << 10);
-    pl->n_seg_max = n_seqs * a->n_kv_heads;  // its counters
   }
 
   const size_t n_part = pl->kernel == LSE_KERNEL_PREFILL
@@ -416,7 +411,7 @@ int lse_attn_plan_query(const lse_attn_plan_t *pl, lse_attn_plan_info *info) {
   info->rows_per_chunk = tc || pf ? pl->rows_per_chunk : 0;
   info->scaled = pl->scaled;
   info->v_stages = tc ? pl->v_stages : 0;
-  info->merge_in_pass = pl->kernel != LSE_KERNEL_CUDA_CORE || pl->cc_fused ? 1 : 0;
+  info->merge_in_pass = pl->kernel != LSE_KERNEL_CUDA_CORE ? 1 : 0;
   return LSE_OK;
 }
 
@@ -599,7 +594,7 @@ int lse_attn_forward(const lse_attn_plan_t *pl, const float *q, const int32_t *k
                      float *lse_out, void *stream, char **err) {
   if (!pl) return fail(err, LSE_ERR_INVALID_ARG, "plan is NULL");
   if (!out) return fail(err, LSE_ERR_INVALID_ARG, "out is NULL");
-  if (pl->kernel != LSE_KERNEL_CUDA_CORE || pl->cc_fused)
+  if (pl->kernel != LSE_KERNEL_CUDA_CORE)
     return launch_partial(pl, q, k_pages, v_pages, seq_lens, row_offsets, row_masks,
                           softmax_scale, ws, out, lse_out, 1, stream, err);
   const int st = launch_partial(pl, q, k_pages, v_pages, seq_lens, row_offsets, row_masks,

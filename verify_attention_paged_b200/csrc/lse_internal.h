@@ -57,8 +57,6 @@ struct lse_attn_plan_s {
   int box_tokens = 0;    // its TMA box height
   int scaled = 0;        // made for an arena with per-vector scales
   int withhold_tile = -1;  // tests of the bounded waits (lse_attn_test_withhold_tile)
-  int cc_fused = 0;      // CUDA-core plan: lse_attn_forward merges in the partial pass
-                         // (the last CTA of each (sequence, kv head) merges its splits)
   // tensor maps of the arena chunks (built on first run, rebuilt on growth);
   // maps_mutex guards them, so threads may run one plan at the same time
   mutable std::vector<uint8_t> maps;

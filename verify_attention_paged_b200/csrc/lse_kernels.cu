@@ -370,48 +370,6 @@ __global__ void __launch_bounds__(kThreads)
     }
     __syncthreads();
   }
-  if (!p.out) return;
-  // One call (lse_attn_forward) on a plan whose merges are small: the last
-  // CTA of this (sequence, kv head) to finish merges the live splits into
-  // out / lse_out (same arithmetic as the merge pass: M = max lse, weights
-  // 2^(lse - M)) and clears the counter for the next call.
-  __shared__ unsigned int s_last;
-  __threadfence();
-  __syncthreads();
-  const int n_live = min((L + p.keys_per_split - 1) / p.keys_per_split, p.n_splits);
-  unsigned int *cnt = p.seg_count + 2 * (s * p.n_kv_heads + g);
-  if (tid == 0) s_last = atomicAdd(cnt, 1u) + 1u == (unsigned)n_live ? 1u : 0u;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  constexpr int kPerLane = D / 32;
-  for (int pr = warp; pr < P; pr += kThreads / 32) {  // a warp per (row, head)
-    const int r = pr / G, h = g * G + (pr - r * G);
-    const long long oi = (long long)(row0 + r) * p.n_q_heads + h;
-    const float *lse = p.lse_part + oi * p.n_splits;
-    const float *o = p.o_part + oi * p.n_splits * D;
-    float M = -INFINITY;
-    for (int i = lane; i < n_live; i += 32) M = fmaxf(M, __ldcg(lse + i));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float W = 0.f, acc[kPerLane];
-#pragma unroll
-    for (int k = 0; k < kPerLane; ++k) acc[k] = 0.f;
-    for (int i = 0; i < n_live; ++i) {
-      const float li = __ldcg(lse + i);
-      const float w = li == -INFINITY ? 0.f : exp2f(li - M);  // empty partial: 0
-      W += w;
-#pragma unroll
-      for (int k = 0; k < kPerLane; ++k)
-        acc[k] = fmaf(w, __ldcg(o + (long long)i * D + lane + 32 * k), acc[k]);
-    }
-    const float inv = W > 0.f ? 1.f / W : 0.f;
-#pragma unroll
-    for (int k = 0; k < kPerLane; ++k) p.out[oi * D + lane + 32 * k] = acc[k] * inv;
-    if (lane == 0 && p.lse_out)
-      p.lse_out[oi] = W > 0.f ? (M + log2f(W)) * 0.69314718055994530942f : -INFINITY;
-  }
-  if (tid == 0) *cnt = 0u;
 }
 
 // ---- merge pass -------------------------------------------------------------
