@@ -78,7 +78,7 @@ constexpr size_t kWsHeader = 256;
 // most kLseSeqTab sequences (the pass keeps them in a shared-memory table)
 // and each working CTA's share is at least kLseSegMinShare tiles.
 constexpr int kLseSeqTab = 96;
-constexpr int kLseSegWeight = 3;
+constexpr int kLseSegWeight = 5;
 constexpr int kLseSegMinShare = 8 * kLseSegWeight;
 
 // Parameters passed by value to the partial and merge kernels.
