@@ -632,7 +632,7 @@ __device__ __noinline__ void fused_end_merge(const TcParams &tp, const EndRec *r
     const int mine = r.piece < P ? (P - 1 - r.piece) / n + 1 : 0;
 #pragma unroll 1
     for (int b = 0; go && b < mine; b += kWarps) {
-      const int np = min(kWarps, mine - b);           // pairs in this round
+      const int np = min(kWarps, mine - b);           // pairs in this batch
       const int kw = kWarps / np;                      // warps per pair
       const int slot = warp / kw, sub = warp - slot * kw;
       const bool active = slot < np;
